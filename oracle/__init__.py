@@ -1,0 +1,222 @@
+"""CPU oracle for paged decode attention — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  It shares no code with the CUDA path (it
+imports nothing from ``serving_attention_paged_b200``) and the CUDA path never
+imports it.
+
+Contents, each written from the FlashInfer README (core features 1-3, the
+single-request decode usage example) and the flashinfer-cubin registry page
+(paged-KV names ``kv_indptr`` / ``kv_indices`` / ``last_page_len``):
+
+* ``paged_decode`` — the attention definition in fp64 (``paged_attention.c``).
+* ``merge_state`` / ``merge_states`` — combining attention states by their
+  log-sum-exp (what split-KV and cascade attention rely on).
+* ``cascade_decode`` — shared prefix merged with per-request suffix.
+* ``plan`` — the split-KV work-list specification restated as a plain
+  linear scan (the library's binary search must agree with it exactly).
+
+Parity status: every function here is pinned by ``tests/test_oracle.py``
+(closed forms, invariants, brute force).  The pages print no worked numeric
+example, so nothing is pinned to a published output value.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "paged_attention.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build_library(force: bool = False) -> str:
+    """Compile the fp64 C oracle with gcc (plain -O2: no fast-math, no FMA)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               _SRC, "-o", _LIB, "-lm"])
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build_library())
+        i32, i64, dbl, vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+        lib.oracle_paged_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                            dbl, vp, i64, vp, vp, i32]
+        lib.oracle_paged_decode.restype = ctypes.c_int
+        lib.oracle_widen.argtypes = [ctypes.c_uint16, i32]
+        lib.oracle_widen.restype = dbl
+        _lib = lib
+    return _lib
+
+
+DTYPE_CODE = {"f16": 0, "bf16": 1}
+
+
+def _as_u16(x) -> np.ndarray:
+    """fp16 / bf16 storage (torch tensor or numpy) as a contiguous uint16 array."""
+    if hasattr(x, "detach"):  # torch tensor: reinterpret its 16-bit storage
+        import torch
+        x = x.detach().cpu().contiguous().view(torch.int16).numpy()
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float16:
+        x = x.view(np.uint16)
+    return x.view(np.uint16)
+
+
+def _as_i32(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def widen(bits: int, dtype: str) -> float:
+    """The oracle's exact fp16 / bf16 -> fp64 widening of one 16-bit pattern."""
+    return _load().oracle_widen(bits, DTYPE_CODE[dtype])
+
+
+def paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, *, num_qo_heads,
+                 num_kv_heads, head_dim, page_size, dtype, sm_scale, rows=None, threads=1):
+    """fp64 attention of every (b, hq) row (or the listed ``rows`` = b*Hq+hq).
+
+    Returns ``(o, lse)``: o ``[n_rows, D]`` fp64 and lse ``[n_rows]`` fp64
+    (natural log; -inf for an empty request).  With ``rows=None`` the result
+    is reshaped to ``[B, Hq, D]`` / ``[B, Hq]``.
+    """
+    lib = _load()
+    qa, ka, va = _as_u16(q), _as_u16(k_pool), _as_u16(v_pool)
+    indptr, indices, last = _as_i32(kv_indptr), _as_i32(kv_indices), _as_i32(last_page_len)
+    batch = len(last)
+    if rows is None:
+        n_rows = batch * num_qo_heads
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = len(rows_arr)
+    o = np.zeros((n_rows, head_dim), dtype=np.float64)
+    lse = np.zeros(n_rows, dtype=np.float64)
+    if indices.size == 0:
+        indices = np.zeros(1, dtype=np.int32)
+    rc = lib.oracle_paged_decode(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, indptr.ctypes.data, indices.ctypes.data,
+        last.ctypes.data if last.size else None, batch, num_qo_heads, num_kv_heads, head_dim,
+        page_size, DTYPE_CODE[dtype], float(sm_scale),
+        rows_arr.ctypes.data if rows_arr is not None else None, n_rows, o.ctypes.data,
+        lse.ctypes.data, int(threads))
+    if rc != 0:
+        raise ValueError("oracle_paged_decode rejected its arguments")
+    if rows is None:
+        return o.reshape(batch, num_qo_heads, head_dim), lse.reshape(batch, num_qo_heads)
+    return o, lse
+
+
+def merge_state(o_a, lse_a, o_b, lse_b):
+    """Combine two attention states over disjoint token sets (fp64).
+
+    With M = max(lse_a, lse_b) and weights w = exp(lse - M):
+    o = (w_a o_a + w_b o_b) / (w_a + w_b),  lse = M + ln(w_a + w_b).
+    Both empty (lse = -inf) gives o = 0, lse = -inf.
+    """
+    return merge_states([(o_a, lse_a), (o_b, lse_b)])
+
+
+def merge_states(states):
+    """Combine any number of attention states ``(o [.., D], lse [..])`` (fp64)."""
+    lses = np.stack([np.asarray(l, dtype=np.float64) for _, l in states])
+    os_ = np.stack([np.asarray(o, dtype=np.float64) for o, _ in states])
+    M = lses.max(axis=0)
+    empty = np.isneginf(M)
+    Ms = np.where(empty, 0.0, M)
+    w = np.exp(lses - Ms)  # exp(-inf) = 0 for empty states
+    wsum = w.sum(axis=0)
+    safe = np.where(empty, 1.0, wsum)
+    o = (w[..., None] * os_).sum(axis=0) / safe[..., None]
+    o = np.where(empty[..., None], 0.0, o)
+    lse = np.where(empty, -np.inf, Ms + np.log(safe))
+    return o, lse
+
+
+def cascade_decode(q, k_pool, v_pool, prefix_indices, prefix_len, kv_indptr, kv_indices,
+                   last_page_len, *, num_qo_heads, num_kv_heads, head_dim, page_size, dtype,
+                   sm_scale, threads=1):
+    """Two-level cascade: attention over the shared prefix, attention over each
+    request's own pages, merged by log-sum-exp (FlashInfer README, core
+    feature 3 "Cascade Attention for hierarchical KV-Cache")."""
+    batch = len(_as_i32(last_page_len))
+    npre = prefix_len // page_size
+    pre_indptr = np.arange(batch + 1, dtype=np.int32) * npre
+    pre_indices = np.tile(_as_i32(prefix_indices)[:npre], batch) if batch else np.zeros(0, np.int32)
+    pre_last = np.full(batch, page_size if npre else 0, dtype=np.int32)
+    kw = dict(num_qo_heads=num_qo_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
+              page_size=page_size, dtype=dtype, sm_scale=sm_scale, threads=threads)
+    o1, l1 = paged_decode(q, k_pool, v_pool, pre_indptr, pre_indices, pre_last, **kw)
+    o2, l2 = paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, **kw)
+    return merge_state(o1, l1, o2, l2)
+
+
+def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per_sm,
+         min_chunk_tokens=256):
+    """Split-KV work list (FlashInfer README core feature 2: variable-length
+    inputs are scheduled in a plan stage to even out the load).
+
+    Specification (the reading adopted where the page is silent):
+      W = num_sms * ctas_per_sm; c_min = max(1, ceil(min_chunk_tokens / P));
+      N = max_b n_b; work(c) = Hkv * sum_b max(1, ceil(n_b / c)).
+      Chunk c (pages): if N <= c_min then max(N, 1); else the smallest c in
+      [c_min, N] with work(c) <= W, or N if none.  Found here by a linear scan.
+      Items: b ascending, chunk j ascending (an empty request has one empty
+      chunk), kv head ascending.  partial_slot is -1 for a one-chunk request,
+      else merge_indptr[b] + j, merge_indptr being the running sum of the
+      chunk counts of the split requests.
+
+    Returns ``(chunk_pages, items, merge_indptr)`` with items an int32 array
+    ``[n, 6]``: request, kv_head, page_begin, page_end, kv_len_in_chunk,
+    partial_slot.
+    """
+    indptr = [int(x) for x in _as_i32(kv_indptr)]
+    last = [int(x) for x in _as_i32(last_page_len)]
+    B, P = len(last), page_size
+    n = [indptr[b + 1] - indptr[b] for b in range(B)]
+    W = num_sms * ctas_per_sm
+    c_min = max(1, -(-min_chunk_tokens // P))
+    N = max(n) if n else 0
+
+    def work(c):
+        return num_kv_heads * sum(max(1, -(-nb // c)) for nb in n)
+
+    if N <= c_min:
+        c = max(N, 1)
+    else:
+        c = N
+        for cand in range(c_min, N + 1):
+            if work(cand) <= W:
+                c = cand
+                break
+
+    chunks = [max(1, -(-nb // c)) for nb in n]
+    merge_indptr = [0]
+    for b in range(B):
+        merge_indptr.append(merge_indptr[-1] + (chunks[b] if chunks[b] > 1 else 0))
+    items = []
+    for b in range(B):
+        for j in range(chunks[b]):
+            pb = indptr[b] + j * c
+            pe = min(pb + c, indptr[b + 1])
+            tokens = (pe - pb) * P
+            if pe == indptr[b + 1] and pe > pb:
+                tokens -= P - last[b]
+            slot = -1 if chunks[b] == 1 else merge_indptr[b] + j
+            for h in range(num_kv_heads):
+                items.append((b, h, pb, pe, tokens, slot))
+    return c, np.array(items, dtype=np.int32).reshape(-1, 6), np.array(merge_indptr, dtype=np.int32)
+
+
+__all__ = ["build_library", "paged_decode", "merge_state", "merge_states", "cascade_decode",
+           "plan", "widen"]
