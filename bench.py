@@ -1,0 +1,406 @@
+#!/usr/bin/env python3
+"""Paged decode attention benchmark: effective KV HBM GB/s, % of peak, µs/step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+
+One step = one decode step of the workload through the run stage (plan made
+beforehand, as a serving engine does once per step and reuses across
+layers): for the plain workloads one ``pa_run`` launch, for the cascade
+``pa_cascade_run``.  Inputs are resident in HBM; L2 is flushed (a 256 MB
+write) before every timed step, outside the CUDA events.  ``value`` is the
+algorithmic K/V bytes of all ranks' steps divided by the max-over-ranks
+device time.  ``e2e`` repeats the step through the public API from host
+buffers: plan on the host, upload of the work list, copies of q and
+kv_indices from pinned memory, the run, and the copy of o and lse back.
+
+With N > 1 (torchrun) every rank runs its own replica of the workload on
+its own GPU (no collective on the data path; the requests of a batch are
+independent), so scaling is weak.
+
+``--impl reference``: the fp64 CPU oracle timed on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode: effective KV HBM GB/s and % of B200 peak; µs per decode step"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="2", help="1 2 3 4 4c 5 (default: 2)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--soak-seconds", type=float, default=1.0,
+                    help="untimed run-in after warm-up so clocks settle and get sampled")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def workload(name):
+    from serving_attention_paged_b200 import workloads as W
+    key = int(name) if name.isdigit() else name
+    return W.WORKLOADS[key]()
+
+
+def workload_config(w):
+    lens = w.kv_lens()
+    cfg = {"workload": w.name, "batch": w.batch, "num_qo_heads": w.num_qo_heads,
+           "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "page_size": w.page_size,
+           "kv_dtype": w.dtype, "accumulate": "f32",
+           "kv_len": (int(lens[0]) if len(set(lens.tolist())) == 1 else
+                      {"min": int(lens.min()), "max": int(lens.max()), "sum": int(lens.sum())}),
+           "pool_pages": w.num_pages, "kv_bytes_per_step": w.kv_bytes(),
+           "l2": "flushed before every timed step (256 MB write, outside the events)"}
+    if w.prefix_len:
+        cfg["shared_prefix_tokens"] = w.prefix_len
+    return cfg
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_sources, workload_name):
+    """DRAM bytes per launch recorded by an ncu capture in profiles/, if the
+    capture's source digest still matches the kernel sources (else None)."""
+    digest = source_digest(kernel_sources)
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for f in sorted(os.listdir(pdir)):
+        if not f.endswith(".md"):
+            continue
+        txt = open(os.path.join(pdir, f)).read()
+        m_w = re.search(r"^workload:\s*(\S+)", txt, re.M)
+        m_d = re.search(r"^source_digest:\s*(\S+)", txt, re.M)
+        m_t = re.search(r"^dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt, re.M)
+        if m_w and m_d and m_t and m_w.group(1) == workload_name and m_d.group(1) == digest:
+            return float(m_t.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.out = tempfile.TemporaryFile(mode="w+")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.seek(0)
+        rows = [r.split(", ") for r in self.out.read().strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 8:
+                continue
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(w, dev, max_requests):
+    """The oracle as it stands, on the host cores, over a bounded sample of
+    the same workload (whole requests, every q head)."""
+    import oracle
+    lens = w.kv_lens()
+    reqs = list(range(min(max_requests, w.batch)))
+    threads = os.cpu_count() or 1
+    indptr, indices, last = w.flat_tables()
+    t0 = time.perf_counter()
+    oracle.paged_decode_requests(dev["q"], dev["k_pool"], dev["v_pool"], indptr, indices, last,
+                                 reqs, num_qo_heads=w.num_qo_heads,
+                                 num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                                 page_size=w.page_size, dtype=w.dtype, sm_scale=w.sm_scale,
+                                 threads=threads)
+    dt = time.perf_counter() - t0
+    toks = sum(int(lens[b]) + w.prefix_len for b in reqs)
+    nbytes = 2 * toks * w.num_kv_heads * w.head_dim * 2
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(reqs)} of {w.batch} requests (all {w.num_qo_heads} q heads each), "
+                      f"{toks} tokens, {nbytes} KV bytes, {dt:.2f} s, fp64"}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 oracle, timed on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = workload(args.workload)
+    # a bounded sample: the first request(s), drawn on the host
+    n_req = 1
+    lens = w.kv_lens()
+    from serving_attention_paged_b200 import workloads as W
+    sub = W.make_workload(w.name, lens[:n_req], num_qo_heads=w.num_qo_heads,
+                          num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                          page_size=w.page_size, dtype=w.dtype, seed=w.seed,
+                          prefix_len=w.prefix_len)
+    t = sub.materialize()
+    indptr, indices, last = sub.flat_tables()
+    threads = os.cpu_count() or 1
+    kw = dict(num_qo_heads=sub.num_qo_heads, num_kv_heads=sub.num_kv_heads,
+              head_dim=sub.head_dim, page_size=sub.page_size, dtype=sub.dtype,
+              sm_scale=sub.sm_scale, threads=threads)
+
+    def step():
+        oracle.paged_decode(t["q"], t["k_pool"], t["v_pool"], indptr, indices, last, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    nbytes = sub.kv_bytes()
+    value = nbytes / sec / 1e9
+    sample = (f"{n_req} of {w.batch} requests per step (all {w.num_qo_heads} q heads), "
+              f"{sub.total_tokens()} tokens, {nbytes} KV bytes, fp64")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}))
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev_t = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev_t,
+                                timeout=datetime.timedelta(seconds=120))
+
+    from serving_attention_paged_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    from serving_attention_paged_b200 import pagedattn as C
+    from serving_attention_paged_b200.wrapper import PagedDecode
+
+    w = workload(args.workload)
+    dev = w.materialize(dev_t)
+    stream = torch.cuda.current_stream(dev_t)
+    t0 = time.perf_counter()
+    pd = PagedDecode(w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
+                     num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
+                     sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
+                     device=dev_t)
+    plan_us = (time.perf_counter() - t0) * 1e6
+    o, lse = pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"],
+                    prefix_indices=dev.get("prefix_indices"))
+    launches_per_step = 2 if (w.prefix_len and w.batch) else 1
+
+    def step():
+        pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"], o, lse,
+               prefix_indices=dev.get("prefix_indices"), stream=stream)
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev_t)
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+
+    uuid = str(torch.cuda.get_device_properties(dev_t).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    t_end = time.perf_counter() + args.soak_seconds
+    while time.perf_counter() < t_end:
+        for _ in range(20):
+            flush.fill_(1.0)
+            step()
+        torch.cuda.synchronize()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
+    for i in range(args.steps):
+        flush.fill_(1.0)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    mean_ms = sum(step_ms) / len(step_ms)
+    t = torch.tensor([mean_ms], dtype=torch.float64, device=dev_t)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+
+    nbytes = w.kv_bytes()
+    value = world * nbytes / (ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    achieved = nbytes / (ms * 1e-3) / 1e9  # one GPU's launch: the dominant (only) kernel
+    kernel_sources = ["serving_attention_paged_b200/csrc/decode.cu",
+                      "serving_attention_paged_b200/csrc/common.cuh"]
+    if w.prefix_len:
+        kernel_sources.append("serving_attention_paged_b200/csrc/cascade.cu")
+    traffic = profiled_traffic(kernel_sources, w.name)
+
+    # end to end through the public API from host buffers
+    e2e = None
+    if not args.no_e2e:
+        q_h = dev["q"].cpu().pin_memory()
+        idx_h = dev["kv_indices"].cpu().pin_memory()
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        q_d = torch.empty_like(dev["q"])
+        idx_d = torch.empty_like(dev["kv_indices"])
+        e2e_s = []
+        for i in range(max(args.warmup, 3) + args.steps):
+            flush.fill_(1.0)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            plan = C.pa_cascade_plan_create(pd.problem, w.prefix_len, w.kv_indptr,
+                                            w.last_page_len) if w.prefix_len else \
+                C.pa_plan_create(pd.problem, w.kv_indptr, w.last_page_len)
+            C.pa_plan_upload(plan, pd.workspace, pd.workspace.numel(), stream)
+            q_d.copy_(q_h, non_blocking=True)
+            idx_d.copy_(idx_h, non_blocking=True)
+            if w.prefix_len:
+                C.pa_cascade_run(plan, q_d, dev["k_pool"], dev["v_pool"], dev["prefix_indices"],
+                                 idx_d, o, lse, pd.workspace, pd.workspace.numel(), stream)
+            else:
+                C.pa_run(plan, q_d, dev["k_pool"], dev["v_pool"], idx_d, o, lse, pd.workspace,
+                         pd.workspace.numel(), stream)
+            o_h.copy_(o, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+            torch.cuda.synchronize()
+            if i >= max(args.warmup, 3):
+                e2e_s.append(time.perf_counter() - t0)
+        e2e_sec = sum(e2e_s) / len(e2e_s)
+        e2e_t = torch.tensor([e2e_sec], dtype=torch.float64, device=dev_t)
+        if world > 1:
+            dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+        items = len(pd.work_items())
+        h2d = (q_h.numel() * q_h.element_size() + idx_h.numel() * 4 + items * 24 +
+               (w.batch + 1) * 4)
+        e2e = {"value": world * nbytes / float(e2e_t.item()) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(o_h.numel() * o_h.element_size() + lse_h.numel() * 4),
+               "us_per_step": float(e2e_t.item()) * 1e6,
+               "includes": "host plan + work-list upload + q/kv_indices H2D + run + o/lse D2H"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        max_req = {"batch_decode_uniform": 16, "single_request_decode": 1}.get(w.name, 4)
+        cpu = cpu_baseline(w, dev, max_req)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "us_per_step": ms * 1e3, "pct_of_peak": 100.0 * achieved / peak,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))",
+            "config": dict(workload_config(w), parallelism=f"replicas x{world}"),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic,
+                         "kernel": "paged_decode_kernel" if not w.prefix_len
+                         else "cascade step (prefix + suffix kernels)"},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": args.steps * launches_per_step,
+            "plan_us": plan_us,
+            "step_ms_p10_p50_p90": [float(np.percentile(step_ms, p)) for p in (10, 50, 90)],
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * pagedattn.h — C ABI of libpagedattn.so: batched decode attention over a
+ * paged KV cache on B200 (sm_100a).
+ *
+ * Where each call comes from (the FlashInfer pages):
+ *   - README, core feature 1: single/batch attention over a sparse (paged)
+ *     KV store; page_size 1 is the "vector-sparse" case.
+ *   - README, core feature 2: the plan/run split.  pa_plan_create is the
+ *     plan stage (host, schedules variable-length requests into a balanced
+ *     split-KV work list); pa_run is the run stage (device).
+ *   - README, core feature 3: cascade attention for a shared prefix
+ *     (pa_cascade_plan_create / pa_cascade_run) and head-query fusion for
+ *     grouped-query attention (every q head of one kv head is computed by
+ *     the same CTA from one load of each K/V row).
+ *   - README, core feature 5: CUDA-graph capture.  pa_run, pa_cascade_run
+ *     and pa_merge_state only enqueue work on the given stream: no host
+ *     synchronisation, no allocation.
+ *   - flashinfer-cubin registry page, quickstart: the paged-table names
+ *     kv_indptr, kv_indices, last_page_len and kv_layout (NHD here).
+ *   - hysenlabs project review, "Installing FlashInfer and running a first
+ *     decode": q is [num_qo_heads, head_dim]; k and v are
+ *     [kv_len, num_kv_heads, head_dim] (NHD).
+ * The merge of partial states by log-sum-exp (pa_merge_state) is not named
+ * on the pages; split-KV and cascade both need it.
+ *
+ * Math (per request b, q head hq, kv head h = hq / (Hq / Hkv)):
+ *   L_b  = 0 if n_b = 0 else (n_b - 1) * P + last_page_len[b]
+ *   row  = kv_indices[kv_indptr[b] + t / P] * P + t % P   for token t < L_b
+ *   s_t  = sm_scale * <q[b,hq,:], k_pool[row,h,:]>
+ *   lse  = ln sum_t exp(s_t)                 (natural log, fp32)
+ *   o    = sum_t exp(s_t - lse) * v_pool[row,h,:]   (rounded once to q's dtype)
+ *   An empty request gives o = 0 and lse = -inf.
+ *
+ * Layouts (all row-major, contiguous, device memory unless marked host):
+ *   q, o        [batch, num_qo_heads, head_dim]          fp16 or bf16
+ *   lse         [batch, num_qo_heads]                    fp32 (may be NULL)
+ *   k/v pool    [num_pages, page_size, num_kv_heads, head_dim]   (NHD)
+ *   kv_indptr   [batch + 1] int32, kv_indices [kv_indptr[batch]] int32,
+ *   last_page_len [batch] int32.
+ *
+ * Ownership: the caller owns every device buffer, the workspace included;
+ * the library never allocates device memory.  A plan owns its host arrays
+ * until pa_plan_destroy.  Functions return a pa_status; nothing throws
+ * across the ABI.  Launch failures return PA_ERR_CUDA.
+ *
+ * Supported: head_dim 128; num_qo_heads / num_kv_heads in {1, 2, 4, 8, 16};
+ * page_size a power of two in [1, 1024]; fp16 and bf16.
+ */
+#ifndef PAGEDATTN_H_
+#define PAGEDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_ABI_VERSION 1
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,          /* malformed tables, null pointers, bad sizes */
+  PA_ERR_UNSUPPORTED = 2,          /* valid but not built (head_dim, group size, page size) */
+  PA_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace shorter than pa_plan_workspace_bytes */
+  PA_ERR_CUDA = 4,                 /* a CUDA runtime call or launch failed */
+  PA_ERR_DEVICE_CHECK = 5,         /* a checked run found an out-of-range page index */
+  PA_ERR_NO_MEMORY = 6             /* host allocation failed */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 /* pa_merge_state only */ } pa_dtype;
+
+/* Flags for pa_problem.flags. */
+#define PA_FLAG_CHECK_INDICES 1u /* kernels bounds-check every page index against
+                                    num_pages; a bad index is skipped (its tokens
+                                    read as zero) and recorded for pa_plan_check */
+
+typedef struct {
+  int32_t batch;            /* requests B >= 0 */
+  int32_t num_qo_heads;     /* Hq */
+  int32_t num_kv_heads;     /* Hkv; Hq % Hkv == 0 */
+  int32_t head_dim;         /* D (128) */
+  int32_t page_size;        /* P, tokens per page */
+  pa_dtype dtype;           /* of q, o, k_pool, v_pool */
+  float sm_scale;           /* softmax scale, always given by the caller (1/sqrt(D) usually) */
+  int32_t num_sms;          /* CTA budget W = num_sms * ctas_per_sm; explicit so that  */
+  int32_t ctas_per_sm;      /*   the plan is a pure function of its inputs              */
+  int32_t min_chunk_tokens; /* smallest split-KV chunk in tokens; 0 means 256 */
+  int64_t num_pages;        /* pages in the pool (bounds for PA_FLAG_CHECK_INDICES) */
+  uint32_t flags;           /* PA_FLAG_* */
+} pa_problem;
+
+/* One unit of run-stage work: kv head `kv_head` of request `request` over
+ * pages kv_indices[page_begin .. page_end) (absolute positions, so the run
+ * stage needs no kv_indptr), holding kv_len_in_chunk tokens.  partial_slot
+ * is -1 when the chunk is the request's only one (the item writes o and lse
+ * itself), else the row of the fp32 partial-state buffer it fills. */
+typedef struct {
+  int32_t request, kv_head, page_begin, page_end, kv_len_in_chunk, partial_slot;
+} pa_work_item;
+
+typedef struct pa_plan_s* pa_plan_t;
+
+/* Plan stage (host only, no CUDA call).  Specification of the work list:
+ *   W = num_sms * ctas_per_sm, c_min = max(1, ceil(min_chunk_tokens / P)),
+ *   N = max_b n_b, work(c) = Hkv * sum_b max(1, ceil(n_b / c)).
+ *   chunk c (pages) = max(N, 1) if N <= c_min, else the smallest c in
+ *   [c_min, N] with work(c) <= W (binary search; N if none).
+ *   Items ordered by request, then chunk, then kv head.  Chunk j of request b
+ *   covers pages [kv_indptr[b] + j*c, min(kv_indptr[b] + (j+1)*c, kv_indptr[b+1])).
+ *   merge_indptr[b+1] - merge_indptr[b] = chunks of b if > 1, else 0.
+ * Validates: kv_indptr[0] == 0 and non-decreasing, 1 <= last_page_len[b] <= P
+ * whenever request b has pages, Hq % Hkv == 0, positive sizes.
+ * Returns PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED otherwise.  The host arrays
+ * are copied; the caller may free them after the call. */
+pa_status pa_plan_create(const pa_problem* problem, const int32_t* kv_indptr_host,
+                         const int32_t* last_page_len_host, pa_plan_t* out);
+
+/* Plan for a two-level cascade: a shared prefix of prefix_len tokens (whole
+ * pages, prefix_len % P == 0) that every request attends to first, plus each
+ * request's own pages described by kv_indptr_host / last_page_len_host.  The
+ * work list is the one pa_plan_create gives for the per-request pages; the
+ * prefix level is scheduled as (kv head, 128-query-row tile, prefix chunk)
+ * tiles on the tensor cores. */
+pa_status pa_cascade_plan_create(const pa_problem* problem, int32_t prefix_len,
+                                 const int32_t* kv_indptr_host,
+                                 const int32_t* last_page_len_host, pa_plan_t* out);
+
+/* Read-only views of the plan (borrowed; valid until pa_plan_destroy). */
+pa_status pa_plan_chunk_pages(pa_plan_t plan, int32_t* chunk_pages);
+pa_status pa_plan_work_items(pa_plan_t plan, const pa_work_item** items, int64_t* n_items);
+pa_status pa_plan_merge_indptr(pa_plan_t plan, const int32_t** merge_indptr /* [B+1] */);
+pa_status pa_plan_num_partials(pa_plan_t plan, int64_t* n_partials);
+pa_status pa_plan_prefix_chunks(pa_plan_t plan, int32_t* n_chunks, int32_t* chunk_tokens);
+
+/* Device workspace the run stage needs: work list, merge offsets, arrival
+ * counters and fp32 partial states.  Caller-allocated, 256-byte aligned. */
+pa_status pa_plan_workspace_bytes(pa_plan_t plan, size_t* bytes);
+
+/* Copy the work list into the workspace and zero its counters (enqueued on
+ * `stream`, a cudaStream_t or NULL for the legacy default stream).  Once per
+ * plan and workspace; any number of runs may follow.  The counters return to
+ * zero at the end of every run, so captured graphs can be replayed. */
+pa_status pa_plan_upload(pa_plan_t plan, void* d_workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Run stage: decode attention for every request of the plan.  kv_indices is
+ * the device copy of the table the plan was made from.  One launch; split
+ * requests are merged inside it by the last CTA to finish (no second
+ * kernel).  lse may be NULL. */
+pa_status pa_run(pa_plan_t plan, const void* q, const void* k_pool, const void* v_pool,
+                 const int32_t* d_kv_indices, void* o, float* lse, void* d_workspace,
+                 size_t workspace_bytes, void* stream);
+
+/* Cascade run: level 1 attends all B * Hq query rows to the shared prefix
+ * (pages d_prefix_indices[0 .. prefix_len / P)) on the tensor cores; level 2
+ * is the paged decode over each request's own pages; both are merged by
+ * log-sum-exp into o and lse.  The plan must come from pa_cascade_plan_create. */
+pa_status pa_cascade_run(pa_plan_t plan, const void* q, const void* k_pool,
+                         const void* v_pool, const int32_t* d_prefix_indices,
+                         const int32_t* d_kv_indices, void* o, float* lse, void* d_workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Combine two attention states over disjoint token sets, row by row:
+ *   M = max(lse_a, lse_b), w_x = exp(lse_x - M),
+ *   o = (w_a o_a + w_b o_b) / (w_a + w_b),   lse = M + ln(w_a + w_b).
+ * Both lse = -inf gives o = 0, lse = -inf.  o_* are [rows, head_dim] in
+ * `dtype` (fp16, bf16 or fp32), lse_* are [rows] fp32 natural-log.  The
+ * outputs may alias either input. */
+pa_status pa_merge_state(const void* o_a, const float* lse_a, const void* o_b,
+                         const float* lse_b, void* o, float* lse, int64_t rows,
+                         int32_t head_dim, pa_dtype dtype, void* stream);
+
+/* After a run with PA_FLAG_CHECK_INDICES: synchronously read the device
+ * error word (PA_OK, or PA_ERR_DEVICE_CHECK with the first bad kv_indices
+ * position in *bad_position) and clear it. */
+pa_status pa_plan_check(pa_plan_t plan, void* d_workspace, int64_t* bad_position, void* stream);
+
+/* Scheduling defaults for `device`: its SM count and how many decode CTAs
+ * of this shape fit on one SM. */
+pa_status pa_default_schedule(int32_t device, int32_t num_qo_heads, int32_t num_kv_heads,
+                              pa_dtype dtype, int32_t* num_sms, int32_t* ctas_per_sm);
+
+void pa_plan_destroy(pa_plan_t plan);
+const char* pa_status_string(pa_status status);
+int32_t pa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H_ */

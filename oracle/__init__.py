@@ -117,6 +117,38 @@ def paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, *, num
     return o, lse
 
 
+def paged_decode_requests(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, requests, *,
+                          num_qo_heads, num_kv_heads, head_dim, page_size, dtype, sm_scale,
+                          threads=1):
+    """``paged_decode`` for every q head of the listed requests only.
+
+    q and the pools may be large torch tensors on any device: only the pages
+    those requests read are copied to the host, as a compact pool with the
+    page table renumbered to match (the tokens each request reads, and their
+    order, are unchanged).  Returns o ``[len(requests), Hq, D]`` and lse.
+    """
+    indptr, indices, last = _as_i32(kv_indptr), _as_i32(kv_indices), _as_i32(last_page_len)
+    pages = [indices[indptr[b]:indptr[b + 1]] for b in requests]
+    used = np.unique(np.concatenate(pages)) if pages else np.zeros(0, np.int64)
+    remap = np.full(int(used.max()) + 1 if used.size else 1, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    sub_indptr = np.zeros(len(requests) + 1, np.int32)
+    sub_indptr[1:] = np.cumsum([len(p) for p in pages])
+    sub_indices = (remap[np.concatenate(pages)] if pages else np.zeros(0)).astype(np.int32)
+    sub_last = last[np.asarray(requests, dtype=np.int64)] if len(requests) else last[:0]
+    if hasattr(k_pool, "detach"):
+        import torch
+        sel = torch.from_numpy(used.astype(np.int64)).to(k_pool.device)
+        kp, vp = k_pool[sel].cpu(), v_pool[sel].cpu()
+        qs = q[torch.as_tensor(list(requests), dtype=torch.int64, device=q.device)].cpu()
+    else:
+        kp, vp, qs = k_pool[used], v_pool[used], q[list(requests)]
+    return paged_decode(qs, kp, vp, sub_indptr, sub_indices, sub_last,
+                        num_qo_heads=num_qo_heads, num_kv_heads=num_kv_heads,
+                        head_dim=head_dim, page_size=page_size, dtype=dtype,
+                        sm_scale=sm_scale, threads=threads)
+
+
 def merge_state(o_a, lse_a, o_b, lse_b):
     """Combine two attention states over disjoint token sets (fp64).
 
@@ -218,5 +250,5 @@ def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per
     return c, np.array(items, dtype=np.int32).reshape(-1, 6), np.array(merge_indptr, dtype=np.int32)
 
 
-__all__ = ["build_library", "paged_decode", "merge_state", "merge_states", "cascade_decode",
+__all__ = ["build_library", "paged_decode", "paged_decode_requests", "merge_state", "merge_states", "cascade_decode",
            "plan", "widen"]

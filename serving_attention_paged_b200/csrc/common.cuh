@@ -1,0 +1,103 @@
+// Small device helpers shared by the kernels of libpagedattn.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace pa {
+
+struct F16 {};   // fp16 storage tag
+struct BF16 {};  // bf16 storage tag
+
+// 8 packed 16-bit values (one 16-byte vector) -> 8 floats.
+__device__ __forceinline__ void to_float8(F16, const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// bf16 is the high half of an fp32: widening is a shift or a mask.
+__device__ __forceinline__ void to_float8(BF16, const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint16_t from_float(F16, float x) {
+  return __half_as_ushort(__float2half_rn(x));
+}
+__device__ __forceinline__ uint16_t from_float(BF16, float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+__device__ __forceinline__ float to_float(F16, uint16_t x) {
+  return __half2float(__ushort_as_half(x));
+}
+__device__ __forceinline__ float to_float(BF16, uint16_t x) {
+  return __uint_as_float(uint32_t(x) << 16);
+}
+
+// Hardware base-2 exponential and logarithm (MUFU), flush-to-zero.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float fast_log2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 16-byte global -> shared copy that bypasses L1; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_addr), "l"(gptr),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Running log-sum-exp merge of attention states, base 2:
+// adding (o, lse2) keeps acc / l = the merged output, m + log2(l) = merged lse.
+struct MergeAcc {
+  float m = -INFINITY, l = 0.f, acc = 0.f;
+  __device__ __forceinline__ void add(float o, float lse2) {
+    if (lse2 == -INFINITY) return;
+    if (lse2 > m) {
+      const float s = fast_exp2(m - lse2);  // m = -inf -> 0
+      l = l * s + 1.f;
+      acc = acc * s + o;
+      m = lse2;
+    } else {
+      const float w = fast_exp2(lse2 - m);
+      l += w;
+      acc += w * o;
+    }
+  }
+  __device__ __forceinline__ float out() const { return m == -INFINITY ? 0.f : acc / l; }
+  __device__ __forceinline__ float lse2() const {
+    return m == -INFINITY ? -INFINITY : m + fast_log2(l);
+  }
+};
+
+}  // namespace pa

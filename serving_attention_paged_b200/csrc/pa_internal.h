@@ -1,0 +1,76 @@
+// Internal declarations shared by the host plan, the C-ABI entry points and
+// the kernels of libpagedattn.so.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "pagedattn.h"
+
+namespace pa {
+
+constexpr int kHeadDim = 128;
+constexpr int kDefaultMinChunkTokens = 256;
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// Device workspace, in this order (each region 256-byte aligned):
+//   items        [n_items]             pa_work_item
+//   merge_indptr [B + 1]               int32
+//   counters     [B * Hkv]             int32, zero between runs
+//   error        [1]                   uint64, first bad kv_indices position (~0 = none)
+//   partial_o    [n_partials, Hq, D]   fp32, split-chunk outputs (normalised)
+//   partial_lse  [n_partials, Hq]      fp32, their log-sum-exp in base 2
+//   prefix_o     [prefix_chunks, B, Hq, D]  fp32 (cascade only)
+//   prefix_lse   [prefix_chunks, B, Hq]     fp32, base 2 (cascade only)
+struct WorkspaceLayout {
+  size_t items = 0, merge_indptr = 0, counters = 0, error = 0, partial_o = 0, partial_lse = 0,
+         prefix_o = 0, prefix_lse = 0, total = 0;
+};
+
+}  // namespace pa
+
+struct pa_plan_s {
+  pa_problem prob{};
+  int32_t group = 1;        // Hq / Hkv
+  int32_t log2_page = 0;    // page_size = 1 << log2_page
+  int32_t chunk_pages = 1;
+  std::vector<int32_t> kv_indptr, last_page_len;
+  std::vector<pa_work_item> items;
+  std::vector<int32_t> merge_indptr;
+  int64_t n_partials = 0;
+  // cascade (level 1 over the shared prefix)
+  bool cascade = false;
+  int32_t prefix_len = 0;
+  int32_t prefix_chunks = 0;        // split of the prefix across CTAs
+  int32_t prefix_chunk_tokens = 0;  // tokens per chunk (multiple of the 128-key tile)
+  int32_t q_tiles = 0;              // 128-row tiles over the B * G query rows of one kv head
+  pa::WorkspaceLayout ws;
+};
+
+namespace pa {
+
+// Kernel launchers (decode.cu, merge_state.cu, cascade.cu).  They return a
+// cudaError_t value as int.
+struct RunPointers {
+  const void* q;
+  const void* k_pool;
+  const void* v_pool;
+  const int32_t* kv_indices;
+  const int32_t* prefix_indices;
+  void* o;
+  float* lse;
+  uint8_t* ws;
+};
+
+int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream);
+int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* stream);
+int launch_merge_state(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                       void* o, float* lse, int64_t rows, int32_t head_dim, pa_dtype dtype,
+                       void* stream);
+int decode_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out);
+bool decode_group_supported(int32_t group);
+
+}  // namespace pa

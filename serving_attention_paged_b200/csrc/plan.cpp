@@ -1,0 +1,254 @@
+// Plan stage: page tables and kv lengths -> load-balanced split-KV work list.
+//
+// FlashInfer README, core feature 2 ("Load-Balanced Scheduling"): the
+// attention computation is split into a plan stage that schedules
+// variable-length inputs and a run stage that computes.  The page gives no
+// algorithm; the specification implemented here is documented with
+// pa_plan_create in pagedattn.h.  Host code only: no CUDA call.
+#include <algorithm>
+#include <cstring>
+#include <new>
+
+#include "pa_internal.h"
+
+namespace {
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int32_t ilog2(int64_t x) {
+  int32_t r = 0;
+  while ((int64_t(1) << r) < x) ++r;
+  return r;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+pa_status validate_problem(const pa_problem* p) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->num_qo_heads <= 0 || p->num_kv_heads <= 0 || p->head_dim <= 0 ||
+      p->page_size <= 0 || p->num_sms <= 0 || p->ctas_per_sm <= 0 || p->min_chunk_tokens < 0 ||
+      p->num_pages < 0)
+    return PA_ERR_INVALID_ARG;
+  if (p->num_qo_heads % p->num_kv_heads) return PA_ERR_INVALID_ARG;
+  if (!(p->sm_scale == p->sm_scale)) return PA_ERR_INVALID_ARG;  // NaN
+  if (p->dtype != PA_F16 && p->dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (p->head_dim != pa::kHeadDim) return PA_ERR_UNSUPPORTED;
+  if (!is_pow2(p->page_size) || p->page_size > 1024) return PA_ERR_UNSUPPORTED;
+  if (!pa::decode_group_supported(p->num_qo_heads / p->num_kv_heads)) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+// Work items for a given chunk size (pages): Hkv * sum_b max(1, ceil(n_b / c)).
+int64_t work(const std::vector<int64_t>& n, int64_t c, int64_t hkv) {
+  int64_t w = 0;
+  for (int64_t nb : n) w += std::max<int64_t>(1, ceil_div(nb, c));
+  return w * hkv;
+}
+
+pa_status build(pa_plan_s* plan, const int32_t* indptr, const int32_t* last) {
+  const pa_problem& p = plan->prob;
+  const int64_t B = p.batch, P = p.page_size, Hkv = p.num_kv_heads;
+  if (B > 0 && (!indptr || !last)) return PA_ERR_INVALID_ARG;
+  if (indptr && indptr[0] != 0) return PA_ERR_INVALID_ARG;
+  std::vector<int64_t> n(B);
+  for (int64_t b = 0; b < B; ++b) {
+    if (indptr[b + 1] < indptr[b]) return PA_ERR_INVALID_ARG;
+    n[b] = int64_t(indptr[b + 1]) - indptr[b];
+    if (n[b] > 0 && (last[b] < 1 || last[b] > P)) return PA_ERR_INVALID_ARG;
+  }
+  plan->kv_indptr.assign(indptr ? indptr : nullptr, indptr ? indptr + B + 1 : nullptr);
+  if (!indptr) plan->kv_indptr.assign(1, 0);
+  plan->last_page_len.assign(last ? last : nullptr, last ? last + B : nullptr);
+
+  // chunk size: smallest c in [c_min, N] with work(c) <= W (work is non-increasing in c)
+  const int64_t W = int64_t(p.num_sms) * p.ctas_per_sm;
+  const int64_t min_tokens = p.min_chunk_tokens ? p.min_chunk_tokens : pa::kDefaultMinChunkTokens;
+  const int64_t c_min = std::max<int64_t>(1, ceil_div(min_tokens, P));
+  const int64_t N = B ? *std::max_element(n.begin(), n.end()) : 0;
+  int64_t c;
+  if (N <= c_min) {
+    c = std::max<int64_t>(N, 1);
+  } else if (work(n, N, Hkv) > W) {
+    c = N;
+  } else {
+    int64_t lo = c_min, hi = N;
+    while (lo < hi) {
+      int64_t mid = lo + (hi - lo) / 2;
+      if (work(n, mid, Hkv) <= W) hi = mid; else lo = mid + 1;
+    }
+    c = lo;
+  }
+  plan->chunk_pages = int32_t(c);
+
+  plan->merge_indptr.assign(B + 1, 0);
+  for (int64_t b = 0; b < B; ++b) {
+    int64_t chunks = std::max<int64_t>(1, ceil_div(n[b], c));
+    plan->merge_indptr[b + 1] = plan->merge_indptr[b] + int32_t(chunks > 1 ? chunks : 0);
+  }
+  plan->n_partials = plan->merge_indptr[B];
+
+  const int64_t total = work(n, c, Hkv);
+  if (total > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  plan->items.clear();
+  plan->items.reserve(size_t(total));
+  for (int64_t b = 0; b < B; ++b) {
+    const int64_t chunks = std::max<int64_t>(1, ceil_div(n[b], c));
+    for (int64_t j = 0; j < chunks; ++j) {
+      const int64_t pb = indptr[b] + j * c;
+      const int64_t pe = std::min<int64_t>(pb + c, indptr[b + 1]);
+      int64_t tokens = (pe - pb) * P;
+      if (pe == indptr[b + 1] && pe > pb) tokens -= P - last[b];
+      const int32_t slot = chunks == 1 ? -1 : int32_t(plan->merge_indptr[b] + j);
+      for (int64_t h = 0; h < Hkv; ++h)
+        plan->items.push_back(pa_work_item{int32_t(b), int32_t(h), int32_t(pb), int32_t(pe),
+                                           int32_t(tokens), slot});
+    }
+  }
+  return PA_OK;
+}
+
+void layout_workspace(pa_plan_s* plan) {
+  const pa_problem& p = plan->prob;
+  pa::WorkspaceLayout& w = plan->ws;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = pa::align_up(off + bytes);
+    return at;
+  };
+  const size_t Hq = p.num_qo_heads, D = p.head_dim, B = p.batch;
+  w.items = take(plan->items.size() * sizeof(pa_work_item));
+  w.merge_indptr = take((B + 1) * sizeof(int32_t));
+  w.counters = take(B * p.num_kv_heads * sizeof(int32_t));
+  w.error = take(sizeof(uint64_t));
+  w.partial_o = take(size_t(plan->n_partials) * Hq * D * sizeof(float));
+  w.partial_lse = take(size_t(plan->n_partials) * Hq * sizeof(float));
+  w.prefix_o = take(size_t(plan->prefix_chunks) * B * Hq * D * sizeof(float));
+  w.prefix_lse = take(size_t(plan->prefix_chunks) * B * Hq * sizeof(float));
+  w.total = off;
+}
+
+// Level-1 cascade schedule: (kv head, 128-row query tile, prefix chunk) tiles,
+// about one per SM; each chunk a whole number of 128-key tiles.
+void schedule_prefix(pa_plan_s* plan) {
+  const pa_problem& p = plan->prob;
+  constexpr int64_t kTileKeys = 128, kTileRows = 128;
+  const int64_t rows = int64_t(p.batch) * plan->group;
+  plan->q_tiles = int32_t(std::max<int64_t>(1, ceil_div(rows, kTileRows)));
+  const int64_t key_tiles = ceil_div(plan->prefix_len, kTileKeys);
+  if (plan->prefix_len == 0 || p.batch == 0) {
+    plan->prefix_chunks = 0;
+    plan->prefix_chunk_tokens = 0;
+    return;
+  }
+  const int64_t base = int64_t(p.num_kv_heads) * plan->q_tiles;
+  int64_t chunks = std::max<int64_t>(1, std::min<int64_t>(int64_t(p.num_sms) / base, key_tiles));
+  const int64_t tiles_per_chunk = ceil_div(key_tiles, chunks);
+  chunks = ceil_div(key_tiles, tiles_per_chunk);
+  plan->prefix_chunks = int32_t(chunks);
+  plan->prefix_chunk_tokens = int32_t(tiles_per_chunk * kTileKeys);
+}
+
+pa_status create(const pa_problem* problem, int32_t prefix_len, bool cascade,
+                 const int32_t* indptr, const int32_t* last, pa_plan_t* out) {
+  if (!out) return PA_ERR_INVALID_ARG;
+  *out = nullptr;
+  pa_status st = validate_problem(problem);
+  if (st != PA_OK) return st;
+  if (cascade && (prefix_len < 0 || prefix_len % problem->page_size)) return PA_ERR_INVALID_ARG;
+  pa_plan_s* plan = new (std::nothrow) pa_plan_s;
+  if (!plan) return PA_ERR_NO_MEMORY;
+  try {
+    plan->prob = *problem;
+    if (plan->prob.min_chunk_tokens == 0) plan->prob.min_chunk_tokens = pa::kDefaultMinChunkTokens;
+    plan->group = problem->num_qo_heads / problem->num_kv_heads;
+    plan->log2_page = ilog2(problem->page_size);
+    plan->cascade = cascade;
+    plan->prefix_len = cascade ? prefix_len : 0;
+    st = build(plan, indptr, last);
+    if (st == PA_OK) {
+      if (cascade) schedule_prefix(plan);
+      layout_workspace(plan);
+    }
+  } catch (const std::bad_alloc&) {
+    st = PA_ERR_NO_MEMORY;
+  }
+  if (st != PA_OK) {
+    delete plan;
+    return st;
+  }
+  *out = plan;
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_plan_create(const pa_problem* problem, const int32_t* kv_indptr_host,
+                         const int32_t* last_page_len_host, pa_plan_t* out) {
+  return create(problem, 0, false, kv_indptr_host, last_page_len_host, out);
+}
+
+pa_status pa_cascade_plan_create(const pa_problem* problem, int32_t prefix_len,
+                                 const int32_t* kv_indptr_host,
+                                 const int32_t* last_page_len_host, pa_plan_t* out) {
+  return create(problem, prefix_len, true, kv_indptr_host, last_page_len_host, out);
+}
+
+pa_status pa_plan_chunk_pages(pa_plan_t plan, int32_t* chunk_pages) {
+  if (!plan || !chunk_pages) return PA_ERR_INVALID_ARG;
+  *chunk_pages = plan->chunk_pages;
+  return PA_OK;
+}
+
+pa_status pa_plan_work_items(pa_plan_t plan, const pa_work_item** items, int64_t* n_items) {
+  if (!plan || !items || !n_items) return PA_ERR_INVALID_ARG;
+  *items = plan->items.data();
+  *n_items = int64_t(plan->items.size());
+  return PA_OK;
+}
+
+pa_status pa_plan_merge_indptr(pa_plan_t plan, const int32_t** merge_indptr) {
+  if (!plan || !merge_indptr) return PA_ERR_INVALID_ARG;
+  *merge_indptr = plan->merge_indptr.data();
+  return PA_OK;
+}
+
+pa_status pa_plan_num_partials(pa_plan_t plan, int64_t* n_partials) {
+  if (!plan || !n_partials) return PA_ERR_INVALID_ARG;
+  *n_partials = plan->n_partials;
+  return PA_OK;
+}
+
+pa_status pa_plan_prefix_chunks(pa_plan_t plan, int32_t* n_chunks, int32_t* chunk_tokens) {
+  if (!plan || !n_chunks || !chunk_tokens) return PA_ERR_INVALID_ARG;
+  *n_chunks = plan->prefix_chunks;
+  *chunk_tokens = plan->prefix_chunk_tokens;
+  return PA_OK;
+}
+
+pa_status pa_plan_workspace_bytes(pa_plan_t plan, size_t* bytes) {
+  if (!plan || !bytes) return PA_ERR_INVALID_ARG;
+  *bytes = plan->ws.total;
+  return PA_OK;
+}
+
+void pa_plan_destroy(pa_plan_t plan) { delete plan; }
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case PA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_DEVICE_CHECK: return "device check failed: page index out of range";
+    case PA_ERR_NO_MEMORY: return "host allocation failed";
+  }
+  return "unknown status";
+}
+
+int32_t pa_abi_version(void) { return PA_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,247 @@
+"""ctypes binding of libpagedattn.so: the C ABI of ``include/pagedattn.h``.
+
+Argument marshalling only.  Every step of the attention path runs in the
+library's CUDA kernels; there is no Python or CPU fallback.  If the library
+is missing the import fails loudly.  Functions keep the C names; device
+buffers may be given as torch tensors (their ``data_ptr()`` is passed) or
+as raw integer addresses, and streams as ``torch.cuda.Stream`` or raw
+``cudaStream_t`` integers (default: torch's current stream).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m serving_attention_paged_b200.build` "
+        "(there is no fallback implementation)")
+lib = ctypes.CDLL(_LIB_PATH)
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL = 0, 1, 2, 3
+PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_NO_MEMORY = 4, 5, 6
+PA_F16, PA_BF16, PA_F32 = 0, 1, 2
+PA_FLAG_CHECK_INDICES = 1
+DTYPE_CODES = {"f16": PA_F16, "bf16": PA_BF16, "f32": PA_F32}
+
+
+class pa_problem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_qo_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("sm_scale", ctypes.c_float), ("num_sms", ctypes.c_int32),
+                ("ctas_per_sm", ctypes.c_int32), ("min_chunk_tokens", ctypes.c_int32),
+                ("num_pages", ctypes.c_int64), ("flags", ctypes.c_uint32)]
+
+
+class pa_work_item(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("request", "kv_head", "page_begin", "page_end", "kv_len_in_chunk", "partial_slot")]
+
+
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_P = ctypes.POINTER
+_SIGS = {
+    "pa_plan_create": [_P(pa_problem), _vp, _vp, _P(_vp)],
+    "pa_cascade_plan_create": [_P(pa_problem), _i32, _vp, _vp, _P(_vp)],
+    "pa_plan_chunk_pages": [_vp, _P(_i32)],
+    "pa_plan_work_items": [_vp, _P(_P(pa_work_item)), _P(_i64)],
+    "pa_plan_merge_indptr": [_vp, _P(_P(_i32))],
+    "pa_plan_num_partials": [_vp, _P(_i64)],
+    "pa_plan_prefix_chunks": [_vp, _P(_i32), _P(_i32)],
+    "pa_plan_workspace_bytes": [_vp, _P(_sz)],
+    "pa_plan_upload": [_vp, _vp, _sz, _vp],
+    "pa_run": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "pa_cascade_run": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "pa_merge_state": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp],
+    "pa_plan_check": [_vp, _vp, _P(_i64), _vp],
+    "pa_default_schedule": [_i32, _i32, _i32, _i32, _P(_i32), _P(_i32)],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = ctypes.c_int
+lib.pa_plan_destroy.argtypes = [_vp]
+lib.pa_plan_destroy.restype = None
+lib.pa_status_string.argtypes = [ctypes.c_int]
+lib.pa_status_string.restype = ctypes.c_char_p
+lib.pa_abi_version.argtypes = []
+lib.pa_abi_version.restype = ctypes.c_int32
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.pa_status_string(status).decode()} (status {status})")
+
+
+def _check(status: int, where: str):
+    if status != PA_OK:
+        raise PagedAttnError(status, where)
+
+
+def _ptr(x):
+    """Device (or host) address of a tensor / integer / None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _host_i32(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+class Plan:
+    """Owns a ``pa_plan_t`` and the host arrays it was made from."""
+
+    def __init__(self, handle: int):
+        self.handle = handle
+
+    def __del__(self):
+        if getattr(self, "handle", None):
+            lib.pa_plan_destroy(self.handle)
+            self.handle = None
+
+
+def make_problem(*, batch, num_qo_heads, num_kv_heads, head_dim=128, page_size, dtype,
+                 sm_scale, num_sms, ctas_per_sm, min_chunk_tokens=0, num_pages=0,
+                 flags=0) -> pa_problem:
+    if isinstance(dtype, str):
+        dtype = DTYPE_CODES[dtype]
+    return pa_problem(batch, num_qo_heads, num_kv_heads, head_dim, page_size, dtype, sm_scale,
+                      num_sms, ctas_per_sm, min_chunk_tokens, num_pages, flags)
+
+
+def pa_plan_create(problem: pa_problem, kv_indptr_host, last_page_len_host) -> Plan:
+    indptr, last = _host_i32(kv_indptr_host), _host_i32(last_page_len_host)
+    h = _vp()
+    _check(lib.pa_plan_create(ctypes.byref(problem), indptr.ctypes.data,
+                              last.ctypes.data if last.size else None, ctypes.byref(h)),
+           "pa_plan_create")
+    return Plan(h.value)
+
+
+def pa_cascade_plan_create(problem: pa_problem, prefix_len: int, kv_indptr_host,
+                           last_page_len_host) -> Plan:
+    indptr, last = _host_i32(kv_indptr_host), _host_i32(last_page_len_host)
+    h = _vp()
+    _check(lib.pa_cascade_plan_create(ctypes.byref(problem), prefix_len, indptr.ctypes.data,
+                                      last.ctypes.data if last.size else None, ctypes.byref(h)),
+           "pa_cascade_plan_create")
+    return Plan(h.value)
+
+
+def pa_plan_chunk_pages(plan: Plan) -> int:
+    c = _i32()
+    _check(lib.pa_plan_chunk_pages(plan.handle, ctypes.byref(c)), "pa_plan_chunk_pages")
+    return c.value
+
+
+def pa_plan_work_items(plan: Plan) -> np.ndarray:
+    """The work list as an int32 array [n, 6] (a copy)."""
+    p, n = _P(pa_work_item)(), _i64()
+    _check(lib.pa_plan_work_items(plan.handle, ctypes.byref(p), ctypes.byref(n)),
+           "pa_plan_work_items")
+    if n.value == 0:
+        return np.zeros((0, 6), dtype=np.int32)
+    buf = ctypes.cast(p, _P(_i32 * (6 * n.value))).contents
+    return np.frombuffer(buf, dtype=np.int32).reshape(n.value, 6).copy()
+
+
+def pa_plan_num_partials(plan: Plan) -> int:
+    n = _i64()
+    _check(lib.pa_plan_num_partials(plan.handle, ctypes.byref(n)), "pa_plan_num_partials")
+    return n.value
+
+
+def pa_plan_merge_indptr(plan: Plan, batch: int) -> np.ndarray:
+    p = _P(_i32)()
+    _check(lib.pa_plan_merge_indptr(plan.handle, ctypes.byref(p)), "pa_plan_merge_indptr")
+    return np.ctypeslib.as_array(p, shape=(batch + 1,)).copy()
+
+
+def pa_plan_prefix_chunks(plan: Plan):
+    n, t = _i32(), _i32()
+    _check(lib.pa_plan_prefix_chunks(plan.handle, ctypes.byref(n), ctypes.byref(t)),
+           "pa_plan_prefix_chunks")
+    return n.value, t.value
+
+
+def pa_plan_workspace_bytes(plan: Plan) -> int:
+    n = _sz()
+    _check(lib.pa_plan_workspace_bytes(plan.handle, ctypes.byref(n)), "pa_plan_workspace_bytes")
+    return n.value
+
+
+def pa_plan_upload(plan: Plan, workspace, workspace_bytes: int, stream=None):
+    _check(lib.pa_plan_upload(plan.handle, _ptr(workspace), workspace_bytes, _stream(stream)),
+           "pa_plan_upload")
+
+
+def pa_run(plan: Plan, q, k_pool, v_pool, kv_indices, o, lse, workspace, workspace_bytes: int,
+           stream=None):
+    _check(lib.pa_run(plan.handle, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(kv_indices),
+                      _ptr(o), _ptr(lse), _ptr(workspace), workspace_bytes, _stream(stream)),
+           "pa_run")
+
+
+def pa_cascade_run(plan: Plan, q, k_pool, v_pool, prefix_indices, kv_indices, o, lse, workspace,
+                   workspace_bytes: int, stream=None):
+    _check(lib.pa_cascade_run(plan.handle, _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                              _ptr(prefix_indices), _ptr(kv_indices), _ptr(o), _ptr(lse),
+                              _ptr(workspace), workspace_bytes, _stream(stream)),
+           "pa_cascade_run")
+
+
+def pa_merge_state(o_a, lse_a, o_b, lse_b, o, lse, rows: int, head_dim: int, dtype,
+                   stream=None):
+    if isinstance(dtype, str):
+        dtype = DTYPE_CODES[dtype]
+    _check(lib.pa_merge_state(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(o), _ptr(lse),
+                              rows, head_dim, dtype, _stream(stream)), "pa_merge_state")
+
+
+def pa_plan_check(plan: Plan, workspace, stream=None) -> int:
+    """-1 when no bad page index was seen, else raises PagedAttnError(DEVICE_CHECK)
+    with ``.position`` set to the first bad kv_indices position."""
+    pos = _i64()
+    st = lib.pa_plan_check(plan.handle, _ptr(workspace), ctypes.byref(pos), _stream(stream))
+    if st == PA_ERR_DEVICE_CHECK:
+        err = PagedAttnError(st, "pa_plan_check")
+        err.position = pos.value
+        raise err
+    _check(st, "pa_plan_check")
+    return pos.value
+
+
+def pa_default_schedule(device: int, num_qo_heads: int, num_kv_heads: int, dtype):
+    if isinstance(dtype, str):
+        dtype = DTYPE_CODES[dtype]
+    sms, k = _i32(), _i32()
+    _check(lib.pa_default_schedule(device, num_qo_heads, num_kv_heads, dtype, ctypes.byref(sms),
+                                   ctypes.byref(k)), "pa_default_schedule")
+    return sms.value, k.value
+
+
+def pa_status_string(status: int) -> str:
+    return lib.pa_status_string(status).decode()
+
+
+def pa_abi_version() -> int:
+    return lib.pa_abi_version()

@@ -1,0 +1,156 @@
+"""The C ABI on the host: exported symbols, plan parity with the oracle's
+restatement (bit-exact), and argument validation.  No GPU needed: the plan
+stage makes no CUDA call and run-stage argument checks happen before any."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from serving_attention_paged_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def C():
+    from serving_attention_paged_b200 import build
+    build.build()
+    from serving_attention_paged_b200 import pagedattn
+    return pagedattn
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "pagedattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(C):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(C.lib, n), n
+    assert C.pa_abi_version() == 1
+
+
+def _problem(C, w, num_sms=148, k=2, mct=0, flags=0):
+    return C.make_problem(batch=w.batch, num_qo_heads=w.num_qo_heads,
+                          num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
+                          sm_scale=w.sm_scale, num_sms=num_sms, ctas_per_sm=k,
+                          min_chunk_tokens=mct, num_pages=w.num_pages, flags=flags)
+
+
+def _compare_plan(C, indptr, last, P, hq, hkv, sms, k, mct):
+    prob = C.make_problem(batch=len(last), num_qo_heads=hq, num_kv_heads=hkv, page_size=P,
+                          dtype="f16", sm_scale=0.1, num_sms=sms, ctas_per_sm=k,
+                          min_chunk_tokens=mct, num_pages=1 << 30)
+    plan = C.pa_plan_create(prob, indptr, last)
+    c, items, mi = oracle.plan(indptr, last, page_size=P, num_kv_heads=hkv, num_sms=sms,
+                               ctas_per_sm=k, min_chunk_tokens=mct if mct else 256)
+    assert C.pa_plan_chunk_pages(plan) == c
+    assert np.array_equal(C.pa_plan_work_items(plan), items)
+    assert np.array_equal(C.pa_plan_merge_indptr(plan, len(last)), mi)
+    assert C.pa_plan_num_partials(plan) == mi[-1]
+    return plan
+
+
+@pytest.mark.parametrize("seed", range(25))
+def test_plan_matches_oracle_bit_exact(C, seed):
+    rng = np.random.default_rng(100 + seed)
+    B = int(rng.integers(0, 70))
+    P = int(rng.choice([1, 4, 16, 64]))
+    lens = rng.integers(0, 5000, size=B) * (rng.random(B) > 0.15)
+    indptr, _, last = W.tables_from_lengths(lens, P)
+    hkv = int(rng.choice([1, 2, 4, 8]))
+    g = int(rng.choice([1, 2, 4, 8]))
+    _compare_plan(C, indptr, last, P, hkv * g, hkv, int(rng.integers(1, 300)),
+                  int(rng.integers(1, 5)), int(rng.choice([0, 1, 100, 512])))
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 5, "4c"])
+def test_plan_matches_oracle_on_benchmark_workloads(C, n):
+    w = W.WORKLOADS[n]()
+    _compare_plan(C, w.kv_indptr, w.last_page_len, w.page_size, w.num_qo_heads, w.num_kv_heads,
+                  148, 3, 0)
+
+
+def test_plan_matches_oracle_vector_sparse(C):
+    w = W.WORKLOADS[4]()
+    _compare_plan(C, w.kv_indptr, w.last_page_len, 1, 64, 8, 148, 3, 0)
+
+
+def test_plan_edge_cases(C):
+    # empty batch, all-empty requests, one page, exactly full pages, B*Hkv above the budget
+    for lens, P, sms in [([], 16, 148), ([0, 0], 16, 148), ([1], 16, 148), ([16, 32, 48], 16, 148),
+                         ([100] * 50, 16, 2), ([3000, 1], 1, 1)]:
+        indptr, _, last = W.tables_from_lengths(lens, P)
+        _compare_plan(C, indptr, last, P, 8, 8, sms, 1, 0)
+
+
+def test_plan_validation(C):
+    w = W.make_workload("v", [20, 40], num_qo_heads=8, num_kv_heads=2, page_size=16,
+                        dtype="f16", seed=1)
+    ok = _problem(C, w)
+    C.pa_plan_create(ok, w.kv_indptr, w.last_page_len)
+
+    def status(prob, indptr=w.kv_indptr, last=w.last_page_len):
+        with pytest.raises(C.PagedAttnError) as e:
+            C.pa_plan_create(prob, indptr, last)
+        return e.value.status
+
+    assert status(ok, indptr=np.array([1, 2, 4])) == C.PA_ERR_INVALID_ARG  # indptr[0] != 0
+    assert status(ok, indptr=np.array([0, 3, 2])) == C.PA_ERR_INVALID_ARG  # decreasing
+    assert status(ok, last=np.array([0, 8])) == C.PA_ERR_INVALID_ARG       # 0 with pages
+    assert status(ok, last=np.array([17, 8])) == C.PA_ERR_INVALID_ARG      # > page_size
+    bad = _problem(C, w); bad.num_qo_heads = 7
+    assert status(bad) == C.PA_ERR_INVALID_ARG                             # Hq % Hkv
+    bad = _problem(C, w); bad.head_dim = 64
+    assert status(bad) == C.PA_ERR_UNSUPPORTED
+    bad = _problem(C, w); bad.page_size = 12
+    assert status(bad) == C.PA_ERR_UNSUPPORTED
+    bad = _problem(C, w); bad.num_qo_heads = 32
+    assert status(bad) == C.PA_ERR_UNSUPPORTED                             # group 16
+    bad = _problem(C, w); bad.dtype = 7
+    assert status(bad) == C.PA_ERR_INVALID_ARG
+    bad = _problem(C, w); bad.num_sms = 0
+    assert status(bad) == C.PA_ERR_INVALID_ARG
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_cascade_plan_create(ok, 24, w.kv_indptr, w.last_page_len)  # not whole pages
+    assert e.value.status == C.PA_ERR_INVALID_ARG
+
+
+def test_run_argument_checks_before_any_launch(C):
+    w = W.make_workload("v", [20, 40], num_qo_heads=8, num_kv_heads=2, page_size=16,
+                        dtype="f16", seed=1)
+    plan = C.pa_plan_create(_problem(C, w), w.kv_indptr, w.last_page_len)
+    nbytes = C.pa_plan_workspace_bytes(plan)
+    assert nbytes % 256 == 0 and nbytes > 0
+    fake = 1 << 40  # never dereferenced: every call below fails its host-side check
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_run(plan, fake, fake, fake, fake, fake, None, fake, nbytes - 256, 0)
+    assert e.value.status == C.PA_ERR_WORKSPACE_TOO_SMALL
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_run(plan, None, fake, fake, fake, fake, None, fake, nbytes, 0)
+    assert e.value.status == C.PA_ERR_INVALID_ARG
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_run(plan, fake + 8, fake, fake, fake, fake, None, fake, nbytes, 0)  # misaligned q
+    assert e.value.status == C.PA_ERR_INVALID_ARG
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_cascade_run(plan, fake, fake, fake, fake, fake, fake, None, fake, nbytes, 0)
+    assert e.value.status == C.PA_ERR_INVALID_ARG  # not a cascade plan
+    C.pa_merge_state(None, None, None, None, None, None, 0, 128, "f16", 0)  # nothing to do
+    with pytest.raises(C.PagedAttnError):
+        C.pa_merge_state(fake, fake, fake, fake, fake, fake, 4, 0, "f16", 0)
+
+
+def test_cascade_plan_shape(C):
+    w = W.WORKLOADS[5]()
+    prob = _problem(C, w)
+    plan = C.pa_cascade_plan_create(prob, w.prefix_len, w.kv_indptr, w.last_page_len)
+    n, tok = C.pa_plan_prefix_chunks(plan)
+    assert n >= 1 and tok % 128 == 0 and n * tok >= w.prefix_len > (n - 1) * tok
+    c, items, mi = oracle.plan(w.kv_indptr, w.last_page_len, page_size=16, num_kv_heads=8,
+                               num_sms=148, ctas_per_sm=2)
+    assert np.array_equal(C.pa_plan_work_items(plan), items)

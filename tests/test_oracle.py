@@ -283,3 +283,16 @@ def test_row_subset_matches_full():
                                  w.last_page_len, num_qo_heads=4, num_kv_heads=2, head_dim=D,
                                  page_size=16, dtype="f16", sm_scale=w.sm_scale, threads=4)
     assert np.array_equal(o3, o) and np.array_equal(l3, lse)
+
+
+def test_request_subset_matches_full_bitwise():
+    w = W.make_workload("subset", [30, 0, 70, 5], num_qo_heads=4, num_kv_heads=2, page_size=16,
+                        dtype="bf16", seed=27, extra_pages=9)
+    t = w.materialize()
+    o, lse = _run(w, t)
+    reqs = [2, 1, 3]
+    o2, l2 = oracle.paged_decode_requests(t["q"], t["k_pool"], t["v_pool"], w.kv_indptr,
+                                          w.kv_indices, w.last_page_len, reqs, num_qo_heads=4,
+                                          num_kv_heads=2, head_dim=D, page_size=16,
+                                          dtype="bf16", sm_scale=w.sm_scale)
+    assert np.array_equal(o2, o[reqs]) and np.array_equal(l2, lse[reqs])
