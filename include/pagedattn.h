@@ -7,7 +7,7 @@
  *     KV store; page_size 1 is the "vector-sparse" case.
  *   - README, core feature 2: the plan/run split.  pa_plan_create is the
  *     plan stage (host, schedules variable-length requests into a balanced
- *     split-KV work list); pa_run is the run stage (device).
+ *     split-KV work list, longest chunks first); pa_run is the run stage.
  *   - README, core feature 3: cascade attention for a shared prefix
  *     (pa_cascade_plan_create / pa_cascade_run) and head-query fusion for
  *     grouped-query attention (every q head of one kv head is computed by
@@ -65,7 +65,8 @@ typedef enum {
   PA_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace shorter than pa_plan_workspace_bytes */
   PA_ERR_CUDA = 4,                 /* a CUDA runtime call or launch failed */
   PA_ERR_DEVICE_CHECK = 5,         /* a checked run found an out-of-range page index */
-  PA_ERR_NO_MEMORY = 6             /* host allocation failed */
+  PA_ERR_NO_MEMORY = 6,            /* host allocation failed */
+  PA_ERR_DEVICE_TIMEOUT = 7        /* a kernel gave up on a bounded wait (see pa_plan_check) */
 } pa_status;
 
 typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 /* pa_merge_state only */ } pa_dtype;
@@ -102,13 +103,17 @@ typedef struct {
 typedef struct pa_plan_s* pa_plan_t;
 
 /* Plan stage (host only, no CUDA call).  Specification of the work list:
- *   W = num_sms * ctas_per_sm, c_min = max(1, ceil(min_chunk_tokens / P)),
- *   N = max_b n_b, work(c) = Hkv * sum_b max(1, ceil(n_b / c)).
- *   chunk c (pages) = max(N, 1) if N <= c_min, else the smallest c in
- *   [c_min, N] with work(c) <= W (binary search; N if none).
- *   Items ordered by request, then chunk, then kv head.  Chunk j of request b
- *   covers pages [kv_indptr[b] + j*c, min(kv_indptr[b] + (j+1)*c, kv_indptr[b+1])).
- *   merge_indptr[b+1] - merge_indptr[b] = chunks of b if > 1, else 0.
+ *   W = num_sms * ctas_per_sm (CTAs resident at once), c_min = max(1,
+ *   ceil(min_chunk_tokens / P)), N = max_b n_b,
+ *   work(c) = Hkv * sum_b max(1, ceil(n_b / c)) (items for chunk size c),
+ *   k = max(1, ceil(Hkv * B / W)) (waves the unsplit batch needs anyway).
+ *   Chunk c (pages) = max(N, 1) if N <= c_min, else the smallest c in
+ *   [c_min, N] with work(c) <= k * W (binary search).
+ *   Items are generated by request, then chunk, then kv head; chunk j of
+ *   request b covers pages [kv_indptr[b] + j*c, min(kv_indptr[b] + (j+1)*c,
+ *   kv_indptr[b+1])).  merge_indptr[b+1] - merge_indptr[b] = chunks of b if
+ *   > 1, else 0, and partial_slot = merge_indptr[b] + j.  The list is then
+ *   stably sorted by kv_len_in_chunk, longest first (launch order).
  * Validates: kv_indptr[0] == 0 and non-decreasing, 1 <= last_page_len[b] <= P
  * whenever request b has pages, Hq % Hkv == 0, positive sizes.
  * Returns PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED otherwise.  The host arrays
@@ -171,9 +176,12 @@ pa_status pa_merge_state(const void* o_a, const float* lse_a, const void* o_b,
                          const float* lse_b, void* o, float* lse, int64_t rows,
                          int32_t head_dim, pa_dtype dtype, void* stream);
 
-/* After a run with PA_FLAG_CHECK_INDICES: synchronously read the device
- * error word (PA_OK, or PA_ERR_DEVICE_CHECK with the first bad kv_indices
- * position in *bad_position) and clear it. */
+/* Synchronously read and clear the device status words of a workspace.
+ * Returns PA_ERR_DEVICE_TIMEOUT if a kernel abandoned one of its bounded
+ * pipeline waits (its outputs are then undefined), else PA_ERR_DEVICE_CHECK
+ * with the first bad kv_indices position in *bad_position if a run with
+ * PA_FLAG_CHECK_INDICES met an out-of-range page index, else PA_OK
+ * (*bad_position = -1). */
 pa_status pa_plan_check(pa_plan_t plan, void* d_workspace, int64_t* bad_position, void* stream);
 
 /* Scheduling defaults for `device`: its SM count and how many decode CTAs

@@ -200,13 +200,15 @@ def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per
 
     Specification (the reading adopted where the page is silent):
       W = num_sms * ctas_per_sm; c_min = max(1, ceil(min_chunk_tokens / P));
-      N = max_b n_b; work(c) = Hkv * sum_b max(1, ceil(n_b / c)).
+      N = max_b n_b; work(c) = Hkv * sum_b max(1, ceil(n_b / c));
+      k = max(1, ceil(Hkv * B / W)), the waves the unsplit batch needs.
       Chunk c (pages): if N <= c_min then max(N, 1); else the smallest c in
-      [c_min, N] with work(c) <= W, or N if none.  Found here by a linear scan.
+      [c_min, N] with work(c) <= k * W.  Found here by a linear scan.
       Items: b ascending, chunk j ascending (an empty request has one empty
       chunk), kv head ascending.  partial_slot is -1 for a one-chunk request,
       else merge_indptr[b] + j, merge_indptr being the running sum of the
-      chunk counts of the split requests.
+      chunk counts of the split requests.  Finally the items are stably
+      ordered by kv_len_in_chunk, longest first.
 
     Returns ``(chunk_pages, items, merge_indptr)`` with items an int32 array
     ``[n, 6]``: request, kv_head, page_begin, page_end, kv_len_in_chunk,
@@ -223,12 +225,13 @@ def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per
     def work(c):
         return num_kv_heads * sum(max(1, -(-nb // c)) for nb in n)
 
+    k = max(1, -(-(num_kv_heads * B) // W))
     if N <= c_min:
         c = max(N, 1)
     else:
         c = N
         for cand in range(c_min, N + 1):
-            if work(cand) <= W:
+            if work(cand) <= k * W:
                 c = cand
                 break
 
@@ -247,6 +250,7 @@ def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per
             slot = -1 if chunks[b] == 1 else merge_indptr[b] + j
             for h in range(num_kv_heads):
                 items.append((b, h, pb, pe, tokens, slot))
+    items.sort(key=lambda item: -item[4])  # Python's sort is stable
     return c, np.array(items, dtype=np.int32).reshape(-1, 6), np.array(merge_indptr, dtype=np.int32)
 
 

@@ -51,6 +51,8 @@ pa_status pa_plan_upload(pa_plan_t plan, void* d_workspace, size_t workspace_byt
     e = cudaMemsetAsync(ws + plan->ws.counters, 0,
                         size_t(p.batch) * p.num_kv_heads * sizeof(int32_t), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws + plan->ws.error, 0xff, sizeof(uint64_t), s);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(ws + plan->ws.error + sizeof(uint64_t), 0, sizeof(uint64_t), s);
   return from_cuda(int(e));
 }
 
@@ -101,12 +103,18 @@ pa_status pa_plan_check(pa_plan_t plan, void* d_workspace, int64_t* bad_position
   if (!plan || !d_workspace) return PA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(d_workspace);
-  unsigned long long word = 0;
-  cudaError_t e = cudaMemcpyAsync(&word, ws + plan->ws.error, sizeof word,
+  unsigned long long words[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(words, ws + plan->ws.error, sizeof words,
                                   cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws + plan->ws.error, 0xff, sizeof(uint64_t), s);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(ws + plan->ws.error + sizeof(uint64_t), 0, sizeof(uint64_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return PA_ERR_CUDA;
+  const unsigned long long word = words[0];
+  if (bad_position) *bad_position = word == ~0ull ? -1 : int64_t(word);
+  if (words[1]) return PA_ERR_DEVICE_TIMEOUT;
   if (word == ~0ull) {
     if (bad_position) *bad_position = -1;
     return PA_OK;

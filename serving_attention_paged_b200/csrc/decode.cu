@@ -7,21 +7,32 @@
 // heads of h, so every K/V row is read from HBM once.
 //
 // Data path.  A K or V row of one (token, kv head) is 128 x 16 bit = 256
-// contiguous bytes of the NHD pool, i.e. 16 lanes x one 16-byte vector.
-// Each stage of a 4-deep cp.async ring holds 32 tokens of K and V (16 KB).
-// Thread (group g = tid / 16, lane c = tid % 16) loads vector c of the rows
-// of tokens g, g + 8, g + 16, g + 24 of every tile and is also the only
-// thread that reads those vectors back, so the ring needs no block barrier:
-// cp.async.wait_group alone orders it.  Page indices are fetched one tile
-// ahead of the copies that use them (this matters for page_size 1).
+// contiguous bytes of the NHD pool: 16 lanes x one 16-byte vector.  Each
+// stage of a 4-deep cp.async ring holds 32 tokens of K and V (16 KB).
+// Thread (group g = tid / 16, lane c = tid % 16) copies vector c of the rows
+// of tokens g, g + 8, g + 16, g + 24 of a tile and is the only thread that
+// reads those vectors back, so the ring needs no barrier at all:
+// cp.async.wait_group orders it.  Rows past the chunk are zero-filled.  Page
+// indices are loaded one tile ahead of the copies that use them.  (Two
+// producer-warp variants were measured and rejected: with per-row 1-D bulk
+// copies the copy engine limits at 256 bytes per operation, and a single
+// warp issuing 16-byte copies for the whole CTA cannot keep HBM busy.)
 //
-// Math.  q is pre-scaled by sm_scale * log2(e) so scores are in base 2.  Each
-// 16-lane group reduces its g partial dot products with a reduce-scatter
-// (G - 1 + 4 - log2 G shuffles for all G heads instead of 4 G), leaving lane c
-// with the score of head c >> (4 - log2 G).  Online softmax state (m, l) is
-// kept per group and head in fp32; o (G x 8 values per lane) accumulates in
-// fp32 registers and is rescaled only when some running max moved.  At the
-// end the 8 groups are combined through shared memory.
+// Math.  16 lanes share one token: lane c holds elements 8c..8c+7 of the row.
+// q stays in its 16-bit storage type and q.k is accumulated with
+// mixed-precision FMAs (16-bit inputs, fp32 accumulate; the products are
+// exact in fp32), so no conversion instructions are spent on K.  The G
+// partial dot products are reduced over the 16 lanes with a reduce-scatter
+// whose operand order is permuted per lane (position i of lane c holds head
+// i ^ (c >> (4 - log2 G))), so no selects are needed and lane c ends with
+// the score of head c >> (4 - log2 G).  Scores are scaled to base 2; the
+// online-softmax state (m, l) is fp32; p reaches the other lanes through
+// shared memory.  o (G x 8 values per lane) accumulates in fp32 registers
+// and is rescaled only when a running max moved.  For fp16 the PV update
+// also uses mixed FMAs with p rounded to fp16 (l accumulates the rounded
+// p, so the normalisation stays exact); for bf16, p stays fp32 and V is
+// widened by a shift or mask.  The 8 token groups are combined at the end
+// through shared memory.
 //
 // Epilogue.  A request served by one chunk writes o (rounded once to the
 // input dtype) and lse (natural log).  A split request writes fp32 partial
@@ -41,14 +52,17 @@ namespace {
 
 constexpr int D = kHeadDim;
 constexpr int kThreads = 128;
-constexpr int kGroups = kThreads / 16;            // 8 token groups of 16 lanes
-constexpr int kTokPerGroup = 4;                    // tokens per group per tile
-constexpr int kTile = kGroups * kTokPerGroup;      // 32 tokens per stage
+constexpr int kGroups = kThreads / 16;                // 8 token groups of 16 lanes
+constexpr int kTokPerGroup = 4;                       // tokens per group per tile
+constexpr int kTile = kGroups * kTokPerGroup;         // 32 tokens per stage
 constexpr int kStages = 4;
-constexpr int kRowBytes = D * 2;                   // one (token, head) row
-constexpr int kStageBytes = 2 * kTile * kRowBytes; // K then V: 16 KB
-constexpr int kSmemBytes = kStages * kStageBytes;  // 64 KB
-constexpr int kMinBlocksPerSm = 3;
+constexpr int kRowBytes = D * 2;                      // one (token, head) row
+constexpr int kHalfStage = kTile * kRowBytes;         // K (or V) rows of a tile: 8 KB
+constexpr int kStageBytes = 2 * kHalfStage;           // 16 KB
+constexpr int kRingBytes = kStages * kStageBytes;     // 64 KB
+constexpr int kPBytesPerGroup = kTokPerGroup * 8 * 4 + 8 * 4;  // p[4][<=8] + alpha[<=8]
+constexpr int kPBytes = kGroups * kPBytesPerGroup;
+constexpr int kSmemBytes = kRingBytes + kPBytes;
 
 struct DecodeArgs {
   const uint16_t* q;
@@ -62,12 +76,12 @@ struct DecodeArgs {
   float* partial_lse;
   const float* prefix_o;
   const float* prefix_lse;
-  unsigned long long* error_pos;
+  unsigned long long* error_pos;  // first bad page position (checked runs)
   uint16_t* o;
   float* lse;
   int64_t num_pages;
   int32_t batch, num_qo_heads, num_kv_heads, log2_page, prefix_chunks;
-  float q_scale;
+  float score_scale;  // sm_scale * log2(e)
 };
 
 template <int G> struct Log2;
@@ -76,32 +90,12 @@ template <> struct Log2<2> { static constexpr int v = 1; };
 template <> struct Log2<4> { static constexpr int v = 2; };
 template <> struct Log2<8> { static constexpr int v = 3; };
 
-// Sum G partial dot products over the 16 lanes of a half warp.  Each of the
-// first log2(G) butterfly steps sends half of the remaining values and keeps
-// the other half, so lane c ends with the total of value c >> (4 - log2 G);
-// the remaining steps add up the copies held by the other lanes.
-template <int G>
-__device__ __forceinline__ float reduce_scatter16(float (&v)[G], int lane16) {
-  constexpr int LG = Log2<G>::v;
-#pragma unroll
-  for (int k = 0; k < LG; ++k) {
-    const int off = 8 >> k;
-    const bool upper = (lane16 & off) != 0;
-    const int half = (G >> k) >> 1;
-#pragma unroll
-    for (int i = 0; i < G / 2; ++i) {
-      if (i < half) {
-        const float send = upper ? v[i] : v[i + half];
-        const float keep = upper ? v[i + half] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-      }
-    }
-  }
-  float r = v[0];
-#pragma unroll
-  for (int k = LG; k < 4; ++k) r += __shfl_xor_sync(0xffffffffu, r, 8 >> k);
-  return r;
-}
+template <int G> struct MinBlocks { static constexpr int v = 3; };
+
+// p as the PV step consumes it: fp16 for fp16 inputs, fp32 for bf16.
+template <typename Tag> struct PType;
+template <> struct PType<F16> { using T = uint16_t; };
+template <> struct PType<BF16> { using T = float; };
 
 template <typename Tag>
 __device__ __forceinline__ void write_final(const DecodeArgs& a, int64_t row, int d, float o,
@@ -110,54 +104,109 @@ __device__ __forceinline__ void write_final(const DecodeArgs& a, int64_t row, in
   if (d == 0 && a.lse) a.lse[row] = lse2 == -INFINITY ? -INFINITY : lse2 * kLn2;
 }
 
+// Reduce G partial dot products over the 16 lanes of a half warp.  Operands
+// are stored in lane-permuted order, so at every butterfly step each lane
+// keeps the low half of its values and sends the high half.
+template <int G>
+__device__ __forceinline__ float reduce_scatter16(float (&v)[G]) {
+  constexpr int LG = Log2<G>::v;
+#pragma unroll
+  for (int k = 0; k < LG; ++k) {
+    const int half = (G >> k) >> 1;
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i)
+      if (i < half) v[i] += __shfl_xor_sync(0xffffffffu, v[i + half], 8 >> k);
+  }
+  float r = v[0];
+#pragma unroll
+  for (int k = LG; k < 4; ++k) r += __shfl_xor_sync(0xffffffffu, r, 8 >> k);
+  return r;
+}
+
+template <typename Tag, int G>
+__device__ __forceinline__ void pv_update(F16, const uint4& v, const uint16_t (&p)[G],
+                                          float (&o)[G][8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) axpy2_f16(p[hh], w[i], o[hh][2 * i], o[hh][2 * i + 1]);
+}
+
+template <typename Tag, int G>
+__device__ __forceinline__ void pv_update(BF16, const uint4& v, const float (&p)[G],
+                                          float (&o)[G][8]) {
+  float vf[8];
+  to_float8(BF16{}, v, vf);
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[hh][i] = fmaf(p[hh], vf[i], o[hh][i]);
+}
+
 template <typename Tag, int G, bool kCheck>
-__global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
+__global__ void __launch_bounds__(kThreads, MinBlocks<G>::v)
     paged_decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_is_last;
+  using PT = typename PType<Tag>::T;
   constexpr int LG = Log2<G>::v;
   constexpr int kLanesPerHead = 16 >> LG;
 
   const int tid = threadIdx.x;
-  const int lane16 = tid & 15;
-  const int grp = tid >> 4;
+  const int lane = tid & 31;
   const pa_work_item it = a.items[blockIdx.x];
   const int b = it.request, h = it.kv_head, len = it.kv_len_in_chunk;
-  const int lp = a.log2_page;
-  const int pmask = (1 << lp) - 1;
+  const int ntiles = (len + kTile - 1) / kTile;
   const int Hq = a.num_qo_heads;
   const int hq0 = h * G;
 
-  float q[G][8];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(
-        a.q + (int64_t(b) * Hq + hq0 + hh) * D + lane16 * 8));
-    to_float8(Tag{}, u, q[hh]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) q[hh][i] *= a.q_scale;
-  }
+  const int lane16 = tid & 15;
+  const int grp = tid >> 4;
+  const int my_head = lane16 >> (4 - LG);  // head whose score this lane ends with
 
+  uint32_t qw[G][4];  // q in storage type; position i holds head i ^ my_head
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+        a.q + (int64_t(b) * Hq + hq0 + (i ^ my_head)) * D + lane16 * 8));
+    qw[i][0] = u.x;
+    qw[i][1] = u.y;
+    qw[i][2] = u.z;
+    qw[i][3] = u.w;
+  }
+  uint8_t* pbuf = smem + kRingBytes + grp * kPBytesPerGroup;
+  PT* pshare = reinterpret_cast<PT*>(pbuf);                       // [kTokPerGroup][G]
+  float* ashare = reinterpret_cast<float*>(pbuf + kTokPerGroup * 8 * 4);  // [G]
+
+  float o[G][8];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[hh][i] = 0.f;
+  float m = -INFINITY, l = 0.f;
+  const bool writer = (lane16 & (kLanesPerHead - 1)) == 0;
+
+  // ---- loads: this thread's 16-byte vectors of its 4 rows per tile ----
+  const int lp = a.log2_page, pmask = (1 << lp) - 1;
   const int64_t row_stride = int64_t(a.num_kv_heads) * D;
   const uint16_t* kbase = a.k_pool + int64_t(h) * D + lane16 * 8;
   const uint16_t* vbase = a.v_pool + int64_t(h) * D + lane16 * 8;
-  const int ntiles = (len + kTile - 1) / kTile;
   const uint32_t my_slot = smem_u32(smem) + grp * kRowBytes + lane16 * 16;
-
   auto load_pages = [&](int tile, int (&pg)[kTokPerGroup]) {
 #pragma unroll
     for (int j = 0; j < kTokPerGroup; ++j) {
       const int pos = tile * kTile + grp + kGroups * j;
-      pg[j] = -1;
+      int p = -1;
       if (pos < len) {
         const int at = it.page_begin + (pos >> lp);
-        int p = __ldg(a.kv_indices + at);
+        p = __ldg(a.kv_indices + at);
         if (kCheck && (p < 0 || int64_t(p) >= a.num_pages)) {
           atomicMin(a.error_pos, (unsigned long long)at);
-          p = -2;  // skipped: reads as zeros
+          p = -1;  // not copied: the row reads as zeros
         }
-        pg[j] = p;
       }
+      pg[j] = p;
     }
   };
   auto issue = [&](int tile, int stage, const int (&pg)[kTokPerGroup]) {
@@ -166,95 +215,94 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
       for (int j = 0; j < kTokPerGroup; ++j) {
         const int pos = tile * kTile + grp + kGroups * j;
         const bool ok = pg[j] >= 0;
-        const int64_t row = ok ? ((int64_t(pg[j]) << lp) | (pos & pmask)) : 0;
+        const int64_t off = ok ? ((int64_t(pg[j]) << lp) | (pos & pmask)) * row_stride : 0;
         const uint32_t dst = my_slot + stage * kStageBytes + j * kGroups * kRowBytes;
-        cp_async16(dst, kbase + row * row_stride, ok ? 16 : 0);
-        cp_async16(dst + kTile * kRowBytes, vbase + row * row_stride, ok ? 16 : 0);
+        cp_async16(dst, kbase + off, ok ? 16 : 0);
+        cp_async16(dst + kHalfStage, vbase + off, ok ? 16 : 0);
       }
     }
     cp_async_commit();
   };
-
   int pg[kTokPerGroup];
 #pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    load_pages(s, pg);
-    issue(s, s, pg);
+  for (int st = 0; st < kStages - 1; ++st) {
+    load_pages(st, pg);
+    issue(st, st, pg);
   }
   load_pages(kStages - 1, pg);
-
-  float o[G][8];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) o[hh][i] = 0.f;
-  float m = -INFINITY, l = 0.f;
 
   for (int t = 0; t < ntiles; ++t) {
     issue(t + kStages - 1, (t + kStages - 1) % kStages, pg);
     load_pages(t + kStages, pg);
     cp_async_wait<kStages - 1>();
+    const int s = t % kStages;
+    const uint8_t* ks = smem + s * kStageBytes + grp * kRowBytes + lane16 * 16;
+    const uint8_t* vs = ks + kHalfStage;
 
-    const uint8_t* ks = smem + (t % kStages) * kStageBytes + grp * kRowBytes + lane16 * 16;
-    const uint8_t* vs = ks + kTile * kRowBytes;
-    float s[kTokPerGroup];
+    float sc[kTokPerGroup];
 #pragma unroll
     for (int j = 0; j < kTokPerGroup; ++j) {
       const uint4 u = *reinterpret_cast<const uint4*>(ks + j * kGroups * kRowBytes);
-      float kf[8];
-      to_float8(Tag{}, u, kf);
       float part[G];
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        float acc = q[hh][0] * kf[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) acc = fmaf(q[hh][i], kf[i], acc);
-        part[hh] = acc;
+      for (int i = 0; i < G; ++i) {
+        float acc = 0.f;
+        acc = dot2(Tag{}, u.x, qw[i][0], acc);
+        acc = dot2(Tag{}, u.y, qw[i][1], acc);
+        acc = dot2(Tag{}, u.z, qw[i][2], acc);
+        acc = dot2(Tag{}, u.w, qw[i][3], acc);
+        part[i] = acc;
       }
-      const float sc = reduce_scatter16<G>(part, lane16);
-      s[j] = (t * kTile + grp + kGroups * j < len) ? sc : -INFINITY;
+      const float r = reduce_scatter16<G>(part);
+      sc[j] = (t * kTile + grp + kGroups * j < len) ? r * a.score_scale : -INFINITY;
     }
 
     float mnew = m;
 #pragma unroll
-    for (int j = 0; j < kTokPerGroup; ++j) mnew = fmaxf(mnew, s[j]);
+    for (int j = 0; j < kTokPerGroup; ++j) mnew = fmaxf(mnew, sc[j]);
     const float msafe = mnew == -INFINITY ? 0.f : mnew;
     const bool moved = mnew != m;
     const float alpha = moved ? fast_exp2(m - msafe) : 1.f;
-    float p[kTokPerGroup];
     float psum = 0.f;
 #pragma unroll
     for (int j = 0; j < kTokPerGroup; ++j) {
-      p[j] = fast_exp2(s[j] - msafe);
-      psum += p[j];
+      float p = fast_exp2(sc[j] - msafe);
+      PT ps;
+      if constexpr (sizeof(PT) == 2) {
+        ps = __half_as_ushort(__float2half_rn(p));
+        p = __half2float(__ushort_as_half(ps));  // l sums exactly what PV multiplies
+      } else {
+        ps = p;
+      }
+      psum += p;
+      if (writer) pshare[j * G + my_head] = ps;
     }
     l = l * alpha + psum;
     m = mnew;
+    if (writer) ashare[my_head] = alpha;
+    __syncwarp();
     if (__any_sync(0xffffffffu, moved)) {
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
-        const float ah = G == 1 ? alpha : __shfl_sync(0xffffffffu, alpha, hh * kLanesPerHead, 16);
+        const float ah = ashare[hh];
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[hh][i] *= ah;
       }
     }
 #pragma unroll
     for (int j = 0; j < kTokPerGroup; ++j) {
-      const uint4 u = *reinterpret_cast<const uint4*>(vs + j * kGroups * kRowBytes);
-      float vf[8];
-      to_float8(Tag{}, u, vf);
+      const uint4 v = *reinterpret_cast<const uint4*>(vs + j * kGroups * kRowBytes);
+      PT pj[G];
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float ph = G == 1 ? p[j] : __shfl_sync(0xffffffffu, p[j], hh * kLanesPerHead, 16);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[hh][i] = fmaf(ph, vf[i], o[hh][i]);
-      }
+      for (int hh = 0; hh < G; ++hh) pj[hh] = pshare[j * G + hh];
+      pv_update<Tag, G>(Tag{}, v, pj, o);
     }
+    __syncwarp();  // p and alpha of this tile consumed before the next tile writes them
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // Combine the 8 token groups through shared memory (the ring is free now).
+  // Combine the 8 token groups through shared memory (the ring is idle now).
   float* Os = reinterpret_cast<float*>(smem);  // [kGroups][G][D]
   float* Ms = Os + kGroups * G * D;            // [kGroups][G]
   float* Ls = Ms + kGroups * G;
@@ -264,10 +312,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
     dst[0] = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
     dst[1] = make_float4(o[hh][4], o[hh][5], o[hh][6], o[hh][7]);
   }
-  if ((lane16 & (kLanesPerHead - 1)) == 0) {
-    const int hs = lane16 / kLanesPerHead;
-    Ms[grp * G + hs] = m;
-    Ls[grp * G + hs] = l;
+  if (writer) {
+    Ms[grp * G + my_head] = m;
+    Ls[grp * G + my_head] = l;
   }
   __syncthreads();
 
@@ -428,7 +475,7 @@ int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream) {
   a.num_kv_heads = pr.num_kv_heads;
   a.log2_page = plan.log2_page;
   a.prefix_chunks = plan.cascade ? plan.prefix_chunks : 0;
-  a.q_scale = pr.sm_scale * kLog2e;
+  a.score_scale = pr.sm_scale * kLog2e;
   const bool check = (pr.flags & PA_FLAG_CHECK_INDICES) != 0;
   const int64_t n = int64_t(plan.items.size());
   cudaStream_t s = static_cast<cudaStream_t>(stream);

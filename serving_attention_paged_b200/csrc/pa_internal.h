@@ -20,7 +20,8 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 //   items        [n_items]             pa_work_item
 //   merge_indptr [B + 1]               int32
 //   counters     [B * Hkv]             int32, zero between runs
-//   error        [1]                   uint64, first bad kv_indices position (~0 = none)
+//   error        [2]                   uint64: first bad kv_indices position (~0 = none),
+//                                      then a timeout flag (0 = none)
 //   partial_o    [n_partials, Hq, D]   fp32, split-chunk outputs (normalised)
 //   partial_lse  [n_partials, Hq]      fp32, their log-sum-exp in base 2
 //   prefix_o     [prefix_chunks, B, Hq, D]  fp32 (cascade only)

@@ -60,21 +60,22 @@ pa_status build(pa_plan_s* plan, const int32_t* indptr, const int32_t* last) {
   if (!indptr) plan->kv_indptr.assign(1, 0);
   plan->last_page_len.assign(last ? last : nullptr, last ? last + B : nullptr);
 
-  // chunk size: smallest c in [c_min, N] with work(c) <= W (work is non-increasing in c)
+  // chunk size: smallest c in [c_min, N] with work(c) <= k * W, where k is the
+  // number of waves the unsplit batch needs anyway (work is non-increasing in c)
   const int64_t W = int64_t(p.num_sms) * p.ctas_per_sm;
   const int64_t min_tokens = p.min_chunk_tokens ? p.min_chunk_tokens : pa::kDefaultMinChunkTokens;
   const int64_t c_min = std::max<int64_t>(1, ceil_div(min_tokens, P));
   const int64_t N = B ? *std::max_element(n.begin(), n.end()) : 0;
+  const int64_t waves = std::max<int64_t>(1, ceil_div(Hkv * B, W));
+  const int64_t budget = waves * W;
   int64_t c;
   if (N <= c_min) {
     c = std::max<int64_t>(N, 1);
-  } else if (work(n, N, Hkv) > W) {
-    c = N;
   } else {
-    int64_t lo = c_min, hi = N;
+    int64_t lo = c_min, hi = N;  // work(N) = Hkv * B <= budget
     while (lo < hi) {
       int64_t mid = lo + (hi - lo) / 2;
-      if (work(n, mid, Hkv) <= W) hi = mid; else lo = mid + 1;
+      if (work(n, mid, Hkv) <= budget) hi = mid; else lo = mid + 1;
     }
     c = lo;
   }
@@ -104,6 +105,12 @@ pa_status build(pa_plan_s* plan, const int32_t* indptr, const int32_t* last) {
                                            int32_t(tokens), slot});
     }
   }
+  // Longest chunks first: the block scheduler hands items to free SMs in
+  // launch order, so this is greedy longest-processing-time-first packing.
+  std::stable_sort(plan->items.begin(), plan->items.end(),
+                   [](const pa_work_item& x, const pa_work_item& y) {
+                     return x.kv_len_in_chunk > y.kv_len_in_chunk;
+                   });
   return PA_OK;
 }
 
@@ -120,7 +127,7 @@ void layout_workspace(pa_plan_s* plan) {
   w.items = take(plan->items.size() * sizeof(pa_work_item));
   w.merge_indptr = take((B + 1) * sizeof(int32_t));
   w.counters = take(B * p.num_kv_heads * sizeof(int32_t));
-  w.error = take(sizeof(uint64_t));
+  w.error = take(2 * sizeof(uint64_t));  // first bad index, timeout flag
   w.partial_o = take(size_t(plan->n_partials) * Hq * D * sizeof(float));
   w.partial_lse = take(size_t(plan->n_partials) * Hq * sizeof(float));
   w.prefix_o = take(size_t(plan->prefix_chunks) * B * Hq * D * sizeof(float));
@@ -245,6 +252,7 @@ const char* pa_status_string(pa_status s) {
     case PA_ERR_CUDA: return "CUDA error";
     case PA_ERR_DEVICE_CHECK: return "device check failed: page index out of range";
     case PA_ERR_NO_MEMORY: return "host allocation failed";
+    case PA_ERR_DEVICE_TIMEOUT: return "a kernel abandoned a bounded wait";
   }
   return "unknown status";
 }

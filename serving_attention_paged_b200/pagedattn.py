@@ -22,7 +22,7 @@ if not os.path.exists(_LIB_PATH):
 lib = ctypes.CDLL(_LIB_PATH)
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL = 0, 1, 2, 3
-PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_NO_MEMORY = 4, 5, 6
+PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_NO_MEMORY, PA_ERR_DEVICE_TIMEOUT = 4, 5, 6, 7
 PA_F16, PA_BF16, PA_F32 = 0, 1, 2
 PA_FLAG_CHECK_INDICES = 1
 DTYPE_CODES = {"f16": PA_F16, "bf16": PA_BF16, "f32": PA_F32}

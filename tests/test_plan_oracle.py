@@ -18,15 +18,16 @@ from serving_attention_paged_b200 import workloads as W
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "plan_small.json")
 
 
-def test_plan_hand_worked_example():
-    g = json.load(open(GOLDEN))
-    c, items, merge_indptr = oracle.plan(g["kv_indptr"], g["last_page_len"],
-                                         page_size=g["page_size"], num_kv_heads=g["num_kv_heads"],
-                                         num_sms=g["num_sms"], ctas_per_sm=g["ctas_per_sm"],
-                                         min_chunk_tokens=g["min_chunk_tokens"])
-    assert c == g["chunk_pages"]
-    assert merge_indptr.tolist() == g["merge_indptr"]
-    assert items.tolist() == g["items"]
+def test_plan_hand_worked_examples():
+    for g in json.load(open(GOLDEN))["cases"]:
+        c, items, merge_indptr = oracle.plan(g["kv_indptr"], g["last_page_len"],
+                                             page_size=g["page_size"],
+                                             num_kv_heads=g["num_kv_heads"],
+                                             num_sms=g["num_sms"], ctas_per_sm=g["ctas_per_sm"],
+                                             min_chunk_tokens=g["min_chunk_tokens"])
+        assert c == g["chunk_pages"]
+        assert merge_indptr.tolist() == g["merge_indptr"]
+        assert items.tolist() == g["items"]
 
 
 def _work(n, c, hkv):
@@ -41,21 +42,23 @@ def check_plan_properties(indptr, last, P, hkv, W_, c_min_tokens, c, items, merg
     lens = np.where(n > 0, (n - 1) * P + last, 0)
     c_min = max(1, -(-c_min_tokens // P))
     N = int(n.max()) if B else 0
-    # chunk size minimal under the budget
+    # chunk size minimal under the budget of k waves
+    budget = max(1, -(-(hkv * B) // W_)) * W_
     if N <= c_min:
         assert c == max(N, 1)
     else:
         assert c_min <= c <= N
-        if c < N:
-            assert _work(n, c, hkv) <= W_
+        assert _work(n, c, hkv) <= budget
         if c > c_min:
-            assert _work(n, c - 1, hkv) > W_
+            assert _work(n, c - 1, hkv) > budget
     assert len(items) == _work(n, c, hkv)
     if B * hkv <= W_:
         assert len(items) <= W_
+    # launch order: longest chunk first
+    assert all(items[i, 4] >= items[i + 1, 4] for i in range(len(items) - 1))
     # coverage: per (b, h) the chunks tile [indptr[b], indptr[b+1]) in order
     cover = {}
-    for (b, h, pb, pe, kl, slot) in items.tolist():
+    for (b, h, pb, pe, kl, slot) in sorted(items.tolist(), key=lambda x: (x[0], x[2], x[1])):
         assert 0 <= pe - pb <= c
         assert pb == indptr[b] or (pb - indptr[b]) % c == 0
         cover.setdefault((b, h), []).append((pb, pe, kl, slot))
