@@ -54,6 +54,10 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="untimed run-in after warm-up so clocks settle and get sampled")
+    ap.add_argument("--min-chunk-tokens", type=int, default=0,
+                    help="split-KV minimum chunk (tokens); 0 = library default")
+    ap.add_argument("--ctas-per-sm", type=int, default=0,
+                    help="CTA budget per SM for the plan; 0 = occupancy of the kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -262,7 +266,8 @@ def run_ours(args):
     pd = PagedDecode(w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
                      num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
                      sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
-                     device=dev_t)
+                     device=dev_t, min_chunk_tokens=args.min_chunk_tokens,
+                     ctas_per_sm=args.ctas_per_sm or None)
     plan_us = (time.perf_counter() - t0) * 1e6
     o, lse = pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"],
                     prefix_indices=dev.get("prefix_indices"))
@@ -356,9 +361,11 @@ def run_ours(args):
         e2e_t = torch.tensor([e2e_sec], dtype=torch.float64, device=dev_t)
         if world > 1:
             dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+        from serving_attention_paged_b200 import pagedattn as Cb
         items = len(pd.work_items())
+        n_cta = len(Cb.pa_plan_cta_indptr(pd.plan)) - 1
         h2d = (q_h.numel() * q_h.element_size() + idx_h.numel() * 4 + items * 24 +
-               (w.batch + 1) * 4)
+               (n_cta + 1) * 4 + (w.batch * w.num_kv_heads + 1) * 4)
         e2e = {"value": world * nbytes / float(e2e_t.item()) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(o_h.numel() * o_h.element_size() + lse_h.numel() * 4),

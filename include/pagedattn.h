@@ -6,8 +6,9 @@
  *   - README, core feature 1: single/batch attention over a sparse (paged)
  *     KV store; page_size 1 is the "vector-sparse" case.
  *   - README, core feature 2: the plan/run split.  pa_plan_create is the
- *     plan stage (host, schedules variable-length requests into a balanced
- *     split-KV work list, longest chunks first); pa_run is the run stage.
+ *     plan stage (host, cuts variable-length requests into equal shares
+ *     per CTA, stream-K style, which the README lists among FlashInfer's
+ *     inspirations); pa_run is the run stage.
  *   - README, core feature 3: cascade attention for a shared prefix
  *     (pa_cascade_plan_create / pa_cascade_run) and head-query fusion for
  *     grouped-query attention (every q head of one kv head is computed by
@@ -86,34 +87,42 @@ typedef struct {
   float sm_scale;           /* softmax scale, always given by the caller (1/sqrt(D) usually) */
   int32_t num_sms;          /* CTA budget W = num_sms * ctas_per_sm; explicit so that  */
   int32_t ctas_per_sm;      /*   the plan is a pure function of its inputs              */
-  int32_t min_chunk_tokens; /* smallest split-KV chunk in tokens; 0 means 256 */
-  int64_t num_pages;        /* pages in the pool (bounds for PA_FLAG_CHECK_INDICES) */
+  int32_t min_chunk_tokens; /* smallest per-CTA quota, in tokens; 0 means 256 */
+  int64_t num_pages;        /* pages in the pool; num_pages * page_size < 2^32 (pool rows
+                               are 32-bit indices); bounds for PA_FLAG_CHECK_INDICES */
   uint32_t flags;           /* PA_FLAG_* */
 } pa_problem;
 
-/* One unit of run-stage work: kv head `kv_head` of request `request` over
- * pages kv_indices[page_begin .. page_end) (absolute positions, so the run
- * stage needs no kv_indptr), holding kv_len_in_chunk tokens.  partial_slot
- * is -1 when the chunk is the request's only one (the item writes o and lse
- * itself), else the row of the fp32 partial-state buffer it fills. */
+/* One piece of run-stage work: tokens [token_begin, token_end) of kv head
+ * `kv_head` of request `request`.  Token t of the request lives on page
+ * kv_indices[page_begin + t / P] at row t % P (page_begin = kv_indptr[request],
+ * so the run stage needs no kv_indptr).  partial_slot is -1 when the piece is
+ * the whole (request, kv head) segment (the piece writes o and lse itself),
+ * else the row of the fp32 partial-state buffer it fills. */
 typedef struct {
-  int32_t request, kv_head, page_begin, page_end, kv_len_in_chunk, partial_slot;
+  int32_t request, kv_head, page_begin, token_begin, token_end, partial_slot;
 } pa_work_item;
 
 typedef struct pa_plan_s* pa_plan_t;
 
-/* Plan stage (host only, no CUDA call).  Specification of the work list:
- *   W = num_sms * ctas_per_sm (CTAs resident at once), c_min = max(1,
- *   ceil(min_chunk_tokens / P)), N = max_b n_b,
- *   work(c) = Hkv * sum_b max(1, ceil(n_b / c)) (items for chunk size c),
- *   k = max(1, ceil(Hkv * B / W)) (waves the unsplit batch needs anyway).
- *   Chunk c (pages) = max(N, 1) if N <= c_min, else the smallest c in
- *   [c_min, N] with work(c) <= k * W (binary search).
- *   Items are generated by request, then chunk, then kv head; chunk j of
- *   request b covers pages [kv_indptr[b] + j*c, min(kv_indptr[b] + (j+1)*c,
- *   kv_indptr[b+1])).  merge_indptr[b+1] - merge_indptr[b] = chunks of b if
- *   > 1, else 0, and partial_slot = merge_indptr[b] + j.  The list is then
- *   stably sorted by kv_len_in_chunk, longest first (launch order).
+/* Plan stage (host only, no CUDA call).  Specification of the work list
+ * (a stream-K style split of the whole decode step over tokens):
+ *   L_b = 0 if n_b = 0 else (n_b - 1) * P + last_page_len[b]; T = sum_b L_b;
+ *   W = num_sms * ctas_per_sm (CTAs resident at once);
+ *   groups = max(1, floor(W / Hkv)) groups of Hkv CTAs, one CTA per kv head;
+ *   quota q = 32 * ceil(max(min_chunk_tokens, ceil(T / groups)) / 32) tokens;
+ *   n_groups = max(1, ceil(T / q)) (0 for an empty batch); n_cta = n_groups * Hkv.
+ *   Group g covers token positions [g q, (g + 1) q) of the requests laid end
+ *   to end; its pieces are the intersections with the requests, in request
+ *   order.  An empty request is a zero-length piece of the group its position
+ *   falls in (the last group at the very end).  CTA g * Hkv + h runs the
+ *   pieces of group g for kv head h, so the Hkv CTAs of a group read the
+ *   same pages at the same time.
+ *   A (request, kv head) segment cut into k > 1 pieces owns partial slots
+ *   merge_indptr[b * Hkv + h] + 0 .. k - 1, in token order; merge_indptr is
+ *   the running sum of those k.
+ * Every group but the last therefore reads exactly q tokens, whatever the
+ * length mix, and no CTA waits for another.
  * Validates: kv_indptr[0] == 0 and non-decreasing, 1 <= last_page_len[b] <= P
  * whenever request b has pages, Hq % Hkv == 0, positive sizes.
  * Returns PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED otherwise.  The host arrays
@@ -132,14 +141,18 @@ pa_status pa_cascade_plan_create(const pa_problem* problem, int32_t prefix_len,
                                  const int32_t* last_page_len_host, pa_plan_t* out);
 
 /* Read-only views of the plan (borrowed; valid until pa_plan_destroy). */
-pa_status pa_plan_chunk_pages(pa_plan_t plan, int32_t* chunk_pages);
+pa_status pa_plan_quota_tokens(pa_plan_t plan, int32_t* quota);
 pa_status pa_plan_work_items(pa_plan_t plan, const pa_work_item** items, int64_t* n_items);
-pa_status pa_plan_merge_indptr(pa_plan_t plan, const int32_t** merge_indptr /* [B+1] */);
+pa_status pa_plan_cta_indptr(pa_plan_t plan, const int32_t** cta_indptr /* [n_cta+1] */,
+                             int64_t* n_cta);
+pa_status pa_plan_merge_indptr(pa_plan_t plan,
+                               const int32_t** merge_indptr /* [B*Hkv+1] */);
 pa_status pa_plan_num_partials(pa_plan_t plan, int64_t* n_partials);
 pa_status pa_plan_prefix_chunks(pa_plan_t plan, int32_t* n_chunks, int32_t* chunk_tokens);
 
-/* Device workspace the run stage needs: work list, merge offsets, arrival
- * counters and fp32 partial states.  Caller-allocated, 256-byte aligned. */
+/* Device workspace the run stage needs: work list, CTA and merge offsets,
+ * arrival counters and fp32 partial states.  Caller-allocated, 256-byte
+ * aligned. */
 pa_status pa_plan_workspace_bytes(pa_plan_t plan, size_t* bytes);
 
 /* Copy the work list into the workspace and zero its counters (enqueued on
@@ -150,9 +163,9 @@ pa_status pa_plan_upload(pa_plan_t plan, void* d_workspace, size_t workspace_byt
                          void* stream);
 
 /* Run stage: decode attention for every request of the plan.  kv_indices is
- * the device copy of the table the plan was made from.  One launch; split
- * requests are merged inside it by the last CTA to finish (no second
- * kernel).  lse may be NULL. */
+ * the device copy of the table the plan was made from.  One launch of n_cta
+ * CTAs; the pieces of a split (request, kv head) are merged inside it by the
+ * last CTA to finish one of them (no second kernel).  lse may be NULL. */
 pa_status pa_run(pa_plan_t plan, const void* q, const void* k_pool, const void* v_pool,
                  const int32_t* d_kv_indices, void* o, float* lse, void* d_workspace,
                  size_t workspace_bytes, void* stream);

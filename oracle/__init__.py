@@ -13,8 +13,8 @@ single-request decode usage example) and the flashinfer-cubin registry page
 * ``merge_state`` / ``merge_states`` — combining attention states by their
   log-sum-exp (what split-KV and cascade attention rely on).
 * ``cascade_decode`` — shared prefix merged with per-request suffix.
-* ``plan`` — the split-KV work-list specification restated as a plain
-  linear scan (the library's binary search must agree with it exactly).
+* ``plan`` — the split-KV work-list specification restated with plain
+  loops (the library's work list must agree with it exactly).
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (closed forms, invariants, brute force).  The pages print no worked numeric
@@ -196,62 +196,73 @@ def cascade_decode(q, k_pool, v_pool, prefix_indices, prefix_len, kv_indptr, kv_
 def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per_sm,
          min_chunk_tokens=256):
     """Split-KV work list (FlashInfer README core feature 2: variable-length
-    inputs are scheduled in a plan stage to even out the load).
+    inputs are scheduled in a plan stage to even out the load; the README
+    also names stream-K among FlashInfer's inspirations).
 
-    Specification (the reading adopted where the page is silent):
-      W = num_sms * ctas_per_sm; c_min = max(1, ceil(min_chunk_tokens / P));
-      N = max_b n_b; work(c) = Hkv * sum_b max(1, ceil(n_b / c));
-      k = max(1, ceil(Hkv * B / W)), the waves the unsplit batch needs.
-      Chunk c (pages): if N <= c_min then max(N, 1); else the smallest c in
-      [c_min, N] with work(c) <= k * W.  Found here by a linear scan.
-      Items: b ascending, chunk j ascending (an empty request has one empty
-      chunk), kv head ascending.  partial_slot is -1 for a one-chunk request,
-      else merge_indptr[b] + j, merge_indptr being the running sum of the
-      chunk counts of the split requests.  Finally the items are stably
-      ordered by kv_len_in_chunk, longest first.
+    Specification (the reading adopted where the page is silent), restated
+    here with plain loops:
+      L_b = 0 if n_b = 0 else (n_b - 1) * P + last_page_len[b]; T = sum_b L_b;
+      W = num_sms * ctas_per_sm; groups = max(1, floor(W / Hkv));
+      quota q = 32 * ceil(max(min_chunk_tokens, ceil(T / groups)) / 32) tokens;
+      n_groups = max(1, ceil(T / q)), or 0 for an empty batch.
+      Group g covers token positions [g q, (g + 1) q) of the requests laid
+      end to end; its pieces are the intersections with the requests (an
+      empty request is a zero-length piece of the group its position falls
+      in; the last group at the very end).  CTA g * Hkv + h runs the pieces of
+      group g for kv head h.  A (request, head) segment cut into k > 1 pieces
+      owns partial slots merge_indptr[b * Hkv + h] + 0 .. k - 1, in order.
 
-    Returns ``(chunk_pages, items, merge_indptr)`` with items an int32 array
-    ``[n, 6]``: request, kv_head, page_begin, page_end, kv_len_in_chunk,
-    partial_slot.
+    Returns ``(quota, items, cta_indptr, merge_indptr)``; items is int32
+    ``[n, 6]``: request, kv_head, page_begin (= kv_indptr[b]), token_begin,
+    token_end, partial_slot.
     """
     indptr = [int(x) for x in _as_i32(kv_indptr)]
     last = [int(x) for x in _as_i32(last_page_len)]
-    B, P = len(last), page_size
-    n = [indptr[b + 1] - indptr[b] for b in range(B)]
+    B, P, Hkv = len(last), page_size, num_kv_heads
+    L = []
+    for b in range(B):
+        n = indptr[b + 1] - indptr[b]
+        L.append((n - 1) * P + last[b] if n > 0 else 0)
+    T = sum(L)
     W = num_sms * ctas_per_sm
-    c_min = max(1, -(-min_chunk_tokens // P))
-    N = max(n) if n else 0
+    groups = max(1, W // Hkv)
+    q = 32 * (-(-max(min_chunk_tokens, -(-T // groups)) // 32))
+    n_groups = 0 if B == 0 else max(1, -(-T // q))
 
-    def work(c):
-        return num_kv_heads * sum(max(1, -(-nb // c)) for nb in n)
-
-    k = max(1, -(-(num_kv_heads * B) // W))
-    if N <= c_min:
-        c = max(N, 1)
-    else:
-        c = N
-        for cand in range(c_min, N + 1):
-            if work(cand) <= k * W:
-                c = cand
+    group_pieces = [[] for _ in range(n_groups)]
+    pos = 0
+    for b in range(B):
+        t = 0
+        while True:
+            g = min(pos // q, n_groups - 1)
+            take = min(L[b] - t, (g + 1) * q - pos)
+            group_pieces[g].append((b, t, t + take))
+            t += take
+            pos += take
+            if t >= L[b]:
                 break
 
-    chunks = [max(1, -(-nb // c)) for nb in n]
-    merge_indptr = [0]
-    for b in range(B):
-        merge_indptr.append(merge_indptr[-1] + (chunks[b] if chunks[b] > 1 else 0))
-    items = []
-    for b in range(B):
-        for j in range(chunks[b]):
-            pb = indptr[b] + j * c
-            pe = min(pb + c, indptr[b + 1])
-            tokens = (pe - pb) * P
-            if pe == indptr[b + 1] and pe > pb:
-                tokens -= P - last[b]
-            slot = -1 if chunks[b] == 1 else merge_indptr[b] + j
-            for h in range(num_kv_heads):
-                items.append((b, h, pb, pe, tokens, slot))
-    items.sort(key=lambda item: -item[4])  # Python's sort is stable
-    return c, np.array(items, dtype=np.int32).reshape(-1, 6), np.array(merge_indptr, dtype=np.int32)
+    items, cta_indptr = [], [0]
+    for g in range(n_groups):
+        for h in range(Hkv):
+            for (b, t0, t1) in group_pieces[g]:
+                items.append([b, h, indptr[b], t0, t1, -1])
+            cta_indptr.append(len(items))
+
+    count = [0] * (B * Hkv)
+    for it in items:
+        count[it[0] * Hkv + it[1]] += 1
+    merge_indptr = [0] * (B * Hkv + 1)
+    for seg in range(B * Hkv):
+        merge_indptr[seg + 1] = merge_indptr[seg] + (count[seg] if count[seg] > 1 else 0)
+    seen = [0] * (B * Hkv)
+    for it in items:
+        seg = it[0] * Hkv + it[1]
+        if count[seg] > 1:
+            it[5] = merge_indptr[seg] + seen[seg]
+            seen[seg] += 1
+    return (q, np.array(items, dtype=np.int32).reshape(-1, 6),
+            np.array(cta_indptr, dtype=np.int32), np.array(merge_indptr, dtype=np.int32))
 
 
 __all__ = ["build_library", "paged_decode", "paged_decode_requests", "merge_state", "merge_states", "cascade_decode",

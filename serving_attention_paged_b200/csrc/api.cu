@@ -45,6 +45,9 @@ pa_status pa_plan_upload(pa_plan_t plan, void* d_workspace, size_t workspace_byt
     e = cudaMemcpyAsync(ws + plan->ws.items, plan->items.data(),
                         plan->items.size() * sizeof(pa_work_item), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess)
+    e = cudaMemcpyAsync(ws + plan->ws.cta_indptr, plan->cta_indptr.data(),
+                        plan->cta_indptr.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
     e = cudaMemcpyAsync(ws + plan->ws.merge_indptr, plan->merge_indptr.data(),
                         plan->merge_indptr.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && p.batch > 0)

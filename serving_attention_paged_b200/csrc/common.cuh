@@ -65,6 +65,14 @@ __device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr,
                "r"(src_bytes)
                : "memory");
 }
+// The same with compile-time byte offsets on the shared (kDst) and global
+// (kSrc) addresses, folded into the instruction.
+template <int kDst, int kSrc = kDst>
+__device__ __forceinline__ void cp_async16_imm(uint32_t smem_addr, uint64_t gaddr, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0+%3], [%1+%4], 16, %2;\n" ::"r"(smem_addr),
+               "l"(gaddr), "r"(src_bytes), "n"(kDst), "n"(kSrc)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }

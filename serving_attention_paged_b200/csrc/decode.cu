@@ -52,17 +52,42 @@ namespace {
 
 constexpr int D = kHeadDim;
 constexpr int kThreads = 128;
-constexpr int kGroups = kThreads / 16;                // 8 token groups of 16 lanes
-constexpr int kTokPerGroup = 4;                       // tokens per group per tile
-constexpr int kTile = kGroups * kTokPerGroup;         // 32 tokens per stage
-constexpr int kStages = 4;
 constexpr int kRowBytes = D * 2;                      // one (token, head) row
-constexpr int kHalfStage = kTile * kRowBytes;         // K (or V) rows of a tile: 8 KB
-constexpr int kStageBytes = 2 * kHalfStage;           // 16 KB
-constexpr int kRingBytes = kStages * kStageBytes;     // 64 KB
-constexpr int kPBytesPerGroup = kTokPerGroup * 8 * 4 + 8 * 4;  // p[4][<=8] + alpha[<=8]
-constexpr int kPBytes = kGroups * kPBytesPerGroup;
-constexpr int kSmemBytes = kRingBytes + kPBytes;
+constexpr int kStages = 3;
+constexpr float kSlack = 8.f;                         // lazy-rescale threshold (base 2)
+
+// Shape of the lane <-> (token, element) mapping for a GQA group size G:
+//   LT lanes share a token; lane c of a token holds the 8-element blocks
+//   c, c + LT, c + 2 LT, ... of the 128-element row (E = 128 / LT elements,
+//   V = E / 8 16-byte vectors), so each vector load of a group of LT lanes
+//   is one contiguous LT * 16-byte piece of the row (conflict-free in shared
+//   memory, full sectors in global memory).  q (16-bit, G x E) and o (fp32,
+//   G x E) stay in registers: E * G <= 64.  Fewer lanes per token means
+//   fewer cross-lane reduction steps and fewer per-token instructions.
+template <int G> struct Shape;
+template <> struct Shape<1> { static constexpr int LT = 4, TPG = 1, LG = 0, MINB = 4; };
+template <> struct Shape<2> { static constexpr int LT = 4, TPG = 1, LG = 1, MINB = 4; };
+template <> struct Shape<4> { static constexpr int LT = 8, TPG = 2, LG = 2, MINB = 3; };
+template <> struct Shape<8> { static constexpr int LT = 16, TPG = 4, LG = 3, MINB = 3; };
+
+template <int G> struct Cfg {
+  static constexpr int LT = Shape<G>::LT;               // lanes per token
+  static constexpr int LG = Shape<G>::LG;               // log2 G
+  static constexpr int LLT = LT == 16 ? 4 : LT == 8 ? 3 : LT == 4 ? 2 : 1;  // log2 LT
+  static constexpr int E = D / LT;                      // elements per lane
+  static constexpr int V = E / 8;                       // 16-byte vectors per lane per row
+  static constexpr int kGroups = kThreads / LT;         // token groups in the CTA
+  static constexpr int TPG = Shape<G>::TPG;             // tokens per group per tile
+  static constexpr int kTile = kGroups * TPG;           // tokens per stage
+  static constexpr int kHalfStage = kTile * kRowBytes;  // K (or V) rows of a tile
+  static constexpr int kStageBytes = 2 * kHalfStage;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kPBytesPerGroup = TPG * 8 * 4 + 8 * 4;  // p[TPG][<=8] + alpha[<=8]
+  static constexpr int kSmemBytes = kRingBytes + kGroups * kPBytesPerGroup;
+  static constexpr int kLanesPerHead = LT >> LG;
+  static_assert(LG <= LLT, "a head's score must fit in the lanes of a token");
+  static_assert(kGroups * G * D * 4 + 2 * kGroups * G * 4 <= kRingBytes, "merge scratch");
+};
 
 struct DecodeArgs {
   const uint16_t* q;
@@ -70,6 +95,7 @@ struct DecodeArgs {
   const uint16_t* v_pool;
   const int32_t* kv_indices;
   const pa_work_item* items;
+  const int32_t* cta_indptr;
   const int32_t* merge_indptr;
   int32_t* counters;
   float* partial_o;
@@ -84,14 +110,6 @@ struct DecodeArgs {
   float score_scale;  // sm_scale * log2(e)
 };
 
-template <int G> struct Log2;
-template <> struct Log2<1> { static constexpr int v = 0; };
-template <> struct Log2<2> { static constexpr int v = 1; };
-template <> struct Log2<4> { static constexpr int v = 2; };
-template <> struct Log2<8> { static constexpr int v = 3; };
-
-template <int G> struct MinBlocks { static constexpr int v = 3; };
-
 // p as the PV step consumes it: fp16 for fp16 inputs, fp32 for bf16.
 template <typename Tag> struct PType;
 template <> struct PType<F16> { using T = uint16_t; };
@@ -104,168 +122,218 @@ __device__ __forceinline__ void write_final(const DecodeArgs& a, int64_t row, in
   if (d == 0 && a.lse) a.lse[row] = lse2 == -INFINITY ? -INFINITY : lse2 * kLn2;
 }
 
-// Reduce G partial dot products over the 16 lanes of a half warp.  Operands
-// are stored in lane-permuted order, so at every butterfly step each lane
-// keeps the low half of its values and sends the high half.
-template <int G>
-__device__ __forceinline__ float reduce_scatter16(float (&v)[G]) {
-  constexpr int LG = Log2<G>::v;
+// Reduce G partial dot products over the LT lanes of a token.  Operands are
+// stored in lane-permuted order, so at every butterfly step each lane keeps
+// the low half of its values and sends the high half; lane c ends with the
+// total of head c >> (log2 LT - log2 G).
+template <int G, int LT>
+__device__ __forceinline__ float reduce_scatter(float (&v)[G]) {
+  constexpr int LG = Cfg<G>::LG;
 #pragma unroll
   for (int k = 0; k < LG; ++k) {
     const int half = (G >> k) >> 1;
 #pragma unroll
     for (int i = 0; i < G / 2; ++i)
-      if (i < half) v[i] += __shfl_xor_sync(0xffffffffu, v[i + half], 8 >> k);
+      if (i < half) v[i] += __shfl_xor_sync(0xffffffffu, v[i + half], (LT / 2) >> k);
   }
   float r = v[0];
 #pragma unroll
-  for (int k = LG; k < 4; ++k) r += __shfl_xor_sync(0xffffffffu, r, 8 >> k);
+  for (int off = (LT / 2) >> LG; off >= 1; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
   return r;
 }
 
-template <typename Tag, int G>
-__device__ __forceinline__ void pv_update(F16, const uint4& v, const uint16_t (&p)[G],
-                                          float (&o)[G][8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Copy G values of p from shared memory with the widest aligned loads.
+template <typename T, int G>
+__device__ __forceinline__ void load_vec(const T* src, T (&dst)[G]) {
+  constexpr int kBytes = G * int(sizeof(T));
+  if constexpr (kBytes % 16 == 0) {
+#pragma unroll
+    for (int i = 0; i < kBytes / 16; ++i)
+      reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
+  } else if constexpr (kBytes == 8) {
+    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+  } else if constexpr (kBytes == 4) {
+    *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
+  } else {
+#pragma unroll
+    for (int i = 0; i < G; ++i) dst[i] = src[i];
+  }
+}
+
+// o[h][8v .. 8v+7] += p[h] * v-vector v, for every head h.
+template <int G, int E>
+__device__ __forceinline__ void pv_update(F16, const uint4& x, int v, const uint16_t (&p)[G],
+                                          float (&o)[G][E]) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
   for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) axpy2_f16(p[hh], w[i], o[hh][2 * i], o[hh][2 * i + 1]);
+    for (int i = 0; i < 4; ++i)
+      axpy2_f16(p[hh], w[i], o[hh][8 * v + 2 * i], o[hh][8 * v + 2 * i + 1]);
 }
-
-template <typename Tag, int G>
-__device__ __forceinline__ void pv_update(BF16, const uint4& v, const float (&p)[G],
-                                          float (&o)[G][8]) {
+template <int G, int E>
+__device__ __forceinline__ void pv_update(BF16, const uint4& x, int v, const float (&p)[G],
+                                          float (&o)[G][E]) {
   float vf[8];
-  to_float8(BF16{}, v, vf);
+  to_float8(BF16{}, x, vf);
 #pragma unroll
   for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) o[hh][i] = fmaf(p[hh], vf[i], o[hh][i]);
+    for (int i = 0; i < 8; ++i) o[hh][8 * v + i] = fmaf(p[hh], vf[i], o[hh][8 * v + i]);
 }
 
+// This lane's V 16-byte vectors of one K row and one V row (vector v of the
+// lane sits v * LT * 16 bytes further in the row and in the ring slot).
+template <int V, int LT, int kHalf, int v = 0>
+__device__ __forceinline__ void copy_row(uint32_t dst, uint64_t ka, uint64_t va, uint32_t nbytes) {
+  if constexpr (v < V) {
+    cp_async16_imm<v * LT * 16>(dst, ka, nbytes);
+    cp_async16_imm<kHalf + v * LT * 16, v * LT * 16>(dst, va, nbytes);
+    copy_row<V, LT, kHalf, v + 1>(dst, ka, va, nbytes);
+  }
+}
+
+// One piece: tokens [token_begin, token_end) of kv head h of request b.
 template <typename Tag, int G, bool kCheck>
-__global__ void __launch_bounds__(kThreads, MinBlocks<G>::v)
-    paged_decode_kernel(const DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ int s_is_last;
+__device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_item& it,
+                                          uint8_t* smem, int& s_is_last) {
+  using C = Cfg<G>;
   using PT = typename PType<Tag>::T;
-  constexpr int LG = Log2<G>::v;
-  constexpr int kLanesPerHead = 16 >> LG;
+  constexpr int LT = C::LT, E = C::E, V = C::V, TPG = C::TPG;
+  constexpr int kGroups = C::kGroups, kTile = C::kTile;
 
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const pa_work_item it = a.items[blockIdx.x];
-  const int b = it.request, h = it.kv_head, len = it.kv_len_in_chunk;
+  const int lt = tid & (LT - 1);   // lane within the token
+  const int grp = tid / LT;        // token group
+  const int b = it.request, h = it.kv_head;
+  const int tb = it.token_begin, len = it.token_end - it.token_begin;
   const int ntiles = (len + kTile - 1) / kTile;
   const int Hq = a.num_qo_heads;
   const int hq0 = h * G;
+  const int my_head = lt >> (C::LLT - C::LG);  // head whose score this lane ends with
 
-  const int lane16 = tid & 15;
-  const int grp = tid >> 4;
-  const int my_head = lane16 >> (4 - LG);  // head whose score this lane ends with
-
-  uint32_t qw[G][4];  // q in storage type; position i holds head i ^ my_head
+  // q in its 16-bit storage type; position i holds head i ^ my_head.
+  uint32_t qw[G][V][4];
 #pragma unroll
-  for (int i = 0; i < G; ++i) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(
-        a.q + (int64_t(b) * Hq + hq0 + (i ^ my_head)) * D + lane16 * 8));
-    qw[i][0] = u.x;
-    qw[i][1] = u.y;
-    qw[i][2] = u.z;
-    qw[i][3] = u.w;
-  }
-  uint8_t* pbuf = smem + kRingBytes + grp * kPBytesPerGroup;
-  PT* pshare = reinterpret_cast<PT*>(pbuf);                       // [kTokPerGroup][G]
-  float* ashare = reinterpret_cast<float*>(pbuf + kTokPerGroup * 8 * 4);  // [G]
+  for (int i = 0; i < G; ++i)
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+          a.q + (int64_t(b) * Hq + hq0 + (i ^ my_head)) * D + (lt + v * LT) * 8));
+      qw[i][v][0] = u.x;
+      qw[i][v][1] = u.y;
+      qw[i][v][2] = u.z;
+      qw[i][v][3] = u.w;
+    }
+  uint8_t* pbuf = smem + C::kRingBytes + grp * C::kPBytesPerGroup;
+  PT* pshare = reinterpret_cast<PT*>(pbuf);                          // [TPG][G]
+  float* ashare = reinterpret_cast<float*>(pbuf + TPG * 8 * 4);      // [G]
 
-  float o[G][8];
+  float o[G][E];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) o[hh][i] = 0.f;
+    for (int i = 0; i < E; ++i) o[hh][i] = 0.f;
   float m = -INFINITY, l = 0.f;
-  const bool writer = (lane16 & (kLanesPerHead - 1)) == 0;
+  const bool writer = (lt & (C::kLanesPerHead - 1)) == 0;
 
-  // ---- loads: this thread's 16-byte vectors of its 4 rows per tile ----
-  const int lp = a.log2_page, pmask = (1 << lp) - 1;
-  const int64_t row_stride = int64_t(a.num_kv_heads) * D;
-  const uint16_t* kbase = a.k_pool + int64_t(h) * D + lane16 * 8;
-  const uint16_t* vbase = a.v_pool + int64_t(h) * D + lane16 * 8;
-  const uint32_t my_slot = smem_u32(smem) + grp * kRowBytes + lane16 * 16;
-  auto load_pages = [&](int tile, int (&pg)[kTokPerGroup]) {
+  // ---- loads: this thread's vectors of its TPG rows per tile ----
+  // Addresses are formed with one 32x32->64-bit multiply-add per row (pool
+  // row index x bytes per pool row + this lane's base), and the V vectors and
+  // the second vector of a row use immediate offsets.
+  const int lp = a.log2_page;
+  const uint32_t pmask = (1u << lp) - 1u;
+  const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * kRowBytes;
+  const uint64_t kaddr0 = reinterpret_cast<uint64_t>(a.k_pool + int64_t(h) * D + lt * 8);
+  const uint64_t vaddr0 = reinterpret_cast<uint64_t>(a.v_pool + int64_t(h) * D + lt * 8);
+  const int32_t* page_list = a.kv_indices + it.page_begin;
+  const uint32_t my_slot = smem_u32(smem) + grp * kRowBytes + lt * 16;
+  auto load_pages = [&](int tile, int (&pg)[TPG]) {
 #pragma unroll
-    for (int j = 0; j < kTokPerGroup; ++j) {
+    for (int j = 0; j < TPG; ++j) {
       const int pos = tile * kTile + grp + kGroups * j;
       int p = -1;
       if (pos < len) {
-        const int at = it.page_begin + (pos >> lp);
-        p = __ldg(a.kv_indices + at);
+        const int idx = (tb + pos) >> lp;
+        p = __ldg(page_list + idx);
         if (kCheck && (p < 0 || int64_t(p) >= a.num_pages)) {
-          atomicMin(a.error_pos, (unsigned long long)at);
+          atomicMin(a.error_pos, (unsigned long long)(it.page_begin + idx));
           p = -1;  // not copied: the row reads as zeros
         }
       }
       pg[j] = p;
     }
   };
-  auto issue = [&](int tile, int stage, const int (&pg)[kTokPerGroup]) {
+  auto issue = [&](int tile, uint32_t stage_off, const int (&pg)[TPG]) {
     if (tile < ntiles) {
 #pragma unroll
-      for (int j = 0; j < kTokPerGroup; ++j) {
-        const int pos = tile * kTile + grp + kGroups * j;
+      for (int j = 0; j < TPG; ++j) {
+        const uint32_t pos = uint32_t(tb + tile * kTile + grp + kGroups * j);
         const bool ok = pg[j] >= 0;
-        const int64_t off = ok ? ((int64_t(pg[j]) << lp) | (pos & pmask)) * row_stride : 0;
-        const uint32_t dst = my_slot + stage * kStageBytes + j * kGroups * kRowBytes;
-        cp_async16(dst, kbase + off, ok ? 16 : 0);
-        cp_async16(dst + kHalfStage, vbase + off, ok ? 16 : 0);
+        const uint32_t row = ok ? ((uint32_t(pg[j]) << lp) | (pos & pmask)) : 0u;
+        const uint32_t nbytes = ok ? 16u : 0u;
+        uint64_t ka, va;
+        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(ka) : "r"(row), "r"(pool_row_bytes), "l"(kaddr0));
+        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(va) : "r"(row), "r"(pool_row_bytes), "l"(vaddr0));
+        const uint32_t dst = my_slot + stage_off + j * kGroups * kRowBytes;
+        copy_row<V, LT, C::kHalfStage>(dst, ka, va, nbytes);
       }
     }
     cp_async_commit();
   };
-  int pg[kTokPerGroup];
+  int pg[TPG];
 #pragma unroll
   for (int st = 0; st < kStages - 1; ++st) {
     load_pages(st, pg);
-    issue(st, st, pg);
+    issue(st, st * C::kStageBytes, pg);
   }
   load_pages(kStages - 1, pg);
 
+  uint32_t issue_off = (kStages - 1) * C::kStageBytes;  // ring slot of tile t + kStages - 1
+  uint32_t read_off = 0;                                 // ring slot of tile t
   for (int t = 0; t < ntiles; ++t) {
-    issue(t + kStages - 1, (t + kStages - 1) % kStages, pg);
+    issue(t + kStages - 1, issue_off, pg);
     load_pages(t + kStages, pg);
+    issue_off = issue_off + C::kStageBytes == C::kRingBytes ? 0u : issue_off + C::kStageBytes;
     cp_async_wait<kStages - 1>();
-    const int s = t % kStages;
-    const uint8_t* ks = smem + s * kStageBytes + grp * kRowBytes + lane16 * 16;
-    const uint8_t* vs = ks + kHalfStage;
+    const uint8_t* ks = smem + read_off + grp * kRowBytes + lt * 16;
+    read_off = read_off + C::kStageBytes == C::kRingBytes ? 0u : read_off + C::kStageBytes;
+    const uint8_t* vs = ks + C::kHalfStage;
 
-    float sc[kTokPerGroup];
+    float sc[TPG];
 #pragma unroll
-    for (int j = 0; j < kTokPerGroup; ++j) {
-      const uint4 u = *reinterpret_cast<const uint4*>(ks + j * kGroups * kRowBytes);
+    for (int j = 0; j < TPG; ++j) {
       float part[G];
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
-        float acc = 0.f;
-        acc = dot2(Tag{}, u.x, qw[i][0], acc);
-        acc = dot2(Tag{}, u.y, qw[i][1], acc);
-        acc = dot2(Tag{}, u.z, qw[i][2], acc);
-        acc = dot2(Tag{}, u.w, qw[i][3], acc);
-        part[i] = acc;
+      for (int i = 0; i < G; ++i) part[i] = 0.f;
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const uint4 u = *reinterpret_cast<const uint4*>(ks + j * kGroups * kRowBytes + v * LT * 16);
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          part[i] = dot2(Tag{}, u.x, qw[i][v][0], part[i]);
+          part[i] = dot2(Tag{}, u.y, qw[i][v][1], part[i]);
+          part[i] = dot2(Tag{}, u.z, qw[i][v][2], part[i]);
+          part[i] = dot2(Tag{}, u.w, qw[i][v][3], part[i]);
+        }
       }
-      const float r = reduce_scatter16<G>(part);
+      const float r = reduce_scatter<G, LT>(part);
       sc[j] = (t * kTile + grp + kGroups * j < len) ? r * a.score_scale : -INFINITY;
     }
 
-    float mnew = m;
+    // Lazy running max: the reference point m moves only when a score beats
+    // it by more than kSlack (base 2), so p = 2^(s - m) <= 2^kSlack and o is
+    // rarely rescaled.  Any reference point gives the same normalised result.
+    float tmax = sc[0];
 #pragma unroll
-    for (int j = 0; j < kTokPerGroup; ++j) mnew = fmaxf(mnew, sc[j]);
+    for (int j = 1; j < TPG; ++j) tmax = fmaxf(tmax, sc[j]);
+    const bool moved = tmax > m + kSlack;
+    const float mnew = moved ? tmax : m;
     const float msafe = mnew == -INFINITY ? 0.f : mnew;
-    const bool moved = mnew != m;
     const float alpha = moved ? fast_exp2(m - msafe) : 1.f;
     float psum = 0.f;
 #pragma unroll
-    for (int j = 0; j < kTokPerGroup; ++j) {
+    for (int j = 0; j < TPG; ++j) {
       float p = fast_exp2(sc[j] - msafe);
       PT ps;
       if constexpr (sizeof(PT) == 2) {
@@ -286,32 +354,36 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<G>::v)
       for (int hh = 0; hh < G; ++hh) {
         const float ah = ashare[hh];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[hh][i] *= ah;
+        for (int i = 0; i < E; ++i) o[hh][i] *= ah;
       }
     }
 #pragma unroll
-    for (int j = 0; j < kTokPerGroup; ++j) {
-      const uint4 v = *reinterpret_cast<const uint4*>(vs + j * kGroups * kRowBytes);
+    for (int j = 0; j < TPG; ++j) {
       PT pj[G];
+      load_vec(pshare + j * G, pj);
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) pj[hh] = pshare[j * G + hh];
-      pv_update<Tag, G>(Tag{}, v, pj, o);
+      for (int v = 0; v < V; ++v) {
+        const uint4 x = *reinterpret_cast<const uint4*>(vs + j * kGroups * kRowBytes + v * LT * 16);
+        pv_update<G, E>(Tag{}, x, v, pj, o);
+      }
     }
     __syncwarp();  // p and alpha of this tile consumed before the next tile writes them
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // Combine the 8 token groups through shared memory (the ring is idle now).
+  // Combine the token groups through shared memory (the ring is idle now).
   float* Os = reinterpret_cast<float*>(smem);  // [kGroups][G][D]
   float* Ms = Os + kGroups * G * D;            // [kGroups][G]
   float* Ls = Ms + kGroups * G;
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    float4* dst = reinterpret_cast<float4*>(Os + (grp * G + hh) * D + lane16 * 8);
-    dst[0] = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
-    dst[1] = make_float4(o[hh][4], o[hh][5], o[hh][6], o[hh][7]);
-  }
+  for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      float4* dst = reinterpret_cast<float4*>(Os + (grp * G + hh) * D + (lt + v * LT) * 8);
+      dst[0] = make_float4(o[hh][8 * v], o[hh][8 * v + 1], o[hh][8 * v + 2], o[hh][8 * v + 3]);
+      dst[1] = make_float4(o[hh][8 * v + 4], o[hh][8 * v + 5], o[hh][8 * v + 6], o[hh][8 * v + 7]);
+    }
   if (writer) {
     Ms[grp * G + my_head] = m;
     Ls[grp * G + my_head] = l;
@@ -323,14 +395,14 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<G>::v)
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
     float M = -INFINITY;
-#pragma unroll
+#pragma unroll 8
     for (int g = 0; g < kGroups; ++g) M = fmaxf(M, Ms[g * G + hh]);
     if (M == -INFINITY) {
       res[hh] = 0.f;
       lse2[hh] = -INFINITY;
     } else {
       float lsum = 0.f, acc = 0.f;
-#pragma unroll
+#pragma unroll 8
       for (int g = 0; g < kGroups; ++g) {
         const float w = fast_exp2(Ms[g * G + hh] - M);
         lsum = fmaf(w, Ls[g * G + hh], lsum);
@@ -363,14 +435,15 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<G>::v)
   const int64_t slot = it.partial_slot;
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
-    a.partial_o[(slot * Hq + hq0 + hh) * D + d] = res[hh];
-    if (d == 0) a.partial_lse[slot * Hq + hq0 + hh] = lse2[hh];
+    a.partial_o[(slot * G + hh) * D + d] = res[hh];
+    if (d == 0) a.partial_lse[slot * G + hh] = lse2[hh];
   }
   __threadfence();
   __syncthreads();
+  const int64_t seg = int64_t(b) * a.num_kv_heads + h;
   if (tid == 0) {
-    const int nchunks = a.merge_indptr[b + 1] - a.merge_indptr[b];
-    int32_t* ctr = a.counters + int64_t(b) * a.num_kv_heads + h;
+    const int nchunks = a.merge_indptr[seg + 1] - a.merge_indptr[seg];
+    int32_t* ctr = a.counters + seg;
     const int prev = atomicAdd(ctr, 1);
     s_is_last = prev == nchunks - 1;
     if (s_is_last) *ctr = 0;  // every other chunk has arrived: safe to reset
@@ -378,36 +451,49 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<G>::v)
   __syncthreads();
   if (!s_is_last) return;
   __threadfence();
-  const int s0 = a.merge_indptr[b], s1 = a.merge_indptr[b + 1];
+  const int s0 = a.merge_indptr[seg], s1 = a.merge_indptr[seg + 1];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
-    const int64_t hq = hq0 + hh;
     MergeAcc acc;
     for (int sl = s0; sl < s1; ++sl)
-      acc.add(__ldcg(a.partial_o + (int64_t(sl) * Hq + hq) * D + d),
-              __ldcg(a.partial_lse + int64_t(sl) * Hq + hq));
-    const int64_t row = int64_t(b) * Hq + hq;
+      acc.add(__ldcg(a.partial_o + (int64_t(sl) * G + hh) * D + d),
+              __ldcg(a.partial_lse + int64_t(sl) * G + hh));
+    const int64_t row = int64_t(b) * Hq + hq0 + hh;
     for (int c = 0; c < a.prefix_chunks; ++c)
       acc.add(a.prefix_o[(c * Bstride + row) * D + d], a.prefix_lse[c * Bstride + row]);
     write_final<Tag>(a, row, d, acc.out(), acc.lse2());
   }
 }
 
+// One CTA per quota: it runs its pieces in order (usually one or two).
 template <typename Tag, int G, bool kCheck>
-cudaError_t launch_t(const DecodeArgs& a, int64_t n_items, cudaStream_t stream) {
+__global__ void __launch_bounds__(kThreads, Shape<G>::MINB)
+    paged_decode_kernel(const DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int s_is_last;
+  const int p0 = a.cta_indptr[blockIdx.x], p1 = a.cta_indptr[blockIdx.x + 1];
+  for (int pi = p0; pi < p1; ++pi) {
+    if (pi > p0) __syncthreads();  // the previous piece is done with shared memory
+    run_piece<Tag, G, kCheck>(a, a.items[pi], smem, s_is_last);
+  }
+}
+
+template <typename Tag, int G, bool kCheck>
+cudaError_t launch_t(const DecodeArgs& a, int64_t n_cta, cudaStream_t stream) {
   auto kern = paged_decode_kernel<Tag, G, kCheck>;
   static std::atomic<uint64_t> configured{0};  // bit per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = uint64_t(1) << (dev & 63);
+  constexpr int kSmem = Cfg<G>::kSmemBytes;
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  if (n_items == 0) return cudaSuccess;
-  kern<<<dim3(unsigned(n_items)), kThreads, kSmemBytes, stream>>>(a);
+  if (n_cta <= 0) return cudaSuccess;
+  kern<<<dim3(unsigned(n_cta)), kThreads, kSmem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -424,17 +510,16 @@ cudaError_t dispatch_group(int group, const DecodeArgs& a, int64_t n, cudaStream
 
 template <typename Tag>
 cudaError_t occupancy_t(int group, int* out) {
-  auto get = [&](auto kern) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+  auto get = [&](auto kern, int smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, kSmemBytes);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, smem);
   };
   switch (group) {
-    case 1: return get(paged_decode_kernel<Tag, 1, false>);
-    case 2: return get(paged_decode_kernel<Tag, 2, false>);
-    case 4: return get(paged_decode_kernel<Tag, 4, false>);
-    case 8: return get(paged_decode_kernel<Tag, 8, false>);
+    case 1: return get(paged_decode_kernel<Tag, 1, false>, Cfg<1>::kSmemBytes);
+    case 2: return get(paged_decode_kernel<Tag, 2, false>, Cfg<2>::kSmemBytes);
+    case 4: return get(paged_decode_kernel<Tag, 4, false>, Cfg<4>::kSmemBytes);
+    case 8: return get(paged_decode_kernel<Tag, 8, false>, Cfg<8>::kSmemBytes);
   }
   return cudaErrorInvalidValue;
 }
@@ -460,6 +545,7 @@ int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream) {
   a.v_pool = static_cast<const uint16_t*>(p.v_pool);
   a.kv_indices = p.kv_indices;
   a.items = reinterpret_cast<const pa_work_item*>(p.ws + plan.ws.items);
+  a.cta_indptr = reinterpret_cast<const int32_t*>(p.ws + plan.ws.cta_indptr);
   a.merge_indptr = reinterpret_cast<const int32_t*>(p.ws + plan.ws.merge_indptr);
   a.counters = reinterpret_cast<int32_t*>(p.ws + plan.ws.counters);
   a.partial_o = reinterpret_cast<float*>(p.ws + plan.ws.partial_o);
@@ -477,7 +563,7 @@ int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream) {
   a.prefix_chunks = plan.cascade ? plan.prefix_chunks : 0;
   a.score_scale = pr.sm_scale * kLog2e;
   const bool check = (pr.flags & PA_FLAG_CHECK_INDICES) != 0;
-  const int64_t n = int64_t(plan.items.size());
+  const int64_t n = int64_t(plan.cta_indptr.size()) - 1;  // CTAs
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (pr.dtype == PA_BF16)

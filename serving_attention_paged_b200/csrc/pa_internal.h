@@ -17,17 +17,19 @@ constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 
 // Device workspace, in this order (each region 256-byte aligned):
-//   items        [n_items]             pa_work_item
-//   merge_indptr [B + 1]               int32
+//   items        [n_items]             pa_work_item (pieces, grouped by CTA)
+//   cta_indptr   [n_cta + 1]           int32, pieces of CTA i
+//   merge_indptr [B * Hkv + 1]         int32, partial slots of segment (b, h)
 //   counters     [B * Hkv]             int32, zero between runs
 //   error        [2]                   uint64: first bad kv_indices position (~0 = none),
 //                                      then a timeout flag (0 = none)
-//   partial_o    [n_partials, Hq, D]   fp32, split-chunk outputs (normalised)
-//   partial_lse  [n_partials, Hq]      fp32, their log-sum-exp in base 2
+//   partial_o    [n_partials, G, D]    fp32, outputs of pieces of split segments
+//                                      (normalised; G = q heads of the kv head)
+//   partial_lse  [n_partials, G]       fp32, their log-sum-exp in base 2
 //   prefix_o     [prefix_chunks, B, Hq, D]  fp32 (cascade only)
 //   prefix_lse   [prefix_chunks, B, Hq]     fp32, base 2 (cascade only)
 struct WorkspaceLayout {
-  size_t items = 0, merge_indptr = 0, counters = 0, error = 0, partial_o = 0, partial_lse = 0,
+  size_t items = 0, cta_indptr = 0, merge_indptr = 0, counters = 0, error = 0, partial_o = 0, partial_lse = 0,
          prefix_o = 0, prefix_lse = 0, total = 0;
 };
 
@@ -37,10 +39,11 @@ struct pa_plan_s {
   pa_problem prob{};
   int32_t group = 1;        // Hq / Hkv
   int32_t log2_page = 0;    // page_size = 1 << log2_page
-  int32_t chunk_pages = 1;
+  int32_t quota = 0;        // (token, kv head) units per CTA
   std::vector<int32_t> kv_indptr, last_page_len;
-  std::vector<pa_work_item> items;
-  std::vector<int32_t> merge_indptr;
+  std::vector<pa_work_item> items;  // pieces, grouped by CTA
+  std::vector<int32_t> cta_indptr;  // [n_cta + 1]
+  std::vector<int32_t> merge_indptr;  // [B * Hkv + 1]
   int64_t n_partials = 0;
   // cascade (level 1 over the shared prefix)
   bool cascade = false;

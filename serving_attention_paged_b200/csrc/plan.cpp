@@ -2,10 +2,14 @@
 //
 // FlashInfer README, core feature 2 ("Load-Balanced Scheduling"): the
 // attention computation is split into a plan stage that schedules
-// variable-length inputs and a run stage that computes.  The page gives no
-// algorithm; the specification implemented here is documented with
-// pa_plan_create in pagedattn.h.  Host code only: no CUDA call.
+// variable-length inputs and a run stage that computes; the same README
+// names stream-K among the designs FlashInfer draws on.  The page gives no
+// algorithm.  The specification implemented here (documented with
+// pa_plan_create in pagedattn.h) is a stream-K style split: every group of
+// Hkv CTAs gets an equal, contiguous share of the concatenated request
+// tokens, one CTA per kv head.  Host code only: no CUDA call.
 #include <algorithm>
+#include <array>
 #include <cstring>
 #include <new>
 
@@ -35,14 +39,9 @@ pa_status validate_problem(const pa_problem* p) {
   if (p->head_dim != pa::kHeadDim) return PA_ERR_UNSUPPORTED;
   if (!is_pow2(p->page_size) || p->page_size > 1024) return PA_ERR_UNSUPPORTED;
   if (!pa::decode_group_supported(p->num_qo_heads / p->num_kv_heads)) return PA_ERR_UNSUPPORTED;
+  // pool rows (page * P + row) are 32-bit indices inside the kernels
+  if (p->num_pages * int64_t(p->page_size) > int64_t(UINT32_MAX)) return PA_ERR_UNSUPPORTED;
   return PA_OK;
-}
-
-// Work items for a given chunk size (pages): Hkv * sum_b max(1, ceil(n_b / c)).
-int64_t work(const std::vector<int64_t>& n, int64_t c, int64_t hkv) {
-  int64_t w = 0;
-  for (int64_t nb : n) w += std::max<int64_t>(1, ceil_div(nb, c));
-  return w * hkv;
 }
 
 pa_status build(pa_plan_s* plan, const int32_t* indptr, const int32_t* last) {
@@ -50,67 +49,71 @@ pa_status build(pa_plan_s* plan, const int32_t* indptr, const int32_t* last) {
   const int64_t B = p.batch, P = p.page_size, Hkv = p.num_kv_heads;
   if (B > 0 && (!indptr || !last)) return PA_ERR_INVALID_ARG;
   if (indptr && indptr[0] != 0) return PA_ERR_INVALID_ARG;
-  std::vector<int64_t> n(B);
+  std::vector<int64_t> L(B);
+  int64_t total = 0;
   for (int64_t b = 0; b < B; ++b) {
     if (indptr[b + 1] < indptr[b]) return PA_ERR_INVALID_ARG;
-    n[b] = int64_t(indptr[b + 1]) - indptr[b];
-    if (n[b] > 0 && (last[b] < 1 || last[b] > P)) return PA_ERR_INVALID_ARG;
+    const int64_t n = int64_t(indptr[b + 1]) - indptr[b];
+    if (n > 0 && (last[b] < 1 || last[b] > P)) return PA_ERR_INVALID_ARG;
+    L[b] = n > 0 ? (n - 1) * P + last[b] : 0;
+    if (L[b] > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    total += L[b];
   }
-  plan->kv_indptr.assign(indptr ? indptr : nullptr, indptr ? indptr + B + 1 : nullptr);
-  if (!indptr) plan->kv_indptr.assign(1, 0);
+  if (indptr) plan->kv_indptr.assign(indptr, indptr + B + 1);
+  else plan->kv_indptr.assign(1, 0);
   plan->last_page_len.assign(last ? last : nullptr, last ? last + B : nullptr);
 
-  // chunk size: smallest c in [c_min, N] with work(c) <= k * W, where k is the
-  // number of waves the unsplit batch needs anyway (work is non-increasing in c)
+  // Token-level stream-K: CTAs come in groups of Hkv (one per kv head); every
+  // group gets the same quota q of the concatenated request tokens (at least
+  // min_chunk_tokens, rounded up to whole 32-token tiles), so the Hkv CTAs of
+  // a group read the same pages at the same time, each its own head.
   const int64_t W = int64_t(p.num_sms) * p.ctas_per_sm;
+  const int64_t groups = std::max<int64_t>(1, W / Hkv);
   const int64_t min_tokens = p.min_chunk_tokens ? p.min_chunk_tokens : pa::kDefaultMinChunkTokens;
-  const int64_t c_min = std::max<int64_t>(1, ceil_div(min_tokens, P));
-  const int64_t N = B ? *std::max_element(n.begin(), n.end()) : 0;
-  const int64_t waves = std::max<int64_t>(1, ceil_div(Hkv * B, W));
-  const int64_t budget = waves * W;
-  int64_t c;
-  if (N <= c_min) {
-    c = std::max<int64_t>(N, 1);
-  } else {
-    int64_t lo = c_min, hi = N;  // work(N) = Hkv * B <= budget
-    while (lo < hi) {
-      int64_t mid = lo + (hi - lo) / 2;
-      if (work(n, mid, Hkv) <= budget) hi = mid; else lo = mid + 1;
-    }
-    c = lo;
-  }
-  plan->chunk_pages = int32_t(c);
+  const int64_t q = ceil_div(std::max<int64_t>(min_tokens, ceil_div(total, groups)), 32) * 32;
+  if (q > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  plan->quota = int32_t(q);
+  const int64_t n_groups = B == 0 ? 0 : std::max<int64_t>(1, ceil_div(total, q));
+  if (n_groups * Hkv > INT32_MAX) return PA_ERR_UNSUPPORTED;
 
-  plan->merge_indptr.assign(B + 1, 0);
+  // Pieces of each group: the requests' token ranges that meet [g q, (g+1) q).
+  // An empty request is a zero-length piece of the group its position falls in.
+  std::vector<std::vector<std::array<int64_t, 3>>> group_pieces(static_cast<size_t>(n_groups));
+  int64_t pos = 0;
   for (int64_t b = 0; b < B; ++b) {
-    int64_t chunks = std::max<int64_t>(1, ceil_div(n[b], c));
-    plan->merge_indptr[b + 1] = plan->merge_indptr[b] + int32_t(chunks > 1 ? chunks : 0);
+    int64_t t = 0;
+    do {
+      const int64_t g = std::min<int64_t>(pos / q, n_groups - 1);
+      const int64_t take = std::min<int64_t>(L[b] - t, (g + 1) * q - pos);
+      group_pieces[size_t(g)].push_back({b, t, t + take});
+      t += take;
+      pos += take;
+    } while (t < L[b]);
   }
-  plan->n_partials = plan->merge_indptr[B];
-
-  const int64_t total = work(n, c, Hkv);
-  if (total > INT32_MAX) return PA_ERR_UNSUPPORTED;
   plan->items.clear();
-  plan->items.reserve(size_t(total));
-  for (int64_t b = 0; b < B; ++b) {
-    const int64_t chunks = std::max<int64_t>(1, ceil_div(n[b], c));
-    for (int64_t j = 0; j < chunks; ++j) {
-      const int64_t pb = indptr[b] + j * c;
-      const int64_t pe = std::min<int64_t>(pb + c, indptr[b + 1]);
-      int64_t tokens = (pe - pb) * P;
-      if (pe == indptr[b + 1] && pe > pb) tokens -= P - last[b];
-      const int32_t slot = chunks == 1 ? -1 : int32_t(plan->merge_indptr[b] + j);
-      for (int64_t h = 0; h < Hkv; ++h)
-        plan->items.push_back(pa_work_item{int32_t(b), int32_t(h), int32_t(pb), int32_t(pe),
-                                           int32_t(tokens), slot});
+  plan->cta_indptr.assign(size_t(n_groups * Hkv) + 1, 0);
+  for (int64_t g = 0; g < n_groups; ++g)
+    for (int64_t h = 0; h < Hkv; ++h) {
+      for (const auto& pc : group_pieces[size_t(g)])
+        plan->items.push_back(pa_work_item{int32_t(pc[0]), int32_t(h), indptr[pc[0]],
+                                           int32_t(pc[1]), int32_t(pc[2]), -1});
+      plan->cta_indptr[size_t(g * Hkv + h) + 1] = int32_t(plan->items.size());
     }
+
+  // Partial slots: a segment (b, h) cut into k > 1 pieces owns k consecutive
+  // slots, in token order (= work-list order, groups being in token order).
+  std::vector<int32_t> count(size_t(B * Hkv), 0);
+  for (const pa_work_item& it : plan->items) ++count[size_t(it.request * Hkv + it.kv_head)];
+  plan->merge_indptr.assign(size_t(B * Hkv) + 1, 0);
+  for (int64_t sgm = 0; sgm < B * Hkv; ++sgm)
+    plan->merge_indptr[sgm + 1] =
+        plan->merge_indptr[sgm] + (count[size_t(sgm)] > 1 ? count[size_t(sgm)] : 0);
+  std::vector<int32_t> seen(size_t(B * Hkv), 0);
+  for (pa_work_item& it : plan->items) {
+    const int64_t sgm = int64_t(it.request) * Hkv + it.kv_head;
+    if (count[size_t(sgm)] > 1) it.partial_slot = plan->merge_indptr[sgm] + seen[size_t(sgm)]++;
   }
-  // Longest chunks first: the block scheduler hands items to free SMs in
-  // launch order, so this is greedy longest-processing-time-first packing.
-  std::stable_sort(plan->items.begin(), plan->items.end(),
-                   [](const pa_work_item& x, const pa_work_item& y) {
-                     return x.kv_len_in_chunk > y.kv_len_in_chunk;
-                   });
+  plan->n_partials = plan->merge_indptr.back();
   return PA_OK;
 }
 
@@ -125,11 +128,13 @@ void layout_workspace(pa_plan_s* plan) {
   };
   const size_t Hq = p.num_qo_heads, D = p.head_dim, B = p.batch;
   w.items = take(plan->items.size() * sizeof(pa_work_item));
-  w.merge_indptr = take((B + 1) * sizeof(int32_t));
+  w.cta_indptr = take(plan->cta_indptr.size() * sizeof(int32_t));
+  w.merge_indptr = take(plan->merge_indptr.size() * sizeof(int32_t));
   w.counters = take(B * p.num_kv_heads * sizeof(int32_t));
   w.error = take(2 * sizeof(uint64_t));  // first bad index, timeout flag
-  w.partial_o = take(size_t(plan->n_partials) * Hq * D * sizeof(float));
-  w.partial_lse = take(size_t(plan->n_partials) * Hq * sizeof(float));
+  const size_t G = plan->group;
+  w.partial_o = take(size_t(plan->n_partials) * G * D * sizeof(float));
+  w.partial_lse = take(size_t(plan->n_partials) * G * sizeof(float));
   w.prefix_o = take(size_t(plan->prefix_chunks) * B * Hq * D * sizeof(float));
   w.prefix_lse = take(size_t(plan->prefix_chunks) * B * Hq * sizeof(float));
   w.total = off;
@@ -203,9 +208,16 @@ pa_status pa_cascade_plan_create(const pa_problem* problem, int32_t prefix_len,
   return create(problem, prefix_len, true, kv_indptr_host, last_page_len_host, out);
 }
 
-pa_status pa_plan_chunk_pages(pa_plan_t plan, int32_t* chunk_pages) {
-  if (!plan || !chunk_pages) return PA_ERR_INVALID_ARG;
-  *chunk_pages = plan->chunk_pages;
+pa_status pa_plan_quota_tokens(pa_plan_t plan, int32_t* quota) {
+  if (!plan || !quota) return PA_ERR_INVALID_ARG;
+  *quota = plan->quota;
+  return PA_OK;
+}
+
+pa_status pa_plan_cta_indptr(pa_plan_t plan, const int32_t** cta_indptr, int64_t* n_cta) {
+  if (!plan || !cta_indptr || !n_cta) return PA_ERR_INVALID_ARG;
+  *cta_indptr = plan->cta_indptr.data();
+  *n_cta = int64_t(plan->cta_indptr.size()) - 1;
   return PA_OK;
 }
 

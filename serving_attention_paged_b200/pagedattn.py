@@ -39,7 +39,7 @@ class pa_problem(ctypes.Structure):
 
 class pa_work_item(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("request", "kv_head", "page_begin", "page_end", "kv_len_in_chunk", "partial_slot")]
+                ("request", "kv_head", "page_begin", "token_begin", "token_end", "partial_slot")]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -47,7 +47,8 @@ _P = ctypes.POINTER
 _SIGS = {
     "pa_plan_create": [_P(pa_problem), _vp, _vp, _P(_vp)],
     "pa_cascade_plan_create": [_P(pa_problem), _i32, _vp, _vp, _P(_vp)],
-    "pa_plan_chunk_pages": [_vp, _P(_i32)],
+    "pa_plan_quota_tokens": [_vp, _P(_i32)],
+    "pa_plan_cta_indptr": [_vp, _P(_P(_i32)), _P(_i64)],
     "pa_plan_work_items": [_vp, _P(_P(pa_work_item)), _P(_i64)],
     "pa_plan_merge_indptr": [_vp, _P(_P(_i32))],
     "pa_plan_num_partials": [_vp, _P(_i64)],
@@ -147,10 +148,17 @@ def pa_cascade_plan_create(problem: pa_problem, prefix_len: int, kv_indptr_host,
     return Plan(h.value)
 
 
-def pa_plan_chunk_pages(plan: Plan) -> int:
+def pa_plan_quota_tokens(plan: Plan) -> int:
     c = _i32()
-    _check(lib.pa_plan_chunk_pages(plan.handle, ctypes.byref(c)), "pa_plan_chunk_pages")
+    _check(lib.pa_plan_quota_tokens(plan.handle, ctypes.byref(c)), "pa_plan_quota_tokens")
     return c.value
+
+
+def pa_plan_cta_indptr(plan: Plan) -> np.ndarray:
+    p, n = _P(_i32)(), _i64()
+    _check(lib.pa_plan_cta_indptr(plan.handle, ctypes.byref(p), ctypes.byref(n)),
+           "pa_plan_cta_indptr")
+    return np.ctypeslib.as_array(p, shape=(n.value + 1,)).copy()
 
 
 def pa_plan_work_items(plan: Plan) -> np.ndarray:
@@ -170,10 +178,11 @@ def pa_plan_num_partials(plan: Plan) -> int:
     return n.value
 
 
-def pa_plan_merge_indptr(plan: Plan, batch: int) -> np.ndarray:
+def pa_plan_merge_indptr(plan: Plan, n_segments: int) -> np.ndarray:
+    """Partial-slot offsets per (request, kv head) segment: [B * Hkv + 1]."""
     p = _P(_i32)()
     _check(lib.pa_plan_merge_indptr(plan.handle, ctypes.byref(p)), "pa_plan_merge_indptr")
-    return np.ctypeslib.as_array(p, shape=(batch + 1,)).copy()
+    return np.ctypeslib.as_array(p, shape=(n_segments + 1,)).copy()
 
 
 def pa_plan_prefix_chunks(plan: Plan):

@@ -45,13 +45,14 @@ def _problem(C, w, num_sms=148, k=2, mct=0, flags=0):
 def _compare_plan(C, indptr, last, P, hq, hkv, sms, k, mct):
     prob = C.make_problem(batch=len(last), num_qo_heads=hq, num_kv_heads=hkv, page_size=P,
                           dtype="f16", sm_scale=0.1, num_sms=sms, ctas_per_sm=k,
-                          min_chunk_tokens=mct, num_pages=1 << 30)
+                          min_chunk_tokens=mct, num_pages=1 << 20)
     plan = C.pa_plan_create(prob, indptr, last)
-    c, items, mi = oracle.plan(indptr, last, page_size=P, num_kv_heads=hkv, num_sms=sms,
-                               ctas_per_sm=k, min_chunk_tokens=mct if mct else 256)
-    assert C.pa_plan_chunk_pages(plan) == c
+    q, items, ci, mi = oracle.plan(indptr, last, page_size=P, num_kv_heads=hkv, num_sms=sms,
+                                   ctas_per_sm=k, min_chunk_tokens=mct if mct else 256)
+    assert C.pa_plan_quota_tokens(plan) == q
     assert np.array_equal(C.pa_plan_work_items(plan), items)
-    assert np.array_equal(C.pa_plan_merge_indptr(plan, len(last)), mi)
+    assert np.array_equal(C.pa_plan_cta_indptr(plan), ci)
+    assert np.array_equal(C.pa_plan_merge_indptr(plan, len(last) * hkv), mi)
     assert C.pa_plan_num_partials(plan) == mi[-1]
     return plan
 
@@ -84,7 +85,7 @@ def test_plan_matches_oracle_vector_sparse(C):
 def test_plan_edge_cases(C):
     # empty batch, all-empty requests, one page, exactly full pages, B*Hkv above the budget
     for lens, P, sms in [([], 16, 148), ([0, 0], 16, 148), ([1], 16, 148), ([16, 32, 48], 16, 148),
-                         ([100] * 50, 16, 2), ([3000, 1], 1, 1)]:
+                         ([100] * 50, 16, 2), ([3000, 1], 1, 1), ([0, 5000, 0], 16, 3)]:
         indptr, _, last = W.tables_from_lengths(lens, P)
         _compare_plan(C, indptr, last, P, 8, 8, sms, 1, 0)
 
@@ -116,6 +117,8 @@ def test_plan_validation(C):
     assert status(bad) == C.PA_ERR_INVALID_ARG
     bad = _problem(C, w); bad.num_sms = 0
     assert status(bad) == C.PA_ERR_INVALID_ARG
+    bad = _problem(C, w); bad.num_pages = (1 << 32) // 16 + 1                # rows need 33 bits
+    assert status(bad) == C.PA_ERR_UNSUPPORTED
     with pytest.raises(C.PagedAttnError) as e:
         C.pa_cascade_plan_create(ok, 24, w.kv_indptr, w.last_page_len)  # not whole pages
     assert e.value.status == C.PA_ERR_INVALID_ARG
@@ -151,6 +154,7 @@ def test_cascade_plan_shape(C):
     plan = C.pa_cascade_plan_create(prob, w.prefix_len, w.kv_indptr, w.last_page_len)
     n, tok = C.pa_plan_prefix_chunks(plan)
     assert n >= 1 and tok % 128 == 0 and n * tok >= w.prefix_len > (n - 1) * tok
-    c, items, mi = oracle.plan(w.kv_indptr, w.last_page_len, page_size=16, num_kv_heads=8,
-                               num_sms=148, ctas_per_sm=2)
+    q, items, ci, mi = oracle.plan(w.kv_indptr, w.last_page_len, page_size=16, num_kv_heads=8,
+                                   num_sms=148, ctas_per_sm=2)
     assert np.array_equal(C.pa_plan_work_items(plan), items)
+    assert np.array_equal(C.pa_plan_cta_indptr(plan), ci)
