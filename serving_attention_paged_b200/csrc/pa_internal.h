@@ -76,5 +76,6 @@ int launch_merge_state(const void* o_a, const float* lse_a, const void* o_b, con
                        void* stream);
 int decode_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out);
 bool decode_group_supported(int32_t group);
+bool cascade_page_size_supported(int32_t page_size);
 
 }  // namespace pa

@@ -168,6 +168,12 @@ pa_status create(const pa_problem* problem, int32_t prefix_len, bool cascade,
   pa_status st = validate_problem(problem);
   if (st != PA_OK) return st;
   if (cascade && (prefix_len < 0 || prefix_len % problem->page_size)) return PA_ERR_INVALID_ARG;
+  // the prefix level moves whole pages (>= 8 rows) with TMA, whose row
+  // coordinates are signed 32-bit
+  if (cascade && prefix_len > 0 &&
+      (!pa::cascade_page_size_supported(problem->page_size) ||
+       problem->num_pages * int64_t(problem->page_size) >= int64_t(INT32_MAX)))
+    return PA_ERR_UNSUPPORTED;
   pa_plan_s* plan = new (std::nothrow) pa_plan_s;
   if (!plan) return PA_ERR_NO_MEMORY;
   try {

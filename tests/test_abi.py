@@ -122,6 +122,11 @@ def test_plan_validation(C):
     with pytest.raises(C.PagedAttnError) as e:
         C.pa_cascade_plan_create(ok, 24, w.kv_indptr, w.last_page_len)  # not whole pages
     assert e.value.status == C.PA_ERR_INVALID_ARG
+    small = _problem(C, w); small.page_size = 4                             # prefix boxes >= 8 rows
+    indptr4, _, last4 = W.tables_from_lengths([20, 40], 4)
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_cascade_plan_create(small, 16, indptr4, last4)
+    assert e.value.status == C.PA_ERR_UNSUPPORTED
 
 
 def test_run_argument_checks_before_any_launch(C):
