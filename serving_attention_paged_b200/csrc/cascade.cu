@@ -276,25 +276,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarSFree + s));
 
+      // Raw scores; the scale is folded into the exponent argument below.
       const int valid = min(kKeys, k1 - (k0 + kt * kKeys));
+      if (valid < kKeys) {  // ragged last tile of the chunk (uniform branch)
+#pragma unroll
+        for (int c = 0; c < kKeys; ++c)
+          if (c >= valid) x[c] = -INFINITY;
+      }
       float tm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
-        x[c] = c < valid ? x[c] * a.score_scale : -INFINITY;
-        tm4[c & 3] = fmaxf(tm4[c & 3], x[c]);
-      }
-      const float tmax = fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3]));
+      for (int c = 0; c < kKeys; ++c) tm4[c & 3] = fmaxf(tm4[c & 3], x[c]);
+      const float tmax = fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3])) * a.score_scale;
       const bool moved = tmax > m + kSlack;
       const float mnew = moved ? tmax : m;
       const float alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
-      // P = 2^(s - m), rounded to the input type (l sums exactly what the MMA
-      // sees), computed before waiting on the tensor core.
+      // P = 2^(s * scale - m), rounded to the input type (l sums exactly what
+      // the MMA sees), computed before waiting on the tensor core.
+      const float nm = -mnew;
       uint32_t w[kKeys / 2];
       float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < kKeys / 2; ++e) {
+        const float p0 = fast_exp2(fmaf(x[2 * e], a.score_scale, nm));
+        const float p1 = fast_exp2(fmaf(x[2 * e + 1], a.score_scale, nm));
         float r0, r1;
-        w[e] = pack2(Tag{}, fast_exp2(x[2 * e] - mnew), fast_exp2(x[2 * e + 1] - mnew), r0, r1);
+        w[e] = pack2(Tag{}, p0, p1, r0, r1);
         ps4[e & 3] += r0 + r1;
       }
       const float psum = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
