@@ -189,6 +189,24 @@ pa_status pa_merge_state(const void* o_a, const float* lse_a, const void* o_b,
                          const float* lse_b, void* o, float* lse, int64_t rows,
                          int32_t head_dim, pa_dtype dtype, void* stream);
 
+/* pa_run without a caller-provided workspace, for callers that cannot
+ * allocate device memory (an engine whose pool already holds all free GPU
+ * memory, a host program that does not own the process's allocator, a path
+ * that must not take cudaMalloc's implicit synchronisation).  The source
+ * pages have no counterpart: this is a convenience of this library.
+ * The workspace is a fixed 8 MiB array inside libpagedattn.so on every GPU
+ * that loads it, held until the process exits; a plan needing more
+ * (pa_plan_workspace_bytes > 8 MiB) is rejected with
+ * PA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued, and cascade plans
+ * with PA_ERR_INVALID_ARG.  Nothing is allocated: each call uploads the plan
+ * into the array (as pa_plan_upload) and runs it (as pa_run).  The first call
+ * on a device looks the array up (cudaGetSymbolAddress), so make it before any
+ * stream capture.  All calls share the array: calls that overlap on the GPU
+ * (different streams or threads) race. */
+pa_status pa_run_static_workspace(pa_plan_t plan, const void* q, const void* k_pool,
+                                  const void* v_pool, const int32_t* d_kv_indices, void* o,
+                                  float* lse, void* stream);
+
 /* Synchronously read and clear the device status words of a workspace.
  * Returns PA_ERR_DEVICE_TIMEOUT if a kernel abandoned one of its bounded
  * pipeline waits (its outputs are then undefined), else PA_ERR_DEVICE_CHECK

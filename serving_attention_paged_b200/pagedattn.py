@@ -58,6 +58,7 @@ _SIGS = {
     "pa_run": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "pa_cascade_run": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "pa_merge_state": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp],
+    "pa_run_static_workspace": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "pa_plan_check": [_vp, _vp, _P(_i64), _vp],
     "pa_default_schedule": [_i32, _i32, _i32, _i32, _P(_i32), _P(_i32)],
 }
@@ -216,6 +217,14 @@ def pa_cascade_run(plan: Plan, q, k_pool, v_pool, prefix_indices, kv_indices, o,
                               _ptr(prefix_indices), _ptr(kv_indices), _ptr(o), _ptr(lse),
                               _ptr(workspace), workspace_bytes, _stream(stream)),
            "pa_cascade_run")
+
+
+def pa_run_static_workspace(plan: Plan, q, k_pool, v_pool, kv_indices, o, lse, stream=None):
+    """pa_run with the library's own fixed 8 MiB device workspace, for callers
+    that cannot allocate device memory (see include/pagedattn.h)."""
+    _check(lib.pa_run_static_workspace(plan.handle, _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                       _ptr(kv_indices), _ptr(o), _ptr(lse), _stream(stream)),
+           "pa_run_static_workspace")
 
 
 def pa_merge_state(o_a, lse_a, o_b, lse_b, o, lse, rows: int, head_dim: int, dtype,
