@@ -58,6 +58,9 @@ def parse_args():
                     help="split-KV minimum chunk (tokens); 0 = library default")
     ap.add_argument("--ctas-per-sm", type=int, default=0,
                     help="CTA budget per SM for the plan; 0 = occupancy of the kernel")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "cuda_cores"],
+                    help="decode kernel: auto (tensor cores for GQA groups 4 and 8) or "
+                         "cuda_cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -283,7 +286,9 @@ def run_ours(args):
                      num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
                      sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
                      device=dev_t, min_chunk_tokens=args.min_chunk_tokens,
-                     ctas_per_sm=args.ctas_per_sm or None)
+                     ctas_per_sm=args.ctas_per_sm or None,
+                     flags=C.PA_FLAG_CUDA_CORES if args.kernel == "cuda_cores" else 0)
+    tensor_cores = C.pa_plan_uses_tensor_cores(pd.plan)
     setup_us = (time.perf_counter() - t0) * 1e6
     reps = 20
     t0 = time.perf_counter()
@@ -345,7 +350,9 @@ def run_ours(args):
     value = aggregate_gbs(world, nbytes, ms * 1e-3)
     peak, peak_kind = measured_peak()
     achieved = nbytes / (ms * 1e-3) / 1e9  # one GPU's launch: the dominant (only) kernel
-    kernel_sources = ["serving_attention_paged_b200/csrc/decode.cu",
+    decode_src = "decode_tc.cu" if tensor_cores else "decode.cu"
+    decode_kernel = "paged_decode_tc_kernel" if tensor_cores else "paged_decode_kernel"
+    kernel_sources = ["serving_attention_paged_b200/csrc/" + decode_src,
                       "serving_attention_paged_b200/csrc/common.cuh"]
     if w.prefix_len:
         kernel_sources.append("serving_attention_paged_b200/csrc/cascade.cu")
@@ -410,8 +417,8 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic,
-                         "kernel": "paged_decode_kernel" if not w.prefix_len
-                         else "cascade step (prefix + suffix kernels)"},
+                         "kernel": decode_kernel if not w.prefix_len
+                         else f"cascade step (prefix kernel + {decode_kernel})"},
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": args.steps * launches_per_step,
             "plan_us": plan_us, "setup_us": setup_us,

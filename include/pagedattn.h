@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 1
+#define PA_ABI_VERSION 2
 
 typedef enum {
   PA_OK = 0,
@@ -76,6 +76,10 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 /* pa_merge_state only */ } p
 #define PA_FLAG_CHECK_INDICES 1u /* kernels bounds-check every page index against
                                     num_pages; a bad index is skipped (its tokens
                                     read as zero) and recorded for pa_plan_check */
+#define PA_FLAG_CUDA_CORES 2u    /* decode with the CUDA-core kernel even where the
+                                    tensor-core one exists (group 4 or 8, fp16/bf16);
+                                    the work list is the same, only the schedule
+                                    defaults differ (pa_default_schedule) */
 
 typedef struct {
   int32_t batch;            /* requests B >= 0 */
@@ -215,10 +219,17 @@ pa_status pa_run_static_workspace(pa_plan_t plan, const void* q, const void* k_p
  * (*bad_position = -1). */
 pa_status pa_plan_check(pa_plan_t plan, void* d_workspace, int64_t* bad_position, void* stream);
 
-/* Scheduling defaults for `device`: its SM count and how many decode CTAs
- * of this shape fit on one SM. */
+/* Scheduling defaults for `device`: its SM count and how many CTAs of the
+ * decode kernel that a problem with this shape, dtype and `flags` (PA_FLAG_*)
+ * runs fit on one SM.  The tensor-core kernel (group 4 or 8, fp16/bf16,
+ * without PA_FLAG_CUDA_CORES) holds one CTA per SM. */
 pa_status pa_default_schedule(int32_t device, int32_t num_qo_heads, int32_t num_kv_heads,
-                              pa_dtype dtype, int32_t* num_sms, int32_t* ctas_per_sm);
+                              pa_dtype dtype, uint32_t flags, int32_t* num_sms,
+                              int32_t* ctas_per_sm);
+
+/* 1 if the plan's decode level runs on the tensor-core kernel, 0 if on the
+ * CUDA-core kernel, -1 for a null plan. */
+int32_t pa_plan_uses_tensor_cores(pa_plan_t plan);
 
 void pa_plan_destroy(pa_plan_t plan);
 const char* pa_status_string(pa_status status);

@@ -13,6 +13,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 pa_status from_cuda(int e) { return e == 0 ? PA_OK : PA_ERR_CUDA; }
 
+int launch_decode_any(const pa_plan_s& plan, const pa::RunPointers& p, void* stream) {
+  return pa::decode_uses_tensor_cores(plan.prob) ? pa::launch_decode_tc(plan, p, stream)
+                                                 : pa::launch_decode(plan, p, stream);
+}
+
 pa_status check_run_args(pa_plan_t plan, const void* q, const void* k_pool, const void* v_pool,
                          const int32_t* kv_indices, void* o, void* ws, size_t ws_bytes) {
   if (!plan || !ws) return PA_ERR_INVALID_ARG;
@@ -52,7 +57,8 @@ pa_status pa_plan_upload(pa_plan_t plan, void* d_workspace, size_t workspace_byt
                         plan->merge_indptr.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && p.batch > 0)
     e = cudaMemsetAsync(ws + plan->ws.counters, 0,
-                        size_t(p.batch) * p.num_kv_heads * sizeof(int32_t), s);
+                        size_t(p.batch) * p.num_kv_heads * pa::kCounterSlots * sizeof(int32_t),
+                        s);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws + plan->ws.error, 0xff, sizeof(uint64_t), s);
   if (e == cudaSuccess)
     e = cudaMemsetAsync(ws + plan->ws.error + sizeof(uint64_t), 0, sizeof(uint64_t), s);
@@ -68,7 +74,7 @@ pa_status pa_run(pa_plan_t plan, const void* q, const void* k_pool, const void* 
   if (plan->cascade) return PA_ERR_INVALID_ARG;  // cascade plans run through pa_cascade_run
   pa::RunPointers p{q, k_pool, v_pool, d_kv_indices, nullptr, o, lse,
                     static_cast<uint8_t*>(d_workspace)};
-  return from_cuda(pa::launch_decode(*plan, p, stream));
+  return from_cuda(launch_decode_any(*plan, p, stream));
 }
 
 pa_status pa_cascade_run(pa_plan_t plan, const void* q, const void* k_pool,
@@ -87,7 +93,7 @@ pa_status pa_cascade_run(pa_plan_t plan, const void* q, const void* k_pool,
     if (e == int(cudaErrorNotSupported)) return PA_ERR_UNSUPPORTED;
     if (e) return PA_ERR_CUDA;
   }
-  return from_cuda(pa::launch_decode(*plan, p, stream));
+  return from_cuda(launch_decode_any(*plan, p, stream));
 }
 
 pa_status pa_merge_state(const void* o_a, const float* lse_a, const void* o_b,
@@ -127,7 +133,8 @@ pa_status pa_plan_check(pa_plan_t plan, void* d_workspace, int64_t* bad_position
 }
 
 pa_status pa_default_schedule(int32_t device, int32_t num_qo_heads, int32_t num_kv_heads,
-                              pa_dtype dtype, int32_t* num_sms, int32_t* ctas_per_sm) {
+                              pa_dtype dtype, uint32_t flags, int32_t* num_sms,
+                              int32_t* ctas_per_sm) {
   if (!num_sms || !ctas_per_sm || num_kv_heads <= 0 || num_qo_heads % num_kv_heads)
     return PA_ERR_INVALID_ARG;
   const int32_t group = num_qo_heads / num_kv_heads;
@@ -138,7 +145,14 @@ pa_status pa_default_schedule(int32_t device, int32_t num_qo_heads, int32_t num_
   int sms = 0;
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
   int32_t k = 0;
-  if (e == cudaSuccess) e = cudaError_t(pa::decode_ctas_per_sm(group, dtype, &k));
+  pa_problem shape{};
+  shape.num_qo_heads = num_qo_heads;
+  shape.num_kv_heads = num_kv_heads;
+  shape.dtype = dtype;
+  shape.flags = flags;
+  if (e == cudaSuccess)
+    e = cudaError_t(pa::decode_uses_tensor_cores(shape) ? pa::decode_tc_ctas_per_sm(group, dtype, &k)
+                                                        : pa::decode_ctas_per_sm(group, dtype, &k));
   cudaSetDevice(prev);
   if (e != cudaSuccess) return PA_ERR_CUDA;
   *num_sms = sms;

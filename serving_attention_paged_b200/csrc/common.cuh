@@ -108,6 +108,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking probe of the same condition, for a thread that polls several
+// barriers in turn (try_wait may suspend the thread for a while).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Every pipeline wait is bounded: a wait that never completes means a broken
 // launch, and the kernel then records a timeout instead of hanging the GPU.
 constexpr uint32_t kSpinLimit = 1u << 22;
@@ -181,5 +193,53 @@ struct MergeAcc {
     return m == -INFINITY ? -INFINITY : m + fast_log2(l);
   }
 };
+
+// Adds, for the G q heads of one kv head at head element d, the partial
+// states in slots [s0, s1) of partial_o [slot, G, D] / partial_lse [slot, G]
+// (base 2) to acc.  Every load of a batch of slots is issued before any of
+// them is used: the merge then costs a few L2 round trips instead of one per
+// head and slot (the output stores in between would otherwise serialise
+// them, since the compiler cannot rule out aliasing).
+template <int G, int D>
+__device__ __forceinline__ void merge_partials(MergeAcc (&acc)[G], const float* partial_o,
+                                               const float* partial_lse, int s0, int s1, int d) {
+  constexpr int kBatch = G >= 8 ? 2 : 4;  // slots per batch of loads
+  for (int sl = s0; sl < s1; sl += kBatch) {
+    float o[kBatch][G], l[kBatch][G];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const bool in = sl + j < s1;
+      const int64_t s = in ? sl + j : s0;  // past the end: a valid slot, ignored below
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        o[j][hh] = __ldcg(partial_o + (s * G + hh) * D + d);
+        l[j][hh] = in ? __ldcg(partial_lse + s * G + hh) : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) acc[hh].add(o[j][hh], l[j][hh]);
+  }
+}
+
+// Adds the cascade prefix states of rows row0 .. row0 + G - 1 at head
+// element d: prefix_o [chunks, B * Hq, D], prefix_lse [chunks, B * Hq].
+template <int G, int D>
+__device__ __forceinline__ void merge_prefix(MergeAcc (&acc)[G], const float* prefix_o,
+                                             const float* prefix_lse, int chunks,
+                                             int64_t rows_per_chunk, int64_t row0, int d) {
+  for (int c = 0; c < chunks; ++c) {
+    float o[G], l[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      const int64_t r = c * rows_per_chunk + row0 + hh;
+      o[hh] = prefix_o[r * D + d];
+      l[hh] = prefix_lse[r];
+    }
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) acc[hh].add(o[hh], l[hh]);
+  }
+}
 
 }  // namespace pa

@@ -414,19 +414,18 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
   }
 
   const int64_t Bstride = int64_t(a.batch) * Hq;
+  const int64_t row0 = int64_t(b) * Hq + hq0;
   if (it.partial_slot < 0) {
+    if (a.prefix_chunks == 0) {
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      const int64_t row = int64_t(b) * Hq + hq0 + hh;
-      if (a.prefix_chunks == 0) {
-        write_final<Tag>(a, row, d, res[hh], lse2[hh]);
-      } else {
-        MergeAcc acc;
-        acc.add(res[hh], lse2[hh]);
-        for (int c = 0; c < a.prefix_chunks; ++c)
-          acc.add(a.prefix_o[(c * Bstride + row) * D + d], a.prefix_lse[c * Bstride + row]);
-        write_final<Tag>(a, row, d, acc.out(), acc.lse2());
-      }
+      for (int hh = 0; hh < G; ++hh) write_final<Tag>(a, row0 + hh, d, res[hh], lse2[hh]);
+    } else {
+      MergeAcc acc[G];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) acc[hh].add(res[hh], lse2[hh]);
+      merge_prefix<G, D>(acc, a.prefix_o, a.prefix_lse, a.prefix_chunks, Bstride, row0, d);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) write_final<Tag>(a, row0 + hh, d, acc[hh].out(), acc[hh].lse2());
     }
     return;
   }
@@ -443,7 +442,7 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
   const int64_t seg = int64_t(b) * a.num_kv_heads + h;
   if (tid == 0) {
     const int nchunks = a.merge_indptr[seg + 1] - a.merge_indptr[seg];
-    int32_t* ctr = a.counters + seg;
+    int32_t* ctr = a.counters + seg * kCounterSlots;
     const int prev = atomicAdd(ctr, 1);
     s_is_last = prev == nchunks - 1;
     if (s_is_last) *ctr = 0;  // every other chunk has arrived: safe to reset
@@ -452,17 +451,11 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
   if (!s_is_last) return;
   __threadfence();
   const int s0 = a.merge_indptr[seg], s1 = a.merge_indptr[seg + 1];
+  MergeAcc acc[G];
+  merge_partials<G, D>(acc, a.partial_o, a.partial_lse, s0, s1, d);
+  merge_prefix<G, D>(acc, a.prefix_o, a.prefix_lse, a.prefix_chunks, Bstride, row0, d);
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    MergeAcc acc;
-    for (int sl = s0; sl < s1; ++sl)
-      acc.add(__ldcg(a.partial_o + (int64_t(sl) * G + hh) * D + d),
-              __ldcg(a.partial_lse + int64_t(sl) * G + hh));
-    const int64_t row = int64_t(b) * Hq + hq0 + hh;
-    for (int c = 0; c < a.prefix_chunks; ++c)
-      acc.add(a.prefix_o[(c * Bstride + row) * D + d], a.prefix_lse[c * Bstride + row]);
-    write_final<Tag>(a, row, d, acc.out(), acc.lse2());
-  }
+  for (int hh = 0; hh < G; ++hh) write_final<Tag>(a, row0 + hh, d, acc[hh].out(), acc[hh].lse2());
 }
 
 // One CTA per quota: it runs its pieces in order (usually one or two).

@@ -1,0 +1,774 @@
+// Batched paged decode with head-query fusion on the sm_100a tensor cores.
+//
+// FlashInfer README, core feature 3 ("Head-Query fusion for accelerating
+// Grouped-Query Attention") and core feature 1 (tensor-core templates for
+// paged KV).  For G = Hq / Hkv >= 4 the G query heads of one kv head turn each
+// 128-token tile into a small dense contraction: S^T = K Q^T (M = 128 tokens,
+// N = 16 with the G heads padded, K = 128) and O^T += V^T P^T (M = 128 head
+// elements, N = 16, K = 128 tokens).  On CUDA cores the same work is issue
+// bound (the FMAs alone take about as long as HBM takes to deliver the
+// bytes); here the tensor core does it and the kernel is left with the data
+// movement.
+//
+// CTA = one group of pieces of the plan (the same work list as the CUDA-core
+// kernel), 416 threads, one CTA per SM:
+//   warps 4-7 (loaders): each 128-token tile of K and V (32 KB each) is copied
+//     with 16-byte cp.async, a half warp per 256-byte row (coalesced), into the
+//     128-byte-swizzled layout the MMA reads; rows past the piece are
+//     zero-filled.  A 3-stage ring: each loader thread hands its copies of a
+//     tile to the stage's mbarrier (cp.async.mbarrier.arrive.noinc), which
+//     completes once all of them have landed, so the loaders block only on
+//     free stages.  Page indices are read per row, so every page size (1
+//     included) works.
+//   warp 8 (MMA): one thread issues S^T(t) into one of two TMEM buffers and
+//     O^T(t) into one of two per-piece accumulators, whichever is ready.
+//   warps 0-3 (softmax): thread i owns token i of the tile (TMEM lane i):
+//     reads its G scores, agrees with the other warps on the tile maximum per
+//     head (lazy running max: the reference moves only when a score beats it
+//     by more than 2^8, and then O^T is rescaled in TMEM), writes P^T in the
+//     input type, and at the end of a piece hands its maxima and row sums to
+//     the epilogue warps and goes on with the next piece.
+//   warps 9-12 (epilogue): load Q^T, and per piece read O^T from TMEM
+//     (thread = head element), normalise it and run the output / partial /
+//     last-arriver merge (each warp merges its own 32 head elements), off the
+//     softmax warps' critical path.
+//     fp16 P keeps 11 significant bits, as in the CUDA-core kernel.  bf16
+//     keeps only 8, which on short rows moves o by ~2^-9 |v|; so a bf16 P is
+//     split into hi = bf16(p) and lo = bf16(p - hi), stored in the padding
+//     rows G..2G-1 of the N = 16 operand: the same single MMA then yields
+//     V^T hi and V^T lo in separate columns, which the epilogue adds.
+// Q^T, S^T, P^T and O^T are double buffered so a CTA's next piece starts while
+// the previous one finishes.  The warps meet only on mbarriers; every wait is
+// bounded, and every parity wait targets a barrier whose previous phase the
+// waiting thread has observed.
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "pa_internal.h"
+#include "tcgen05.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int D = kHeadDim;
+constexpr int kTok = 128;                    // tokens per tile (MMA M of S^T)
+constexpr int kN = 16;                       // padded heads (MMA N)
+constexpr int kStages = 3;
+constexpr int kHalfKV = kTok * 128;          // 128 token rows x 64 elements: 16 KB
+constexpr int kTileKV = 2 * kHalfKV;         // K or V of a tile: 32 KB
+constexpr int kStageBytes = 2 * kTileKV;     // K then V
+constexpr int kHalfQ = kN * 128;             // 16 head rows x 64 elements: 2 KB
+constexpr int kQBytes = 2 * kHalfQ;          // Q^T: 16 rows x 128 elements
+constexpr int kPHalf = kN * 128;             // 16 head rows x 64 tokens: 2 KB
+constexpr int kPBytes = 2 * kPHalf;          // P^T: 16 rows x 128 tokens
+constexpr int kOffRing = 0;
+constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+constexpr int kOffP = kOffQ + 2 * kQBytes;
+constexpr int kOffX = kOffP + 2 * kPBytes;     // tile maxima [2][4 warps][16]
+constexpr int kOffL = kOffX + 2 * 4 * kN * 4;  // row sums    [2][4 warps][16]
+constexpr int kOffM = kOffL + 2 * 4 * kN * 4;  // a piece's final maxima [2][16]
+constexpr int kOffBar = kOffM + 2 * kN * 4;
+
+// mbarriers: a K/V ring of full / empty pairs, then double-buffered pairs.
+constexpr int kBarFull = 0, kBarEmpty = kStages;
+constexpr int kBarS = 2 * kStages;      // S^T(t) written              (MMA commit)
+constexpr int kBarSFree = kBarS + 2;    // S^T(t) read                 (4 softmax warps)
+constexpr int kBarPReady = kBarS + 4;   // P^T(t) written, O^T rescaled (4 softmax warps)
+constexpr int kBarPFree = kBarS + 6;    // PV(t) done                  (MMA commit)
+constexpr int kBarQReady = kBarS + 8;   // Q^T of a piece written      (4 epilogue warps)
+constexpr int kBarODone = kBarS + 10;   // last PV of a piece done     (MMA commit)
+constexpr int kBarOFree = kBarS + 12;   // O^T of a piece read         (4 epilogue warps)
+constexpr int kBarXReady = kBarS + 14;  // tile maxima written         (4 softmax warps)
+constexpr int kBarLReady = kBarS + 16;  // piece maxima, row sums written (4 softmax warps)
+constexpr int kBarLFree = kBarS + 18;   // ... and read                (4 epilogue warps)
+constexpr int kNumBars = kBarS + 20;
+
+constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;  // + alignment slack
+constexpr int kThreads = 13 * 32;
+constexpr uint32_t kTmemCols = 64;  // S0, S1, O0, O1: 16 columns each
+constexpr float kSlack = 8.f;       // lazy max: rescale only past 2^8
+
+static_assert(kSmemBytes <= 232448, "shared memory");
+static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "128-byte swizzle atoms need 1 KB alignment");
+
+struct TcArgs {
+  const uint16_t* q;
+  const uint16_t* k_pool;
+  const uint16_t* v_pool;
+  const int32_t* kv_indices;
+  const pa_work_item* items;
+  const int32_t* cta_indptr;
+  const int32_t* merge_indptr;
+  int32_t* counters;  // [B * Hkv * kCounterSlots]
+  float* partial_o;
+  float* partial_lse;
+  const float* prefix_o;
+  const float* prefix_lse;
+  unsigned long long* error_pos;  // [0] first bad page position, [1] timeout flag
+  uint16_t* o;
+  float* lse;
+  int64_t num_pages;
+  int32_t batch, num_qo_heads, num_kv_heads, log2_page, prefix_chunks;
+  float score_scale;
+};
+
+template <typename Tag> struct Fmt;
+template <> struct Fmt<F16> { static constexpr int v = 0; };
+template <> struct Fmt<BF16> { static constexpr int v = 1; };
+
+__device__ __forceinline__ uint16_t round16(F16, float x, float& r) {
+  const __half h = __float2half_rn(x);
+  r = __half2float(h);
+  return __half_as_ushort(h);
+}
+__device__ __forceinline__ uint16_t round16(BF16, float x, float& r) {
+  const uint16_t u = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+  r = __uint_as_float(uint32_t(u) << 16);
+  return u;
+}
+
+// N consecutive fp32 columns of this thread's TMEM lane.
+template <int N> __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]);
+template <> __device__ __forceinline__ void tmem_ld<4>(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+template <> __device__ __forceinline__ void tmem_ld<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+template <> __device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+template <int N> __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]);
+template <> __device__ __forceinline__ void tmem_st<4>(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+template <> __device__ __forceinline__ void tmem_st<8>(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+template <> __device__ __forceinline__ void tmem_st<16>(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+// Byte offset of 16-byte chunk c (0..15) of row r in a 128-byte-swizzled
+// tile stored as two 64-element halves of `half_bytes` each.
+__device__ __forceinline__ uint32_t sw_chunk(int r, int c, int half_bytes) {
+  return uint32_t((c >> 3) * half_bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <typename Tag>
+__device__ __forceinline__ void write_out(const TcArgs& a, int64_t row, int d, float o, float lse2) {
+  a.o[row * D + d] = from_float(Tag{}, o);
+  if (d == 0 && a.lse) a.lse[row] = lse2 == -INFINITY ? -INFINITY : lse2 * kLn2;
+}
+
+__device__ __forceinline__ void flag_timeout(const TcArgs& a) { atomicOr(a.error_pos + 1, 1ull); }
+
+__device__ __forceinline__ int next_nonempty(const pa_work_item* items, int pc, int p1) {
+  while (pc < p1 && items[pc].token_end == items[pc].token_begin) ++pc;
+  return pc;
+}
+
+template <typename Tag, int G, bool kCheck>
+__global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcArgs a) {
+  // bf16: P^T rows [0, G) hold hi, rows [G, 2G) lo; O^T columns likewise
+  constexpr bool kSplit = Fmt<Tag>::v == 1;
+  constexpr int kCols = kSplit ? 2 * G : G;
+  static_assert(kCols <= kN, "hi and lo rows must fit the padded MMA N");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) { return sb + kOffBar + 8 * i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p0 = a.cta_indptr[blockIdx.x], p1 = a.cta_indptr[blockIdx.x + 1];
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarFull + s), 128);
+      mbar_init(bar(kBarEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(kBarS + b), 1);
+      mbar_init(bar(kBarSFree + b), 4);
+      mbar_init(bar(kBarPReady + b), 4);
+      mbar_init(bar(kBarPFree + b), 1);
+      mbar_init(bar(kBarQReady + b), 4);
+      mbar_init(bar(kBarODone + b), 1);
+      mbar_init(bar(kBarOFree + b), 4);
+      mbar_init(bar(kBarXReady + b), 4);
+      mbar_init(bar(kBarLReady + b), 4);
+      mbar_init(bar(kBarLFree + b), 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp >= 4 && warp < 8) {
+    // ------------------------------ loaders ------------------------------
+    const int lw = warp - 4;
+    const int lp = a.log2_page;
+    const uint32_t pmask = (1u << lp) - 1u;
+    const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * D * 2;
+    const int c = lane & 15;  // 16-byte chunk of a 256-byte row
+    // Page of this lane's row (32 * lw + lane) of tile tt of a piece; -1 past
+    // the piece or rejected by the bounds check.
+    auto page_of = [&](const pa_work_item& w, int wlen, int wtt) -> int {
+      const int mypos = wtt * kTok + 32 * lw + lane;
+      if (mypos >= wlen) return -1;
+      const int idx = (w.token_begin + mypos) >> lp;
+      int pg = __ldg(a.kv_indices + w.page_begin + idx);
+      if (kCheck && (pg < 0 || int64_t(pg) >= a.num_pages)) {
+        atomicMin(a.error_pos, (unsigned long long)(w.page_begin + idx));
+        pg = -1;
+      }
+      return pg;
+    };
+    // One walk over the tiles of the CTA's non-empty pieces.  The next tile's
+    // page indices are fetched before waiting for its stage, so the lookup
+    // overlaps the wait.
+    int pi = next_nonempty(a.items, p0, p1);
+    pa_work_item it{};
+    int len = 0, tt = 0;
+    if (pi < p1) {
+      it = a.items[pi];
+      len = it.token_end - it.token_begin;
+    }
+    int pg = pi < p1 ? page_of(it, len, 0) : -1;
+    int t = 0;
+    bool ok = true;
+    while (pi < p1) {
+      const int s = t % kStages;
+      if (t >= kStages && !mbar_wait(bar(kBarEmpty + s), ((t / kStages) - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint64_t kb = reinterpret_cast<uint64_t>(a.k_pool + int64_t(it.kv_head) * D) + c * 16;
+      const uint64_t vb = reinterpret_cast<uint64_t>(a.v_pool + int64_t(it.kv_head) * D) + c * 16;
+      const uint32_t kdst = sb + kOffRing + s * kStageBytes;
+      const uint32_t vdst = kdst + kTileKV;
+#pragma unroll 4
+      for (int k = 0; k < 16; ++k) {
+        const int rr = 2 * k + (lane >> 4);  // row within the warp's 32
+        const int r = 32 * lw + rr;           // row within the tile
+        const int rpg = __shfl_sync(0xffffffffu, pg, rr);
+        const uint32_t pos = uint32_t(it.token_begin + tt * kTok + r);
+        const uint32_t row = rpg >= 0 ? ((uint32_t(rpg) << lp) | (pos & pmask)) : 0u;
+        const uint32_t nbytes = rpg >= 0 ? 16u : 0u;  // 0: zero-fill, nothing read
+        uint64_t ka, va;
+        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(ka) : "r"(row), "r"(pool_row_bytes), "l"(kb));
+        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(va) : "r"(row), "r"(pool_row_bytes), "l"(vb));
+        const uint32_t off = sw_chunk(r, c, kHalfKV);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(kdst + off),
+                     "l"(ka), "r"(nbytes)
+                     : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(vdst + off),
+                     "l"(va), "r"(nbytes)
+                     : "memory");
+      }
+      // the stage's barrier counts this thread once all its copies above land
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(
+                       bar(kBarFull + s))
+                   : "memory");
+      ++t;
+      if (++tt * kTok >= len) {
+        tt = 0;
+        pi = next_nonempty(a.items, pi + 1, p1);
+        if (pi < p1) {
+          it = a.items[pi];
+          len = it.token_end - it.token_begin;
+        }
+      }
+      if (pi < p1) pg = page_of(it, len, tt);
+    }
+    if (!ok) {
+      asm volatile("cp.async.wait_all;\n" ::: "memory");
+      if (lane == 0) flag_timeout(a);
+    }
+  } else if (warp == 8) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = tc::idesc_f16(Fmt<Tag>::v, 0, kTok, kN);
+      // O^T = V^T P^T: A = V^T (M = head elements, MN-major), B = P^T (K-major)
+      constexpr uint32_t kIdescO = tc::idesc_f16(Fmt<Tag>::v, 0, D, kN) | (1u << 15);
+      const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffRing, 16, 1024);
+      const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffRing + kTileKV, kHalfKV, 1024);
+      const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
+      const uint64_t dp0 = tc::smem_desc_sw128(sb + kOffP, 16, 1024);
+      // S^T(ts) and PV(tv) walk the pieces in step with their counters
+      int s_piece = next_nonempty(a.items, p0, p1), s_tile = 0, s_np = 0;
+      int v_piece = s_piece, v_tile = 0, v_np = 0;
+      auto ntiles_of = [&](int pc) {
+        return (a.items[pc].token_end - a.items[pc].token_begin + kTok - 1) / kTok;
+      };
+      int s_ntiles = s_piece < p1 ? ntiles_of(s_piece) : 0;
+      int v_ntiles = s_ntiles;
+      int ts = 0, tv = 0;
+      uint32_t idle = 0;
+      bool ok = true;
+      while (v_piece < p1) {
+        bool progress = false;
+        if (s_piece < p1 &&
+            (ts < 2 || mbar_test_wait(bar(kBarSFree + (ts & 1)), ((ts - 2) >> 1) & 1)) &&
+            mbar_test_wait(bar(kBarFull + ts % kStages), (ts / kStages) & 1) &&
+            mbar_test_wait(bar(kBarQReady + (s_np & 1)), (s_np >> 1) & 1)) {
+          fence_proxy_async_smem();  // the loaders' cp.async writes, seen by the tensor core
+          tc::fence_after_sync();
+          const uint64_t kd = dk0 + uint64_t(((ts % kStages) * kStageBytes) >> 4);
+          const uint64_t qd = dq0 + uint64_t(((s_np & 1) * kQBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = ((kk >> 2) * kHalfKV + (kk & 3) * 32) >> 4;
+            const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
+            tc::mma_f16_ss(tmem + (ts & 1) * kN, kd + koff, qd + qoff, kIdescS, kk > 0);
+          }
+          tc::commit(bar(kBarS + (ts & 1)));
+          ++ts;
+          if (++s_tile == s_ntiles) {
+            s_tile = 0;
+            ++s_np;
+            s_piece = next_nonempty(a.items, s_piece + 1, p1);
+            s_ntiles = s_piece < p1 ? ntiles_of(s_piece) : 0;
+          }
+          progress = true;
+        }
+        if (tv < ts && mbar_test_wait(bar(kBarPReady + (tv & 1)), (tv >> 1) & 1) &&
+            (v_tile > 0 || v_np < 2 ||
+             mbar_test_wait(bar(kBarOFree + (v_np & 1)), ((v_np - 2) >> 1) & 1))) {
+          tc::fence_after_sync();
+          const uint64_t vd = dv0 + uint64_t(((tv % kStages) * kStageBytes) >> 4);
+          const uint64_t pd = dp0 + uint64_t(((tv & 1) * kPBytes) >> 4);
+          const uint32_t od = tmem + 2 * kN + (v_np & 1) * kN;
+#pragma unroll
+          for (int kk = 0; kk < kTok / 16; ++kk) {
+            const uint32_t voff = (kk * 16 * 128) >> 4;  // 16 token rows
+            const uint32_t poff = ((kk >> 2) * kPHalf + (kk & 3) * 32) >> 4;
+            tc::mma_f16_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::commit(bar(kBarPFree + (tv & 1)));
+          tc::commit(bar(kBarEmpty + tv % kStages));
+          ++tv;
+          if (++v_tile == v_ntiles) {
+            tc::commit(bar(kBarODone + (v_np & 1)));
+            v_tile = 0;
+            ++v_np;
+            v_piece = next_nonempty(a.items, v_piece + 1, p1);
+            v_ntiles = v_piece < p1 ? ntiles_of(v_piece) : 0;
+          }
+          progress = true;
+        }
+        idle = progress ? 0u : idle + 1u;
+        if (idle > kSpinLimit) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) flag_timeout(a);
+    }
+  } else if (warp < 4) {
+    // ------------------------------- softmax -------------------------------
+    const int i = threadIdx.x;  // token row of a tile (TMEM lane)
+    const uint32_t lane_addr = tmem + (uint32_t(warp * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(smem + kOffX);  // [2][4][kN]
+    float* xsum = reinterpret_cast<float*>(smem + kOffL);  // [2][4][kN]
+    float* xm_piece = reinterpret_cast<float*>(smem + kOffM);  // [2][kN]
+    // P^T rows past the used ones stay zero for the whole kernel
+    for (int e = i; e < 2 * kPBytes / 16; e += 128)
+      reinterpret_cast<uint4*>(smem + kOffP)[e] = make_uint4(0, 0, 0, 0);
+    int t = 0, np = 0;
+    bool ok = true;
+    for (int pi = p0; ok && pi < p1; ++pi) {
+      const pa_work_item it = a.items[pi];
+      const int len = it.token_end - it.token_begin;
+      const int ntiles = (len + kTok - 1) / kTok;
+      if (ntiles == 0) continue;  // the epilogue warps write its (0, -inf)
+      float m[G], lsum[G];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        m[hh] = -INFINITY;
+        lsum[hh] = 0.f;
+      }
+      for (int tt = 0; tt < ntiles; ++tt, ++t) {
+        const int sbuf = t & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarS + sbuf), (t >> 1) & 1));
+        if (!ok) break;
+        tc::fence_after_sync();
+        float sv[G];
+        {
+          uint32_t r[G];
+          tmem_ld<G>(lane_addr + sbuf * kN, r);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) sv[hh] = __uint_as_float(r[hh]);
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarSFree + sbuf));
+        const bool valid = tt * kTok + i < len;
+        // tile maximum per head over the 128 tokens: shuffles, then the 4 warps
+        float* xm = xmax + sbuf * 4 * kN;
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          float v = valid ? sv[hh] : -INFINITY;
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+          if (lane == 0) xm[warp * kN + hh] = v;
+        }
+        if (lane == 0) mbar_arrive(bar(kBarXReady + sbuf));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarXReady + sbuf), (t >> 1) & 1));
+        if (!ok) break;
+        bool moved = false;
+        float alpha[G], mn[G];
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float tmax =
+              fmaxf(fmaxf(xm[hh], xm[kN + hh]), fmaxf(xm[2 * kN + hh], xm[3 * kN + hh])) *
+              a.score_scale;
+          alpha[hh] = 1.f;
+          mn[hh] = m[hh];
+          if (tmax > m[hh] + kSlack) {
+            mn[hh] = tmax;
+            alpha[hh] = fast_exp2(m[hh] - tmax);  // m = -inf -> 0
+            moved = true;
+          }
+        }
+        // the reference moved: rescale this piece's O^T (lane = head element)
+        // once PV(t - 1) has landed; the first tile's PV overwrites O^T
+        if (moved && tt > 0) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(bar(kBarPFree + ((t - 1) & 1)), ((t - 1) >> 1) & 1));
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t oaddr = lane_addr + 2 * kN + (np & 1) * kN;
+          uint32_t r[kCols];
+          tmem_ld<kCols>(oaddr, r);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int cc = 0; cc < kCols; ++cc)
+            r[cc] = __float_as_uint(__uint_as_float(r[cc]) * alpha[cc % G]);
+          tmem_st<kCols>(oaddr, r);
+          tc::tmem_wait_st();
+        }
+        // P^T(t) for this thread's token; the row sums add the rounded values
+        if (t >= 2) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarPFree + sbuf), ((t - 2) >> 1) & 1));
+          if (!ok) break;
+        }
+        uint8_t* pt = smem + kOffP + sbuf * kPBytes + (i >> 6) * kPHalf + (i & 7) * 2;
+        const int pc = (i >> 3) & 7;  // 16-byte chunk of the token within its 128-byte row
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float p = valid ? fast_exp2(fmaf(sv[hh], a.score_scale, -mn[hh])) : 0.f;
+          float pr;
+          const uint16_t bits = round16(Tag{}, p, pr);
+          *reinterpret_cast<uint16_t*>(pt + hh * 128 + ((pc ^ (hh & 7)) << 4)) = bits;
+          if constexpr (kSplit) {  // p - hi is exact in fp32
+            float lo;
+            const uint16_t lbits = round16(Tag{}, p - pr, lo);
+            *reinterpret_cast<uint16_t*>(pt + (G + hh) * 128 + ((pc ^ ((G + hh) & 7)) << 4)) = lbits;
+            pr += lo;
+          }
+          lsum[hh] = fmaf(lsum[hh], alpha[hh], pr);
+          m[hh] = mn[hh];
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarPReady + sbuf));
+      }
+      if (!ok) break;
+      // hand the piece's maxima and row sums to the epilogue warps, once they
+      // have read those of the piece two back from the same buffer
+      if (np >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarLFree + (np & 1)), ((np - 2) >> 1) & 1));
+        if (!ok) break;
+      }
+      float* xs = xsum + (np & 1) * 4 * kN;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        float v = lsum[hh];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) xs[warp * kN + hh] = v;
+        if (i == 0) xm_piece[(np & 1) * kN + hh] = m[hh];
+      }
+      if (lane == 0) mbar_arrive(bar(kBarLReady + (np & 1)));
+      ++np;
+    }
+    if (!ok && lane == 0) flag_timeout(a);
+  } else if (warp >= 9) {
+    // ------------------------------- epilogue -------------------------------
+    // Warp 9 + j reads TMEM lanes 32 (warp % 4) .. + 31: head elements d.
+    const int quarter = warp & 3;
+    const int d = 32 * quarter + lane;
+    const int j = (warp - 9) * 32 + lane;  // 0..127, for the Q^T copies
+    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
+    const float* xsum = reinterpret_cast<const float*>(smem + kOffL);
+    const float* xm_piece = reinterpret_cast<const float*>(smem + kOffM);
+    const int Hq = a.num_qo_heads;
+    const int64_t Bstride = int64_t(a.batch) * Hq;
+    // Q^T of a piece, 16 rows x 16 chunks of 16 bytes (rows past G zero):
+    // thread j fetches chunks j and j + 128 into registers, and later stores
+    // them into buffer np & 1 for the np-th non-empty piece.
+    auto fetch_q = [&](int pc, uint4 (&v)[2]) {
+      const pa_work_item w = a.items[pc];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = j + 128 * k, r = e >> 4, ch = e & 15;
+        v[k] = r < G ? __ldg(reinterpret_cast<const uint4*>(
+                           a.q + (int64_t(w.request) * Hq + w.kv_head * G + r) * D + ch * 8))
+                     : make_uint4(0, 0, 0, 0);
+      }
+    };
+    auto store_q = [&](const uint4 (&v)[2], int np) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = j + 128 * k;
+        *reinterpret_cast<uint4*>(smem + kOffQ + (np & 1) * kQBytes +
+                                  sw_chunk(e >> 4, e & 15, kHalfQ)) = v[k];
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarQReady + (np & 1)));
+    };
+    {
+      const int pc = next_nonempty(a.items, p0, p1);
+      if (pc < p1) {
+        uint4 v[2];
+        fetch_q(pc, v);
+        store_q(v, 0);
+        const int pc2 = next_nonempty(a.items, pc + 1, p1);
+        if (pc2 < p1) {
+          fetch_q(pc2, v);
+          store_q(v, 1);
+        }
+      }
+    }
+    int np = 0;
+    bool ok = true;
+    for (int pi = p0; pi < p1; ++pi) {
+      const pa_work_item it = a.items[pi];
+      const int b = it.request, h = it.kv_head;
+      const int ntiles = (it.token_end - it.token_begin + kTok - 1) / kTok;
+      float res[G], lse2[G];
+      if (ntiles > 0) {
+        // Q^T of the non-empty piece after next goes into this piece's buffer
+        // once this piece's MMAs are done
+        const int pn = next_nonempty(a.items, pi + 1, p1);
+        const int pnn = pn < p1 ? next_nonempty(a.items, pn + 1, p1) : p1;
+        uint4 qn[2];
+        if (pnn < p1) fetch_q(pnn, qn);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarLReady + (np & 1)), (np >> 1) & 1));
+        if (!ok) break;
+        const float* xs = xsum + (np & 1) * 4 * kN;
+        float l[G], m[G];
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          l[hh] = (xs[hh] + xs[kN + hh]) + (xs[2 * kN + hh] + xs[3 * kN + hh]);
+          m[hh] = xm_piece[(np & 1) * kN + hh];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarLFree + (np & 1)));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + (np & 1)), (np >> 1) & 1));
+        if (!ok) break;
+        tc::fence_after_sync();
+        uint32_t r[kCols];
+        tmem_ld<kCols>(lane_addr + 2 * kN + (np & 1) * kN, r);
+        tc::tmem_wait_ld();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarOFree + (np & 1)));
+        // every MMA reading this piece's Q^T buffer is done
+        if (pnn < p1) store_q(qn, np + 2);
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float acc = kSplit ? __uint_as_float(r[hh]) + __uint_as_float(r[(G + hh) % kCols])
+                                   : __uint_as_float(r[hh]);
+          res[hh] = acc / l[hh];
+          lse2[hh] = m[hh] + fast_log2(l[hh]);
+        }
+        ++np;
+      } else {
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          res[hh] = 0.f;
+          lse2[hh] = -INFINITY;
+        }
+      }
+
+      const int64_t row0 = int64_t(b) * Hq + h * G;
+      if (it.partial_slot < 0) {
+        if (a.prefix_chunks == 0) {
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) write_out<Tag>(a, row0 + hh, d, res[hh], lse2[hh]);
+        } else {
+          MergeAcc acc[G];
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) acc[hh].add(res[hh], lse2[hh]);
+          merge_prefix<G, D>(acc, a.prefix_o, a.prefix_lse, a.prefix_chunks, Bstride, row0, d);
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh)
+            write_out<Tag>(a, row0 + hh, d, acc[hh].out(), acc[hh].lse2());
+        }
+        continue;
+      }
+      // split segment: store this piece's state; the warp that arrives last on
+      // its counter merges its 32 head elements of the segment
+      const int64_t slot = it.partial_slot;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) a.partial_o[(slot * G + hh) * D + d] = res[hh];
+      if (lane < G) {  // every warp stores the same values, so each warp's merge sees them
+        float v = lse2[0];
+#pragma unroll
+        for (int hh = 1; hh < G; ++hh) v = lane == hh ? lse2[hh] : v;
+        a.partial_lse[slot * G + lane] = v;
+      }
+      __threadfence();
+      __syncwarp();
+      const int64_t seg = int64_t(b) * a.num_kv_heads + h;
+      int last = 0;
+      if (lane == 0) {
+        const int nchunks = a.merge_indptr[seg + 1] - a.merge_indptr[seg];
+        int32_t* ctr = a.counters + seg * kCounterSlots + quarter;
+        last = atomicAdd(ctr, 1) == nchunks - 1;
+        if (last) *ctr = 0;
+      }
+      if (!__shfl_sync(0xffffffffu, last, 0)) continue;
+      __threadfence();
+      const int s0 = a.merge_indptr[seg], s1 = a.merge_indptr[seg + 1];
+      MergeAcc acc[G];
+      merge_partials<G, D>(acc, a.partial_o, a.partial_lse, s0, s1, d);
+      merge_prefix<G, D>(acc, a.prefix_o, a.prefix_lse, a.prefix_chunks, Bstride, row0, d);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+        write_out<Tag>(a, row0 + hh, d, acc[hh].out(), acc[hh].lse2());
+    }
+    if (!ok && lane == 0) flag_timeout(a);
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+template <typename Tag, int G, bool kCheck>
+cudaError_t launch_tc_t(const TcArgs& a, int64_t n_cta, cudaStream_t stream) {
+  auto kern = paged_decode_tc_kernel<Tag, G, kCheck>;
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = uint64_t(1) << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  if (n_cta <= 0) return cudaSuccess;
+  kern<<<dim3(unsigned(n_cta)), kThreads, kSmemBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename Tag, bool kCheck>
+cudaError_t dispatch_tc(int group, const TcArgs& a, int64_t n, cudaStream_t s) {
+  switch (group) {
+    case 4: return launch_tc_t<Tag, 4, kCheck>(a, n, s);
+    case 8: return launch_tc_t<Tag, 8, kCheck>(a, n, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool decode_tc_supported(int32_t group, pa_dtype dtype) {
+  return (group == 4 || group == 8) && (dtype == PA_F16 || dtype == PA_BF16);
+}
+
+int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out) {
+  auto get = [&](auto kern) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, kSmemBytes);
+  };
+  const bool bf = dtype == PA_BF16;
+  if (group == 4)
+    return int(bf ? get(paged_decode_tc_kernel<BF16, 4, false>) : get(paged_decode_tc_kernel<F16, 4, false>));
+  if (group == 8)
+    return int(bf ? get(paged_decode_tc_kernel<BF16, 8, false>) : get(paged_decode_tc_kernel<F16, 8, false>));
+  return int(cudaErrorInvalidValue);
+}
+
+int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream) {
+  const pa_problem& pr = plan.prob;
+  TcArgs a{};
+  a.q = static_cast<const uint16_t*>(p.q);
+  a.k_pool = static_cast<const uint16_t*>(p.k_pool);
+  a.v_pool = static_cast<const uint16_t*>(p.v_pool);
+  a.kv_indices = p.kv_indices;
+  a.items = reinterpret_cast<const pa_work_item*>(p.ws + plan.ws.items);
+  a.cta_indptr = reinterpret_cast<const int32_t*>(p.ws + plan.ws.cta_indptr);
+  a.merge_indptr = reinterpret_cast<const int32_t*>(p.ws + plan.ws.merge_indptr);
+  a.counters = reinterpret_cast<int32_t*>(p.ws + plan.ws.counters);
+  a.partial_o = reinterpret_cast<float*>(p.ws + plan.ws.partial_o);
+  a.partial_lse = reinterpret_cast<float*>(p.ws + plan.ws.partial_lse);
+  a.prefix_o = reinterpret_cast<const float*>(p.ws + plan.ws.prefix_o);
+  a.prefix_lse = reinterpret_cast<const float*>(p.ws + plan.ws.prefix_lse);
+  a.error_pos = reinterpret_cast<unsigned long long*>(p.ws + plan.ws.error);
+  a.o = static_cast<uint16_t*>(p.o);
+  a.lse = p.lse;
+  a.num_pages = pr.num_pages;
+  a.batch = pr.batch;
+  a.num_qo_heads = pr.num_qo_heads;
+  a.num_kv_heads = pr.num_kv_heads;
+  a.log2_page = plan.log2_page;
+  a.prefix_chunks = plan.cascade ? plan.prefix_chunks : 0;
+  a.score_scale = pr.sm_scale * kLog2e;
+  const bool check = (pr.flags & PA_FLAG_CHECK_INDICES) != 0;
+  const int64_t n = int64_t(plan.cta_indptr.size()) - 1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (pr.dtype == PA_BF16)
+    e = check ? dispatch_tc<BF16, true>(plan.group, a, n, s)
+              : dispatch_tc<BF16, false>(plan.group, a, n, s);
+  else
+    e = check ? dispatch_tc<F16, true>(plan.group, a, n, s)
+              : dispatch_tc<F16, false>(plan.group, a, n, s);
+  return int(e);
+}
+
+}  // namespace pa

@@ -13,6 +13,9 @@ namespace pa {
 constexpr int kHeadDim = 128;
 constexpr int kDefaultMinChunkTokens = 256;
 constexpr size_t kAlign = 256;
+// Arrival counters per (request, kv head): the tensor-core decode kernel
+// merges split segments per epilogue warp (4), the CUDA-core kernel uses slot 0.
+constexpr int kCounterSlots = 4;
 
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 
@@ -20,7 +23,7 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 //   items        [n_items]             pa_work_item (pieces, grouped by CTA)
 //   cta_indptr   [n_cta + 1]           int32, pieces of CTA i
 //   merge_indptr [B * Hkv + 1]         int32, partial slots of segment (b, h)
-//   counters     [B * Hkv]             int32, zero between runs
+//   counters     [B * Hkv * kCounterSlots]  int32, zero between runs
 //   error        [2]                   uint64: first bad kv_indices position (~0 = none),
 //                                      then a timeout flag (0 = none)
 //   partial_o    [n_partials, G, D]    fp32, outputs of pieces of split segments
@@ -70,6 +73,15 @@ struct RunPointers {
 };
 
 int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream);
+int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream);
+bool decode_tc_supported(int32_t group, pa_dtype dtype);
+int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out);
+// The decode kernel a problem runs: tensor cores where built, unless the
+// caller asked for the CUDA-core kernel.
+inline bool decode_uses_tensor_cores(const pa_problem& p) {
+  return decode_tc_supported(p.num_qo_heads / p.num_kv_heads, p.dtype) &&
+         !(p.flags & PA_FLAG_CUDA_CORES);
+}
 int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* stream);
 int launch_merge_state(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
                        void* o, float* lse, int64_t rows, int32_t head_dim, pa_dtype dtype,

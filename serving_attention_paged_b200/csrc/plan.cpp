@@ -130,7 +130,7 @@ void layout_workspace(pa_plan_s* plan) {
   w.items = take(plan->items.size() * sizeof(pa_work_item));
   w.cta_indptr = take(plan->cta_indptr.size() * sizeof(int32_t));
   w.merge_indptr = take(plan->merge_indptr.size() * sizeof(int32_t));
-  w.counters = take(B * p.num_kv_heads * sizeof(int32_t));
+  w.counters = take(B * p.num_kv_heads * pa::kCounterSlots * sizeof(int32_t));
   w.error = take(2 * sizeof(uint64_t));  // first bad index, timeout flag
   const size_t G = plan->group;
   w.partial_o = take(size_t(plan->n_partials) * G * D * sizeof(float));
@@ -273,6 +273,10 @@ const char* pa_status_string(pa_status s) {
     case PA_ERR_DEVICE_TIMEOUT: return "a kernel abandoned a bounded wait";
   }
   return "unknown status";
+}
+
+int32_t pa_plan_uses_tensor_cores(pa_plan_t plan) {
+  return plan ? int32_t(pa::decode_uses_tensor_cores(plan->prob)) : -1;
 }
 
 int32_t pa_abi_version(void) { return PA_ABI_VERSION; }

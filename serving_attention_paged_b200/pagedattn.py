@@ -25,6 +25,7 @@ PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL = 0, 1
 PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_NO_MEMORY, PA_ERR_DEVICE_TIMEOUT = 4, 5, 6, 7
 PA_F16, PA_BF16, PA_F32 = 0, 1, 2
 PA_FLAG_CHECK_INDICES = 1
+PA_FLAG_CUDA_CORES = 2
 DTYPE_CODES = {"f16": PA_F16, "bf16": PA_BF16, "f32": PA_F32}
 
 
@@ -60,7 +61,7 @@ _SIGS = {
     "pa_merge_state": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp],
     "pa_run_static_workspace": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "pa_plan_check": [_vp, _vp, _P(_i64), _vp],
-    "pa_default_schedule": [_i32, _i32, _i32, _i32, _P(_i32), _P(_i32)],
+    "pa_default_schedule": [_i32, _i32, _i32, _i32, ctypes.c_uint32, _P(_i32), _P(_i32)],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name)
@@ -72,6 +73,8 @@ lib.pa_status_string.argtypes = [ctypes.c_int]
 lib.pa_status_string.restype = ctypes.c_char_p
 lib.pa_abi_version.argtypes = []
 lib.pa_abi_version.restype = ctypes.c_int32
+lib.pa_plan_uses_tensor_cores.argtypes = [_vp]
+lib.pa_plan_uses_tensor_cores.restype = ctypes.c_int32
 
 
 class PagedAttnError(RuntimeError):
@@ -114,10 +117,11 @@ class Plan:
 
     def __init__(self, handle: int):
         self.handle = handle
+        self._destroy = lib.pa_plan_destroy  # still reachable during interpreter shutdown
 
     def __del__(self):
         if getattr(self, "handle", None):
-            lib.pa_plan_destroy(self.handle)
+            self._destroy(self.handle)
             self.handle = None
 
 
@@ -248,17 +252,21 @@ def pa_plan_check(plan: Plan, workspace, stream=None) -> int:
     return pos.value
 
 
-def pa_default_schedule(device: int, num_qo_heads: int, num_kv_heads: int, dtype):
+def pa_default_schedule(device: int, num_qo_heads: int, num_kv_heads: int, dtype, flags: int = 0):
     if isinstance(dtype, str):
         dtype = DTYPE_CODES[dtype]
     sms, k = _i32(), _i32()
-    _check(lib.pa_default_schedule(device, num_qo_heads, num_kv_heads, dtype, ctypes.byref(sms),
-                                   ctypes.byref(k)), "pa_default_schedule")
+    _check(lib.pa_default_schedule(device, num_qo_heads, num_kv_heads, dtype, flags,
+                                   ctypes.byref(sms), ctypes.byref(k)), "pa_default_schedule")
     return sms.value, k.value
 
 
 def pa_status_string(status: int) -> str:
     return lib.pa_status_string(status).decode()
+
+
+def pa_plan_uses_tensor_cores(plan: Plan) -> bool:
+    return lib.pa_plan_uses_tensor_cores(plan.handle) == 1
 
 
 def pa_abi_version() -> int:

@@ -28,7 +28,7 @@ class PagedDecode:
         self.device = torch.device(device if device is not None else "cuda")
         dev_index = self.device.index if self.device.index is not None else torch.cuda.current_device()
         if num_sms is None or ctas_per_sm is None:
-            sms, k = C.pa_default_schedule(dev_index, num_qo_heads, num_kv_heads, dtype)
+            sms, k = C.pa_default_schedule(dev_index, num_qo_heads, num_kv_heads, dtype, flags)
             num_sms = sms if num_sms is None else num_sms
             ctas_per_sm = k if ctas_per_sm is None else ctas_per_sm
         self.dtype = dtype

@@ -1,8 +1,9 @@
 """Paged decode on the GPU against the fp64 oracle (element by element).
 
-Small cases span several 32-token tiles, ragged tails, empty requests, every
-supported GQA group, page sizes 1 / 16 / 64, both dtypes, and forced
-split-KV.  Full-size benchmark workloads run in the bench's launch
+Small cases span several 32-token (CUDA-core) and 128-token (tensor-core)
+tiles, ragged tails, empty requests, every supported GQA group, page sizes
+1 / 16 / 64, both dtypes, forced split-KV and both decode kernels for groups
+4 and 8.  Full-size benchmark workloads run in the bench's launch
 configuration and are checked on sampled requests (every q head of each).
 """
 import numpy as np
@@ -26,17 +27,24 @@ def _decode(w, dev, **kw):
     o, lse = pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"],
                     prefix_indices=dev.get("prefix_indices"))
     torch.cuda.synchronize()
+    assert pd.check() == -1  # no bounded wait gave up
     return pd, o, lse
+
+
+KERNELS = {"auto": 0, "cuda_cores": 2}  # 2 = PA_FLAG_CUDA_CORES
 
 
 def _to_dev(t):
     return {k: v.cuda() for k, v in t.items()}
 
 
+@pytest.mark.parametrize("kernel", ["auto", "cuda_cores"])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("P", [1, 16, 64])
-def test_small_parity(dtype, group, P):
+def test_small_parity(dtype, group, P, kernel):
+    if kernel == "cuda_cores" and group < 4:
+        pytest.skip("groups 1 and 2 always run on CUDA cores")
     hkv = 2
     w = W.make_workload("small", EDGE_LENS, num_qo_heads=hkv * group, num_kv_heads=hkv,
                         page_size=P, dtype=dtype, seed=40 + group + P, extra_pages=3)
@@ -46,8 +54,44 @@ def test_small_parity(dtype, group, P):
     # no split (large budget) and forced split (tiny budget, 16-token chunks)
     for kw in (dict(num_sms=10000, ctas_per_sm=1),
                dict(num_sms=3, ctas_per_sm=1, min_chunk_tokens=16)):
-        pd, o, lse = _decode(w, dev, **kw)
-        assert_close(to_np(o), to_np(lse), o_ref, l_ref, dtype, f"G={group} P={P} {kw}")
+        pd, o, lse = _decode(w, dev, flags=KERNELS[kernel], **kw)
+        assert_close(to_np(o), to_np(lse), o_ref, l_ref, dtype,
+                     f"G={group} P={P} {kernel} {kw}")
+
+
+@pytest.mark.parametrize("kernel", ["auto", "cuda_cores"])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("group", [4, 8])
+@pytest.mark.parametrize("sm_scale", [1.0, 3.0])
+def test_sharp_softmax_moves_the_running_max(dtype, group, sm_scale, kernel):
+    """Scores spread over tens of units in log2: the running maximum of a long
+    piece moves many times past the lazy-rescale slack, so the rescale of the
+    accumulated output (TMEM on the tensor-core path) runs."""
+    w = W.make_workload("sharp", [2000, 700, 129, 5000, 1], num_qo_heads=2 * group,
+                        num_kv_heads=2, page_size=16, dtype=dtype, seed=90 + group,
+                        sm_scale=sm_scale)
+    t = w.materialize()
+    o_ref, l_ref = oracle_full(w, t)
+    dev = _to_dev(t)
+    for kw in (dict(num_sms=10000, ctas_per_sm=1),
+               dict(num_sms=5, ctas_per_sm=1, min_chunk_tokens=300)):
+        pd, o, lse = _decode(w, dev, flags=KERNELS[kernel], **kw)
+        assert_close(to_np(o), to_np(lse), o_ref, l_ref, dtype,
+                     f"sharp G={group} scale={sm_scale} {kernel} {kw}")
+
+
+@pytest.mark.parametrize("group", [4, 8])
+def test_tensor_core_and_cuda_core_kernels_agree(group):
+    """The two decode kernels on the same plan shape agree to rounding."""
+    w = W.make_workload("agree", [4096, 3000, 17, 0, 1200], num_qo_heads=4 * group,
+                        num_kv_heads=4, page_size=16, dtype="bf16", seed=95 + group)
+    dev = _to_dev(w.materialize())
+    _, o_tc, l_tc = _decode(w, dev, num_sms=148, ctas_per_sm=1)
+    _, o_cc, l_cc = _decode(w, dev, num_sms=148, ctas_per_sm=1, flags=KERNELS["cuda_cores"])
+    assert (o_tc.float() - o_cc.float()).abs().max().item() <= 2 * 2e-3
+    fin = torch.isfinite(l_cc)
+    assert torch.equal(fin, torch.isfinite(l_tc))
+    assert (l_tc[fin] - l_cc[fin]).abs().max().item() <= 2e-3
 
 
 def test_split_chunks_are_exercised():
@@ -117,7 +161,8 @@ def test_cuda_graph_replay():
         assert torch.equal(o, o_eager) and torch.equal(lse, l_eager)
 
 
-def test_bounds_checked_run_reports_bad_index():
+@pytest.mark.parametrize("kernel", ["auto", "cuda_cores"])
+def test_bounds_checked_run_reports_bad_index(kernel):
     from serving_attention_paged_b200 import pagedattn as C
     w = W.make_workload("chk", [40, 40], num_qo_heads=8, num_kv_heads=2, page_size=16,
                         dtype="f16", seed=10)
@@ -128,7 +173,7 @@ def test_bounds_checked_run_reports_bad_index():
     from serving_attention_paged_b200.wrapper import PagedDecode
     pd = PagedDecode(w.kv_indptr, w.last_page_len, num_qo_heads=8, num_kv_heads=2,
                      page_size=16, dtype="f16", sm_scale=w.sm_scale, num_pages=w.num_pages,
-                     flags=C.PA_FLAG_CHECK_INDICES)
+                     flags=C.PA_FLAG_CHECK_INDICES | KERNELS[kernel])
     pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"])
     assert pd.check() == -1
     pd.run(dev["q"], dev["k_pool"], dev["v_pool"], bad)
