@@ -58,9 +58,9 @@ def parse_args():
                     help="split-KV minimum chunk (tokens); 0 = library default")
     ap.add_argument("--ctas-per-sm", type=int, default=0,
                     help="CTA budget per SM for the plan; 0 = occupancy of the kernel")
-    ap.add_argument("--kernel", default="auto", choices=["auto", "cuda_cores"],
-                    help="decode kernel: auto (tensor cores for GQA groups 4 and 8) or "
-                         "cuda_cores")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"],
+                    help="decode kernel: auto (tensor cores for GQA groups 4 and 8, CUDA cores "
+                         "for 1 and 2), cuda_cores or tensor_cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -287,7 +287,8 @@ def run_ours(args):
                      sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
                      device=dev_t, min_chunk_tokens=args.min_chunk_tokens,
                      ctas_per_sm=args.ctas_per_sm or None,
-                     flags=C.PA_FLAG_CUDA_CORES if args.kernel == "cuda_cores" else 0)
+                     flags={"auto": 0, "cuda_cores": C.PA_FLAG_CUDA_CORES,
+                            "tensor_cores": C.PA_FLAG_TENSOR_CORES}[args.kernel])
     tensor_cores = C.pa_plan_uses_tensor_cores(pd.plan)
     setup_us = (time.perf_counter() - t0) * 1e6
     reps = 20

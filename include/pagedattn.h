@@ -76,10 +76,13 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 /* pa_merge_state only */ } p
 #define PA_FLAG_CHECK_INDICES 1u /* kernels bounds-check every page index against
                                     num_pages; a bad index is skipped (its tokens
                                     read as zero) and recorded for pa_plan_check */
-#define PA_FLAG_CUDA_CORES 2u    /* decode with the CUDA-core kernel even where the
-                                    tensor-core one exists (group 4 or 8, fp16/bf16);
-                                    the work list is the same, only the schedule
-                                    defaults differ (pa_default_schedule) */
+/* Decode kernel choice.  By default GQA groups 4 and 8 run on the tensor-core
+ * kernel and groups 1 and 2 on the CUDA-core kernel (the faster of the two at
+ * those shapes on B200); the work list is the same either way, only the
+ * schedule defaults differ (pa_default_schedule). */
+#define PA_FLAG_CUDA_CORES 2u    /* CUDA-core decode kernel for every group */
+#define PA_FLAG_TENSOR_CORES 4u  /* tensor-core decode kernel for every group (fp16/bf16);
+                                    PA_FLAG_CUDA_CORES wins if both are set */
 
 typedef struct {
   int32_t batch;            /* requests B >= 0 */
@@ -221,8 +224,7 @@ pa_status pa_plan_check(pa_plan_t plan, void* d_workspace, int64_t* bad_position
 
 /* Scheduling defaults for `device`: its SM count and how many CTAs of the
  * decode kernel that a problem with this shape, dtype and `flags` (PA_FLAG_*)
- * runs fit on one SM.  The tensor-core kernel (group 4 or 8, fp16/bf16,
- * without PA_FLAG_CUDA_CORES) holds one CTA per SM. */
+ * runs fit on one SM.  The tensor-core kernel holds one CTA per SM. */
 pa_status pa_default_schedule(int32_t device, int32_t num_qo_heads, int32_t num_kv_heads,
                               pa_dtype dtype, uint32_t flags, int32_t* num_sms,
                               int32_t* ctas_per_sm);

@@ -42,26 +42,11 @@ pa_status pa_plan_upload(pa_plan_t plan, void* d_workspace, size_t workspace_byt
   if (!plan || !d_workspace) return PA_ERR_INVALID_ARG;
   if (workspace_bytes < plan->ws.total) return PA_ERR_WORKSPACE_TOO_SMALL;
   if (reinterpret_cast<uintptr_t>(d_workspace) & (pa::kAlign - 1)) return PA_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(d_workspace);
-  const pa_problem& p = plan->prob;
-  cudaError_t e = cudaSuccess;
-  if (!plan->items.empty())
-    e = cudaMemcpyAsync(ws + plan->ws.items, plan->items.data(),
-                        plan->items.size() * sizeof(pa_work_item), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(ws + plan->ws.cta_indptr, plan->cta_indptr.data(),
-                        plan->cta_indptr.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(ws + plan->ws.merge_indptr, plan->merge_indptr.data(),
-                        plan->merge_indptr.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess && p.batch > 0)
-    e = cudaMemsetAsync(ws + plan->ws.counters, 0,
-                        size_t(p.batch) * p.num_kv_heads * pa::kCounterSlots * sizeof(int32_t),
-                        s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ws + plan->ws.error, 0xff, sizeof(uint64_t), s);
-  if (e == cudaSuccess)
-    e = cudaMemsetAsync(ws + plan->ws.error + sizeof(uint64_t), 0, sizeof(uint64_t), s);
+  // one copy of the plan's image of the workspace head (work list, offsets,
+  // zeroed counters, cleared status words)
+  const std::vector<uint8_t>& img = plan->upload_image;
+  const cudaError_t e = cudaMemcpyAsync(d_workspace, img.data(), img.size(),
+                                        cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
   return from_cuda(int(e));
 }
 

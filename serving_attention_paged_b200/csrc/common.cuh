@@ -224,21 +224,29 @@ __device__ __forceinline__ void merge_partials(MergeAcc (&acc)[G], const float* 
 }
 
 // Adds the cascade prefix states of rows row0 .. row0 + G - 1 at head
-// element d: prefix_o [chunks, B * Hq, D], prefix_lse [chunks, B * Hq].
+// element d: prefix_o [chunks, B * Hq, D], prefix_lse [chunks, B * Hq].  As
+// above, every load of a batch of chunks is issued before any is used.
 template <int G, int D>
 __device__ __forceinline__ void merge_prefix(MergeAcc (&acc)[G], const float* prefix_o,
                                              const float* prefix_lse, int chunks,
                                              int64_t rows_per_chunk, int64_t row0, int d) {
-  for (int c = 0; c < chunks; ++c) {
-    float o[G], l[G];
+  constexpr int kBatch = G >= 8 ? 2 : 4;  // chunks per batch of loads
+  for (int c0 = 0; c0 < chunks; c0 += kBatch) {
+    float o[kBatch][G], l[kBatch][G];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      const int64_t r = c * rows_per_chunk + row0 + hh;
-      o[hh] = prefix_o[r * D + d];
-      l[hh] = prefix_lse[r];
+    for (int j = 0; j < kBatch; ++j) {
+      const bool in = c0 + j < chunks;
+      const int64_t base = int64_t(in ? c0 + j : 0) * rows_per_chunk + row0;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        o[j][hh] = prefix_o[(base + hh) * D + d];
+        l[j][hh] = in ? prefix_lse[base + hh] : -INFINITY;
+      }
     }
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) acc[hh].add(o[hh], l[hh]);
+    for (int j = 0; j < kBatch; ++j)
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) acc[hh].add(o[j][hh], l[j][hh]);
   }
 }
 

@@ -131,6 +131,14 @@ __device__ __forceinline__ uint16_t round16(BF16, float x, float& r) {
 
 // N consecutive fp32 columns of this thread's TMEM lane.
 template <int N> __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]);
+template <> __device__ __forceinline__ void tmem_ld<1>(uint32_t taddr, uint32_t (&r)[1]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n" : "=r"(r[0]) : "r"(taddr));
+}
+template <> __device__ __forceinline__ void tmem_ld<2>(uint32_t taddr, uint32_t (&r)[2]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(taddr));
+}
 template <> __device__ __forceinline__ void tmem_ld<4>(uint32_t taddr, uint32_t (&r)[4]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -152,6 +160,15 @@ template <> __device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t
       : "r"(taddr));
 }
 template <int N> __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]);
+template <> __device__ __forceinline__ void tmem_st<1>(uint32_t taddr, const uint32_t (&r)[1]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n" ::"r"(taddr), "r"(r[0])
+               : "memory");
+}
+template <> __device__ __forceinline__ void tmem_st<2>(uint32_t taddr, const uint32_t (&r)[2]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};\n" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1])
+               : "memory");
+}
 template <> __device__ __forceinline__ void tmem_st<4>(uint32_t taddr, const uint32_t (&r)[4]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(taddr),
                "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
@@ -706,6 +723,8 @@ cudaError_t launch_tc_t(const TcArgs& a, int64_t n_cta, cudaStream_t stream) {
 template <typename Tag, bool kCheck>
 cudaError_t dispatch_tc(int group, const TcArgs& a, int64_t n, cudaStream_t s) {
   switch (group) {
+    case 1: return launch_tc_t<Tag, 1, kCheck>(a, n, s);
+    case 2: return launch_tc_t<Tag, 2, kCheck>(a, n, s);
     case 4: return launch_tc_t<Tag, 4, kCheck>(a, n, s);
     case 8: return launch_tc_t<Tag, 8, kCheck>(a, n, s);
   }
@@ -715,7 +734,8 @@ cudaError_t dispatch_tc(int group, const TcArgs& a, int64_t n, cudaStream_t s) {
 }  // namespace
 
 bool decode_tc_supported(int32_t group, pa_dtype dtype) {
-  return (group == 4 || group == 8) && (dtype == PA_F16 || dtype == PA_BF16);
+  return (group == 1 || group == 2 || group == 4 || group == 8) &&
+         (dtype == PA_F16 || dtype == PA_BF16);
 }
 
 int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out) {
@@ -726,6 +746,10 @@ int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out) {
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, kSmemBytes);
   };
   const bool bf = dtype == PA_BF16;
+  if (group == 1)
+    return int(bf ? get(paged_decode_tc_kernel<BF16, 1, false>) : get(paged_decode_tc_kernel<F16, 1, false>));
+  if (group == 2)
+    return int(bf ? get(paged_decode_tc_kernel<BF16, 2, false>) : get(paged_decode_tc_kernel<F16, 2, false>));
   if (group == 4)
     return int(bf ? get(paged_decode_tc_kernel<BF16, 4, false>) : get(paged_decode_tc_kernel<F16, 4, false>));
   if (group == 8)

@@ -55,6 +55,10 @@ struct pa_plan_s {
   int32_t prefix_chunk_tokens = 0;  // tokens per chunk (multiple of the 128-key tile)
   int32_t q_tiles = 0;              // 128-row tiles over the B * G query rows of one kv head
   pa::WorkspaceLayout ws;
+  // Bytes [0, ws.partial_o) of the workspace as pa_plan_upload writes them:
+  // work list, CTA and merge offsets, zeroed counters and the status words
+  // (no bad index, no timeout), so the upload is a single copy.
+  std::vector<uint8_t> upload_image;
 };
 
 namespace pa {
@@ -76,11 +80,13 @@ int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream);
 int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream);
 bool decode_tc_supported(int32_t group, pa_dtype dtype);
 int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out);
-// The decode kernel a problem runs: tensor cores where built, unless the
-// caller asked for the CUDA-core kernel.
+// The decode kernel a problem runs: the caller's choice if any, else tensor
+// cores for GQA groups of 4 and more (measured faster there; at groups 1 and
+// 2 the padded MMA buys nothing and the CUDA-core kernel is quicker).
 inline bool decode_uses_tensor_cores(const pa_problem& p) {
-  return decode_tc_supported(p.num_qo_heads / p.num_kv_heads, p.dtype) &&
-         !(p.flags & PA_FLAG_CUDA_CORES);
+  const int32_t group = p.num_qo_heads / p.num_kv_heads;
+  if (!decode_tc_supported(group, p.dtype) || (p.flags & PA_FLAG_CUDA_CORES)) return false;
+  return (p.flags & PA_FLAG_TENSOR_CORES) || group >= 4;
 }
 int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* stream);
 int launch_merge_state(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,

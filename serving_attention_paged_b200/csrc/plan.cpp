@@ -140,6 +140,19 @@ void layout_workspace(pa_plan_s* plan) {
   w.total = off;
 }
 
+void build_upload_image(pa_plan_s* plan) {
+  const pa::WorkspaceLayout& w = plan->ws;
+  std::vector<uint8_t>& img = plan->upload_image;
+  img.assign(w.partial_o, 0);  // counters stay zero
+  if (!plan->items.empty())
+    std::memcpy(img.data() + w.items, plan->items.data(), plan->items.size() * sizeof(pa_work_item));
+  std::memcpy(img.data() + w.cta_indptr, plan->cta_indptr.data(),
+              plan->cta_indptr.size() * sizeof(int32_t));
+  std::memcpy(img.data() + w.merge_indptr, plan->merge_indptr.data(),
+              plan->merge_indptr.size() * sizeof(int32_t));
+  std::memset(img.data() + w.error, 0xff, sizeof(uint64_t));  // first bad index: none
+}
+
 // Level-1 cascade schedule: (kv head, 128-row query tile, prefix chunk) tiles,
 // about one per SM; each chunk a whole number of 128-key tiles.
 void schedule_prefix(pa_plan_s* plan) {
@@ -187,6 +200,7 @@ pa_status create(const pa_problem* problem, int32_t prefix_len, bool cascade,
     if (st == PA_OK) {
       if (cascade) schedule_prefix(plan);
       layout_workspace(plan);
+      build_upload_image(plan);
     }
   } catch (const std::bad_alloc&) {
     st = PA_ERR_NO_MEMORY;

@@ -26,6 +26,7 @@ PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_NO_MEMORY, PA_ERR_DEVICE_TIMEOUT = 4, 5
 PA_F16, PA_BF16, PA_F32 = 0, 1, 2
 PA_FLAG_CHECK_INDICES = 1
 PA_FLAG_CUDA_CORES = 2
+PA_FLAG_TENSOR_CORES = 4
 DTYPE_CODES = {"f16": PA_F16, "bf16": PA_BF16, "f32": PA_F32}
 
 

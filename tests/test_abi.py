@@ -163,3 +163,20 @@ def test_cascade_plan_shape(C):
                                    num_sms=148, ctas_per_sm=2)
     assert np.array_equal(C.pa_plan_work_items(plan), items)
     assert np.array_equal(C.pa_plan_cta_indptr(plan), ci)
+
+
+def test_decode_kernel_choice(C):
+    """Default: tensor cores for GQA groups 4 and 8, CUDA cores for 1 and 2;
+    PA_FLAG_CUDA_CORES / PA_FLAG_TENSOR_CORES override (CUDA cores win)."""
+    w = W.make_workload("k", [20, 40], num_qo_heads=8, num_kv_heads=2, page_size=16,
+                        dtype="f16", seed=1)
+    cases = [(1, 0, False), (2, 0, False), (4, 0, True), (8, 0, True),
+             (4, C.PA_FLAG_CUDA_CORES, False), (8, C.PA_FLAG_CUDA_CORES, False),
+             (1, C.PA_FLAG_TENSOR_CORES, True), (2, C.PA_FLAG_TENSOR_CORES, True),
+             (4, C.PA_FLAG_CUDA_CORES | C.PA_FLAG_TENSOR_CORES, False)]
+    for group, flags, expect in cases:
+        prob = C.make_problem(batch=w.batch, num_qo_heads=2 * group, num_kv_heads=2,
+                              page_size=16, dtype="bf16", sm_scale=0.1, num_sms=148,
+                              ctas_per_sm=1, num_pages=w.num_pages, flags=flags)
+        plan = C.pa_plan_create(prob, w.kv_indptr, w.last_page_len)
+        assert C.pa_plan_uses_tensor_cores(plan) is expect, (group, flags)

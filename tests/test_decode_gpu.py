@@ -2,8 +2,7 @@
 
 Small cases span several 32-token (CUDA-core) and 128-token (tensor-core)
 tiles, ragged tails, empty requests, every supported GQA group, page sizes
-1 / 16 / 64, both dtypes, forced split-KV and both decode kernels for groups
-4 and 8.  Full-size benchmark workloads run in the bench's launch
+1 / 16 / 64, both dtypes, forced split-KV and both decode kernels.  Full-size benchmark workloads run in the bench's launch
 configuration and are checked on sampled requests (every q head of each).
 """
 import numpy as np
@@ -31,20 +30,18 @@ def _decode(w, dev, **kw):
     return pd, o, lse
 
 
-KERNELS = {"auto": 0, "cuda_cores": 2}  # 2 = PA_FLAG_CUDA_CORES
+KERNELS = {"auto": 0, "cuda_cores": 2, "tensor_cores": 4}  # PA_FLAG_CUDA_CORES / _TENSOR_CORES
 
 
 def _to_dev(t):
     return {k: v.cuda() for k, v in t.items()}
 
 
-@pytest.mark.parametrize("kernel", ["auto", "cuda_cores"])
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("P", [1, 16, 64])
 def test_small_parity(dtype, group, P, kernel):
-    if kernel == "cuda_cores" and group < 4:
-        pytest.skip("groups 1 and 2 always run on CUDA cores")
     hkv = 2
     w = W.make_workload("small", EDGE_LENS, num_qo_heads=hkv * group, num_kv_heads=hkv,
                         page_size=P, dtype=dtype, seed=40 + group + P, extra_pages=3)
