@@ -59,8 +59,8 @@ def parse_args():
     ap.add_argument("--ctas-per-sm", type=int, default=0,
                     help="CTA budget per SM for the plan; 0 = occupancy of the kernel")
     ap.add_argument("--kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"],
-                    help="decode kernel: auto (tensor cores for GQA groups 4 and 8, CUDA cores "
-                         "for 1 and 2), cuda_cores or tensor_cores")
+                    help="decode kernel: auto (tensor cores for GQA group 8, CUDA cores for "
+                         "1, 2 and 4), cuda_cores or tensor_cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()

@@ -76,8 +76,8 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 /* pa_merge_state only */ } p
 #define PA_FLAG_CHECK_INDICES 1u /* kernels bounds-check every page index against
                                     num_pages; a bad index is skipped (its tokens
                                     read as zero) and recorded for pa_plan_check */
-/* Decode kernel choice.  By default GQA groups 4 and 8 run on the tensor-core
- * kernel and groups 1 and 2 on the CUDA-core kernel (the faster of the two at
+/* Decode kernel choice.  By default GQA group 8 runs on the tensor-core kernel
+ * and groups 1, 2 and 4 on the CUDA-core kernel (the faster of the two at
  * those shapes on B200); the work list is the same either way, only the
  * schedule defaults differ (pa_default_schedule). */
 #define PA_FLAG_CUDA_CORES 2u    /* CUDA-core decode kernel for every group */

@@ -81,12 +81,13 @@ int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream);
 bool decode_tc_supported(int32_t group, pa_dtype dtype);
 int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out);
 // The decode kernel a problem runs: the caller's choice if any, else tensor
-// cores for GQA groups of 4 and more (measured faster there; at groups 1 and
-// 2 the padded MMA buys nothing and the CUDA-core kernel is quicker).
+// cores for GQA groups of 8, where the CUDA-core kernel is issue-bound (1.4x
+// slower on B200); at groups 1 to 4 the CUDA-core kernel measured as fast or
+// faster, the padded MMA buying nothing once HBM is the bound.
 inline bool decode_uses_tensor_cores(const pa_problem& p) {
   const int32_t group = p.num_qo_heads / p.num_kv_heads;
   if (!decode_tc_supported(group, p.dtype) || (p.flags & PA_FLAG_CUDA_CORES)) return false;
-  return (p.flags & PA_FLAG_TENSOR_CORES) || group >= 4;
+  return (p.flags & PA_FLAG_TENSOR_CORES) || group >= 8;
 }
 int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* stream);
 int launch_merge_state(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,

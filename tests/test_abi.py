@@ -166,11 +166,12 @@ def test_cascade_plan_shape(C):
 
 
 def test_decode_kernel_choice(C):
-    """Default: tensor cores for GQA groups 4 and 8, CUDA cores for 1 and 2;
+    """Default: tensor cores for GQA group 8, CUDA cores for 1, 2 and 4;
     PA_FLAG_CUDA_CORES / PA_FLAG_TENSOR_CORES override (CUDA cores win)."""
     w = W.make_workload("k", [20, 40], num_qo_heads=8, num_kv_heads=2, page_size=16,
                         dtype="f16", seed=1)
-    cases = [(1, 0, False), (2, 0, False), (4, 0, True), (8, 0, True),
+    cases = [(1, 0, False), (2, 0, False), (4, 0, False), (8, 0, True),
+             (4, C.PA_FLAG_TENSOR_CORES, True),
              (4, C.PA_FLAG_CUDA_CORES, False), (8, C.PA_FLAG_CUDA_CORES, False),
              (1, C.PA_FLAG_TENSOR_CORES, True), (2, C.PA_FLAG_TENSOR_CORES, True),
              (4, C.PA_FLAG_CUDA_CORES | C.PA_FLAG_TENSOR_CORES, False)]
