@@ -61,6 +61,9 @@ def parse_args():
     ap.add_argument("--kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"],
                     help="decode kernel: auto (tensor cores for GQA group 8, CUDA cores for "
                          "1, 2 and 4), cuda_cores or tensor_cores")
+    ap.add_argument("--piece-cost-tokens", type=int, default=0,
+                    help="plan cost of a piece boundary in tokens; 0 = the kernel's default, "
+                         "< 0 = none")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -288,7 +291,8 @@ def run_ours(args):
                      device=dev_t, min_chunk_tokens=args.min_chunk_tokens,
                      ctas_per_sm=args.ctas_per_sm or None,
                      flags={"auto": 0, "cuda_cores": C.PA_FLAG_CUDA_CORES,
-                            "tensor_cores": C.PA_FLAG_TENSOR_CORES}[args.kernel])
+                            "tensor_cores": C.PA_FLAG_TENSOR_CORES}[args.kernel],
+                     piece_cost_tokens=args.piece_cost_tokens)
     tensor_cores = C.pa_plan_uses_tensor_cores(pd.plan)
     setup_us = (time.perf_counter() - t0) * 1e6
     reps = 20

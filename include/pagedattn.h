@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 2
+#define PA_ABI_VERSION 3
 
 typedef enum {
   PA_OK = 0,
@@ -98,6 +98,10 @@ typedef struct {
   int64_t num_pages;        /* pages in the pool; num_pages * page_size < 2^32 (pool rows
                                are 32-bit indices); bounds for PA_FLAG_CHECK_INDICES */
   uint32_t flags;           /* PA_FLAG_* */
+  int32_t piece_cost_tokens; /* plan budget charged for each further piece of a CTA
+                                (see pa_plan_create): 0 = the default of the decode
+                                kernel the problem runs (400 CUDA cores, 128 tensor
+                                cores), > 0 that many tokens, < 0 none */
 } pa_problem;
 
 /* One piece of run-stage work: tokens [token_begin, token_end) of kv head
@@ -113,23 +117,31 @@ typedef struct {
 typedef struct pa_plan_s* pa_plan_t;
 
 /* Plan stage (host only, no CUDA call).  Specification of the work list
- * (a stream-K style split of the whole decode step over tokens):
+ * (a stream-K style split of the whole decode step over tokens, each piece
+ * boundary charged a cost c = piece_cost_tokens in token time):
  *   L_b = 0 if n_b = 0 else (n_b - 1) * P + last_page_len[b]; T = sum_b L_b;
+ *   N = number of requests with L_b > 0;
  *   W = num_sms * ctas_per_sm (CTAs resident at once);
- *   groups = max(1, floor(W / Hkv)) groups of Hkv CTAs, one CTA per kv head;
- *   quota q = 32 * ceil(max(min_chunk_tokens, ceil(T / groups)) / 32) tokens;
- *   n_groups = max(1, ceil(T / q)) (0 for an empty batch); n_cta = n_groups * Hkv.
- *   Group g covers token positions [g q, (g + 1) q) of the requests laid end
- *   to end; its pieces are the intersections with the requests, in request
- *   order.  An empty request is a zero-length piece of the group its position
- *   falls in (the last group at the very end).  CTA g * Hkv + h runs the
- *   pieces of group g for kv head h, so the Hkv CTAs of a group read the
- *   same pages at the same time.
+ *   groups = max(1, floor(W / Hkv)) groups of Hkv CTAs, one CTA per kv head.
+ *   Walk for a budget q: the requests' tokens, laid end to end, fill groups
+ *   in order.  A group takes pieces (request, [t0, t1)) in request order; a
+ *   piece after the group's first one costs c + (t1 - t0) of its budget q,
+ *   the first one t1 - t0.  A group is full when the next token would not
+ *   fit (it holds a piece and used + c >= q); the next token then opens the
+ *   next group, and a request cut there continues as the first piece of that
+ *   group.  An empty request is a zero-length piece of the group the next
+ *   token goes to (the last group at the very end) and costs nothing.
+ *   q = 32 * ceil(max(min_chunk_tokens, ceil((T + c * max(N - 1, 0)) / groups)) / 32);
+ *   n_groups is the number of groups the walk fills, never more than groups
+ *   (0 for an empty batch, 1 when every request is empty); n_cta = n_groups * Hkv.
+ *   With c = 0 group g holds exactly the token positions [g q, (g + 1) q).
+ *   CTA g * Hkv + h runs the pieces of group g for kv head h, so the Hkv CTAs
+ *   of a group read the same pages at the same time.
  *   A (request, kv head) segment cut into k > 1 pieces owns partial slots
  *   merge_indptr[b * Hkv + h] + 0 .. k - 1, in token order; merge_indptr is
  *   the running sum of those k.
- * Every group but the last therefore reads exactly q tokens, whatever the
- * length mix, and no CTA waits for another.
+ * Every CTA is resident from the start and no CTA waits for another; the
+ * costs make a CTA with more pieces take fewer tokens, so all finish together.
  * Validates: kv_indptr[0] == 0 and non-decreasing, 1 <= last_page_len[b] <= P
  * whenever request b has pages, Hq % Hkv == 0, positive sizes.
  * Returns PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED otherwise.  The host arrays

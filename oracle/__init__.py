@@ -194,23 +194,30 @@ def cascade_decode(q, k_pool, v_pool, prefix_indices, prefix_len, kv_indptr, kv_
 
 
 def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per_sm,
-         min_chunk_tokens=256):
+         min_chunk_tokens=256, piece_cost=0):
     """Split-KV work list (FlashInfer README core feature 2: variable-length
     inputs are scheduled in a plan stage to even out the load; the README
     also names stream-K among FlashInfer's inspirations).
 
     Specification (the reading adopted where the page is silent), restated
-    here with plain loops:
+    here with plain loops; c = piece_cost is the budget a piece boundary
+    costs, in tokens:
       L_b = 0 if n_b = 0 else (n_b - 1) * P + last_page_len[b]; T = sum_b L_b;
-      W = num_sms * ctas_per_sm; groups = max(1, floor(W / Hkv));
-      quota q = 32 * ceil(max(min_chunk_tokens, ceil(T / groups)) / 32) tokens;
-      n_groups = max(1, ceil(T / q)), or 0 for an empty batch.
-      Group g covers token positions [g q, (g + 1) q) of the requests laid
-      end to end; its pieces are the intersections with the requests (an
-      empty request is a zero-length piece of the group its position falls
-      in; the last group at the very end).  CTA g * Hkv + h runs the pieces of
-      group g for kv head h.  A (request, head) segment cut into k > 1 pieces
-      owns partial slots merge_indptr[b * Hkv + h] + 0 .. k - 1, in order.
+      N = number of non-empty requests; W = num_sms * ctas_per_sm;
+      groups = max(1, floor(W / Hkv)).
+      Walk for budget q: requests in order fill groups in order; a group's
+      first piece costs its token count, each later piece c more; a group
+      is full once it holds a piece and used + c >= q, and the next token
+      then opens the next group (a request cut there goes on as that group's
+      first piece).  An empty request is a zero-length, free piece of the
+      group the next token goes to (the last group at the very end).
+      q = 32 * ceil(max(min_chunk_tokens, ceil((T + c * max(N - 1, 0)) / groups)) / 32);
+      n_groups = the groups the walk fills (0 for an empty batch), which is
+      at most `groups`.  With c = 0, group g is token positions
+      [g q, (g + 1) q) of the requests laid end to end.
+      CTA g * Hkv + h runs the pieces of group g for kv head h.  A (request,
+      head) segment cut into k > 1 pieces owns partial slots
+      merge_indptr[b * Hkv + h] + 0 .. k - 1, in order.
 
     Returns ``(quota, items, cta_indptr, merge_indptr)``; items is int32
     ``[n, 6]``: request, kv_head, page_begin (= kv_indptr[b]), token_begin,
@@ -218,29 +225,53 @@ def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per
     """
     indptr = [int(x) for x in _as_i32(kv_indptr)]
     last = [int(x) for x in _as_i32(last_page_len)]
-    B, P, Hkv = len(last), page_size, num_kv_heads
+    B, P, Hkv, c = len(last), page_size, num_kv_heads, piece_cost
     L = []
     for b in range(B):
         n = indptr[b + 1] - indptr[b]
         L.append((n - 1) * P + last[b] if n > 0 else 0)
     T = sum(L)
-    W = num_sms * ctas_per_sm
-    groups = max(1, W // Hkv)
-    q = 32 * (-(-max(min_chunk_tokens, -(-T // groups)) // 32))
-    n_groups = 0 if B == 0 else max(1, -(-T // q))
+    N = sum(1 for x in L if x > 0)
+    groups = max(1, (num_sms * ctas_per_sm) // Hkv)
 
-    group_pieces = [[] for _ in range(n_groups)]
-    pos = 0
-    for b in range(B):
-        t = 0
-        while True:
-            g = min(pos // q, n_groups - 1)
-            take = min(L[b] - t, (g + 1) * q - pos)
-            group_pieces[g].append((b, t, t + take))
-            t += take
-            pos += take
-            if t >= L[b]:
-                break
+    def fill(q):
+        """Pieces (b, t0, t1) per group for budget q."""
+        out = [[]]
+        load = 0          # budget used by the group being filled
+        opened = False    # it holds a non-empty piece
+        for b in range(B):
+            if L[b] == 0:
+                gi = len(out) - 1
+                if opened and load + c >= q:
+                    gi += 1
+                    out.append([])
+                    # the next token goes there: start it fresh
+                    load, opened = 0, False
+                out[gi].append((b, 0, 0))
+                continue
+            t = 0
+            while t < L[b]:
+                extra = c if opened else 0
+                if opened and load + extra >= q:
+                    out.append([])
+                    load, opened = 0, False
+                    continue
+                n = min(L[b] - t, q - load - extra)
+                out[-1].append((b, t, t + n))
+                load += extra + n
+                opened = True
+                t += n
+        # groups that received only empty requests after the last token
+        while len(out) > 1 and all(t1 == t0 for (_, t0, t1) in out[-1]) and \
+                not any(t1 > t0 for (_, t0, t1) in out[-1]):
+            tail = out.pop()
+            out[-1].extend(tail)
+        return out
+
+    q = 32 * (-(-max(min_chunk_tokens, -(-(T + c * max(N - 1, 0)) // groups)) // 32))
+    group_pieces = fill(q) if B > 0 else []
+    n_groups = len(group_pieces)
+    assert n_groups <= groups
 
     items, cta_indptr = [], [0]
     for g in range(n_groups):

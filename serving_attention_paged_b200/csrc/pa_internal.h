@@ -89,6 +89,17 @@ inline bool decode_uses_tensor_cores(const pa_problem& p) {
   if (!decode_tc_supported(group, p.dtype) || (p.flags & PA_FLAG_CUDA_CORES)) return false;
   return (p.flags & PA_FLAG_TENSOR_CORES) || group >= 8;
 }
+// Plan cost of a piece boundary, in tokens of the kernel's steady-state rate.
+// Per-CTA clock traces on B200 put the extra time of a further piece of a CTA
+// at several us for the CUDA-core kernel (each piece refills its pipeline and
+// runs its epilogue in line; ~16 KB/us per CTA) and near none for the
+// tensor-core kernel (its loaders run across pieces and epilogue warps work
+// off the critical path); the values are the best of a sweep on the uniform
+// and ragged batches.
+constexpr int32_t kPieceCostCudaCores = 400, kPieceCostTensorCores = 128;
+inline int32_t default_piece_cost_tokens(const pa_problem& p) {
+  return decode_uses_tensor_cores(p) ? kPieceCostTensorCores : kPieceCostCudaCores;
+}
 int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* stream);
 int launch_merge_state(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
                        void* o, float* lse, int64_t rows, int32_t head_dim, pa_dtype dtype,

@@ -63,33 +63,77 @@ pa_status build(pa_plan_s* plan, const int32_t* indptr, const int32_t* last) {
   else plan->kv_indptr.assign(1, 0);
   plan->last_page_len.assign(last ? last : nullptr, last ? last + B : nullptr);
 
-  // Token-level stream-K: CTAs come in groups of Hkv (one per kv head); every
-  // group gets the same quota q of the concatenated request tokens (at least
-  // min_chunk_tokens, rounded up to whole 32-token tiles), so the Hkv CTAs of
-  // a group read the same pages at the same time, each its own head.
+  // Token-level stream-K with a cost per piece: CTAs come in groups of Hkv
+  // (one per kv head), so the Hkv CTAs of a group read the same pages at the
+  // same time, each its own head.  Every group has the same budget q, filled
+  // with the requests' tokens laid end to end; a piece that a group starts
+  // after its first one (a new request) also charges c tokens, the measured
+  // cost of a piece boundary (pipeline refill and epilogue) in token time.
   const int64_t W = int64_t(p.num_sms) * p.ctas_per_sm;
   const int64_t groups = std::max<int64_t>(1, W / Hkv);
   const int64_t min_tokens = p.min_chunk_tokens ? p.min_chunk_tokens : pa::kDefaultMinChunkTokens;
-  const int64_t q = ceil_div(std::max<int64_t>(min_tokens, ceil_div(total, groups)), 32) * 32;
+  const int64_t c = p.piece_cost_tokens > 0    ? p.piece_cost_tokens
+                    : p.piece_cost_tokens == 0 ? pa::default_piece_cost_tokens(p)
+                                               : 0;
+  int64_t nonempty = 0;
+  for (int64_t b = 0; b < B; ++b) nonempty += L[b] > 0;
+  std::vector<std::vector<std::array<int64_t, 3>>> group_pieces;
+  // The walk for budget q; returns the number of groups it fills.
+  auto walk = [&](int64_t q) -> int64_t {
+    group_pieces.assign(1, {});
+    size_t g = 0;
+    int64_t used = 0;
+    bool has_piece = false;  // group g holds a non-empty piece
+    for (int64_t b = 0; b < B; ++b) {
+      if (L[b] == 0) {  // zero-length piece in the group the next token goes to
+        const size_t target = has_piece && used + c >= q ? g + 1 : g;
+        if (target == group_pieces.size()) group_pieces.emplace_back();
+        group_pieces[target].push_back({b, 0, 0});
+        continue;
+      }
+      int64_t t = 0;
+      while (t < L[b]) {
+        const int64_t cost = has_piece ? c : 0;
+        if (has_piece && used + cost >= q) {  // the next token does not fit
+          if (++g == group_pieces.size()) group_pieces.emplace_back();
+          used = 0;
+          has_piece = false;
+          continue;
+        }
+        const int64_t take = std::min<int64_t>(L[b] - t, q - used - cost);
+        group_pieces[g].push_back({b, t, t + take});
+        used += cost + take;
+        has_piece = true;
+        t += take;
+      }
+    }
+    // zero-length pieces past the last group with tokens join that group
+    const size_t n = std::max<size_t>(1, g + 1);
+    for (size_t k = n; k < group_pieces.size(); ++k)
+      group_pieces[n - 1].insert(group_pieces[n - 1].end(), group_pieces[k].begin(),
+                                 group_pieces[k].end());
+    group_pieces.resize(n);
+    return int64_t(n);
+  };
+  // q: the even share of the tokens plus one piece cost per further request.
+  // The walk then always fits in `groups`: a group that closes with budget
+  // left over (less than c) is followed by a group whose first piece starts
+  // a request, a cost the share counted but the walk does not charge, so
+  // (n_groups - 1) q < T + c (N - 1) <= groups q.
+  const int64_t q = ceil_div(std::max<int64_t>(min_tokens,
+                                               ceil_div(total + c * std::max<int64_t>(nonempty - 1, 0),
+                                                        groups)),
+                             32) * 32;
   if (q > INT32_MAX) return PA_ERR_UNSUPPORTED;
-  plan->quota = int32_t(q);
-  const int64_t n_groups = B == 0 ? 0 : std::max<int64_t>(1, ceil_div(total, q));
-  if (n_groups * Hkv > INT32_MAX) return PA_ERR_UNSUPPORTED;
-
-  // Pieces of each group: the requests' token ranges that meet [g q, (g+1) q).
-  // An empty request is a zero-length piece of the group its position falls in.
-  std::vector<std::vector<std::array<int64_t, 3>>> group_pieces(static_cast<size_t>(n_groups));
-  int64_t pos = 0;
-  for (int64_t b = 0; b < B; ++b) {
-    int64_t t = 0;
-    do {
-      const int64_t g = std::min<int64_t>(pos / q, n_groups - 1);
-      const int64_t take = std::min<int64_t>(L[b] - t, (g + 1) * q - pos);
-      group_pieces[size_t(g)].push_back({b, t, t + take});
-      t += take;
-      pos += take;
-    } while (t < L[b]);
+  int64_t n_groups = 0;
+  if (B > 0) {
+    n_groups = walk(q);
+    if (n_groups > groups) return PA_ERR_UNSUPPORTED;  // cannot happen (see above)
+  } else {
+    group_pieces.clear();
   }
+  plan->quota = int32_t(q);
+  if (n_groups * Hkv > INT32_MAX) return PA_ERR_UNSUPPORTED;
   plan->items.clear();
   plan->cta_indptr.assign(size_t(n_groups * Hkv) + 1, 0);
   for (int64_t g = 0; g < n_groups; ++g)

@@ -36,7 +36,8 @@ class pa_problem(ctypes.Structure):
                 ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("sm_scale", ctypes.c_float), ("num_sms", ctypes.c_int32),
                 ("ctas_per_sm", ctypes.c_int32), ("min_chunk_tokens", ctypes.c_int32),
-                ("num_pages", ctypes.c_int64), ("flags", ctypes.c_uint32)]
+                ("num_pages", ctypes.c_int64), ("flags", ctypes.c_uint32),
+                ("piece_cost_tokens", ctypes.c_int32)]
 
 
 class pa_work_item(ctypes.Structure):
@@ -128,11 +129,12 @@ class Plan:
 
 def make_problem(*, batch, num_qo_heads, num_kv_heads, head_dim=128, page_size, dtype,
                  sm_scale, num_sms, ctas_per_sm, min_chunk_tokens=0, num_pages=0,
-                 flags=0) -> pa_problem:
+                 flags=0, piece_cost_tokens=0) -> pa_problem:
     if isinstance(dtype, str):
         dtype = DTYPE_CODES[dtype]
     return pa_problem(batch, num_qo_heads, num_kv_heads, head_dim, page_size, dtype, sm_scale,
-                      num_sms, ctas_per_sm, min_chunk_tokens, num_pages, flags)
+                      num_sms, ctas_per_sm, min_chunk_tokens, num_pages, flags,
+                      piece_cost_tokens)
 
 
 def pa_plan_create(problem: pa_problem, kv_indptr_host, last_page_len_host) -> Plan:

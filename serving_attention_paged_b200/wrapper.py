@@ -24,7 +24,8 @@ class PagedDecode:
 
     def __init__(self, kv_indptr, last_page_len, *, num_qo_heads, num_kv_heads, page_size,
                  dtype, sm_scale, num_pages, head_dim=128, device=None, num_sms=None,
-                 ctas_per_sm=None, min_chunk_tokens=0, prefix_len=0, flags=0, stream=None):
+                 ctas_per_sm=None, min_chunk_tokens=0, prefix_len=0, flags=0,
+                 piece_cost_tokens=0, stream=None):
         self.device = torch.device(device if device is not None else "cuda")
         dev_index = self.device.index if self.device.index is not None else torch.cuda.current_device()
         if num_sms is None or ctas_per_sm is None:
@@ -40,7 +41,7 @@ class PagedDecode:
                                       page_size=page_size, dtype=dtype, sm_scale=sm_scale,
                                       num_sms=num_sms, ctas_per_sm=ctas_per_sm,
                                       min_chunk_tokens=min_chunk_tokens, num_pages=num_pages,
-                                      flags=flags)
+                                      flags=flags, piece_cost_tokens=piece_cost_tokens)
         if prefix_len:
             self.plan = C.pa_cascade_plan_create(self.problem, prefix_len, kv_indptr, last_page_len)
         else:

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(C):
     assert len(names) >= 15
     for n in names:
         assert hasattr(C.lib, n), n
-    assert C.pa_abi_version() == 2
+    assert C.pa_abi_version() == 3
 
 
 def _problem(C, w, num_sms=148, k=2, mct=0, flags=0):
@@ -42,13 +42,15 @@ def _problem(C, w, num_sms=148, k=2, mct=0, flags=0):
                           min_chunk_tokens=mct, num_pages=w.num_pages, flags=flags)
 
 
-def _compare_plan(C, indptr, last, P, hq, hkv, sms, k, mct):
+def _compare_plan(C, indptr, last, P, hq, hkv, sms, k, mct, c=0):
     prob = C.make_problem(batch=len(last), num_qo_heads=hq, num_kv_heads=hkv, page_size=P,
                           dtype="f16", sm_scale=0.1, num_sms=sms, ctas_per_sm=k,
-                          min_chunk_tokens=mct, num_pages=1 << 20)
+                          min_chunk_tokens=mct, num_pages=1 << 20,
+                          piece_cost_tokens=c if c > 0 else -1)
     plan = C.pa_plan_create(prob, indptr, last)
     q, items, ci, mi = oracle.plan(indptr, last, page_size=P, num_kv_heads=hkv, num_sms=sms,
-                                   ctas_per_sm=k, min_chunk_tokens=mct if mct else 256)
+                                   ctas_per_sm=k, min_chunk_tokens=mct if mct else 256,
+                                   piece_cost=c)
     assert C.pa_plan_quota_tokens(plan) == q
     assert np.array_equal(C.pa_plan_work_items(plan), items)
     assert np.array_equal(C.pa_plan_cta_indptr(plan), ci)
@@ -67,19 +69,21 @@ def test_plan_matches_oracle_bit_exact(C, seed):
     hkv = int(rng.choice([1, 2, 4, 8]))
     g = int(rng.choice([1, 2, 4, 8]))
     _compare_plan(C, indptr, last, P, hkv * g, hkv, int(rng.integers(1, 300)),
-                  int(rng.integers(1, 5)), int(rng.choice([0, 1, 100, 512])))
+                  int(rng.integers(1, 5)), int(rng.choice([0, 1, 100, 512])),
+                  int(rng.choice([0, 1, 37, 160, 256, 1000])))
 
 
+@pytest.mark.parametrize("c", [0, 160, 256])
 @pytest.mark.parametrize("n", [1, 2, 3, 5, "4c"])
-def test_plan_matches_oracle_on_benchmark_workloads(C, n):
+def test_plan_matches_oracle_on_benchmark_workloads(C, n, c):
     w = W.WORKLOADS[n]()
     _compare_plan(C, w.kv_indptr, w.last_page_len, w.page_size, w.num_qo_heads, w.num_kv_heads,
-                  148, 3, 0)
+                  148, 3, 0, c)
 
 
 def test_plan_matches_oracle_vector_sparse(C):
     w = W.WORKLOADS[4]()
-    _compare_plan(C, w.kv_indptr, w.last_page_len, 1, 64, 8, 148, 3, 0)
+    _compare_plan(C, w.kv_indptr, w.last_page_len, 1, 64, 8, 148, 1, 0, 256)
 
 
 def test_plan_edge_cases(C):
@@ -87,7 +91,8 @@ def test_plan_edge_cases(C):
     for lens, P, sms in [([], 16, 148), ([0, 0], 16, 148), ([1], 16, 148), ([16, 32, 48], 16, 148),
                          ([100] * 50, 16, 2), ([3000, 1], 1, 1), ([0, 5000, 0], 16, 3)]:
         indptr, _, last = W.tables_from_lengths(lens, P)
-        _compare_plan(C, indptr, last, P, 8, 8, sms, 1, 0)
+        for c in (0, 160):
+            _compare_plan(C, indptr, last, P, 8, 8, sms, 1, 0, c)
 
 
 def test_plan_validation(C):
@@ -160,7 +165,7 @@ def test_cascade_plan_shape(C):
     n, tok = C.pa_plan_prefix_chunks(plan)
     assert n >= 1 and tok % 128 == 0 and n * tok >= w.prefix_len > (n - 1) * tok
     q, items, ci, mi = oracle.plan(w.kv_indptr, w.last_page_len, page_size=16, num_kv_heads=8,
-                                   num_sms=148, ctas_per_sm=2)
+                                   num_sms=148, ctas_per_sm=2, piece_cost=400)
     assert np.array_equal(C.pa_plan_work_items(plan), items)
     assert np.array_equal(C.pa_plan_cta_indptr(plan), ci)
 
@@ -181,3 +186,18 @@ def test_decode_kernel_choice(C):
                               ctas_per_sm=1, num_pages=w.num_pages, flags=flags)
         plan = C.pa_plan_create(prob, w.kv_indptr, w.last_page_len)
         assert C.pa_plan_uses_tensor_cores(plan) is expect, (group, flags)
+
+
+def test_default_piece_cost_follows_the_kernel(C):
+    """piece_cost_tokens = 0 takes the default of the decode kernel the plan
+    runs: 400 tokens for the CUDA-core kernel, 128 for the tensor-core one."""
+    w = W.WORKLOADS[3]()
+    for flags, c in ((0, 400), (C.PA_FLAG_TENSOR_CORES, 128)):
+        base = dict(batch=w.batch, num_qo_heads=w.num_qo_heads, num_kv_heads=w.num_kv_heads,
+                    page_size=w.page_size, dtype=w.dtype, sm_scale=w.sm_scale, num_sms=148,
+                    ctas_per_sm=2, num_pages=w.num_pages, flags=flags)
+        default = C.pa_plan_create(C.make_problem(**base), w.kv_indptr, w.last_page_len)
+        explicit = C.pa_plan_create(C.make_problem(piece_cost_tokens=c, **base), w.kv_indptr,
+                                    w.last_page_len)
+        assert np.array_equal(C.pa_plan_work_items(default), C.pa_plan_work_items(explicit))
+        assert C.pa_plan_quota_tokens(default) == C.pa_plan_quota_tokens(explicit)

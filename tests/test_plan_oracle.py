@@ -25,7 +25,7 @@ def test_plan_hand_worked_examples():
         q, items, cta_indptr, merge_indptr = oracle.plan(
             g["kv_indptr"], g["last_page_len"], page_size=g["page_size"],
             num_kv_heads=g["num_kv_heads"], num_sms=g["num_sms"], ctas_per_sm=g["ctas_per_sm"],
-            min_chunk_tokens=g["min_chunk_tokens"])
+            min_chunk_tokens=g["min_chunk_tokens"], piece_cost=g.get("piece_cost_tokens", 0))
         assert q == g["quota"]
         assert cta_indptr.tolist() == g["cta_indptr"]
         assert merge_indptr.tolist() == g["merge_indptr"]
@@ -33,19 +33,22 @@ def test_plan_hand_worked_examples():
 
 
 def check_plan_properties(indptr, last, P, hkv, W_, min_tokens, q, items, cta_indptr,
-                          merge_indptr):
+                          merge_indptr, c=0):
     indptr = np.asarray(indptr, np.int64)
     last = np.asarray(last, np.int64)
     B = len(last)
     n = np.diff(indptr)
     lens = np.where(n > 0, (n - 1) * P + last, 0)
     T = int(lens.sum())
+    N = int((lens > 0).sum())
     groups = max(1, W_ // hkv)
-    share = max(min_tokens, -(-T // groups))
+    share = max(min_tokens, -(-(T + c * max(N - 1, 0)) // groups))
     assert q % 32 == 0 and share <= q < share + 32
     n_cta = len(cta_indptr) - 1
-    n_groups = 0 if B == 0 else max(1, -(-T // q))
-    assert n_cta == n_groups * hkv
+    n_groups = n_cta // hkv
+    assert n_cta == n_groups * hkv and n_groups <= groups  # one wave: every CTA resident
+    if c == 0:
+        assert n_groups == (0 if B == 0 else max(1, -(-T // q)))
     assert cta_indptr[0] == 0 and cta_indptr[-1] == len(items)
     assert all(cta_indptr[i] <= cta_indptr[i + 1] for i in range(n_cta))
     cta = [items[cta_indptr[i]:cta_indptr[i + 1]] for i in range(n_cta)]
@@ -58,10 +61,11 @@ def check_plan_properties(indptr, last, P, hkv, W_, min_tokens, q, items, cta_in
             ranges = r if ranges is None else ranges
             assert r == ranges  # the Hkv CTAs of a group read the same tokens
         tokens = sum(t1 - t0 for _, t0, t1 in ranges)
+        used = tokens + c * max(sum(1 for _, t0, t1 in ranges if t1 > t0) - 1, 0)
+        assert used <= q  # the budget holds
         if g < n_groups - 1:
-            assert tokens == q  # balance: every group but the last reads exactly q tokens
-        else:
-            assert 0 <= tokens <= q
+            # balance: a group closes only when the next token would not fit
+            assert used + c >= q and (c > 0 or tokens == q)
     # coverage: per (b, h) the pieces tile [0, L_b) in token order
     for b in range(B):
         for h in range(hkv):
@@ -79,8 +83,9 @@ def check_plan_properties(indptr, last, P, hkv, W_, min_tokens, q, items, cta_in
                                             list(range(merge_indptr[seg], merge_indptr[seg + 1])))
 
 
+@pytest.mark.parametrize("c", [0, 37, 160])
 @pytest.mark.parametrize("seed", range(12))
-def test_plan_properties_random(seed):
+def test_plan_properties_random(seed, c):
     rng = np.random.default_rng(seed)
     B = int(rng.integers(0, 40))
     P = int(rng.choice([1, 2, 16, 64]))
@@ -90,8 +95,8 @@ def test_plan_properties_random(seed):
     sms, k = int(rng.integers(1, 200)), int(rng.integers(1, 4))
     mct = int(rng.choice([1, 64, 256, 1000]))
     q, items, ci, mi = oracle.plan(indptr, last, page_size=P, num_kv_heads=hkv, num_sms=sms,
-                                   ctas_per_sm=k, min_chunk_tokens=mct)
-    check_plan_properties(indptr, last, P, hkv, sms * k, mct, q, items, ci, mi)
+                                   ctas_per_sm=k, min_chunk_tokens=mct, piece_cost=c)
+    check_plan_properties(indptr, last, P, hkv, sms * k, mct, q, items, ci, mi, c)
 
 
 def test_plan_empty_batch():
@@ -101,10 +106,32 @@ def test_plan_empty_batch():
     assert q == 256
 
 
-def test_plan_benchmark_shapes():
+@pytest.mark.parametrize("c", [0, 160, 256])
+def test_plan_benchmark_shapes(c):
     for n in (1, 2, 3):
         w = W.WORKLOADS[n]()
         q, items, ci, mi = oracle.plan(w.kv_indptr, w.last_page_len, page_size=w.page_size,
-                                       num_kv_heads=w.num_kv_heads, num_sms=148, ctas_per_sm=4)
+                                       num_kv_heads=w.num_kv_heads, num_sms=148, ctas_per_sm=4,
+                                       piece_cost=c)
         check_plan_properties(w.kv_indptr, w.last_page_len, w.page_size, w.num_kv_heads, 592,
-                              256, q, items, ci, mi)
+                              256, q, items, ci, mi, c)
+
+
+def test_piece_cost_shifts_tokens_to_single_piece_groups():
+    """With a piece cost c, a group of k pieces reads between q - c k and
+    q - c (k - 1) tokens (it closes once the next piece would not fit), so a
+    two-piece group reads about c fewer tokens than a one-piece group
+    (uniform batch: 16 x 4096 tokens)."""
+    w = W.WORKLOADS[2]()
+    for c in (160, 256):
+        q, items, ci, _ = oracle.plan(w.kv_indptr, w.last_page_len, page_size=16, num_kv_heads=8,
+                                      num_sms=148, ctas_per_sm=3, piece_cost=c)
+        groups = [items[ci[g * 8]:ci[g * 8 + 1]] for g in range((len(ci) - 1) // 8)]
+        by_k = {}
+        for pcs in groups[:-1]:
+            k = len(pcs)
+            tok = int((pcs[:, 4] - pcs[:, 3]).sum())
+            assert q - c * k <= tok <= q - c * (k - 1)
+            by_k.setdefault(k, []).append(tok)
+        assert set(by_k) == {1, 2}
+        assert np.mean(by_k[1]) - np.mean(by_k[2]) > c / 2
