@@ -77,6 +77,21 @@ def test_sharp_softmax_moves_the_running_max(dtype, group, sm_scale, kernel):
                      f"sharp G={group} scale={sm_scale} {kernel} {kw}")
 
 
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+@pytest.mark.parametrize("cost", [-1, 1, 1000])
+def test_piece_cost_plans(kernel, cost):
+    """Plans with no piece cost, a tiny one and a huge one (many short
+    pieces, many split segments) give the same attention."""
+    w = W.make_workload("cost", [0, 3, 700, 5000, 1, 129, 2000], num_qo_heads=16,
+                        num_kv_heads=2, page_size=16, dtype="bf16", seed=120)
+    t = w.materialize()
+    o_ref, l_ref = oracle_full(w, t)
+    dev = _to_dev(t)
+    pd, o, lse = _decode(w, dev, num_sms=7, ctas_per_sm=1, min_chunk_tokens=32,
+                         flags=KERNELS[kernel], piece_cost_tokens=cost)
+    assert_close(to_np(o), to_np(lse), o_ref, l_ref, "bf16", f"{kernel} cost={cost}")
+
+
 @pytest.mark.parametrize("group", [4, 8])
 def test_tensor_core_and_cuda_core_kernels_agree(group):
     """The two decode kernels on the same plan shape agree to rounding."""
