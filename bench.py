@@ -50,7 +50,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="2", help="1 2 3 4 4c 5 (default: 2)")
+    ap.add_argument("--workload", default="2", help="1 2 3 4 4c 4s 5 (default: 2)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="untimed run-in after warm-up so clocks settle and get sampled")

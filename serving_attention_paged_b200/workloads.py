@@ -359,6 +359,19 @@ def vector_sparse_decode(seed=1004, pool_tokens=1 << 21) -> PagedWorkload:
                          last_page_len=last)
 
 
+def vector_sparse_small(seed=1004, batch=48, pool_tokens=1 << 19) -> PagedWorkload:
+    """The first 48 requests of ``vector_sparse_decode`` (same length draws,
+    GQA 64/8, P=1, bf16) in a 512K-token pool: small enough (2 x 1 GB pools)
+    for a full counter capture of one launch."""
+    lens = vector_sparse_lengths(seed, batch)
+    order = permutation(stream_key(seed, STREAM_PERM), pool_tokens)
+    indptr, indices, last = tables_from_lengths(lens, 1, order)
+    return PagedWorkload(name="vector_sparse_small", batch=len(lens), num_qo_heads=64,
+                         num_kv_heads=8, head_dim=128, page_size=1, dtype="bf16", seed=seed,
+                         num_pages=pool_tokens, kv_indptr=indptr, kv_indices=indices,
+                         last_page_len=last)
+
+
 def vector_sparse_contiguous_twin(seed=1004) -> PagedWorkload:
     """The same requests and token values as ``vector_sparse_decode`` with
     P=16 and each request's pages contiguous and ascending in the pool."""
@@ -388,4 +401,5 @@ WORKLOADS = {
     4: vector_sparse_decode,
     5: cascade_shared_prefix,
     "4c": vector_sparse_contiguous_twin,
+    "4s": vector_sparse_small,
 }
