@@ -56,7 +56,7 @@ def test_small_parity(dtype, group, P, kernel):
                      f"G={group} P={P} {kernel} {kw}")
 
 
-@pytest.mark.parametrize("kernel", ["auto", "cuda_cores"])
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("group", [4, 8])
 @pytest.mark.parametrize("sm_scale", [1.0, 3.0])
@@ -98,7 +98,7 @@ def test_tensor_core_and_cuda_core_kernels_agree(group):
     w = W.make_workload("agree", [4096, 3000, 17, 0, 1200], num_qo_heads=4 * group,
                         num_kv_heads=4, page_size=16, dtype="bf16", seed=95 + group)
     dev = _to_dev(w.materialize())
-    _, o_tc, l_tc = _decode(w, dev, num_sms=148, ctas_per_sm=1)
+    _, o_tc, l_tc = _decode(w, dev, num_sms=148, ctas_per_sm=1, flags=KERNELS["tensor_cores"])
     _, o_cc, l_cc = _decode(w, dev, num_sms=148, ctas_per_sm=1, flags=KERNELS["cuda_cores"])
     assert (o_tc.float() - o_cc.float()).abs().max().item() <= 2 * 2e-3
     fin = torch.isfinite(l_cc)
@@ -106,13 +106,14 @@ def test_tensor_core_and_cuda_core_kernels_agree(group):
     assert (l_tc[fin] - l_cc[fin]).abs().max().item() <= 2e-3
 
 
-def test_split_chunks_are_exercised():
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+def test_split_chunks_are_exercised(kernel):
     w = W.make_workload("split", [5000, 3, 700], num_qo_heads=32, num_kv_heads=8, page_size=16,
                         dtype="bf16", seed=5)
     t = w.materialize()
     o_ref, l_ref = oracle_full(w, t)
     dev = _to_dev(t)
-    pd, o, lse = _decode(w, dev, num_sms=148, ctas_per_sm=2)
+    pd, o, lse = _decode(w, dev, num_sms=148, ctas_per_sm=2, flags=KERNELS[kernel])
     items = pd.work_items()
     assert (items[:, 5] >= 0).any()  # some requests really were split
     assert_close(to_np(o), to_np(lse), o_ref, l_ref, "bf16", "split")
@@ -153,12 +154,13 @@ def test_page_permutation_invariance_gpu():
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
-def test_cuda_graph_replay():
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+def test_cuda_graph_replay(kernel):
     w = W.make_workload("graph", [4000, 50, 2000, 9], num_qo_heads=32, num_kv_heads=8,
                         page_size=16, dtype="f16", seed=9)
     t = w.materialize()
     dev = _to_dev(t)
-    pd, o_eager, l_eager = _decode(w, dev, num_sms=148, ctas_per_sm=2)
+    pd, o_eager, l_eager = _decode(w, dev, num_sms=148, ctas_per_sm=2, flags=KERNELS[kernel])
     o = torch.zeros_like(o_eager)
     lse = torch.zeros_like(l_eager)
     s = torch.cuda.Stream()
@@ -173,7 +175,7 @@ def test_cuda_graph_replay():
         assert torch.equal(o, o_eager) and torch.equal(lse, l_eager)
 
 
-@pytest.mark.parametrize("kernel", ["auto", "cuda_cores"])
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
 def test_bounds_checked_run_reports_bad_index(kernel):
     from serving_attention_paged_b200 import pagedattn as C
     w = W.make_workload("chk", [40, 40], num_qo_heads=8, num_kv_heads=2, page_size=16,
