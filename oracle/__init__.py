@@ -13,6 +13,8 @@ single-request decode usage example) and the flashinfer-cubin registry page
 * ``merge_state`` / ``merge_states`` — combining attention states by their
   log-sum-exp (what split-KV and cascade attention rely on).
 * ``cascade_decode`` — shared prefix merged with per-request suffix.
+* ``paged_prefill`` — causal attention of new (appended) query tokens over
+  the paged KV (README usage example: prefill / append attention).
 * ``plan`` — the split-KV work-list specification restated with plain
   loops (the library's work list must agree with it exactly).
 
@@ -193,6 +195,54 @@ def cascade_decode(q, k_pool, v_pool, prefix_indices, prefix_len, kv_indptr, kv_
     return merge_state(o1, l1, o2, l2)
 
 
+def paged_prefill(q, k_pool, v_pool, qo_indptr, kv_indptr, kv_indices, last_page_len, *,
+                  num_qo_heads, num_kv_heads, head_dim, page_size, dtype, sm_scale,
+                  queries=None, threads=1):
+    """Prefill / append attention (README usage example: prefill and append
+    attention over a paged KV cache, causal).
+
+    Request b has L_b keys (its page table) of which its Q_b new query tokens
+    are the last Q_b (qo_indptr[b + 1] - qo_indptr[b] = Q_b <= L_b).  Query i
+    (0-based) of request b attends causally to keys t < L_b - Q_b + i + 1.
+    That is exactly a decode over the request's pages cut at that limit, so
+    each query becomes one row of ``paged_decode`` with its own page list.
+
+    q is ``[total_q, Hq, D]``.  Returns o ``[n, Hq, D]`` and lse ``[n, Hq]``
+    for every query (``queries=None``) or the listed global query indices.
+    """
+    qo = [int(x) for x in _as_i32(qo_indptr)]
+    indptr = [int(x) for x in _as_i32(kv_indptr)]
+    indices = _as_i32(kv_indices)
+    last = [int(x) for x in _as_i32(last_page_len)]
+    B, P = len(last), page_size
+    owner = []
+    for b in range(B):
+        n = indptr[b + 1] - indptr[b]
+        L = (n - 1) * P + last[b] if n > 0 else 0
+        Q = qo[b + 1] - qo[b]
+        if Q > L:
+            raise ValueError(f"request {b}: {Q} queries but only {L} keys")
+        owner += [(b, L, Q, i) for i in range(Q)]
+    sel = list(range(len(owner))) if queries is None else [int(x) for x in queries]
+    q_indptr, q_indices, q_last = [0], [], []
+    for g in sel:
+        b, L, Q, i = owner[g]
+        lim = L - Q + i + 1
+        n = -(-lim // P)
+        q_indices.extend(indices[indptr[b]:indptr[b] + n].tolist())
+        q_indptr.append(len(q_indices))
+        q_last.append(lim - (n - 1) * P)
+    if hasattr(q, "detach"):
+        import torch
+        qs = q[torch.as_tensor(sel, dtype=torch.int64, device=q.device)].cpu()
+        kp, vp = k_pool.cpu(), v_pool.cpu()
+    else:
+        qs, kp, vp = np.asarray(q)[sel], k_pool, v_pool
+    return paged_decode(qs, kp, vp, q_indptr, q_indices, q_last, num_qo_heads=num_qo_heads,
+                        num_kv_heads=num_kv_heads, head_dim=head_dim, page_size=page_size,
+                        dtype=dtype, sm_scale=sm_scale, threads=threads)
+
+
 def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per_sm,
          min_chunk_tokens=256, piece_cost=0):
     """Split-KV work list (FlashInfer README core feature 2: variable-length
@@ -297,4 +347,4 @@ def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per
 
 
 __all__ = ["build_library", "paged_decode", "paged_decode_requests", "merge_state", "merge_states", "cascade_decode",
-           "plan", "widen"]
+           "paged_prefill", "plan", "widen"]

@@ -151,6 +151,7 @@ class PagedWorkload:
     sm_scale: float = 0.0
     prefix_len: int = 0
     prefix_indices: Optional[np.ndarray] = None
+    qo_lens: Optional[np.ndarray] = None  # prefill / append: new tokens per request
     extra: dict = field(default_factory=dict)
 
     def __post_init__(self):
@@ -161,6 +162,8 @@ class PagedWorkload:
         self.last_page_len = np.ascontiguousarray(self.last_page_len, dtype=np.int32)
         if self.prefix_indices is not None:
             self.prefix_indices = np.ascontiguousarray(self.prefix_indices, dtype=np.int32)
+        if self.qo_lens is not None:
+            self.qo_lens = np.ascontiguousarray(self.qo_lens, dtype=np.int64)
 
     # -- derived sizes -------------------------------------------------------
     @property
@@ -216,11 +219,32 @@ class PagedWorkload:
             parts.append(pages[t // P] * P + t % P)
         return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
 
+    @property
+    def qo_indptr(self) -> Optional[np.ndarray]:
+        """Prefill / append: query-token offsets per request (int32 [B+1])."""
+        if self.qo_lens is None:
+            return None
+        ind = np.zeros(self.batch + 1, dtype=np.int64)
+        ind[1:] = np.cumsum(self.qo_lens)
+        return ind.astype(np.int32)
+
+    def query_rows(self) -> int:
+        """q rows: one per request for decode, one per new token for prefill."""
+        return self.batch if self.qo_lens is None else int(self.qo_lens.sum())
+
+    def prefill_flops(self) -> int:
+        """Causal attention flops of a prefill step (4 per query-key pair and element)."""
+        lens = self.kv_lens()
+        pairs = sum(int(Q) * int(L - Q) + int(Q) * (int(Q) + 1) // 2
+                    for Q, L in zip(self.qo_lens, lens))
+        return 4 * pairs * self.num_qo_heads * self.head_dim
+
     # -- tensors ---------------------------------------------------------------
     def make_q(self, device="cpu") -> torch.Tensor:
-        n = self.batch * self.num_qo_heads * self.head_dim
+        rows = self.query_rows()
+        n = rows * self.num_qo_heads * self.head_dim
         q = normal_as(stream_key(self.seed, STREAM_Q), 0, n, self.dtype, device)
-        return q.view(self.batch, self.num_qo_heads, self.head_dim)
+        return q.view(rows, self.num_qo_heads, self.head_dim)
 
     def make_pool(self, which: str, device="cpu", chunk_tokens: int = 1 << 15,
                   rows: Optional[np.ndarray] = None) -> torch.Tensor:
@@ -289,7 +313,7 @@ def tables_from_lengths(lens, page_size: int, page_order: Optional[np.ndarray] =
 
 def make_workload(name, lens, *, num_qo_heads, num_kv_heads, head_dim=128, page_size=16,
                   dtype="f16", seed=0, shuffle=True, extra_pages=0, prefix_len=0,
-                  sm_scale=0.0) -> PagedWorkload:
+                  sm_scale=0.0, qo_lens=None) -> PagedWorkload:
     """A paged problem whose pool holds exactly the pages used (+ ``extra_pages``).
 
     ``shuffle`` places every page at a random pool position (one permutation
@@ -310,7 +334,7 @@ def make_workload(name, lens, *, num_qo_heads, num_kv_heads, head_dim=128, page_
                          num_kv_heads=num_kv_heads, head_dim=head_dim, page_size=page_size,
                          dtype=dtype, seed=seed, num_pages=num_pages, kv_indptr=indptr,
                          kv_indices=indices, last_page_len=last, prefix_len=prefix_len,
-                         prefix_indices=prefix_indices, sm_scale=sm_scale)
+                         prefix_indices=prefix_indices, sm_scale=sm_scale, qo_lens=qo_lens)
 
 
 # ---------------------------------------------------------------------------
@@ -394,6 +418,13 @@ def cascade_shared_prefix(seed=1005, prefix_len=16384) -> PagedWorkload:
                          prefix_len=prefix_len)
 
 
+def prefill_append(seed=1006) -> PagedWorkload:
+    """B=8 requests appending 1024 new tokens to 1024 cached ones (kv_len 2048,
+    causal), GQA 32/8, P=16, fp16, shuffled exact pool."""
+    return make_workload("prefill_append", [2048] * 8, num_qo_heads=32, num_kv_heads=8,
+                         page_size=16, dtype="f16", seed=seed, qo_lens=[1024] * 8)
+
+
 WORKLOADS = {
     1: single_request_decode,
     2: batch_decode_uniform,
@@ -402,4 +433,5 @@ WORKLOADS = {
     5: cascade_shared_prefix,
     "4c": vector_sparse_contiguous_twin,
     "4s": vector_sparse_small,
+    6: prefill_append,
 }

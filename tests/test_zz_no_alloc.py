@@ -19,20 +19,24 @@ from serving_attention_paged_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def _problem(C, w, num_sms=148, ctas_per_sm=3):
+def _problem(C, w, num_sms=148, ctas_per_sm=3, flags=0):
     return C.make_problem(batch=w.batch, num_qo_heads=w.num_qo_heads,
                           num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
                           sm_scale=w.sm_scale, num_sms=num_sms, ctas_per_sm=ctas_per_sm,
-                          num_pages=w.num_pages)
+                          num_pages=w.num_pages, flags=flags)
 
 
-def test_static_workspace_matches_caller_workspace_twice():
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+def test_static_workspace_matches_caller_workspace_twice(kernel):
     from serving_attention_paged_b200 import pagedattn as C
     lens = [3000, 0, 17, 900, 4096, 1]
     w = W.make_workload("static_ws", lens, num_qo_heads=32, num_kv_heads=8, page_size=16,
                         dtype="bf16", seed=91)
     dev = {k: v.cuda() for k, v in w.materialize().items()}
-    plan = C.pa_plan_create(_problem(C, w), w.kv_indptr, w.last_page_len)
+    flags = C.PA_FLAG_TENSOR_CORES if kernel == "tensor_cores" else C.PA_FLAG_CUDA_CORES
+    plan = C.pa_plan_create(_problem(C, w, ctas_per_sm=1 if kernel == "tensor_cores" else 3,
+                                     flags=flags), w.kv_indptr, w.last_page_len)
+    assert C.pa_plan_uses_tensor_cores(plan) == (kernel == "tensor_cores")
     assert C.pa_plan_num_partials(plan) > 0  # the split path (partials, counters) is exercised
     nbytes = C.pa_plan_workspace_bytes(plan)
     ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
