@@ -42,6 +42,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode: effective KV HBM GB/s and % of B200 peak; µs per decode step"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -50,7 +51,8 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="2", help="1 2 3 4 4c 4s 5 (default: 2)")
+    ap.add_argument("--workload", default="2",
+                    help="1 2 3 4 4c 4s 5 (decode), 6 (prefill / append); default: 2")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="untimed run-in after warm-up so clocks settle and get sampled")
@@ -216,6 +218,9 @@ def run_reference(args):
         return
     import oracle
     w = workload(args.workload)
+    if w.qo_lens is not None:
+        run_reference_prefill(args, w)
+        return
     # a bounded sample: the first request(s), drawn on the host
     n_req = 1
     lens = w.kv_lens()
@@ -257,58 +262,56 @@ def run_reference(args):
                 "d2h_bytes_per_step": 0}}))
 
 
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device")
-    torch.cuda.set_device(local)
-    dev_t = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", device_id=dev_t,
-                                timeout=datetime.timedelta(seconds=120))
-
-    from serving_attention_paged_b200 import build
-    if rank == 0 or world == 1:
-        build.build()
-    if world > 1:
-        dist.barrier()
-    from serving_attention_paged_b200 import pagedattn as C
-    from serving_attention_paged_b200.wrapper import PagedDecode
-
-    w = workload(args.workload)
-    dev = w.materialize(dev_t)
-    stream = torch.cuda.current_stream(dev_t)
-    t0 = time.perf_counter()
-    pd = PagedDecode(w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
-                     num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
-                     sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
-                     device=dev_t, min_chunk_tokens=args.min_chunk_tokens,
-                     ctas_per_sm=args.ctas_per_sm or None,
-                     flags={"auto": 0, "cuda_cores": C.PA_FLAG_CUDA_CORES,
-                            "tensor_cores": C.PA_FLAG_TENSOR_CORES}[args.kernel],
-                     piece_cost_tokens=args.piece_cost_tokens)
-    tensor_cores = C.pa_plan_uses_tensor_cores(pd.plan)
-    setup_us = (time.perf_counter() - t0) * 1e6
-    reps = 20
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        (C.pa_cascade_plan_create(pd.problem, w.prefix_len, w.kv_indptr, w.last_page_len)
-         if w.prefix_len else C.pa_plan_create(pd.problem, w.kv_indptr, w.last_page_len))
-    plan_us = (time.perf_counter() - t0) * 1e6 / reps
-    o, lse = pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"],
-                    prefix_indices=dev.get("prefix_indices"))
-    launches_per_step = 2 if (w.prefix_len and w.batch) else 1
+def run_reference_prefill(args, w):
+    """Reference arm for prefill: the oracle on every 16th new token of the
+    first request, drawn on the host."""
+    import oracle
+    from serving_attention_paged_b200 import workloads as W
+    lens = w.kv_lens()
+    sub = W.make_workload(w.name, lens[:1], num_qo_heads=w.num_qo_heads,
+                          num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                          page_size=w.page_size, dtype=w.dtype, seed=w.seed,
+                          qo_lens=w.qo_lens[:1])
+    t = sub.materialize()
+    sel = np.arange(0, sub.query_rows(), 16)
+    threads = os.cpu_count() or 1
 
     def step():
-        pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"], o, lse,
-               prefix_indices=dev.get("prefix_indices"), stream=stream)
+        oracle.paged_prefill(t["q"], t["k_pool"], t["v_pool"], sub.qo_indptr, sub.kv_indptr,
+                             sub.kv_indices, sub.last_page_len, num_qo_heads=sub.num_qo_heads,
+                             num_kv_heads=sub.num_kv_heads, head_dim=sub.head_dim,
+                             page_size=sub.page_size, dtype=sub.dtype, sm_scale=sub.sm_scale,
+                             queries=sel, threads=threads)
 
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    flops = prefill_query_flops(sub, sel)
+    value = flops / sec / 1e12
+    sample = (f"every 16th new token of request 0 ({len(sel)} of {w.query_rows()} tokens, all "
+              f"{w.num_qo_heads} q heads), {flops / 1e9:.2f} GFLOP per step, fp64")
+    print(json.dumps({
+        "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "batch": w.batch,
+                                        "num_qo_heads": w.num_qo_heads,
+                                        "num_kv_heads": w.num_kv_heads, "causal": True},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}))
+
+def make_l2_flush(dev_t):
+    """A 256 MB write, then a 256 MB read of another buffer so the dirty lines
+    of that write are written back too (both outside the timed events)."""
+    import torch
     flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev_t)
     flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev_t)
     flush_sink = torch.empty((), dtype=torch.float32, device=dev_t)
@@ -317,6 +320,16 @@ def run_ours(args):
         flush_w.fill_(1.0)                       # evicts the inputs ...
         torch.sum(flush_r, dim=0, out=flush_sink)  # ... and the dirty lines of that write
 
+    return flush_l2
+
+
+def timed_steps(step, flush_l2, args, stream, dev_t, world):
+    """W warm-up steps, an untimed soak while the clocks are sampled, then K
+    steps each bracketed by CUDA events on the launching stream (L2 flushed
+    before each, outside the events).  Returns the max-over-ranks mean step
+    time (ms), this rank's step times and the clock record."""
+    import torch
+    import torch.distributed as dist
     for _ in range(max(args.warmup, 3)):
         flush_l2()
         step()
@@ -348,8 +361,207 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    step_ms = [st.elapsed_time(en) for st, en in zip(starts, ends)]
     ms = max_over_ranks(sum(step_ms) / len(step_ms), dev_t)
+    return ms, step_ms, clocks
+
+
+PREFILL_METRIC = ("paged prefill / append (causal): attention TFLOP/s and % of B200 dense "
+                  "tensor peak; µs per step")
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(path))["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def prefill_cpu_baseline(w, dev, stride):
+    """The oracle as it stands, on the host cores, over every ``stride``-th new
+    token of the workload (all q heads)."""
+    import oracle
+    threads = os.cpu_count() or 1
+    sel = np.arange(0, w.query_rows(), stride)
+    t0 = time.perf_counter()
+    oracle.paged_prefill(dev["q"], dev["k_pool"], dev["v_pool"], w.qo_indptr, w.kv_indptr,
+                         w.kv_indices, w.last_page_len, num_qo_heads=w.num_qo_heads,
+                         num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                         page_size=w.page_size, dtype=w.dtype, sm_scale=w.sm_scale,
+                         queries=sel, threads=threads)
+    dt = time.perf_counter() - t0
+    flops = prefill_query_flops(w, sel)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"every {stride}th new token ({len(sel)} of {w.query_rows()}, all "
+                      f"{w.num_qo_heads} q heads), {flops / 1e9:.2f} GFLOP, {dt:.2f} s, fp64"}
+
+
+def prefill_query_flops(w, queries):
+    """Attention flops of the listed new tokens (4 per visible key and element)."""
+    qo, lens = w.qo_indptr, w.kv_lens()
+    b = np.searchsorted(qo, queries, side="right") - 1
+    i = queries - qo[b]
+    visible = lens[b] - (qo[b + 1] - qo[b]) + i + 1
+    return int(4 * visible.sum() * w.num_qo_heads * w.head_dim)
+
+
+def run_prefill(args, w, dev, stream, dev_t, world, rank):
+    """Prefill / append step: one pa_prefill_run launch over all new tokens."""
+    import torch
+    from serving_attention_paged_b200 import pagedattn as C
+    from serving_attention_paged_b200.wrapper import PagedPrefill
+    t0 = time.perf_counter()
+    pf = PagedPrefill(w.qo_indptr, w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
+                      num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
+                      sm_scale=w.sm_scale, num_pages=w.num_pages, causal=True, device=dev_t)
+    setup_us = (time.perf_counter() - t0) * 1e6
+    reps = 20
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        C.pa_prefill_plan_create(pf.problem, True, w.qo_indptr, w.kv_indptr, w.last_page_len)
+    plan_us = (time.perf_counter() - t0) * 1e6 / reps
+    o, lse = pf.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"])
+
+    def step():
+        pf.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"], o, lse, stream=stream)
+
+    flush_l2 = make_l2_flush(dev_t)
+    ms, step_ms, clocks = timed_steps(step, flush_l2, args, stream, dev_t, world)
+    flops = w.prefill_flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+    traffic = profiled_traffic(["serving_attention_paged_b200/csrc/prefill.cu",
+                                "serving_attention_paged_b200/csrc/common.cuh"], w.name)
+
+    e2e = None
+    if not args.no_e2e:
+        q_h = dev["q"].cpu().pin_memory()
+        idx_h = dev["kv_indices"].cpu().pin_memory()
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        q_d = torch.empty_like(dev["q"])
+        idx_d = torch.empty_like(dev["kv_indices"])
+        e2e_s = []
+        for i in range(max(args.warmup, 3) + args.steps):
+            flush_l2()
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            plan = C.pa_prefill_plan_create(pf.problem, True, w.qo_indptr, w.kv_indptr,
+                                            w.last_page_len)
+            C.pa_plan_upload(plan, pf.workspace, pf.workspace.numel(), stream)
+            q_d.copy_(q_h, non_blocking=True)
+            idx_d.copy_(idx_h, non_blocking=True)
+            C.pa_prefill_run(plan, q_d, dev["k_pool"], dev["v_pool"], idx_d, o, lse,
+                             pf.workspace, pf.workspace.numel(), stream)
+            o_h.copy_(o, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+            torch.cuda.synchronize()
+            if i >= max(args.warmup, 3):
+                e2e_s.append(time.perf_counter() - t0)
+        e2e_max = max_over_ranks(sum(e2e_s) / len(e2e_s), dev_t)
+        h2d = q_h.numel() * q_h.element_size() + idx_h.numel() * 4 + len(pf.tiles()) * 24
+        e2e = {"value": world * flops / e2e_max / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(o_h.numel() * o_h.element_size() + lse_h.numel() * 4),
+               "us_per_step": e2e_max * 1e6,
+               "includes": "host plan + tile upload + q/kv_indices H2D + run + o/lse D2H"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = prefill_cpu_baseline(w, dev, stride=8)
+
+    if rank == 0:
+        lens = w.kv_lens()
+        cfg = {"workload": w.name, "batch": w.batch, "num_qo_heads": w.num_qo_heads,
+               "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+               "page_size": w.page_size, "kv_dtype": w.dtype, "accumulate": "f32",
+               "kv_len": int(lens[0]) if len(set(lens.tolist())) == 1 else int(lens.sum()),
+               "qo_len": int(w.qo_lens[0]) if len(set(w.qo_lens.tolist())) == 1
+               else int(w.qo_lens.sum()),
+               "causal": True, "flops_per_step": flops, "pool_pages": w.num_pages,
+               "l2": "flushed before every timed step: 256 MB write, then a 256 MB read of "
+                     "another buffer (both untimed)",
+               "parallelism": f"replicas x{world}"}
+        print(json.dumps({
+            "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "us_per_step": ms * 1e3, "pct_of_peak": 100.0 * achieved / peak,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))",
+            "config": cfg,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind + " (bf16 cuBLAS burst; fp16 has the same "
+                                                  "nominal dense rate)",
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "paged_prefill_kernel"},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": args.steps,
+            "plan_us": plan_us, "setup_us": setup_us,
+            "step_ms_p10_p50_p90": [float(np.percentile(step_ms, p)) for p in (10, 50, 90)],
+        }))
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev_t = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev_t,
+                                timeout=datetime.timedelta(seconds=120))
+
+    from serving_attention_paged_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    from serving_attention_paged_b200 import pagedattn as C
+    from serving_attention_paged_b200.wrapper import PagedDecode
+
+    w = workload(args.workload)
+    dev = w.materialize(dev_t)
+    stream = torch.cuda.current_stream(dev_t)
+    if w.qo_lens is not None:
+        run_prefill(args, w, dev, stream, dev_t, world, rank)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    t0 = time.perf_counter()
+    pd = PagedDecode(w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
+                     num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
+                     sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
+                     device=dev_t, min_chunk_tokens=args.min_chunk_tokens,
+                     ctas_per_sm=args.ctas_per_sm or None,
+                     flags={"auto": 0, "cuda_cores": C.PA_FLAG_CUDA_CORES,
+                            "tensor_cores": C.PA_FLAG_TENSOR_CORES}[args.kernel],
+                     piece_cost_tokens=args.piece_cost_tokens)
+    tensor_cores = C.pa_plan_uses_tensor_cores(pd.plan)
+    setup_us = (time.perf_counter() - t0) * 1e6
+    reps = 20
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        (C.pa_cascade_plan_create(pd.problem, w.prefix_len, w.kv_indptr, w.last_page_len)
+         if w.prefix_len else C.pa_plan_create(pd.problem, w.kv_indptr, w.last_page_len))
+    plan_us = (time.perf_counter() - t0) * 1e6 / reps
+    o, lse = pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"],
+                    prefix_indices=dev.get("prefix_indices"))
+    launches_per_step = 2 if (w.prefix_len and w.batch) else 1
+
+    def step():
+        pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"], o, lse,
+               prefix_indices=dev.get("prefix_indices"), stream=stream)
+
+    flush_l2 = make_l2_flush(dev_t)
+    ms, step_ms, clocks = timed_steps(step, flush_l2, args, stream, dev_t, world)
 
     nbytes = w.kv_bytes()
     value = aggregate_gbs(world, nbytes, ms * 1e-3)

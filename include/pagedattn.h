@@ -13,9 +13,13 @@
  *     (pa_cascade_plan_create / pa_cascade_run) and head-query fusion for
  *     grouped-query attention (every q head of one kv head is computed by
  *     the same CTA from one load of each K/V row).
- *   - README, core feature 5: CUDA-graph capture.  pa_run, pa_cascade_run
- *     and pa_merge_state only enqueue work on the given stream: no host
- *     synchronisation, no allocation.
+ *   - README, core feature 1 and its usage example of append (causal mask)
+ *     and prefill attention: pa_prefill_plan_create / pa_prefill_run (new
+ *     query tokens of each request against its paged keys, on the tensor
+ *     cores).
+ *   - README, core feature 5: CUDA-graph capture.  pa_run, pa_cascade_run,
+ *     pa_prefill_run and pa_merge_state only enqueue work on the given
+ *     stream: no host synchronisation, no allocation.
  *   - flashinfer-cubin registry page, quickstart: the paged-table names
  *     kv_indptr, kv_indices, last_page_len and kv_layout (NHD here).
  *   - hysenlabs project review, "Installing FlashInfer and running a first
@@ -57,7 +61,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 3
+#define PA_ABI_VERSION 4
 
 typedef enum {
   PA_OK = 0,
@@ -159,6 +163,40 @@ pa_status pa_cascade_plan_create(const pa_problem* problem, int32_t prefix_len,
                                  const int32_t* kv_indptr_host,
                                  const int32_t* last_page_len_host, pa_plan_t* out);
 
+/* One query tile of a prefill plan: query tokens [q_begin, q_begin + n_q)
+ * (rows of q and o) of request `request`; token q_begin + j sees keys
+ * [0, min(kv_base + j + 1, kv_end)) of the request, page_begin =
+ * kv_indptr[request].  Causal plans have kv_end = kv_base + n_q, plans
+ * without the mask kv_base = kv_end - 1 = L_b - 1. */
+typedef struct {
+  int32_t request, q_begin, n_q, page_begin, kv_base, kv_end;
+} pa_prefill_tile;
+/* Plan for prefill / append attention (host only, no CUDA call).  Request b
+ * has Q_b = qo_indptr[b + 1] - qo_indptr[b] new query tokens, rows
+ * qo_indptr[b] .. qo_indptr[b + 1] - 1 of q and o, and L_b keys in its pages
+ * (kv_indptr / last_page_len as for pa_plan_create).  With causal != 0 the
+ * last Q_b keys are the new tokens' own and new token i (0-based within the
+ * request) attends to keys t < L_b - Q_b + i + 1 (Q_b = L_b is prefill,
+ * Q_b < L_b append); with causal == 0 every token attends to all L_b keys.
+ *   s_t = sm_scale <q[qo_indptr[b] + i, hq, :], k_pool[row(b, t), h, :]>,
+ *   lse = ln sum_t exp(s_t) (fp32), o = sum_t exp(s_t - lse) v_pool[row(b, t), h, :]
+ *   rounded once to the input type; a token that sees no key gets o = 0,
+ *   lse = -inf.
+ * Layouts: q and o are [total_q, num_qo_heads, head_dim] with total_q =
+ * qo_indptr[batch]; lse is [total_q, num_qo_heads]; the pools as above.
+ * Work: the query tokens of each request are cut into tiles of 128 / G
+ * consecutive tokens (G = Hq / Hkv; the last tile of a request may be
+ * shorter); the run launches one CTA per (tile, kv head), tiles in
+ * decreasing order of 64-key tiles ceil(kv_end / 64), ties in request then
+ * token order.  num_sms, ctas_per_sm, min_chunk_tokens and
+ * piece_cost_tokens are not used.
+ * Validates as pa_plan_create, plus: qo_indptr[0] == 0 and non-decreasing,
+ * total_q < 2^31, and Q_b <= L_b when causal.  page_size must be >= 8
+ * (pages move as tensor-memory-access boxes of >= 8 rows) and num_pages *
+ * page_size < 2^31 - 1: PA_ERR_UNSUPPORTED otherwise. */
+pa_status pa_prefill_plan_create(const pa_problem* problem, int32_t causal,
+                                 const int32_t* qo_indptr_host, const int32_t* kv_indptr_host,
+                                 const int32_t* last_page_len_host, pa_plan_t* out);
 /* Read-only views of the plan (borrowed; valid until pa_plan_destroy). */
 pa_status pa_plan_quota_tokens(pa_plan_t plan, int32_t* quota);
 pa_status pa_plan_work_items(pa_plan_t plan, const pa_work_item** items, int64_t* n_items);
@@ -168,6 +206,8 @@ pa_status pa_plan_merge_indptr(pa_plan_t plan,
                                const int32_t** merge_indptr /* [B*Hkv+1] */);
 pa_status pa_plan_num_partials(pa_plan_t plan, int64_t* n_partials);
 pa_status pa_plan_prefix_chunks(pa_plan_t plan, int32_t* n_chunks, int32_t* chunk_tokens);
+/* The tiles of a prefill plan in launch order (0 tiles for other plans). */
+pa_status pa_plan_prefill_tiles(pa_plan_t plan, const pa_prefill_tile** tiles, int64_t* n_tiles);
 
 /* Device workspace the run stage needs: work list, CTA and merge offsets,
  * arrival counters and fp32 partial states.  Caller-allocated, 256-byte
@@ -198,6 +238,15 @@ pa_status pa_cascade_run(pa_plan_t plan, const void* q, const void* k_pool,
                          const int32_t* d_kv_indices, void* o, float* lse, void* d_workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Prefill / append run: attention of every new query token of the plan
+ * (pa_prefill_plan_create) to its request's keys, written to o and
+ * lse (lse may be NULL).  One launch; the plan's tiles must have been
+ * uploaded (pa_plan_upload) into d_workspace.  PA_FLAG_CHECK_INDICES
+ * bounds-checks page indices as for pa_run.  Other plans are rejected with
+ * PA_ERR_INVALID_ARG, as prefill plans are by pa_run and pa_cascade_run. */
+pa_status pa_prefill_run(pa_plan_t plan, const void* q, const void* k_pool, const void* v_pool,
+                         const int32_t* d_kv_indices, void* o, float* lse, void* d_workspace,
+                         size_t workspace_bytes, void* stream);
 /* Combine two attention states over disjoint token sets, row by row:
  *   M = max(lse_a, lse_b), w_x = exp(lse_x - M),
  *   o = (w_a o_a + w_b o_b) / (w_a + w_b),   lse = M + ln(w_a + w_b).
@@ -216,8 +265,8 @@ pa_status pa_merge_state(const void* o_a, const float* lse_a, const void* o_b,
  * The workspace is a fixed 8 MiB array inside libpagedattn.so on every GPU
  * that loads it, held until the process exits; a plan needing more
  * (pa_plan_workspace_bytes > 8 MiB) is rejected with
- * PA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued, and cascade plans
- * with PA_ERR_INVALID_ARG.  Nothing is allocated: each call uploads the plan
+ * PA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued, and cascade and
+ * prefill plans with PA_ERR_INVALID_ARG.  Nothing is allocated: each call uploads the plan
  * into the array (as pa_plan_upload) and runs it (as pa_run).  The first call
  * on a device looks the array up (cudaGetSymbolAddress), so make it before any
  * stream capture.  All calls share the array: calls that overlap on the GPU

@@ -197,15 +197,18 @@ def cascade_decode(q, k_pool, v_pool, prefix_indices, prefix_len, kv_indptr, kv_
 
 def paged_prefill(q, k_pool, v_pool, qo_indptr, kv_indptr, kv_indices, last_page_len, *,
                   num_qo_heads, num_kv_heads, head_dim, page_size, dtype, sm_scale,
-                  queries=None, threads=1):
-    """Prefill / append attention (README usage example: prefill and append
-    attention over a paged KV cache, causal).
+                  causal=True, queries=None, threads=1):
+    """Prefill / append attention (README usage example: append attention
+    with a causal mask, the new tokens being the last ones in the KV-Cache;
+    prefill attention without the mask).
 
-    Request b has L_b keys (its page table) of which its Q_b new query tokens
-    are the last Q_b (qo_indptr[b + 1] - qo_indptr[b] = Q_b <= L_b).  Query i
-    (0-based) of request b attends causally to keys t < L_b - Q_b + i + 1.
-    That is exactly a decode over the request's pages cut at that limit, so
-    each query becomes one row of ``paged_decode`` with its own page list.
+    Request b has L_b keys (its page table) and Q_b = qo_indptr[b + 1] -
+    qo_indptr[b] new query tokens.  With ``causal`` those are its last Q_b
+    keys (Q_b <= L_b) and query i (0-based) attends to keys
+    t < L_b - Q_b + i + 1; without it every query attends to all L_b keys.
+    Either way that is exactly a decode over the request's pages cut at the
+    query's limit, so each query becomes one row of ``paged_decode`` with its
+    own page list.
 
     q is ``[total_q, Hq, D]``.  Returns o ``[n, Hq, D]`` and lse ``[n, Hq]``
     for every query (``queries=None``) or the listed global query indices.
@@ -220,14 +223,14 @@ def paged_prefill(q, k_pool, v_pool, qo_indptr, kv_indptr, kv_indices, last_page
         n = indptr[b + 1] - indptr[b]
         L = (n - 1) * P + last[b] if n > 0 else 0
         Q = qo[b + 1] - qo[b]
-        if Q > L:
+        if causal and Q > L:
             raise ValueError(f"request {b}: {Q} queries but only {L} keys")
         owner += [(b, L, Q, i) for i in range(Q)]
     sel = list(range(len(owner))) if queries is None else [int(x) for x in queries]
     q_indptr, q_indices, q_last = [0], [], []
     for g in sel:
         b, L, Q, i = owner[g]
-        lim = L - Q + i + 1
+        lim = L - Q + i + 1 if causal else L
         n = -(-lim // P)
         q_indices.extend(indices[indptr[b]:indptr[b] + n].tolist())
         q_indptr.append(len(q_indices))

@@ -22,7 +22,7 @@ OUT_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpagedattn.so")
 
 SOURCES = ["plan.cpp", "api.cu", "decode.cu", "decode_tc.cu", "merge_state.cu", "cascade.cu",
-           "static_workspace.cu"]
+           "prefill.cu", "static_workspace.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -1,8 +1,8 @@
 // C-ABI entry points of libpagedattn.so that touch the device: workspace
-// upload, the run stage, cascade run, merge_state, the index check and the
-// scheduling defaults.  Argument checking happens here, on the host, before
-// anything is enqueued; pointers must be device pointers (16-byte aligned
-// for q, o and the pools).
+// upload, the run stage, cascade run, prefill run, merge_state, the index
+// check and the scheduling defaults.  Argument checking happens here, on the
+// host, before anything is enqueued; pointers must be device pointers
+// (16-byte aligned for q, o and the pools).
 #include <cuda_runtime.h>
 
 #include "pa_internal.h"
@@ -56,7 +56,8 @@ pa_status pa_run(pa_plan_t plan, const void* q, const void* k_pool, const void* 
   pa_status st =
       check_run_args(plan, q, k_pool, v_pool, d_kv_indices, o, d_workspace, workspace_bytes);
   if (st != PA_OK) return st;
-  if (plan->cascade) return PA_ERR_INVALID_ARG;  // cascade plans run through pa_cascade_run
+  // cascade and prefill plans run through pa_cascade_run and pa_prefill_run
+  if (plan->cascade || plan->prefill) return PA_ERR_INVALID_ARG;
   pa::RunPointers p{q, k_pool, v_pool, d_kv_indices, nullptr, o, lse,
                     static_cast<uint8_t*>(d_workspace)};
   return from_cuda(launch_decode_any(*plan, p, stream));
@@ -79,6 +80,18 @@ pa_status pa_cascade_run(pa_plan_t plan, const void* q, const void* k_pool,
     if (e) return PA_ERR_CUDA;
   }
   return from_cuda(launch_decode_any(*plan, p, stream));
+}
+
+pa_status pa_prefill_run(pa_plan_t plan, const void* q, const void* k_pool, const void* v_pool,
+                         const int32_t* d_kv_indices, void* o, float* lse, void* d_workspace,
+                         size_t workspace_bytes, void* stream) {
+  pa_status st =
+      check_run_args(plan, q, k_pool, v_pool, d_kv_indices, o, d_workspace, workspace_bytes);
+  if (st != PA_OK) return st;
+  if (!plan->prefill) return PA_ERR_INVALID_ARG;
+  pa::RunPointers p{q, k_pool, v_pool, d_kv_indices, nullptr, o, lse,
+                    static_cast<uint8_t*>(d_workspace)};
+  return from_cuda(pa::launch_prefill(*plan, p, stream));
 }
 
 pa_status pa_merge_state(const void* o_a, const float* lse_a, const void* o_b,

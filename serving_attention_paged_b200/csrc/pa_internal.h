@@ -21,9 +21,10 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 
 // Device workspace, in this order (each region 256-byte aligned):
 //   items        [n_items]             pa_work_item (pieces, grouped by CTA)
+//   prefill_tiles [n_tiles]            pa_prefill_tile (prefill plans only)
 //   cta_indptr   [n_cta + 1]           int32, pieces of CTA i
 //   merge_indptr [B * Hkv + 1]         int32, partial slots of segment (b, h)
-//   counters     [B * Hkv * kCounterSlots]  int32, zero between runs
+//   counters     [B * Hkv * kCounterSlots]  int32, zero between runs (decode levels only)
 //   error        [2]                   uint64: first bad kv_indices position (~0 = none),
 //                                      then a timeout flag (0 = none)
 //   partial_o    [n_partials, G, D]    fp32, outputs of pieces of split segments
@@ -32,8 +33,8 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 //   prefix_o     [prefix_chunks, B, Hq, D]  fp32 (cascade only)
 //   prefix_lse   [prefix_chunks, B, Hq]     fp32, base 2 (cascade only)
 struct WorkspaceLayout {
-  size_t items = 0, cta_indptr = 0, merge_indptr = 0, counters = 0, error = 0, partial_o = 0, partial_lse = 0,
-         prefix_o = 0, prefix_lse = 0, total = 0;
+  size_t items = 0, prefill_tiles = 0, cta_indptr = 0, merge_indptr = 0, counters = 0, error = 0,
+         partial_o = 0, partial_lse = 0, prefix_o = 0, prefix_lse = 0, total = 0;
 };
 
 }  // namespace pa
@@ -54,6 +55,11 @@ struct pa_plan_s {
   int32_t prefix_chunks = 0;        // split of the prefix across CTAs
   int32_t prefix_chunk_tokens = 0;  // tokens per chunk (multiple of the 128-key tile)
   int32_t q_tiles = 0;              // 128-row tiles over the B * G query rows of one kv head
+  // prefill / append (pa_prefill_plan_create): query tiles, longest first
+  bool prefill = false;
+  int64_t total_q = 0;
+  std::vector<int32_t> qo_indptr;
+  std::vector<pa_prefill_tile> prefill_tiles;
   pa::WorkspaceLayout ws;
   // Bytes [0, ws.partial_o) of the workspace as pa_plan_upload writes them:
   // work list, CTA and merge offsets, zeroed counters and the status words
@@ -63,8 +69,8 @@ struct pa_plan_s {
 
 namespace pa {
 
-// Kernel launchers (decode.cu, merge_state.cu, cascade.cu).  They return a
-// cudaError_t value as int.
+// Kernel launchers (decode.cu, decode_tc.cu, merge_state.cu, cascade.cu,
+// prefill.cu).  They return a cudaError_t value as int.
 struct RunPointers {
   const void* q;
   const void* k_pool;
@@ -101,6 +107,7 @@ inline int32_t default_piece_cost_tokens(const pa_problem& p) {
   return decode_uses_tensor_cores(p) ? kPieceCostTensorCores : kPieceCostCudaCores;
 }
 int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* stream);
+int launch_prefill(const pa_plan_s& plan, const RunPointers& p, void* stream);
 int launch_merge_state(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
                        void* o, float* lse, int64_t rows, int32_t head_dim, pa_dtype dtype,
                        void* stream);

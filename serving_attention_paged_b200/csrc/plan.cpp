@@ -172,9 +172,10 @@ void layout_workspace(pa_plan_s* plan) {
   };
   const size_t Hq = p.num_qo_heads, D = p.head_dim, B = p.batch;
   w.items = take(plan->items.size() * sizeof(pa_work_item));
+  w.prefill_tiles = take(plan->prefill_tiles.size() * sizeof(pa_prefill_tile));
   w.cta_indptr = take(plan->cta_indptr.size() * sizeof(int32_t));
   w.merge_indptr = take(plan->merge_indptr.size() * sizeof(int32_t));
-  w.counters = take(B * p.num_kv_heads * pa::kCounterSlots * sizeof(int32_t));
+  w.counters = take(plan->prefill ? 0 : B * p.num_kv_heads * pa::kCounterSlots * sizeof(int32_t));
   w.error = take(2 * sizeof(uint64_t));  // first bad index, timeout flag
   const size_t G = plan->group;
   w.partial_o = take(size_t(plan->n_partials) * G * D * sizeof(float));
@@ -190,6 +191,9 @@ void build_upload_image(pa_plan_s* plan) {
   img.assign(w.partial_o, 0);  // counters stay zero
   if (!plan->items.empty())
     std::memcpy(img.data() + w.items, plan->items.data(), plan->items.size() * sizeof(pa_work_item));
+  if (!plan->prefill_tiles.empty())
+    std::memcpy(img.data() + w.prefill_tiles, plan->prefill_tiles.data(),
+                plan->prefill_tiles.size() * sizeof(pa_prefill_tile));
   std::memcpy(img.data() + w.cta_indptr, plan->cta_indptr.data(),
               plan->cta_indptr.size() * sizeof(int32_t));
   std::memcpy(img.data() + w.merge_indptr, plan->merge_indptr.data(),
@@ -218,8 +222,56 @@ void schedule_prefix(pa_plan_s* plan) {
   plan->prefix_chunk_tokens = int32_t(tiles_per_chunk * kTileKeys);
 }
 
-pa_status create(const pa_problem* problem, int32_t prefix_len, bool cascade,
-                 const int32_t* indptr, const int32_t* last, pa_plan_t* out) {
+// Prefill / append tiles: each request's new tokens cut into runs of 128 / G
+// (one 128-row tensor-core tile of (token, q head) rows per kv head), listed
+// in decreasing order of 64-key tiles so that the long ones start first.
+pa_status build_prefill(pa_plan_s* plan, bool causal, const int32_t* qo, const int32_t* indptr,
+                        const int32_t* last) {
+  const pa_problem& p = plan->prob;
+  const int64_t B = p.batch, P = p.page_size;
+  if (B > 0 && (!qo || !indptr || !last)) return PA_ERR_INVALID_ARG;
+  if ((qo && qo[0] != 0) || (indptr && indptr[0] != 0)) return PA_ERR_INVALID_ARG;
+  const int64_t per_tile = 128 / plan->group;
+  constexpr int64_t kTileKeys = 64;
+  std::vector<pa_prefill_tile> tiles;
+  for (int64_t b = 0; b < B; ++b) {
+    if (indptr[b + 1] < indptr[b] || qo[b + 1] < qo[b]) return PA_ERR_INVALID_ARG;
+    const int64_t n = int64_t(indptr[b + 1]) - indptr[b];
+    if (n > 0 && (last[b] < 1 || last[b] > P)) return PA_ERR_INVALID_ARG;
+    const int64_t L = n > 0 ? (n - 1) * P + last[b] : 0;
+    if (L > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    const int64_t Q = int64_t(qo[b + 1]) - qo[b];
+    if (causal && Q > L) return PA_ERR_INVALID_ARG;
+    for (int64_t t0 = 0; t0 < Q; t0 += per_tile) {
+      const int64_t nq = std::min(per_tile, Q - t0);
+      const int64_t base = causal ? L - Q + t0 : L - 1;
+      const int64_t end = causal ? base + nq : L;
+      tiles.push_back(pa_prefill_tile{int32_t(b), int32_t(qo[b] + t0), int32_t(nq), indptr[b],
+                                      int32_t(base), int32_t(end)});
+    }
+  }
+  std::stable_sort(tiles.begin(), tiles.end(), [](const pa_prefill_tile& x, const pa_prefill_tile& y) {
+    return ceil_div(x.kv_end, kTileKeys) > ceil_div(y.kv_end, kTileKeys);
+  });
+  plan->prefill_tiles = std::move(tiles);
+  plan->total_q = B > 0 ? qo[B] : 0;
+  if (B > 0) plan->kv_indptr.assign(indptr, indptr + B + 1);
+  else plan->kv_indptr.assign(1, 0);
+  plan->last_page_len.assign(last ? last : nullptr, last ? last + B : nullptr);
+  if (B > 0) plan->qo_indptr.assign(qo, qo + B + 1);
+  else plan->qo_indptr.assign(1, 0);
+  plan->cta_indptr.assign(1, 0);
+  plan->merge_indptr.assign(1, 0);
+  if (plan->prefill_tiles.size() * size_t(p.num_kv_heads) > size_t(INT32_MAX))
+    return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+enum class Mode { kDecode, kCascade, kPrefill };
+
+pa_status create(const pa_problem* problem, int32_t prefix_len, Mode mode, bool causal,
+                 const int32_t* qo, const int32_t* indptr, const int32_t* last, pa_plan_t* out) {
+  const bool cascade = mode == Mode::kCascade;
   if (!out) return PA_ERR_INVALID_ARG;
   *out = nullptr;
   pa_status st = validate_problem(problem);
@@ -227,7 +279,7 @@ pa_status create(const pa_problem* problem, int32_t prefix_len, bool cascade,
   if (cascade && (prefix_len < 0 || prefix_len % problem->page_size)) return PA_ERR_INVALID_ARG;
   // the prefix level moves whole pages (>= 8 rows) with TMA, whose row
   // coordinates are signed 32-bit
-  if (cascade && prefix_len > 0 &&
+  if (((cascade && prefix_len > 0) || mode == Mode::kPrefill) &&
       (!pa::cascade_page_size_supported(problem->page_size) ||
        problem->num_pages * int64_t(problem->page_size) >= int64_t(INT32_MAX)))
     return PA_ERR_UNSUPPORTED;
@@ -239,8 +291,9 @@ pa_status create(const pa_problem* problem, int32_t prefix_len, bool cascade,
     plan->group = problem->num_qo_heads / problem->num_kv_heads;
     plan->log2_page = ilog2(problem->page_size);
     plan->cascade = cascade;
+    plan->prefill = mode == Mode::kPrefill;
     plan->prefix_len = cascade ? prefix_len : 0;
-    st = build(plan, indptr, last);
+    st = plan->prefill ? build_prefill(plan, causal, qo, indptr, last) : build(plan, indptr, last);
     if (st == PA_OK) {
       if (cascade) schedule_prefix(plan);
       layout_workspace(plan);
@@ -263,13 +316,29 @@ extern "C" {
 
 pa_status pa_plan_create(const pa_problem* problem, const int32_t* kv_indptr_host,
                          const int32_t* last_page_len_host, pa_plan_t* out) {
-  return create(problem, 0, false, kv_indptr_host, last_page_len_host, out);
+  return create(problem, 0, Mode::kDecode, false, nullptr, kv_indptr_host, last_page_len_host,
+                out);
 }
 
 pa_status pa_cascade_plan_create(const pa_problem* problem, int32_t prefix_len,
                                  const int32_t* kv_indptr_host,
                                  const int32_t* last_page_len_host, pa_plan_t* out) {
-  return create(problem, prefix_len, true, kv_indptr_host, last_page_len_host, out);
+  return create(problem, prefix_len, Mode::kCascade, false, nullptr, kv_indptr_host,
+                last_page_len_host, out);
+}
+
+pa_status pa_prefill_plan_create(const pa_problem* problem, int32_t causal,
+                                 const int32_t* qo_indptr_host, const int32_t* kv_indptr_host,
+                                 const int32_t* last_page_len_host, pa_plan_t* out) {
+  return create(problem, 0, Mode::kPrefill, causal != 0, qo_indptr_host, kv_indptr_host,
+                last_page_len_host, out);
+}
+
+pa_status pa_plan_prefill_tiles(pa_plan_t plan, const pa_prefill_tile** tiles, int64_t* n_tiles) {
+  if (!plan || !tiles || !n_tiles) return PA_ERR_INVALID_ARG;
+  *tiles = plan->prefill_tiles.data();
+  *n_tiles = int64_t(plan->prefill_tiles.size());
+  return PA_OK;
 }
 
 pa_status pa_plan_quota_tokens(pa_plan_t plan, int32_t* quota) {

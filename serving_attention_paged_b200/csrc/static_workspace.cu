@@ -52,7 +52,7 @@ pa_status static_workspace_address(void** out) {
 extern "C" pa_status pa_run_static_workspace(pa_plan_t plan, const void* q, const void* k_pool,
                                              const void* v_pool, const int32_t* d_kv_indices,
                                              void* o, float* lse, void* stream) {
-  if (!plan || plan->cascade) return PA_ERR_INVALID_ARG;
+  if (!plan || plan->cascade || plan->prefill) return PA_ERR_INVALID_ARG;
   if (plan->ws.total > kStaticWorkspaceBytes) return PA_ERR_WORKSPACE_TOO_SMALL;
   void* ws = nullptr;
   pa_status st = static_workspace_address(&ws);

@@ -45,11 +45,19 @@ class pa_work_item(ctypes.Structure):
                 ("request", "kv_head", "page_begin", "token_begin", "token_end", "partial_slot")]
 
 
+class pa_prefill_tile(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("request", "q_begin", "n_q", "page_begin", "kv_base", "kv_end")]
+
+
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 _P = ctypes.POINTER
 _SIGS = {
     "pa_plan_create": [_P(pa_problem), _vp, _vp, _P(_vp)],
     "pa_cascade_plan_create": [_P(pa_problem), _i32, _vp, _vp, _P(_vp)],
+    "pa_prefill_plan_create": [_P(pa_problem), _i32, _vp, _vp, _vp, _P(_vp)],
+    "pa_plan_prefill_tiles": [_vp, _P(_P(pa_prefill_tile)), _P(_i64)],
+    "pa_prefill_run": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "pa_plan_quota_tokens": [_vp, _P(_i32)],
     "pa_plan_cta_indptr": [_vp, _P(_P(_i32)), _P(_i64)],
     "pa_plan_work_items": [_vp, _P(_P(pa_work_item)), _P(_i64)],
@@ -156,6 +164,30 @@ def pa_cascade_plan_create(problem: pa_problem, prefix_len: int, kv_indptr_host,
     return Plan(h.value)
 
 
+def pa_prefill_plan_create(problem: pa_problem, causal: bool, qo_indptr_host, kv_indptr_host,
+                           last_page_len_host) -> Plan:
+    qo = _host_i32(qo_indptr_host)
+    indptr, last = _host_i32(kv_indptr_host), _host_i32(last_page_len_host)
+    h = _vp()
+    _check(lib.pa_prefill_plan_create(ctypes.byref(problem), int(bool(causal)), qo.ctypes.data,
+                                      indptr.ctypes.data, last.ctypes.data if last.size else None,
+                                      ctypes.byref(h)),
+           "pa_prefill_plan_create")
+    return Plan(h.value)
+
+
+def pa_plan_prefill_tiles(plan: Plan) -> np.ndarray:
+    """The prefill tiles in launch order as an int32 array [n, 6] (a copy):
+    request, q_begin, n_q, page_begin, kv_base, kv_end."""
+    p, n = _P(pa_prefill_tile)(), _i64()
+    _check(lib.pa_plan_prefill_tiles(plan.handle, ctypes.byref(p), ctypes.byref(n)),
+           "pa_plan_prefill_tiles")
+    if n.value == 0:
+        return np.zeros((0, 6), dtype=np.int32)
+    buf = ctypes.cast(p, _P(_i32 * (6 * n.value))).contents
+    return np.frombuffer(buf, dtype=np.int32).reshape(n.value, 6).copy()
+
+
 def pa_plan_quota_tokens(plan: Plan) -> int:
     c = _i32()
     _check(lib.pa_plan_quota_tokens(plan.handle, ctypes.byref(c)), "pa_plan_quota_tokens")
@@ -224,6 +256,14 @@ def pa_cascade_run(plan: Plan, q, k_pool, v_pool, prefix_indices, kv_indices, o,
                               _ptr(prefix_indices), _ptr(kv_indices), _ptr(o), _ptr(lse),
                               _ptr(workspace), workspace_bytes, _stream(stream)),
            "pa_cascade_run")
+
+
+def pa_prefill_run(plan: Plan, q, k_pool, v_pool, kv_indices, o, lse, workspace,
+                   workspace_bytes: int, stream=None):
+    _check(lib.pa_prefill_run(plan.handle, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(kv_indices),
+                              _ptr(o), _ptr(lse), _ptr(workspace), workspace_bytes,
+                              _stream(stream)),
+           "pa_prefill_run")
 
 
 def pa_run_static_workspace(plan: Plan, q, k_pool, v_pool, kv_indices, o, lse, stream=None):

@@ -2,8 +2,9 @@
 
 ``PagedDecode`` holds a plan and its device workspace (allocated through
 torch, the library itself never allocates) and calls ``pa_run`` /
-``pa_cascade_run``.  It only marshals arguments; all attention work is done
-by the library's kernels.
+``pa_cascade_run``; ``PagedPrefill`` does the same for ``pa_prefill_run``.
+They only marshal arguments; all attention work is done by the library's
+kernels.
 """
 from __future__ import annotations
 
@@ -68,6 +69,51 @@ class PagedDecode:
         else:
             C.pa_run(self.plan, q, k_pool, v_pool, kv_indices, o, lse, self.workspace,
                      self.workspace.numel(), stream)
+        return o, lse
+
+    def check(self, stream=None) -> int:
+        return C.pa_plan_check(self.plan, self.workspace, stream)
+
+
+class PagedPrefill:
+    """Prefill / append attention: plan once per batch of new tokens (host),
+    run once per layer (device).  ``qo_indptr`` gives each request's new query
+    tokens (rows of q); with ``causal`` they are the last of its keys and
+    each sees the keys up to its own position, else every token sees all of
+    its request's keys."""
+
+    def __init__(self, qo_indptr, kv_indptr, last_page_len, *, num_qo_heads, num_kv_heads,
+                 page_size, dtype, sm_scale, num_pages, causal=True, head_dim=128, device=None,
+                 flags=0, stream=None):
+        self.device = torch.device(device if device is not None else "cuda")
+        self.dtype = dtype
+        self.batch = len(last_page_len)
+        self.total_q = int(qo_indptr[-1]) if self.batch else 0
+        self.num_qo_heads, self.head_dim = num_qo_heads, head_dim
+        # the schedule fields do not apply to prefill plans; they only need to be valid
+        self.problem = C.make_problem(batch=self.batch, num_qo_heads=num_qo_heads,
+                                      num_kv_heads=num_kv_heads, head_dim=head_dim,
+                                      page_size=page_size, dtype=dtype, sm_scale=sm_scale,
+                                      num_sms=1, ctas_per_sm=1, num_pages=num_pages, flags=flags)
+        self.plan = C.pa_prefill_plan_create(self.problem, causal, qo_indptr, kv_indptr,
+                                             last_page_len)
+        self.workspace_bytes = C.pa_plan_workspace_bytes(self.plan)
+        self.workspace = torch.empty(max(self.workspace_bytes, 256), dtype=torch.uint8,
+                                     device=self.device)
+        C.pa_plan_upload(self.plan, self.workspace, self.workspace.numel(), stream)
+
+    def tiles(self):
+        return C.pa_plan_prefill_tiles(self.plan)
+
+    def run(self, q, k_pool, v_pool, kv_indices, o=None, lse=None, stream=None):
+        if o is None:
+            o = torch.empty(self.total_q, self.num_qo_heads, self.head_dim,
+                            dtype=_TORCH_DTYPES[self.dtype], device=self.device)
+        if lse is None:
+            lse = torch.empty(self.total_q, self.num_qo_heads, dtype=torch.float32,
+                              device=self.device)
+        C.pa_prefill_run(self.plan, q, k_pool, v_pool, kv_indices, o, lse, self.workspace,
+                         self.workspace.numel(), stream)
         return o, lse
 
     def check(self, stream=None) -> int:

@@ -2,9 +2,10 @@
 prefill and append attention over a paged KV cache, causal).
 
 The oracle evaluates each new query token as a decode over its request's
-pages cut at the causal limit.  The pins check that against what the
-definition fixes independently: dense causal attention written out with a
-naive softmax on contiguous tensors, the first query of a fresh prefill
+pages cut at the query's limit (its causal position, or all keys without
+the mask).  The pins check that against what the definition fixes
+independently: dense attention written out with a naive softmax on
+contiguous tensors (causal and not), the first query of a fresh prefill
 (one visible key: o = V_0, lse = s_0), and causality itself (a key's values
 change only the queries that may see it).
 """
@@ -25,9 +26,10 @@ def _widen(t, dtype):
     return table[bits].reshape(tuple(t.shape))
 
 
-def _dense_causal(w, t):
-    """Causal attention on contiguous per-request K/V in the generator's logical
-    token order (no pages), naive softmax in fp64."""
+def _dense(w, t, causal=True):
+    """Attention on contiguous per-request K/V in the generator's logical token
+    order (no pages), naive softmax in fp64; a query that sees no key gets
+    o = 0, lse = -inf."""
     G, D = w.group, w.head_dim
     q = _widen(t["q"], w.dtype)
     lens, qo = w.kv_lens(), w.qo_indptr
@@ -39,7 +41,10 @@ def _dense_causal(w, t):
         V = _widen(w.logical_kv("v", int(start[b]), int(start[b + 1])), w.dtype)
         Q = qo[b + 1] - qo[b]
         for i in range(Q):
-            lim = int(lens[b]) - Q + i + 1
+            lim = int(lens[b]) - Q + i + 1 if causal else int(lens[b])
+            if lim == 0:
+                lse[qo[b] + i] = -np.inf
+                continue
             for hq in range(w.num_qo_heads):
                 s = w.sm_scale * (K[:lim, hq // G, :] @ q[qo[b] + i, hq])
                 e = np.exp(s)  # tiny inputs: no max subtraction needed
@@ -61,7 +66,7 @@ def test_prefill_matches_dense_causal_brute_force(dtype):
                         page_size=4, dtype=dtype, seed=31, qo_lens=[3, 5, 1, 0])
     t = w.materialize()
     o, lse = _prefill(w, t)
-    o_ref, l_ref = _dense_causal(w, t)
+    o_ref, l_ref = _dense(w, t)
     assert np.abs(o - o_ref).max() < 1e-12 and np.abs(lse - l_ref).max() < 1e-12
 
 
@@ -121,3 +126,18 @@ def test_prefill_rejects_more_queries_than_keys():
     t = w.materialize()
     with pytest.raises(ValueError):
         _prefill(w, t)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_prefill_without_mask_matches_dense_brute_force(dtype):
+    """No causal mask: every query sees all of its request's keys; more
+    queries than keys and a request without keys are allowed."""
+    w = W.make_workload("pf_nomask", [7, 0, 9, 2], num_qo_heads=4, num_kv_heads=2, head_dim=16,
+                        page_size=4, dtype=dtype, seed=36, qo_lens=[3, 2, 1, 5])
+    t = w.materialize()
+    o, lse = _prefill(w, t, causal=False)
+    o_ref, l_ref = _dense(w, t, causal=False)
+    empty = np.isneginf(l_ref)
+    assert empty.sum() == 2 * w.num_qo_heads
+    assert np.array_equal(np.isneginf(lse), empty) and np.all(o[empty] == 0)
+    assert np.abs(o - o_ref).max() < 1e-12 and np.abs(lse[~empty] - l_ref[~empty]).max() < 1e-12

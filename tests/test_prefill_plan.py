@@ -1,0 +1,129 @@
+"""The prefill / append plan on the host (no GPU): its tiles cover every new
+query token of every request exactly once, in runs of at most 128 / G
+tokens of one request, with the key range of the causal rule (or all keys
+without the mask), longest first; malformed tables are rejected before
+anything runs."""
+import numpy as np
+import pytest
+
+from serving_attention_paged_b200 import workloads as W
+
+
+@pytest.fixture(scope="module")
+def C():
+    from serving_attention_paged_b200 import build
+    build.build()
+    from serving_attention_paged_b200 import pagedattn
+    return pagedattn
+
+
+def _problem(C, batch, hq=32, hkv=8, P=16, flags=0):
+    return C.make_problem(batch=batch, num_qo_heads=hq, num_kv_heads=hkv, page_size=P,
+                          dtype="f16", sm_scale=0.088, num_sms=1, ctas_per_sm=1,
+                          num_pages=1 << 16, flags=flags)
+
+
+def _tables(kv_lens, P):
+    n = [-(-L // P) for L in kv_lens]
+    indptr = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    last = np.array([L - (k - 1) * P if k else 0 for L, k in zip(kv_lens, n)], np.int32)
+    return indptr, last
+
+
+def _expected_tiles(kv_lens, qo_lens, G, causal):
+    """The tile rule written out: per request, runs of 128 / G new tokens."""
+    per = 128 // G
+    out, qo = [], 0
+    indptr, _ = _tables(kv_lens, 16)
+    for b, (L, Q) in enumerate(zip(kv_lens, qo_lens)):
+        for t0 in range(0, Q, per):
+            n = min(per, Q - t0)
+            base, end = (L - Q + t0, L - Q + t0 + n) if causal else (L - 1, L)
+            out.append((b, qo + t0, n, int(indptr[b]), base, end))
+        qo += Q
+    return out
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (32, 4), (16, 8)])
+def test_tiles_cover_every_query_once_longest_first(C, causal, hq, hkv):
+    rng = np.random.default_rng(5 + hq + hkv)
+    kv_lens = [int(x) for x in rng.integers(1, 3000, 23)] + [0, 1, 64, 65]
+    qo_lens = [int(rng.integers(0, L + 1)) for L in kv_lens]
+    qo_lens[3] = kv_lens[3]  # a fresh prefill
+    indptr, last = _tables(kv_lens, 16)
+    qo_indptr = np.concatenate([[0], np.cumsum(qo_lens)]).astype(np.int32)
+    plan = C.pa_prefill_plan_create(_problem(C, len(kv_lens), hq, hkv), causal, qo_indptr,
+                                    indptr, last)
+    tiles = C.pa_plan_prefill_tiles(plan)
+    G = hq // hkv
+    expected = _expected_tiles(kv_lens, qo_lens, G, causal)
+    # the same set of tiles ...
+    assert sorted(map(tuple, tiles.tolist())) == sorted(expected)
+    # ... in decreasing order of 64-key tiles, ties in (request, token) order
+    keys = -(-tiles[:, 5] // 64)
+    assert np.all(np.diff(keys) <= 0)
+    for k in np.unique(keys):
+        grp = tiles[keys == k]
+        assert np.all(np.diff(grp[:, 1]) > 0)
+    # every new token of every request exactly once
+    seen = np.zeros(qo_indptr[-1], np.int32)
+    for r, q0, n, pb, base, end in tiles:
+        assert 1 <= n <= 128 // G and pb == indptr[r]
+        assert qo_indptr[r] <= q0 and q0 + n <= qo_indptr[r + 1]
+        seen[q0:q0 + n] += 1
+    assert np.all(seen == 1)
+    assert C.pa_plan_workspace_bytes(plan) >= tiles.nbytes
+
+
+def test_tiles_of_the_prefill_workload(C):
+    w = W.WORKLOADS[6]()
+    plan = C.pa_prefill_plan_create(_problem(C, w.batch, w.num_qo_heads, w.num_kv_heads,
+                                             w.page_size), True, w.qo_indptr, w.kv_indptr,
+                                    w.last_page_len)
+    tiles = C.pa_plan_prefill_tiles(plan)
+    G = w.num_qo_heads // w.num_kv_heads
+    assert len(tiles) == w.batch * (1024 // (128 // G))
+    # the last token of each request sees every key of it
+    lens = w.kv_lens()
+    for r in range(w.batch):
+        mine = tiles[tiles[:, 0] == r]
+        assert mine[:, 5].max() == lens[r] and mine[:, 4].min() == lens[r] - 1024
+
+
+def test_prefill_plan_validation(C):
+    indptr, last = _tables([40, 10], 16)
+    ok = np.array([0, 40, 50], np.int32)
+    C.pa_prefill_plan_create(_problem(C, 2), True, ok, indptr, last)
+    for bad in ([0, 41, 51], [1, 40, 50], [0, 40, 39]):  # more queries than keys, bad start, decreasing
+        with pytest.raises(C.PagedAttnError) as e:
+            C.pa_prefill_plan_create(_problem(C, 2), True, np.array(bad, np.int32), indptr, last)
+        assert e.value.status == C.PA_ERR_INVALID_ARG
+    # without the mask more queries than keys are fine
+    C.pa_prefill_plan_create(_problem(C, 2), False, np.array([0, 41, 51], np.int32), indptr, last)
+    # pages must be whole tensor-memory-access boxes (>= 8 rows)
+    i4, l4 = _tables([40, 10], 4)
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_prefill_plan_create(_problem(C, 2, P=4), True, ok, i4, l4)
+    assert e.value.status == C.PA_ERR_UNSUPPORTED
+
+
+def test_plans_run_only_through_their_own_entry_point(C):
+    indptr, last = _tables([40, 10], 16)
+    pf = C.pa_prefill_plan_create(_problem(C, 2), True, np.array([0, 4, 6], np.int32), indptr,
+                                  last)
+    dec = C.pa_plan_create(_problem(C, 2), indptr, last)
+    big = 1 << 40  # never dereferenced: the host check fails first
+    ws_pf, ws_dec = C.pa_plan_workspace_bytes(pf), C.pa_plan_workspace_bytes(dec)
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_run(pf, big, big, big, big, big, None, big, ws_pf, 0)
+    assert e.value.status == C.PA_ERR_INVALID_ARG
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_prefill_run(dec, big, big, big, big, big, None, big, ws_dec, 0)
+    assert e.value.status == C.PA_ERR_INVALID_ARG
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_run_static_workspace(pf, big, big, big, big, big, None, 0)
+    assert e.value.status == C.PA_ERR_INVALID_ARG
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_prefill_run(pf, big, big, big, big, big, None, big, ws_pf - 1, 0)
+    assert e.value.status == C.PA_ERR_WORKSPACE_TOO_SMALL
