@@ -184,7 +184,7 @@ typedef struct {
  *   lse = -inf.
  * Layouts: q and o are [total_q, num_qo_heads, head_dim] with total_q =
  * qo_indptr[batch]; lse is [total_q, num_qo_heads]; the pools as above.
- * Work: the query tokens of each request are cut into tiles of 128 / G
+ * Work: the query tokens of each request are cut into tiles of 256 / G
  * consecutive tokens (G = Hq / Hkv; the last tile of a request may be
  * shorter); the run launches one CTA per (tile, kv head), tiles in
  * decreasing order of 64-key tiles ceil(kv_end / 64), ties in request then

@@ -222,16 +222,16 @@ void schedule_prefix(pa_plan_s* plan) {
   plan->prefix_chunk_tokens = int32_t(tiles_per_chunk * kTileKeys);
 }
 
-// Prefill / append tiles: each request's new tokens cut into runs of 128 / G
-// (one 128-row tensor-core tile of (token, q head) rows per kv head), listed
-// in decreasing order of 64-key tiles so that the long ones start first.
+// Prefill / append tiles: each request's new tokens cut into runs of 256 / G
+// (two 128-row tensor-core tiles of (token, q head) rows per kv head, one CTA),
+// listed in decreasing order of 64-key tiles so that the long ones start first.
 pa_status build_prefill(pa_plan_s* plan, bool causal, const int32_t* qo, const int32_t* indptr,
                         const int32_t* last) {
   const pa_problem& p = plan->prob;
   const int64_t B = p.batch, P = p.page_size;
   if (B > 0 && (!qo || !indptr || !last)) return PA_ERR_INVALID_ARG;
   if ((qo && qo[0] != 0) || (indptr && indptr[0] != 0)) return PA_ERR_INVALID_ARG;
-  const int64_t per_tile = 128 / plan->group;
+  const int64_t per_tile = 256 / plan->group;
   constexpr int64_t kTileKeys = 64;
   std::vector<pa_prefill_tile> tiles;
   for (int64_t b = 0; b < B; ++b) {

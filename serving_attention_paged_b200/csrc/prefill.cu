@@ -11,32 +11,40 @@
 // tile sees keys [0, min(kv_base + j + 1, kv_end)).
 //
 // CTA = (query tile, kv head h); one CTA per SM.  A query tile is up to
-// 128 / G consecutive new tokens of one request; its 128 rows are the
-// (token, q head of h) pairs, token-major, so one K/V load serves all G
-// heads of the kv head (head-query fusion).  The host plan lists the tiles
+// 256 / G consecutive new tokens of one request, as two halves of 128 rows
+// (M of one MMA); a half's rows are its (token, q head of h) pairs,
+// token-major, so one K/V load serves all G heads of the kv head
+// (head-query fusion) and both halves.  The host plan lists the tiles
 // longest first, so the block scheduler starts the long ones first.
-//   warp 4  (TMA):     Q tile once; K and V of each 64-key tile as page-row
-//                      boxes, 128-byte swizzle, into a 4-stage ring; boxes
-//                      wholly past the tile's last key read out of range
-//                      (zero fill).
-//   warp 5  (MMA):     S = Q K^T into one of two TMEM buffers (M = 128,
-//                      N = 64, K = 128), then O += P V (V as an MN-major
-//                      operand) into a third; completion goes to mbarriers.
-//                      Before the last P V it zeroes the V rows that were
-//                      copied from a page but lie past the tile's keys (a
-//                      partly used last page may hold anything, NaN
-//                      included, and 0 * NaN would reach O).
-//   warps 0-3 (rows):  thread i owns tile row i = TMEM lane i: reads S with
-//                      tcgen05.ld, masks the keys its token may not see,
-//                      keeps a lazy running max (O is rescaled in TMEM only
-//                      when the max grows by more than 2^8), writes P in the
-//                      input type into shared memory in the swizzled K-major
-//                      layout, and at the end writes o = O / l in the input
-//                      type and lse = ln l + max straight to the outputs.
+//   warp 8  (TMA):     both halves of Q once; K and V of each 64-key tile as
+//                      page-row boxes, 128-byte swizzle, into a 3-stage ring;
+//                      boxes wholly past the tile's last key read out of
+//                      range (zero fill).
+//   warp 9  (MMA):     per half, S = Q K^T into one of two TMEM buffers
+//                      (M = 128, N = 64, K = 128) and O += P V (V as an
+//                      MN-major operand) into the half's O; completion goes
+//                      to mbarriers, and a K/V stage is released when both
+//                      halves are done with it.  Before the first P V of the
+//                      last tile it zeroes the V rows that were copied from
+//                      a page but lie past the tile's keys (a partly used
+//                      last page may hold anything, NaN included, and
+//                      0 * NaN would reach O).
+//   warps 0-3, 4-7:    one warpgroup per half; thread i owns row i of its
+//                      half = TMEM lane i: reads S with tcgen05.ld, masks
+//                      the keys its token may not see, keeps a lazy running
+//                      max (O is rescaled in TMEM only when the max grows by
+//                      more than 2^8), writes P in the input type into
+//                      shared memory in the swizzled K-major layout, and at
+//                      the end writes o = O / l in the input type and
+//                      lse = ln l + max straight to the outputs.  Two
+//                      independent softmax chains per SM keep the tensor
+//                      core fed while each waits on its own latencies.
 //                      For bf16, P is written as two bf16 terms (hi and the
-//                      rounding remainder lo) and P V is issued for both, so
-//                      the weights carry ~16 bits like the fp16 path
-//                      instead of bf16's 8.
+//                      rounding remainder lo; one P slot per half, single-
+//                      buffered) and P V is issued for both, so the weights
+//                      carry ~16 bits like the fp16 path instead of 8.
+// TMEM: S (half, buffer) at columns 64 (2 half + buffer), O of a half at
+// 256 + 128 half: all 512 columns, one CTA per SM.
 // Every mbarrier wait is bounded; on a timeout the kernel records it in the
 // workspace status word and unwinds instead of hanging.  Waits are by phase
 // parity, and every wait targets a barrier whose previous phase the waiting
@@ -57,34 +65,40 @@ namespace pa {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int kRows = 128;                  // tile rows (M): query tokens x G heads
+constexpr int kRows = 128;                  // rows of one MMA tile (M): query tokens x G heads
+constexpr int kHalves = 2;                  // MMA tiles per CTA, one softmax warpgroup each
 constexpr int kKeys = 64;                   // keys per K/V tile
-constexpr int kThreads = 32 * 6;            // 4 row warps, 1 TMA warp, 1 MMA warp
+constexpr int kThreads = 32 * 10;           // 8 softmax warps, 1 TMA warp, 1 MMA warp
+constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr int kQHalf = kRows * 128;         // 128 rows x 64 16-bit columns (16 KB)
 constexpr int kKVHalf = kKeys * 128;        // 64 keys x 64 16-bit columns (8 KB)
-constexpr int kQBytes = 2 * kQHalf;
+constexpr int kQBytes = 2 * kQHalf;         // one MMA tile of Q: 128 rows x 128 elements
 constexpr int kKVBytes = 2 * kKVHalf;
 constexpr int kPBytes = kRows * kKeys * 2;  // 128 rows x 64 keys, one 128-byte row each
-constexpr int kStages = 4;
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kStages = 3;
+constexpr int kOffQ = 0;                                  // Q of half 0, then half 1
+constexpr int kOffK = kOffQ + kHalves * kQBytes;
 constexpr int kOffV = kOffK + kStages * kKVBytes;
-constexpr int kOffP = kOffV + kStages * kKVBytes;  // two P buffers (+ two lo buffers for bf16)
-constexpr int kNumBars = 21;
-constexpr uint32_t kTmemCols = 256;  // S0 [0,64) S1 [64,128) O [128,256)
-constexpr uint32_t kColO = 128;
+constexpr int kOffP = kOffV + kStages * kKVBytes;         // 2 P slots per half
+constexpr int kOffBar = kOffP + kHalves * 2 * kPBytes;
+constexpr uint32_t kTmemCols = 512;  // S: 4 x 64 columns, O: 2 x 128 columns
+constexpr uint32_t kColO = 256;
 constexpr float kSlack = 8.f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr int kBarQ = 0, kBarFullK = 1, kBarFullV = 5, kBarEmpty = 9, kBarS = 13, kBarSFree = 15,
-              kBarPReady = 17, kBarPFree = 19;
+// mbarriers: Q, then per K/V stage full K, full V, empty; then per (half,
+// buffer) S ready, S read, P ready, P read.
+constexpr int kBarQ = 0, kBarFullK = 1, kBarFullV = kBarFullK + kStages,
+              kBarEmpty = kBarFullV + kStages, kBarS = kBarEmpty + kStages, kBarSFree = kBarS + 4,
+              kBarPReady = kBarSFree + 4, kBarPFree = kBarPReady + 4, kNumBars = kBarPFree + 4;
+constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 8 + 1024;  // + 1 KB alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
-template <typename Tag> struct Layout {
-  static constexpr bool kSplit = std::is_same<Tag, BF16>::value;  // P as hi + lo
-  static constexpr int kOffPLo = kOffP + 2 * kPBytes;
-  static constexpr int kOffBar = kOffP + (kSplit ? 4 : 2) * kPBytes;
-  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 8 + 1024;  // + 1 KB alignment slack
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+// fp16 double-buffers P per half; bf16 holds P as hi + lo in the same two
+// slots, single-buffered.
+template <typename Tag> struct PTraits {
+  static constexpr bool kSplit = std::is_same<Tag, BF16>::value;
+  static constexpr int kBufs = kSplit ? 1 : 2;
 };
 
 struct PrefillArgs {
@@ -128,13 +142,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v, const PrefillArgs a) {
-  using L = Layout<Tag>;
+  using PT = PTraits<Tag>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  auto bar = [&](int i) { return sb + L::kOffBar + 8 * i; };
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffBar + kNumBars * 8);
+  auto bar = [&](int i) { return sb + kOffBar + 8 * i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.group;
@@ -145,7 +159,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int page_begin = __ldg(&tp->page_begin);
   const int kv_base = __ldg(&tp->kv_base);
   const int kv_end = __ldg(&tp->kv_end);
-  const int ntiles = (kv_end + kKeys - 1) / kKeys;
+  // Half 0 holds tokens [0, per_half) of the tile, half 1 the rest; half 0's
+  // last token sees fewer keys, so it may need fewer K/V tiles.
+  const int per_half = kRows / G;
+  const int nq0 = min(n_q, per_half), nq1 = n_q - nq0;
+  const int nt0 = (min(kv_base + nq0, kv_end) + kKeys - 1) / kKeys;
+  const int nt1 = nq1 > 0 ? (kv_end + kKeys - 1) / kKeys : 0;
+  const int ntiles = max(nt0, nt1);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
@@ -154,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarFullV + s), 1);
       mbar_init(bar(kBarEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 4; ++s) {
       mbar_init(bar(kBarS + s), 1);
       mbar_init(bar(kBarSFree + s), 4);
       mbar_init(bar(kBarPReady + s), 4);
@@ -171,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == kWarpTma) {
     // ------------------------------ TMA producer ------------------------------
     // Lane j owns box j of every tile (a page, or a 64-row part of one): it
     // reads that page's index one tile ahead and issues the box's copies.
@@ -190,9 +210,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       return page * a.page_size + (key & pmask);
     };
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(kBarQ), kQBytes);
-      tc::tma_load_3d(sb + kOffQ, &tmap_q, 0, h * G, q_begin, bar(kBarQ));
-      tc::tma_load_3d(sb + kOffQ + kQHalf, &tmap_q, 64, h * G, q_begin, bar(kBarQ));
+      mbar_arrive_expect_tx(bar(kBarQ), kHalves * kQBytes);
+      for (int hf = 0; hf < kHalves; ++hf) {
+        const uint32_t dq = sb + kOffQ + hf * kQBytes;
+        tc::tma_load_3d(dq, &tmap_q, 0, h * G, q_begin + hf * per_half, bar(kBarQ));
+        tc::tma_load_3d(dq + kQHalf, &tmap_q, 64, h * G, q_begin + hf * per_half, bar(kBarQ));
+      }
     }
     int rowA = row_of(0), rowB = row_of(1);  // unrolled by two: no copy of a pending load
     auto produce = [&](int kt, int row) -> bool {
@@ -223,96 +246,114 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!ok && lane == 0) flag_timeout(a);
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ------------------------------ MMA issuer ------------------------------
-    // The whole warp runs the loop (it zeroes stale V rows before the last
-    // P V); lane 0 polls the barriers and issues, the others follow its
-    // decisions.
+    // The whole warp runs the loop (it zeroes stale V rows before the first
+    // P V of the last tile); lane 0 polls the barriers and issues, the others
+    // follow its decisions.  Each half runs its own S and P V sequence over
+    // the shared K/V ring; a stage is released once every half that uses the
+    // tile has issued its P V.
     // Rows [zero_from, zero_to) of the last tile were copied from the page
     // that holds the tile's last key but lie past it.
     const int zero_from = kv_end - (ntiles - 1) * kKeys;
     const int zero_to = min(kKeys, (zero_from + a.box_rows - 1) / a.box_rows * a.box_rows);
+    bool zeroed = !(ntiles > 0 && zero_from < zero_to);
     constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
     constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
     // descriptors are built once; a k-step adds its byte offset / 16
-    const uint64_t dq = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
+    const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
     const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffK, 16, 1024);
     const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffV, kKVHalf, 1024);
     const uint64_t dp0 = tc::smem_desc_sw128(sb + kOffP, 16, 1024);
+    const int nt[2] = {nt0, nt1};
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarQ), 0));
-    int ns = 0, npv = 0;
+    int ns[2] = {0, 0}, npv[2] = {0, 0};
     uint32_t idle = 0;
-    while (ok && npv < ntiles) {
+    while (ok && (npv[0] < nt[0] || npv[1] < nt[1])) {
       bool progress = false;
-      // S(ns) into buffer ns & 1, free once softmax has read S(ns - 2)
-      int go = 0;
-      if (lane == 0)
-        go = ns < ntiles && ns <= npv + 2 &&
-             (ns < 2 || mbar_try_wait(bar(kBarSFree + (ns & 1)), ((ns - 2) >> 1) & 1)) &&
-             mbar_try_wait(bar(kBarFullK + ns % kStages), (ns / kStages) & 1);
-      if (__shfl_sync(0xffffffffu, go, 0)) {
-        if (lane == 0) {
-          tc::fence_after_sync();
-          const uint64_t kd = dk0 + ((ns % kStages) * kKVBytes >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-            const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
-            tc::mma_f16_ss(tmem + (ns & 1) * kKeys, dq + off, kd + koff, kIdescQK, kk > 0);
-          }
-          tc::commit(bar(kBarS + (ns & 1)));
-        }
-        __syncwarp();
-        ++ns;
-        progress = true;
-      }
-      // O += P(npv) V(npv)
-      go = 0;
-      if (lane == 0)
-        go = npv < ns && mbar_try_wait(bar(kBarPReady + (npv & 1)), (npv >> 1) & 1) &&
-             mbar_try_wait(bar(kBarFullV + npv % kStages), (npv / kStages) & 1);
-      if (__shfl_sync(0xffffffffu, go, 0)) {
-        const int s = npv % kStages;
-        if (npv == ntiles - 1 && zero_from < zero_to) {
-          // every lane observes the landed copy itself before overwriting it
-          const bool landed = mbar_wait(bar(kBarFullV + s), (npv / kStages) & 1);
-          if (landed) {
-            uint8_t* vt = smem + kOffV + s * kKVBytes;
-            const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
-            for (int c = lane; c < n16; c += 32) {
-              const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
-              *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
-                  make_uint4(0u, 0u, 0u, 0u);
+      for (int hf = 0; hf < kHalves; ++hf) {
+        // S(ns) of this half into its buffer ns & 1, free once the half's
+        // softmax has read S(ns - 2)
+        int go = 0;
+        const int n = ns[hf];
+        if (lane == 0)
+          go = n < nt[hf] && n <= npv[hf] + 2 &&
+               (n < 2 || mbar_try_wait(bar(kBarSFree + 2 * hf + (n & 1)), ((n - 2) >> 1) & 1)) &&
+               mbar_try_wait(bar(kBarFullK + n % kStages), (n / kStages) & 1);
+        if (__shfl_sync(0xffffffffu, go, 0)) {
+          if (lane == 0) {
+            tc::fence_after_sync();
+            const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
+            const uint64_t kd = dk0 + ((n % kStages) * kKVBytes >> 4);
+            const uint32_t dst = tmem + (2 * hf + (n & 1)) * kKeys;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+              const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+              tc::mma_f16_ss(dst, qd + off, kd + koff, kIdescQK, kk > 0);
             }
-            fence_proxy_async_smem();
+            tc::commit(bar(kBarS + 2 * hf + (n & 1)));
           }
-          __syncwarp();  // the zeros are written (and fenced) before lane 0 issues
-          if (!__all_sync(0xffffffffu, landed)) {
-            ok = false;
-            break;
-          }
+          __syncwarp();
+          ns[hf] = n + 1;
+          progress = true;
         }
-        if (lane == 0) {
-          tc::fence_after_sync();
-          const uint64_t pd = dp0 + (((npv & 1) * kPBytes) >> 4);
-          const uint64_t vd = dv0 + ((s * kKVBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < kKeys / 16; ++kk)
-            tc::mma_f16_ss(tmem + kColO, pd + ((kk * 32) >> 4), vd + ((kk * 16 * 128) >> 4),
-                           kIdescPV, (npv > 0 || kk > 0) ? 1u : 0u);
-          if (L::kSplit) {
-            const uint64_t pl = pd + ((L::kOffPLo - kOffP) >> 4);
+        // O(half) += P(npv) V(npv)
+        go = 0;
+        const int v = npv[hf];
+        const int pb = v % PT::kBufs;
+        if (lane == 0)
+          go = v < ns[hf] &&
+               mbar_try_wait(bar(kBarPReady + 2 * hf + pb), (v / PT::kBufs) & 1) &&
+               mbar_try_wait(bar(kBarFullV + v % kStages), (v / kStages) & 1);
+        if (__shfl_sync(0xffffffffu, go, 0)) {
+          const int s = v % kStages;
+          if (!zeroed && v == ntiles - 1) {
+            // every lane observes the landed copy itself before overwriting it
+            const bool landed = mbar_wait(bar(kBarFullV + s), (v / kStages) & 1);
+            if (landed) {
+              uint8_t* vt = smem + kOffV + s * kKVBytes;
+              const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
+              for (int c = lane; c < n16; c += 32) {
+                const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
+                *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+              }
+              fence_proxy_async_smem();
+            }
+            __syncwarp();  // the zeros are written (and fenced) before lane 0 issues
+            if (!__all_sync(0xffffffffu, landed)) {
+              ok = false;
+              break;
+            }
+            zeroed = true;
+          }
+          if (lane == 0) {
+            tc::fence_after_sync();
+            const uint64_t pd = dp0 + (((2 * hf + pb) * kPBytes) >> 4);
+            const uint64_t vd = dv0 + ((s * kKVBytes) >> 4);
+            const uint32_t dst = tmem + kColO + hf * D;
 #pragma unroll
             for (int kk = 0; kk < kKeys / 16; ++kk)
-              tc::mma_f16_ss(tmem + kColO, pl + ((kk * 32) >> 4), vd + ((kk * 16 * 128) >> 4),
-                             kIdescPV, 1u);
+              tc::mma_f16_ss(dst, pd + ((kk * 32) >> 4), vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                             (v > 0 || kk > 0) ? 1u : 0u);
+            if (PT::kSplit) {  // the lo term sits in the half's second slot
+              const uint64_t pl = pd + (kPBytes >> 4);
+#pragma unroll
+              for (int kk = 0; kk < kKeys / 16; ++kk)
+                tc::mma_f16_ss(dst, pl + ((kk * 32) >> 4), vd + ((kk * 16 * 128) >> 4),
+                               kIdescPV, 1u);
+            }
+            tc::commit(bar(kBarPFree + 2 * hf + pb));
+            // the stage is free once the other half is done with this tile too
+            const int other = 1 - hf;
+            if (npv[other] > v || v >= nt[other]) tc::commit(bar(kBarEmpty + s));
           }
-          tc::commit(bar(kBarPFree + (npv & 1)));
-          tc::commit(bar(kBarEmpty + s));
+          __syncwarp();
+          npv[hf] = v + 1;
+          progress = true;
         }
-        __syncwarp();
-        ++npv;
-        progress = true;
       }
       idle = progress ? 0u : idle + 1u;
       if (idle > kSpinLimit) ok = false;
@@ -320,37 +361,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) flag_timeout(a);
   } else {
     // ------------------------- softmax / epilogue rows -------------------------
-    const int i = threadIdx.x;  // tile row == TMEM lane
-    const int jq = i / G, jh = i - jq * G;
-    // keys this row may see (rows past the tile's tokens: all of the tile's keys)
+    const int hf = warp >> 2;              // which half (warpgroup)
+    const int i = threadIdx.x & 127;       // row within the half == TMEM lane
+    const int jq = hf * per_half + i / G;  // token within the tile
+    const int jh = i % G;
+    const int nt = hf ? nt1 : nt0;
+    const int nqh = hf ? nq1 : nq0;
+    // keys this row may see (rows past the tile's tokens: all of the tile's
+    // keys), and the fewest any row of the half sees
     const int lim = min(kv_base + jq + 1, kv_end);
-    const uint32_t lane_addr = tmem + (uint32_t(warp * 32) << 16);
+    const int lim_min = min(kv_base + hf * per_half + 1, kv_end);
+    const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16);
+    const uint32_t col_s = 2 * hf * kKeys, col_o = kColO + hf * D;
+    uint8_t* p_slots = smem + kOffP + 2 * hf * kPBytes;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int kt = 0; kt < ntiles; ++kt) {
+    for (int kt = 0; kt < nt; ++kt) {
       const int s = kt & 1;  // S buffer
-      ok = mbar_wait(bar(kBarS + s), (kt >> 1) & 1);
+      ok = mbar_wait(bar(kBarS + 2 * hf + s), (kt >> 1) & 1);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::fence_after_sync();
       float x[kKeys];
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
         float t32[32];
-        tc::tmem_ld32(lane_addr + s * kKeys + 32 * c, t32);
+        tc::tmem_ld32(lane_addr + col_s + s * kKeys + 32 * c, t32);
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[32 * c + e] = t32[e];
       }
       tc::tmem_wait_ld();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarSFree + s));
+      if (lane == 0) mbar_arrive(bar(kBarSFree + 2 * hf + s));
 
       // Raw scores; the scale is folded into the exponent argument below.
       // Keys at or past a row's limit are masked (a select: the score of a
-      // stale row may be anything).  Tiles wholly below the first token's
-      // limit need no mask (uniform branch).
+      // stale row may be anything).  Tiles wholly below every row's limit
+      // need no mask (uniform branch).
       const int key0 = kt * kKeys;
-      if (key0 + kKeys > kv_base + 1) {
+      if (key0 + kKeys > lim_min) {
 #pragma unroll
         for (int c = 0; c < kKeys; ++c) x[c] = key0 + c < lim ? x[c] : -INFINITY;
       }
@@ -361,76 +410,78 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool moved = tmax > m + kSlack;
       const float mnew = moved ? tmax : m;
       const float alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
-      // P = 2^(s * scale - m) in the input type (l sums exactly what the
-      // tensor core multiplies), computed before waiting on the tensor core.
-      const float nm = -mnew;
-      uint32_t w[kKeys / 2];
-      uint32_t wl[L::kSplit ? kKeys / 2 : 1];
-      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int e = 0; e < kKeys / 2; ++e) {
-        const float p0 = fast_exp2(fmaf(x[2 * e], a.score_scale, nm));
-        const float p1 = fast_exp2(fmaf(x[2 * e + 1], a.score_scale, nm));
-        float r0, r1;
-        w[e] = pack2(Tag{}, p0, p1, r0, r1);
-        if constexpr (L::kSplit) {
-          float q0, q1;
-          wl[e] = pack2(Tag{}, p0 - r0, p1 - r1, q0, q1);
-          r0 += q0;
-          r1 += q1;
-        }
-        ps4[e & 3] += r0 + r1;
-      }
-      const float psum = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
-      l = l * alpha + psum;
-      m = mnew;
       // O is rescaled in TMEM once the previous tile's P V is complete,
-      // waited for on the P buffer it read: this thread already saw that
-      // barrier's previous phase (P V of tile kt - 3), so the parity is exact.
+      // waited for on the P slot it read.  This thread already saw that
+      // barrier's previous phase (when it last refilled the slot), so the
+      // parity is exact.
       if (kt > 0 && __any_sync(0xffffffffu, moved)) {
-        ok = mbar_wait(bar(kBarPFree + ((kt - 1) & 1)), ((kt - 1) >> 1) & 1);
+        const int pv = kt - 1;
+        ok = mbar_wait(bar(kBarPFree + 2 * hf + pv % PT::kBufs), (pv / PT::kBufs) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc::fence_after_sync();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float ov[32];
-          tc::tmem_ld32(lane_addr + kColO + 32 * c, ov);
+          tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-          tc::tmem_st32(lane_addr + kColO + 32 * c, ov);
+          tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
         }
         tc::tmem_wait_st();
       }
-      // This tile's P buffer was last read by the P V of tile kt - 2.
-      if (kt >= 2) {
-        ok = mbar_wait(bar(kBarPFree + (kt & 1)), ((kt - 2) >> 1) & 1);
+      // This tile's P slot was last read by the P V of tile kt - kBufs.
+      const int pb = kt % PT::kBufs;
+      if (kt >= PT::kBufs) {
+        const int pv = kt - PT::kBufs;
+        ok = mbar_wait(bar(kBarPFree + 2 * hf + pb), (pv / PT::kBufs) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
       }
-      uint8_t* prow = smem + kOffP + (kt & 1) * kPBytes + i * 128;
+      // P = 2^(s * scale - m) in the input type, eight keys (one 16-byte
+      // chunk of the swizzled 128-byte row) at a time; l sums what the
+      // tensor core multiplies.
+      const float nm = -mnew;
+      uint8_t* prow = p_slots + pb * kPBytes + i * 128;
+      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c8 = 0; c8 < kKeys / 8; ++c8)  // 16-byte chunk c8 of the 128-byte row
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (i & 7)) << 4)) =
-            make_uint4(w[4 * c8], w[4 * c8 + 1], w[4 * c8 + 2], w[4 * c8 + 3]);
-      if constexpr (L::kSplit) {
-        uint8_t* lrow = prow + (L::kOffPLo - kOffP);
+      for (int c8 = 0; c8 < kKeys / 8; ++c8) {
+        uint32_t w[4], wl[4];
 #pragma unroll
-        for (int c8 = 0; c8 < kKeys / 8; ++c8)
-          *reinterpret_cast<uint4*>(lrow + ((c8 ^ (i & 7)) << 4)) =
-              make_uint4(wl[4 * c8], wl[4 * c8 + 1], wl[4 * c8 + 2], wl[4 * c8 + 3]);
+        for (int e = 0; e < 4; ++e) {
+          const int c = 8 * c8 + 2 * e;
+          const float p0 = fast_exp2(fmaf(x[c], a.score_scale, nm));
+          const float p1 = fast_exp2(fmaf(x[c + 1], a.score_scale, nm));
+          float r0, r1;
+          w[e] = pack2(Tag{}, p0, p1, r0, r1);
+          if constexpr (PT::kSplit) {  // hi + lo carries p to ~2^-16: sum p itself
+            float q0, q1;
+            wl[e] = pack2(Tag{}, p0 - r0, p1 - r1, q0, q1);
+            ps4[e] += p0 + p1;
+          } else {
+            ps4[e] += r0 + r1;
+          }
+        }
+        *reinterpret_cast<uint4*>(prow + ((c8 ^ (i & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        if constexpr (PT::kSplit)  // the lo term in the half's second slot
+          *reinterpret_cast<uint4*>(prow + kPBytes + ((c8 ^ (i & 7)) << 4)) =
+              make_uint4(wl[0], wl[1], wl[2], wl[3]);
       }
+      l = l * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
+      m = mnew;
       fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarPReady + (kt & 1)));
+      if (lane == 0) mbar_arrive(bar(kBarPReady + 2 * hf + pb));
     }
     // epilogue: o = O / l in the input type and lse = (m + log2 l) ln 2; a
-    // tile without keys (no mask, empty request) writes o = 0, lse = -inf
-    if (ok && ntiles > 0)
-      ok = mbar_wait(bar(kBarPFree + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1);
+    // half without keys (no mask, empty request) writes o = 0, lse = -inf
+    if (ok && nt > 0) {
+      const int pv = nt - 1;
+      ok = mbar_wait(bar(kBarPFree + 2 * hf + pv % PT::kBufs), (pv / PT::kBufs) & 1);
+    }
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (!all_ok && lane == 0) flag_timeout(a);
-    if (all_ok) {
+    if (all_ok && nqh > 0) {
       tc::fence_after_sync();
       const bool valid = jq < n_q;
       const int64_t orow = int64_t(q_begin + jq) * a.num_qo_heads + h * G + jh;
@@ -439,8 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float ov[32];
-        if (ntiles > 0) {
-          tc::tmem_ld32(lane_addr + kColO + 32 * c, ov);
+        if (nt > 0) {
+          tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
           tc::tmem_wait_ld();
         } else {
 #pragma unroll
@@ -501,7 +552,7 @@ template <typename Tag, bool kCheck>
 cudaError_t launch_t(const PrefillArgs& args, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t stream) {
   auto kern = paged_prefill_kernel<Tag, kCheck>;
-  constexpr int smem = Layout<Tag>::kSmemBytes;
+  constexpr int smem = kSmemBytes;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -52,8 +52,8 @@ def _check(w, dev, o_ref, l_ref, causal, what):
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 def test_prefill_small(dtype, group):
     """Fresh prefill, append, single-token append and an idle request; keys
-    span several 64-key tiles with ragged ends; query tiles of 128 / G tokens
-    with a ragged last one."""
+    span several 64-key tiles with ragged ends; query tiles of 256 / G tokens
+    (two halves of 128 / G) with ragged last ones, some without a second half."""
     hkv = 2
     kv = [200, 77, 1, 150, 64]
     qo = [200, 40, 1, 0, 33]
@@ -105,7 +105,7 @@ def test_stale_rows_of_partly_used_pages_do_not_leak(dtype):
 
 
 def test_prefill_many_tiles_per_request():
-    """One long fresh prefill (1000 tokens, 32 tiles at G = 4) next to short
+    """One long fresh prefill (1000 tokens, 16 tiles at G = 4) next to short
     appends: tiles of very different lengths in one launch."""
     w = W.make_workload("pf_long", [1000, 300, 2000], num_qo_heads=32, num_kv_heads=8,
                         page_size=16, dtype="bf16", seed=140, qo_lens=[1000, 17, 130])

@@ -1,5 +1,5 @@
 """The prefill / append plan on the host (no GPU): its tiles cover every new
-query token of every request exactly once, in runs of at most 128 / G
+query token of every request exactly once, in runs of at most 256 / G
 tokens of one request, with the key range of the causal rule (or all keys
 without the mask), longest first; malformed tables are rejected before
 anything runs."""
@@ -31,8 +31,8 @@ def _tables(kv_lens, P):
 
 
 def _expected_tiles(kv_lens, qo_lens, G, causal):
-    """The tile rule written out: per request, runs of 128 / G new tokens."""
-    per = 128 // G
+    """The tile rule written out: per request, runs of 256 / G new tokens."""
+    per = 256 // G
     out, qo = [], 0
     indptr, _ = _tables(kv_lens, 16)
     for b, (L, Q) in enumerate(zip(kv_lens, qo_lens)):
@@ -69,7 +69,7 @@ def test_tiles_cover_every_query_once_longest_first(C, causal, hq, hkv):
     # every new token of every request exactly once
     seen = np.zeros(qo_indptr[-1], np.int32)
     for r, q0, n, pb, base, end in tiles:
-        assert 1 <= n <= 128 // G and pb == indptr[r]
+        assert 1 <= n <= 256 // G and pb == indptr[r]
         assert qo_indptr[r] <= q0 and q0 + n <= qo_indptr[r + 1]
         seen[q0:q0 + n] += 1
     assert np.all(seen == 1)
@@ -83,7 +83,7 @@ def test_tiles_of_the_prefill_workload(C):
                                     w.last_page_len)
     tiles = C.pa_plan_prefill_tiles(plan)
     G = w.num_qo_heads // w.num_kv_heads
-    assert len(tiles) == w.batch * (1024 // (128 // G))
+    assert len(tiles) == w.batch * (1024 // (256 // G))
     # the last token of each request sees every key of it
     lens = w.kv_lens()
     for r in range(w.batch):
