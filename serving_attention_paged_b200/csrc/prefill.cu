@@ -17,34 +17,37 @@
 // (head-query fusion) and both halves.  The host plan lists the tiles
 // longest first, so the block scheduler starts the long ones first.
 //   warp 8  (TMA):     both halves of Q once; K and V of each 64-key tile as
-//                      page-row boxes, 128-byte swizzle, into a 3-stage ring;
+//                      page-row boxes, 128-byte swizzle, into a 5-stage ring;
 //                      boxes wholly past the tile's last key read out of
 //                      range (zero fill).
 //   warp 9  (MMA):     per half, S = Q K^T into one of two TMEM buffers
-//                      (M = 128, N = 64, K = 128) and O += P V (V as an
-//                      MN-major operand) into the half's O; completion goes
-//                      to mbarriers, and a K/V stage is released when both
-//                      halves are done with it.  Before the first P V of the
-//                      last tile it zeroes the V rows that were copied from
-//                      a page but lie past the tile's keys (a partly used
-//                      last page may hold anything, NaN included, and
-//                      0 * NaN would reach O).
+//                      (M = 128, N = 64, K = 128) and O += P V with P read
+//                      from TMEM (V an MN-major operand in shared memory)
+//                      into the half's O; completion goes to mbarriers, and
+//                      a K/V stage is released when both halves are done
+//                      with it.  Before the first P V of the last tile it
+//                      zeroes the V rows that were copied from a page but
+//                      lie past the tile's keys (a partly used last page may
+//                      hold anything, NaN included, and 0 * NaN would reach
+//                      O).
 //   warps 0-3, 4-7:    one warpgroup per half; thread i owns row i of its
 //                      half = TMEM lane i: reads S with tcgen05.ld, masks
 //                      the keys its token may not see, keeps a lazy running
 //                      max (O is rescaled in TMEM only when the max grows by
-//                      more than 2^8), writes P in the input type into
-//                      shared memory in the swizzled K-major layout, and at
-//                      the end writes o = O / l in the input type and
-//                      lse = ln l + max straight to the outputs.  Two
-//                      independent softmax chains per SM keep the tensor
-//                      core fed while each waits on its own latencies.
-//                      For bf16, P is written as two bf16 terms (hi and the
-//                      rounding remainder lo; one P slot per half, single-
-//                      buffered) and P V is issued for both, so the weights
-//                      carry ~16 bits like the fp16 path instead of 8.
-// TMEM: S (half, buffer) at columns 64 (2 half + buffer), O of a half at
-// 256 + 128 half: all 512 columns, one CTA per SM.
+//                      more than 2^8), writes P in the input type over S in
+//                      TMEM with tcgen05.st, and at the end writes o = O / l
+//                      in the input type and lse = ln l + max straight to
+//                      the outputs.  Two independent softmax chains per SM
+//                      keep the tensor core fed while each waits on its own
+//                      latencies.  For bf16, P is written as two bf16 terms
+//                      (hi and the rounding remainder lo, in the buffer's
+//                      two 32-column halves) and P V is issued for both, so
+//                      the weights carry ~16 bits like the fp16 path
+//                      instead of 8.
+// TMEM: S / P (half, buffer) at columns 64 (2 half + buffer), O of a half at
+// 256 + 128 half: all 512 columns, one CTA per SM.  Keeping P out of shared
+// memory leaves room for five K/V stages: the K/V tiles come through L2 with
+// microseconds of latency, and the ring depth sets how many are in flight.
 // Every mbarrier wait is bounded; on a timeout the kernel records it in the
 // workspace status word and unwinds instead of hanging.  Waits are by phase
 // parity, and every wait targets a barrier whose previous phase the waiting
@@ -74,31 +77,28 @@ constexpr int kQHalf = kRows * 128;         // 128 rows x 64 16-bit columns (16 
 constexpr int kKVHalf = kKeys * 128;        // 64 keys x 64 16-bit columns (8 KB)
 constexpr int kQBytes = 2 * kQHalf;         // one MMA tile of Q: 128 rows x 128 elements
 constexpr int kKVBytes = 2 * kKVHalf;
-constexpr int kPBytes = kRows * kKeys * 2;  // 128 rows x 64 keys, one 128-byte row each
-constexpr int kStages = 3;
+constexpr int kStages = 5;
 constexpr int kOffQ = 0;                                  // Q of half 0, then half 1
 constexpr int kOffK = kOffQ + kHalves * kQBytes;
 constexpr int kOffV = kOffK + kStages * kKVBytes;
-constexpr int kOffP = kOffV + kStages * kKVBytes;         // 2 P slots per half
-constexpr int kOffBar = kOffP + kHalves * 2 * kPBytes;
+constexpr int kOffBar = kOffV + kStages * kKVBytes;
 constexpr uint32_t kTmemCols = 512;  // S: 4 x 64 columns, O: 2 x 128 columns
 constexpr uint32_t kColO = 256;
 constexpr float kSlack = 8.f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // mbarriers: Q, then per K/V stage full K, full V, empty; then per (half,
-// buffer) S ready, S read, P ready, P read.
+// buffer) S ready, P ready (in TMEM, over S), P V done.
 constexpr int kBarQ = 0, kBarFullK = 1, kBarFullV = kBarFullK + kStages,
-              kBarEmpty = kBarFullV + kStages, kBarS = kBarEmpty + kStages, kBarSFree = kBarS + 4,
-              kBarPReady = kBarSFree + 4, kBarPFree = kBarPReady + 4, kNumBars = kBarPFree + 4;
+              kBarEmpty = kBarFullV + kStages, kBarS = kBarEmpty + kStages,
+              kBarPReady = kBarS + 4, kBarPFree = kBarPReady + 4, kNumBars = kBarPFree + 4;
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 8 + 1024;  // + 1 KB alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
-// fp16 double-buffers P per half; bf16 holds P as hi + lo in the same two
-// slots, single-buffered.
+// P is written over its own S in TMEM: 64 keys of 16 bits fill 32 of the
+// buffer's 64 columns; bf16 puts its lo term in the other 32.
 template <typename Tag> struct PTraits {
   static constexpr bool kSplit = std::is_same<Tag, BF16>::value;
-  static constexpr int kBufs = kSplit ? 1 : 2;
 };
 
 struct PrefillArgs {
@@ -176,7 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 4; ++s) {
       mbar_init(bar(kBarS + s), 1);
-      mbar_init(bar(kBarSFree + s), 4);
       mbar_init(bar(kBarPReady + s), 4);
       mbar_init(bar(kBarPFree + s), 1);
     }
@@ -264,7 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
     const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffK, 16, 1024);
     const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffV, kKVHalf, 1024);
-    const uint64_t dp0 = tc::smem_desc_sw128(sb + kOffP, 16, 1024);
     const int nt[2] = {nt0, nt1};
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarQ), 0));
     int ns[2] = {0, 0}, npv[2] = {0, 0};
@@ -273,13 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool progress = false;
 #pragma unroll
       for (int hf = 0; hf < kHalves; ++hf) {
-        // S(ns) of this half into its buffer ns & 1, free once the half's
-        // softmax has read S(ns - 2)
+        // S(ns) of this half into its buffer ns & 1, free once P V(ns - 2)
+        // has read the P written over S(ns - 2).  This thread waits for every
+        // P V of a buffer in order, so the parity is exact.
         int go = 0;
         const int n = ns[hf];
         if (lane == 0)
-          go = n < nt[hf] && n <= npv[hf] + 2 &&
-               (n < 2 || mbar_try_wait(bar(kBarSFree + 2 * hf + (n & 1)), ((n - 2) >> 1) & 1)) &&
+          go = n < nt[hf] && n <= npv[hf] + 1 &&
+               (n < 2 || mbar_try_wait(bar(kBarPFree + 2 * hf + (n & 1)), ((n - 2) >> 1) & 1)) &&
                mbar_try_wait(bar(kBarFullK + n % kStages), (n / kStages) & 1);
         if (__shfl_sync(0xffffffffu, go, 0)) {
           if (lane == 0) {
@@ -299,13 +298,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ns[hf] = n + 1;
           progress = true;
         }
-        // O(half) += P(npv) V(npv)
+        // O(half) += P(npv) V(npv), P read from TMEM
         go = 0;
         const int v = npv[hf];
-        const int pb = v % PT::kBufs;
+        const int pb = v & 1;
         if (lane == 0)
-          go = v < ns[hf] &&
-               mbar_try_wait(bar(kBarPReady + 2 * hf + pb), (v / PT::kBufs) & 1) &&
+          go = v < ns[hf] && mbar_try_wait(bar(kBarPReady + 2 * hf + pb), (v >> 1) & 1) &&
                mbar_try_wait(bar(kBarFullV + v % kStages), (v / kStages) & 1);
         if (__shfl_sync(0xffffffffu, go, 0)) {
           const int s = v % kStages;
@@ -331,18 +329,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (lane == 0) {
             tc::fence_after_sync();
-            const uint64_t pd = dp0 + (((2 * hf + pb) * kPBytes) >> 4);
+            const uint32_t pt = tmem + (2 * hf + pb) * kKeys;  // P over S(v)
             const uint64_t vd = dv0 + ((s * kKVBytes) >> 4);
             const uint32_t dst = tmem + kColO + hf * D;
 #pragma unroll
             for (int kk = 0; kk < kKeys / 16; ++kk)
-              tc::mma_f16_ss(dst, pd + ((kk * 32) >> 4), vd + ((kk * 16 * 128) >> 4), kIdescPV,
+              tc::mma_f16_ts(dst, pt + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
                              (v > 0 || kk > 0) ? 1u : 0u);
-            if (PT::kSplit) {  // the lo term sits in the half's second slot
-              const uint64_t pl = pd + (kPBytes >> 4);
+            if (PT::kSplit) {  // the lo term in the buffer's other 32 columns
 #pragma unroll
               for (int kk = 0; kk < kKeys / 16; ++kk)
-                tc::mma_f16_ss(dst, pl + ((kk * 32) >> 4), vd + ((kk * 16 * 128) >> 4),
+                tc::mma_f16_ts(dst, pt + kKeys / 2 + kk * 8, vd + ((kk * 16 * 128) >> 4),
                                kIdescPV, 1u);
             }
             tc::commit(bar(kBarPFree + 2 * hf + pb));
@@ -373,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lim_min = min(kv_base + hf * per_half + 1, kv_end);
     const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16);
     const uint32_t col_s = 2 * hf * kKeys, col_o = kColO + hf * D;
-    uint8_t* p_slots = smem + kOffP + 2 * hf * kPBytes;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int kt = 0; kt < nt; ++kt) {
@@ -390,9 +386,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; ++e) x[32 * c + e] = t32[e];
       }
       tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarSFree + 2 * hf + s));
 
       // Raw scores; the scale is folded into the exponent argument below.
       // Keys at or past a row's limit are masked (a select: the score of a
@@ -410,45 +403,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool moved = tmax > m + kSlack;
       const float mnew = moved ? tmax : m;
       const float alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
-      // O is rescaled in TMEM once the previous tile's P V is complete,
-      // waited for on the P slot it read.  This thread already saw that
-      // barrier's previous phase (when it last refilled the slot), so the
-      // parity is exact.
-      if (kt > 0 && __any_sync(0xffffffffu, moved)) {
+      // The previous tile's P V must be complete before O is rescaled; it is
+      // waited for every tile, so this thread sees every phase of the
+      // barrier in order and the parity is exact.
+      if (kt > 0) {
         const int pv = kt - 1;
-        ok = mbar_wait(bar(kBarPFree + 2 * hf + pv % PT::kBufs), (pv / PT::kBufs) & 1);
+        ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
-        tc::fence_after_sync();
+        if (__any_sync(0xffffffffu, moved)) {
+          tc::fence_after_sync();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float ov[32];
-          tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
-          tc::tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
+            tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-          tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
+          }
         }
-        tc::tmem_wait_st();
       }
-      // This tile's P slot was last read by the P V of tile kt - kBufs.
-      const int pb = kt % PT::kBufs;
-      if (kt >= PT::kBufs) {
-        const int pv = kt - PT::kBufs;
-        ok = mbar_wait(bar(kBarPFree + 2 * hf + pb), (pv / PT::kBufs) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      // P = 2^(s * scale - m) in the input type, eight keys (one 16-byte
-      // chunk of the swizzled 128-byte row) at a time; l sums what the
-      // tensor core multiplies.
+      // P = 2^(s * scale - m) in the input type, written over S in TMEM (the
+      // P V that last read this buffer finished before S was written), 32
+      // keys at a time; l sums what the tensor core multiplies.
       const float nm = -mnew;
-      uint8_t* prow = p_slots + pb * kPBytes + i * 128;
+      const uint32_t p_addr = lane_addr + col_s + s * kKeys;
       float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c8 = 0; c8 < kKeys / 8; ++c8) {
-        uint32_t w[4], wl[4];
+      for (int c16 = 0; c16 < kKeys / 32; ++c16) {
+        uint32_t w[16], wl[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 8 * c8 + 2 * e;
+        for (int e = 0; e < 16; ++e) {
+          const int c = 32 * c16 + 2 * e;
           const float p0 = fast_exp2(fmaf(x[c], a.score_scale, nm));
           const float p1 = fast_exp2(fmaf(x[c + 1], a.score_scale, nm));
           float r0, r1;
@@ -456,28 +442,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (PT::kSplit) {  // hi + lo carries p to ~2^-16: sum p itself
             float q0, q1;
             wl[e] = pack2(Tag{}, p0 - r0, p1 - r1, q0, q1);
-            ps4[e] += p0 + p1;
+            ps4[e & 3] += p0 + p1;
           } else {
-            ps4[e] += r0 + r1;
+            ps4[e & 3] += r0 + r1;
           }
         }
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (i & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        if constexpr (PT::kSplit)  // the lo term in the half's second slot
-          *reinterpret_cast<uint4*>(prow + kPBytes + ((c8 ^ (i & 7)) << 4)) =
-              make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        tc::tmem_st16(p_addr + 16 * c16, w);
+        if constexpr (PT::kSplit) tc::tmem_st16(p_addr + kKeys / 2 + 16 * c16, wl);
       }
       l = l * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
       m = mnew;
-      fence_proxy_async_smem();
+      tc::tmem_wait_st();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarPReady + 2 * hf + pb));
+      if (lane == 0) mbar_arrive(bar(kBarPReady + 2 * hf + s));
     }
     // epilogue: o = O / l in the input type and lse = (m + log2 l) ln 2; a
     // half without keys (no mask, empty request) writes o = 0, lse = -inf
     if (ok && nt > 0) {
       const int pv = nt - 1;
-      ok = mbar_wait(bar(kBarPFree + 2 * hf + pv % PT::kBufs), (pv / PT::kBufs) & 1);
+      ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
     }
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (!all_ok && lane == 0) flag_timeout(a);
