@@ -249,7 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ MMA issuer ------------------------------
     // The whole warp runs the loop (it zeroes stale V rows before the first
     // P V of the last tile); lane 0 polls the barriers and issues, the others
-    // follow its decisions.  Each half runs its own S and P V sequence over
+    // follow its decisions.  Polling uses test_wait, which never suspends:
+    // try_wait on a barrier that is not ready may park the thread for a
+    // while, delaying work another barrier has already released.  Each half runs its own S and P V sequence over
     // the shared K/V ring; a stage is released once every half that uses the
     // tile has issued its P V.
     // Rows [zero_from, zero_to) of the last tile were copied from the page
@@ -278,8 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = ns[hf];
         if (lane == 0)
           go = n < nt[hf] && n <= npv[hf] + 1 &&
-               (n < 2 || mbar_try_wait(bar(kBarPFree + 2 * hf + (n & 1)), ((n - 2) >> 1) & 1)) &&
-               mbar_try_wait(bar(kBarFullK + n % kStages), (n / kStages) & 1);
+               (n < 2 ||
+                mbar_test_wait(bar(kBarPFree + 2 * hf + (n & 1)), ((n - 2) >> 1) & 1)) &&
+               mbar_test_wait(bar(kBarFullK + n % kStages), (n / kStages) & 1);
         if (__shfl_sync(0xffffffffu, go, 0)) {
           if (lane == 0) {
             tc::fence_after_sync();
@@ -303,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int v = npv[hf];
         const int pb = v & 1;
         if (lane == 0)
-          go = v < ns[hf] && mbar_try_wait(bar(kBarPReady + 2 * hf + pb), (v >> 1) & 1) &&
-               mbar_try_wait(bar(kBarFullV + v % kStages), (v / kStages) & 1);
+          go = v < ns[hf] && mbar_test_wait(bar(kBarPReady + 2 * hf + pb), (v >> 1) & 1) &&
+               mbar_test_wait(bar(kBarFullV + v % kStages), (v / kStages) & 1);
         if (__shfl_sync(0xffffffffu, go, 0)) {
           const int s = v % kStages;
           if (!zeroed && v == ntiles - 1) {
