@@ -247,18 +247,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) flag_timeout(a);
   } else if (warp == kWarpMma) {
     // ------------------------------ MMA issuer ------------------------------
-    // The whole warp runs the loop (it zeroes stale V rows before the first
-    // P V of the last tile); lane 0 polls the barriers and issues, the others
-    // follow its decisions.  Polling uses test_wait, which never suspends:
-    // try_wait on a barrier that is not ready may park the thread for a
-    // while, delaying work another barrier has already released.  Each half runs its own S and P V sequence over
-    // the shared K/V ring; a stage is released once every half that uses the
-    // tile has issued its P V.
+    // The whole warp runs the schedule (it zeroes stale V rows before the
+    // P V of the last tile); every lane waits, lane 0 issues.  Each half runs
+    // its own S and P V sequence over the shared K/V ring; a stage is
+    // released once every half that uses the tile has issued its P V.
     // Rows [zero_from, zero_to) of the last tile were copied from the page
     // that holds the tile's last key but lie past it.
     const int zero_from = kv_end - (ntiles - 1) * kKeys;
     const int zero_to = min(kKeys, (zero_from + a.box_rows - 1) / a.box_rows * a.box_rows);
-    bool zeroed = !(ntiles > 0 && zero_from < zero_to);
     constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
     constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
     // descriptors are built once; a k-step adds its byte offset / 16
@@ -266,73 +262,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffK, 16, 1024);
     const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffV, kKVHalf, 1024);
     const int nt[2] = {nt0, nt1};
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarQ), 0));
-    int ns[2] = {0, 0}, npv[2] = {0, 0};
-    uint32_t idle = 0;
-    while (ok && (npv[0] < nt[0] || npv[1] < nt[1])) {
-      bool progress = false;
+    // Fixed order, one blocking wait per input: S of tile kt for both halves,
+    // then P V of tile kt - 1 for both.  The softmax of a half always finds
+    // the next S issued while it works on the current tile.  S(kt) goes into
+    // the buffer P V(kt - 2) read P from, so it waits for that P V to finish;
+    // this warp waits for every P V of a buffer in order, so the parity is
+    // exact.
+    // Every lane waits and ok stays warp-uniform, so the lanes take the same
+    // branches to the __syncwarp calls.
+    auto wait_all = [&](int b, int parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar(b), parity));
+    };
+    bool ok = wait_all(kBarQ, 0);
+    for (int kt = 0; ok && kt <= ntiles; ++kt) {
+      if (kt < ntiles) {
+        const int s = kt % kStages;
+        ok = wait_all(kBarFullK + s, (kt / kStages) & 1);
 #pragma unroll
-      for (int hf = 0; hf < kHalves; ++hf) {
-        // S(ns) of this half into its buffer ns & 1, free once P V(ns - 2)
-        // has read the P written over S(ns - 2).  This thread waits for every
-        // P V of a buffer in order, so the parity is exact.
-        int go = 0;
-        const int n = ns[hf];
-        if (lane == 0)
-          go = n < nt[hf] && n <= npv[hf] + 1 &&
-               (n < 2 ||
-                mbar_test_wait(bar(kBarPFree + 2 * hf + (n & 1)), ((n - 2) >> 1) & 1)) &&
-               mbar_test_wait(bar(kBarFullK + n % kStages), (n / kStages) & 1);
-        if (__shfl_sync(0xffffffffu, go, 0)) {
-          if (lane == 0) {
+        for (int hf = 0; hf < kHalves; ++hf) {
+          if (!ok || kt >= nt[hf]) continue;
+          if (kt >= 2) ok = wait_all(kBarPFree + 2 * hf + (kt & 1), ((kt - 2) >> 1) & 1);
+          if (ok && lane == 0) {
             tc::fence_after_sync();
             const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
-            const uint64_t kd = dk0 + ((n % kStages) * kKVBytes >> 4);
-            const uint32_t dst = tmem + (2 * hf + (n & 1)) * kKeys;
+            const uint64_t kd = dk0 + ((s * kKVBytes) >> 4);
+            const uint32_t dst = tmem + (2 * hf + (kt & 1)) * kKeys;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
               const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
               tc::mma_f16_ss(dst, qd + off, kd + koff, kIdescQK, kk > 0);
             }
-            tc::commit(bar(kBarS + 2 * hf + (n & 1)));
+            tc::commit(bar(kBarS + 2 * hf + (kt & 1)));
           }
           __syncwarp();
-          ns[hf] = n + 1;
-          progress = true;
         }
-        // O(half) += P(npv) V(npv), P read from TMEM
-        go = 0;
-        const int v = npv[hf];
-        const int pb = v & 1;
-        if (lane == 0)
-          go = v < ns[hf] && mbar_test_wait(bar(kBarPReady + 2 * hf + pb), (v >> 1) & 1) &&
-               mbar_test_wait(bar(kBarFullV + v % kStages), (v / kStages) & 1);
-        if (__shfl_sync(0xffffffffu, go, 0)) {
-          const int s = v % kStages;
-          if (!zeroed && v == ntiles - 1) {
-            // every lane observes the landed copy itself before overwriting it
-            const bool landed = mbar_wait(bar(kBarFullV + s), (v / kStages) & 1);
-            if (landed) {
-              uint8_t* vt = smem + kOffV + s * kKVBytes;
-              const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
-              for (int c = lane; c < n16; c += 32) {
-                const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
-                *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
-                    make_uint4(0u, 0u, 0u, 0u);
-              }
-              fence_proxy_async_smem();
-            }
-            __syncwarp();  // the zeros are written (and fenced) before lane 0 issues
-            if (!__all_sync(0xffffffffu, landed)) {
-              ok = false;
-              break;
-            }
-            zeroed = true;
+      }
+      if (ok && kt >= 1) {
+        // O(half) += P(v) V(v), P read from TMEM
+        const int v = kt - 1, s = v % kStages;
+        ok = wait_all(kBarFullV + s, (v / kStages) & 1);
+        if (ok && v == ntiles - 1 && zero_from < zero_to) {
+          // every lane has observed the landed copy itself before overwriting it
+          uint8_t* vt = smem + kOffV + s * kKVBytes;
+          const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
+          for (int c = lane; c < n16; c += 32) {
+            const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
+            *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
           }
-          if (lane == 0) {
+          fence_proxy_async_smem();
+          __syncwarp();  // the zeros are written (and fenced) before lane 0 issues
+        }
+#pragma unroll
+        for (int hf = 0; hf < kHalves; ++hf) {
+          if (!ok || v >= nt[hf]) continue;
+          ok = wait_all(kBarPReady + 2 * hf + (v & 1), (v >> 1) & 1);
+          if (ok && lane == 0) {
             tc::fence_after_sync();
-            const uint32_t pt = tmem + (2 * hf + pb) * kKeys;  // P over S(v)
+            const uint32_t pt = tmem + (2 * hf + (v & 1)) * kKeys;  // P over S(v)
             const uint64_t vd = dv0 + ((s * kKVBytes) >> 4);
             const uint32_t dst = tmem + kColO + hf * D;
 #pragma unroll
@@ -345,18 +333,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::mma_f16_ts(dst, pt + kKeys / 2 + kk * 8, vd + ((kk * 16 * 128) >> 4),
                                kIdescPV, 1u);
             }
-            tc::commit(bar(kBarPFree + 2 * hf + pb));
-            // the stage is free once the other half is done with this tile too
-            const int other = 1 - hf;
-            if (npv[other] > v || v >= nt[other]) tc::commit(bar(kBarEmpty + s));
+            tc::commit(bar(kBarPFree + 2 * hf + (v & 1)));
           }
           __syncwarp();
-          npv[hf] = v + 1;
-          progress = true;
         }
+        if (ok && lane == 0) tc::commit(bar(kBarEmpty + s));  // both halves are done with v
       }
-      idle = progress ? 0u : idle + 1u;
-      if (idle > kSpinLimit) ok = false;
     }
     if (!ok && lane == 0) flag_timeout(a);
   } else {
