@@ -388,24 +388,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool moved = tmax > m + kSlack;
       const float mnew = moved ? tmax : m;
       const float alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
-      // The previous tile's P V must be complete before O is rescaled; it is
-      // waited for every tile, so this thread sees every phase of the
-      // barrier in order and the parity is exact.
-      if (kt > 0) {
+      // O is rescaled in TMEM once the previous tile's P V is complete.  The
+      // wait is exact without having seen the barrier's earlier phases: S(kt - 1)
+      // was issued only after P V(kt - 3) (same buffer) had finished, and
+      // P V(kt + 1) cannot start before this thread writes P(kt + 1), so the
+      // barrier is in P V(kt - 1)'s phase or just past it.
+      if (kt > 0 && __any_sync(0xffffffffu, moved)) {
         const int pv = kt - 1;
         ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
-        if (__any_sync(0xffffffffu, moved)) {
-          tc::fence_after_sync();
+        tc::fence_after_sync();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float ov[32];
-            tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
-            tc::tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
+          tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-            tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
-          }
+          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+          tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
         }
       }
       // P = 2^(s * scale - m) in the input type, written over S in TMEM (the
@@ -443,7 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar(kBarPReady + 2 * hf + s));
     }
     // epilogue: o = O / l in the input type and lse = (m + log2 l) ln 2; a
-    // half without keys (no mask, empty request) writes o = 0, lse = -inf
+    // half without keys (no mask, empty request) writes o = 0, lse = -inf.
+    // The wait for the last P V is exact for the reason given above.
     if (ok && nt > 0) {
       const int pv = nt - 1;
       ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
