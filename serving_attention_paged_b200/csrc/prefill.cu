@@ -264,10 +264,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nt[2] = {nt0, nt1};
     // Fixed order, one blocking wait per input: S of tile kt for both halves,
     // then P V of tile kt - 1 for both.  The softmax of a half always finds
-    // the next S issued while it works on the current tile.  S(kt) goes into
-    // the buffer P V(kt - 2) read P from, so it waits for that P V to finish;
-    // this warp waits for every P V of a buffer in order, so the parity is
-    // exact.
+    // the next S issued while it works on the current tile.  S(kt) overwrites
+    // the TMEM buffer P V(kt - 2) reads P from; it is issued after that P V by
+    // this same thread, and the tensor pipe runs one thread's tcgen05.mma in
+    // issue order, so it is queued without waiting for the P V to finish and
+    // the pipe never drains between tiles.
     // Every lane waits and ok stays warp-uniform, so the lanes take the same
     // branches to the __syncwarp calls.
     auto wait_all = [&](int b, int parity) {
@@ -281,7 +282,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int hf = 0; hf < kHalves; ++hf) {
           if (!ok || kt >= nt[hf]) continue;
-          if (kt >= 2) ok = wait_all(kBarPFree + 2 * hf + (kt & 1), ((kt - 2) >> 1) & 1);
           if (ok && lane == 0) {
             tc::fence_after_sync();
             const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
@@ -388,11 +388,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool moved = tmax > m + kSlack;
       const float mnew = moved ? tmax : m;
       const float alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
-      // O is rescaled in TMEM once the previous tile's P V is complete.  The
-      // wait is exact without having seen the barrier's earlier phases: S(kt - 1)
-      // was issued only after P V(kt - 3) (same buffer) had finished, and
-      // P V(kt + 1) cannot start before this thread writes P(kt + 1), so the
-      // barrier is in P V(kt - 1)'s phase or just past it.
+      // P V(kt - 2) has finished: S(kt) was issued after it and its commit
+      // counts every earlier MMA.  Waiting for it anyway (it returns at once)
+      // lets this thread see every phase of each P V barrier in order, which
+      // keeps the rescale wait below exact.
+      if (kt >= 2) {
+        const int pv = kt - 2;
+        ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      // O is rescaled in TMEM once the previous tile's P V is complete.
       if (kt > 0 && __any_sync(0xffffffffu, moved)) {
         const int pv = kt - 1;
         ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
@@ -409,8 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // P = 2^(s * scale - m) in the input type, written over S in TMEM (the
-      // P V that last read this buffer finished before S was written), 32
-      // keys at a time; l sums what the tensor core multiplies.
+      // P V that last read this buffer has finished, see above), 32 keys at a
+      // time; l sums what the tensor core multiplies.
       const float nm = -mnew;
       const uint32_t p_addr = lane_addr + col_s + s * kKeys;
       float ps4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -444,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // epilogue: o = O / l in the input type and lse = (m + log2 l) ln 2; a
     // half without keys (no mask, empty request) writes o = 0, lse = -inf.
-    // The wait for the last P V is exact for the reason given above.
+    // The wait for the last P V is exact: this thread saw P V(nt - 3) finish.
     if (ok && nt > 0) {
       const int pv = nt - 1;
       ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
