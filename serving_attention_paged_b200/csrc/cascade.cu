@@ -201,10 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 5) {
     // ------------------------------ MMA issuer ------------------------------
     // S of the next tile and P V of the current one are issued as soon as
-    // their inputs are ready, whichever comes first.  Polling uses
-    // test_wait, which never suspends: try_wait on a barrier that is not
-    // ready may park the thread for a while, delaying work another barrier
-    // has already released.
+    // their inputs are ready, whichever comes first.
     if (lane == 0) {
       constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
       constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
@@ -220,8 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool progress = false;
         // S(ns) into buffer ns & 1, free once softmax has read S(ns - 2)
         if (ns < ntiles && ns <= npv + 2 &&
-            (ns < 2 || mbar_test_wait(bar(kBarSFree + (ns & 1)), ((ns - 2) >> 1) & 1)) &&
-            mbar_test_wait(bar(kBarFullK + ns % kStages), (ns / kStages) & 1)) {
+            (ns < 2 || mbar_try_wait(bar(kBarSFree + (ns & 1)), ((ns - 2) >> 1) & 1)) &&
+            mbar_try_wait(bar(kBarFullK + ns % kStages), (ns / kStages) & 1)) {
           tc::fence_after_sync();
           const uint64_t kd = dk0 + ((ns % kStages) * kKVBytes >> 4);
 #pragma unroll
@@ -235,8 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           progress = true;
         }
         // O += P(npv) V(npv)
-        if (npv < ns && mbar_test_wait(bar(kBarPReady + (npv & 1)), (npv >> 1) & 1) &&
-            mbar_test_wait(bar(kBarFullV + npv % kStages), (npv / kStages) & 1)) {
+        if (npv < ns && mbar_try_wait(bar(kBarPReady + (npv & 1)), (npv >> 1) & 1) &&
+            mbar_try_wait(bar(kBarFullV + npv % kStages), (npv / kStages) & 1)) {
           tc::fence_after_sync();
           const int s = npv % kStages;
           const uint64_t pd = dp0 + (((npv & 1) * kPBytes) >> 4);
