@@ -9,7 +9,9 @@ Contents, each written from the FlashInfer README (core features 1-3, the
 single-request decode usage example) and the flashinfer-cubin registry page
 (paged-KV names ``kv_indptr`` / ``kv_indices`` / ``last_page_len``):
 
-* ``paged_decode`` — the attention definition in fp64 (``paged_attention.c``).
+* ``paged_decode`` — the attention definition in fp64 (``paged_attention.c``),
+  over 16-bit pools or 8-bit (FP8 E4M3 / E5M2) pools with a K and a V scale
+  (README core feature 3: low-precision attention for a compressed KV-Cache).
 * ``merge_state`` / ``merge_states`` — combining attention states by their
   log-sum-exp (what split-KV and cascade attention rely on).
 * ``cascade_decode`` — shared prefix merged with per-request suffix.
@@ -18,9 +20,11 @@ single-request decode usage example) and the flashinfer-cubin registry page
 * ``plan`` — the split-KV work-list specification restated with plain
   loops (the library's work list must agree with it exactly).
 
-Parity status: every function here is pinned by ``tests/test_oracle.py``
-(closed forms, invariants, brute force).  The pages print no worked numeric
-example, so nothing is pinned to a published output value.
+Parity status: every function here is pinned by ``tests/test_oracle.py``,
+``tests/test_plan_oracle.py``, ``tests/test_prefill_oracle.py`` and
+``tests/test_fp8_oracle.py`` (closed forms, invariants, brute force, and
+torch's own FP8 conversion for the 8-bit widening).  The pages print no
+worked numeric example, so nothing is pinned to a published output value.
 """
 from __future__ import annotations
 
@@ -55,6 +59,11 @@ def _load():
         lib.oracle_paged_decode.restype = ctypes.c_int
         lib.oracle_widen.argtypes = [ctypes.c_uint16, i32]
         lib.oracle_widen.restype = dbl
+        lib.oracle_paged_decode_kv.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                               i32, i32, dbl, dbl, dbl, vp, i64, vp, vp, i32]
+        lib.oracle_paged_decode_kv.restype = ctypes.c_int
+        lib.oracle_widen8.argtypes = [ctypes.c_uint8, i32]
+        lib.oracle_widen8.restype = dbl
         _lib = lib
     return _lib
 
@@ -73,6 +82,17 @@ def _as_u16(x) -> np.ndarray:
     return x.view(np.uint16)
 
 
+def _as_u8(x) -> np.ndarray:
+    """8-bit float storage (torch float8 tensor or uint8 numpy) as contiguous uint8."""
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().cpu().contiguous().view(torch.uint8).numpy()
+    return np.ascontiguousarray(x).view(np.uint8)
+
+
+KV8_CODE = {"e4m3": 0, "e5m2": 1}
+
+
 def _as_i32(x) -> np.ndarray:
     if hasattr(x, "detach"):
         x = x.detach().cpu().numpy()
@@ -84,16 +104,32 @@ def widen(bits: int, dtype: str) -> float:
     return _load().oracle_widen(bits, DTYPE_CODE[dtype])
 
 
+def widen8(code: int, kv_dtype: str) -> float:
+    """The oracle's exact FP8 (``e4m3``: OCP E4M3 without infinities, max 448;
+    ``e5m2``: OCP E5M2) -> fp64 widening of one 8-bit pattern."""
+    return _load().oracle_widen8(code, KV8_CODE[kv_dtype])
+
+
 def paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, *, num_qo_heads,
-                 num_kv_heads, head_dim, page_size, dtype, sm_scale, rows=None, threads=1):
+                 num_kv_heads, head_dim, page_size, dtype, sm_scale, rows=None, threads=1,
+                 kv_dtype=None, k_scale=1.0, v_scale=1.0):
     """fp64 attention of every (b, hq) row (or the listed ``rows`` = b*Hq+hq).
+
+    ``dtype`` is q's (fp16 / bf16).  With ``kv_dtype=None`` the pools hold the
+    same 16-bit type; with ``kv_dtype`` ``"e4m3"`` or ``"e5m2"`` they hold
+    8-bit codes and each cached key is ``k_scale * code`` (values:
+    ``v_scale * code``).
 
     Returns ``(o, lse)``: o ``[n_rows, D]`` fp64 and lse ``[n_rows]`` fp64
     (natural log; -inf for an empty request).  With ``rows=None`` the result
     is reshaped to ``[B, Hq, D]`` / ``[B, Hq]``.
     """
     lib = _load()
-    qa, ka, va = _as_u16(q), _as_u16(k_pool), _as_u16(v_pool)
+    qa = _as_u16(q)
+    if kv_dtype is None:
+        ka, va, fmt = _as_u16(k_pool), _as_u16(v_pool), -1
+    else:
+        ka, va, fmt = _as_u8(k_pool), _as_u8(v_pool), KV8_CODE[kv_dtype]
     indptr, indices, last = _as_i32(kv_indptr), _as_i32(kv_indices), _as_i32(last_page_len)
     batch = len(last)
     if rows is None:
@@ -106,10 +142,10 @@ def paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, *, num
     lse = np.zeros(n_rows, dtype=np.float64)
     if indices.size == 0:
         indices = np.zeros(1, dtype=np.int32)
-    rc = lib.oracle_paged_decode(
+    rc = lib.oracle_paged_decode_kv(
         qa.ctypes.data, ka.ctypes.data, va.ctypes.data, indptr.ctypes.data, indices.ctypes.data,
         last.ctypes.data if last.size else None, batch, num_qo_heads, num_kv_heads, head_dim,
-        page_size, DTYPE_CODE[dtype], float(sm_scale),
+        page_size, DTYPE_CODE[dtype], fmt, float(sm_scale), float(k_scale), float(v_scale),
         rows_arr.ctypes.data if rows_arr is not None else None, n_rows, o.ctypes.data,
         lse.ctypes.data, int(threads))
     if rc != 0:
@@ -121,7 +157,7 @@ def paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, *, num
 
 def paged_decode_requests(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, requests, *,
                           num_qo_heads, num_kv_heads, head_dim, page_size, dtype, sm_scale,
-                          threads=1):
+                          threads=1, kv_dtype=None, k_scale=1.0, v_scale=1.0):
     """``paged_decode`` for every q head of the listed requests only.
 
     q and the pools may be large torch tensors on any device: only the pages
@@ -148,7 +184,8 @@ def paged_decode_requests(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_le
     return paged_decode(qs, kp, vp, sub_indptr, sub_indices, sub_last,
                         num_qo_heads=num_qo_heads, num_kv_heads=num_kv_heads,
                         head_dim=head_dim, page_size=page_size, dtype=dtype,
-                        sm_scale=sm_scale, threads=threads)
+                        sm_scale=sm_scale, threads=threads, kv_dtype=kv_dtype,
+                        k_scale=k_scale, v_scale=v_scale)
 
 
 def merge_state(o_a, lse_a, o_b, lse_b):
@@ -350,4 +387,4 @@ def plan(kv_indptr, last_page_len, *, page_size, num_kv_heads, num_sms, ctas_per
 
 
 __all__ = ["build_library", "paged_decode", "paged_decode_requests", "merge_state", "merge_states", "cascade_decode",
-           "paged_prefill", "plan", "widen"]
+           "paged_prefill", "plan", "widen", "widen8"]

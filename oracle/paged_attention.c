@@ -22,6 +22,12 @@
  * An empty request (L_b = 0) gives o = 0 and lse = -inf.  The fp16 / bf16
  * inputs are widened to fp64 exactly; all arithmetic is fp64 in plain
  * token order.  Work is spread over POSIX threads by (b, hq) row only.
+ *
+ * Low-precision KV cache (README core feature 3: efficient kernels for
+ * low-precision attention for compressed KV-Cache): the pools may hold
+ * 8-bit floats (OCP FP8 E4M3 without infinities, or E5M2) with one scale
+ * for K and one for V; the cached value is scale * code, and q stays fp16 /
+ * bf16.
  */
 #include <math.h>
 #include <pthread.h>
@@ -54,14 +60,54 @@ static double bf16_to_f64(uint16_t b) {
 
 static double widen(uint16_t x, int dtype) { return dtype ? bf16_to_f64(x) : f16_to_f64(x); }
 
+/* OCP FP8 E4M3 ("FN" variant): 1 sign bit, 4 exponent bits (bias 7), 3
+ * fraction bits; no infinities, exponent and fraction all ones is NaN, so
+ * the largest value is 448. */
+static double e4m3_to_f64(uint8_t c) {
+  int sign = (c >> 7) & 1;
+  int e = (c >> 3) & 0xf;
+  int f = c & 0x7;
+  double v;
+  if (e == 0xf && f == 0x7)
+    v = NAN;
+  else if (e == 0)
+    v = ldexp((double)f, -9); /* subnormal: f/8 * 2^-6 */
+  else
+    v = ldexp((double)(f + 8), e - 10); /* (1 + f/8) * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+/* OCP FP8 E5M2: 1 sign bit, 5 exponent bits (bias 15), 2 fraction bits, with
+ * IEEE infinities and NaNs. */
+static double e5m2_to_f64(uint8_t c) {
+  int sign = (c >> 7) & 1;
+  int e = (c >> 2) & 0x1f;
+  int f = c & 0x3;
+  double v;
+  if (e == 0)
+    v = ldexp((double)f, -16); /* subnormal: f/4 * 2^-14 */
+  else if (e == 31)
+    v = f ? NAN : INFINITY;
+  else
+    v = ldexp((double)(f + 4), e - 17); /* (1 + f/4) * 2^(e-15) */
+  return sign ? -v : v;
+}
+
+/* kv_fmt: -1 = the 16-bit q dtype, 0 = E4M3, 1 = E5M2. */
+static double widen8(uint8_t c, int kv_fmt) { return kv_fmt ? e5m2_to_f64(c) : e4m3_to_f64(c); }
+
+/* Exposed so that the tests can pin the 8-bit widening against torch. */
+double oracle_widen8(uint8_t x, int32_t kv_fmt) { return widen8(x, kv_fmt); }
+
 /* Exposed so that the tests can pin the widening against numpy / torch. */
 double oracle_widen(uint16_t x, int32_t dtype) { return widen(x, dtype); }
 
 typedef struct {
-  const uint16_t *q, *k_pool, *v_pool;
+  const uint16_t *q;
+  const void *k_pool, *v_pool;
   const int32_t *kv_indptr, *kv_indices, *last_page_len;
-  int32_t batch, num_qo_heads, num_kv_heads, head_dim, page_size, dtype;
-  double sm_scale;
+  int32_t batch, num_qo_heads, num_kv_heads, head_dim, page_size, dtype, kv_fmt;
+  double sm_scale, k_scale, v_scale;
   const int64_t *rows;
   int64_t n_rows;
   double *out_o, *out_lse;
@@ -69,6 +115,12 @@ typedef struct {
   pthread_mutex_t lock;
   int error;
 } job_t;
+
+/* Element i of a K or V pool, widened (and scaled, for 8-bit pools). */
+static double kv_elem(const job_t *J, const void *pool, int64_t i, double scale) {
+  if (J->kv_fmt < 0) return widen(((const uint16_t *)pool)[i], J->dtype);
+  return scale * widen8(((const uint8_t *)pool)[i], J->kv_fmt);
+}
 
 static void one_row(job_t *J, int64_t r, int64_t out_index, double *s, double *q) {
   const int32_t Hq = J->num_qo_heads, Hkv = J->num_kv_heads, D = J->head_dim, P = J->page_size;
@@ -88,9 +140,9 @@ static void one_row(job_t *J, int64_t r, int64_t out_index, double *s, double *q
   double M = -INFINITY;
   for (int64_t t = 0; t < L; ++t) {
     int64_t row = (int64_t)J->kv_indices[J->kv_indptr[b] + t / P] * P + t % P;
-    const uint16_t *k = J->k_pool + (row * Hkv + h) * D;
+    const int64_t k0 = (row * Hkv + h) * D;
     double acc = 0.0;
-    for (int d = 0; d < D; ++d) acc += q[d] * widen(k[d], J->dtype);
+    for (int d = 0; d < D; ++d) acc += q[d] * kv_elem(J, J->k_pool, k0 + d, J->k_scale);
     s[t] = J->sm_scale * acc;
     if (s[t] > M) M = s[t];
   }
@@ -102,9 +154,9 @@ static void one_row(job_t *J, int64_t r, int64_t out_index, double *s, double *q
   /* softmax-weighted values */
   for (int64_t t = 0; t < L; ++t) {
     int64_t row = (int64_t)J->kv_indices[J->kv_indptr[b] + t / P] * P + t % P;
-    const uint16_t *v = J->v_pool + (row * Hkv + h) * D;
+    const int64_t v0 = (row * Hkv + h) * D;
     double w = exp(s[t] - lse);
-    for (int d = 0; d < D; ++d) o[d] += w * widen(v[d], J->dtype);
+    for (int d = 0; d < D; ++d) o[d] += w * kv_elem(J, J->v_pool, v0 + d, J->v_scale);
   }
 }
 
@@ -147,16 +199,19 @@ static void *worker(void *arg) {
 /*
  * Attention rows r = b * Hq + hq listed in rows[0..n_rows) (rows == NULL:
  * all B * Hq rows in order).  out_o is [n_rows, D] fp64, out_lse [n_rows].
- * dtype: 0 = fp16, 1 = bf16.  Returns 0, or 1 on bad arguments / no memory.
+ * dtype (of q, and of the pools when kv_fmt < 0): 0 = fp16, 1 = bf16.
+ * kv_fmt: -1 = 16-bit pools; 0 = E4M3 or 1 = E5M2 pools, each value times
+ * k_scale (K) or v_scale (V).  Returns 0, or 1 on bad arguments / no memory.
  */
-int oracle_paged_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool,
-                        const int32_t *kv_indptr, const int32_t *kv_indices,
-                        const int32_t *last_page_len, int32_t batch, int32_t num_qo_heads,
-                        int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
-                        int32_t dtype, double sm_scale, const int64_t *rows, int64_t n_rows,
-                        double *out_o, double *out_lse, int32_t n_threads) {
+int oracle_paged_decode_kv(const uint16_t *q, const void *k_pool, const void *v_pool,
+                           const int32_t *kv_indptr, const int32_t *kv_indices,
+                           const int32_t *last_page_len, int32_t batch, int32_t num_qo_heads,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
+                           int32_t dtype, int32_t kv_fmt, double sm_scale, double k_scale,
+                           double v_scale, const int64_t *rows, int64_t n_rows, double *out_o,
+                           double *out_lse, int32_t n_threads) {
   if (batch < 0 || num_kv_heads <= 0 || num_qo_heads % num_kv_heads || head_dim <= 0 ||
-      page_size <= 0)
+      page_size <= 0 || kv_fmt < -1 || kv_fmt > 1)
     return 1;
   job_t J;
   memset(&J, 0, sizeof J);
@@ -172,7 +227,10 @@ int oracle_paged_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_
   J.head_dim = head_dim;
   J.page_size = page_size;
   J.dtype = dtype;
+  J.kv_fmt = kv_fmt;
   J.sm_scale = sm_scale;
+  J.k_scale = k_scale;
+  J.v_scale = v_scale;
   J.rows = rows;
   J.n_rows = rows ? n_rows : (int64_t)batch * num_qo_heads;
   J.out_o = out_o;
@@ -188,4 +246,16 @@ int oracle_paged_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_
   for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
   pthread_mutex_destroy(&J.lock);
   return J.error;
+}
+
+/* The 16-bit decode above with both pools in q's dtype. */
+int oracle_paged_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool,
+                        const int32_t *kv_indptr, const int32_t *kv_indices,
+                        const int32_t *last_page_len, int32_t batch, int32_t num_qo_heads,
+                        int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
+                        int32_t dtype, double sm_scale, const int64_t *rows, int64_t n_rows,
+                        double *out_o, double *out_lse, int32_t n_threads) {
+  return oracle_paged_decode_kv(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, batch,
+                                num_qo_heads, num_kv_heads, head_dim, page_size, dtype, -1,
+                                sm_scale, 1.0, 1.0, rows, n_rows, out_o, out_lse, n_threads);
 }

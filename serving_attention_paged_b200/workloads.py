@@ -50,6 +50,7 @@ STREAM_LEN = 4
 STREAM_PERM = 5
 
 DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16}
+KV8_DTYPES = {"e4m3": torch.float8_e4m3fn, "e5m2": torch.float8_e5m2}
 DTYPE_CODES = {"f16": 0, "bf16": 1}
 
 
@@ -152,6 +153,10 @@ class PagedWorkload:
     prefix_len: int = 0
     prefix_indices: Optional[np.ndarray] = None
     qo_lens: Optional[np.ndarray] = None  # prefill / append: new tokens per request
+    # 8-bit KV cache: pools hold FP8 codes c, the cached key / value is scale * c
+    kv_dtype: Optional[str] = None         # None (pools in `dtype`), "e4m3" or "e5m2"
+    k_scale: float = 1.0
+    v_scale: float = 1.0
     extra: dict = field(default_factory=dict)
 
     def __post_init__(self):
@@ -180,7 +185,7 @@ class PagedWorkload:
 
     def kv_bytes(self) -> int:
         """Algorithmic K+V bytes one decode step reads (prefix counted once)."""
-        e = 2
+        e = 1 if self.kv_dtype else 2
         return 2 * self.total_tokens() * self.num_kv_heads * self.head_dim * e
 
     def flat_tables(self):
@@ -248,26 +253,41 @@ class PagedWorkload:
 
     def make_pool(self, which: str, device="cpu", chunk_tokens: int = 1 << 15,
                   rows: Optional[np.ndarray] = None) -> torch.Tensor:
-        """K (``which='k'``) or V pool ``[num_pages, P, Hkv, D]``; unused rows are 0."""
+        """K (``which='k'``) or V pool ``[num_pages, P, Hkv, D]``; unused rows are 0.
+
+        An 8-bit pool holds each N(0, 1) draw (rounded to fp32) divided by the
+        pool's scale and rounded to the FP8 format (torch's conversion, RNE)."""
         stream = STREAM_K if which == "k" else STREAM_V
         key = stream_key(self.seed, stream)
         w = self.num_kv_heads * self.head_dim
-        pool = torch.zeros(self.num_pages * self.page_size, w, dtype=DTYPES[self.dtype], device=device)
+        pool_dtype = KV8_DTYPES[self.kv_dtype] if self.kv_dtype else DTYPES[self.dtype]
+        pool = torch.zeros(self.num_pages * self.page_size, w, dtype=pool_dtype, device=device)
         if rows is None:
             rows = self.token_rows()
         rows_t = torch.from_numpy(rows).to(device)
         for j0 in range(0, len(rows), chunk_tokens):
             j1 = min(len(rows), j0 + chunk_tokens)
-            vals = normal_as(key, j0 * w, (j1 - j0) * w, self.dtype, device).view(j1 - j0, w)
+            if self.kv_dtype:
+                scale = self.k_scale if which == "k" else self.v_scale
+                x = normal(key, j0 * w, (j1 - j0) * w, device).to(torch.float32) / scale
+                vals = x.to(pool_dtype).view(j1 - j0, w)
+            else:
+                vals = normal_as(key, j0 * w, (j1 - j0) * w, self.dtype, device).view(j1 - j0, w)
             pool[rows_t[j0:j1]] = vals
         return pool.view(self.num_pages, self.page_size, self.num_kv_heads, self.head_dim)
 
     def logical_kv(self, which: str, token_begin: int, token_end: int, device="cpu") -> torch.Tensor:
-        """K or V of logical tokens [token_begin, token_end) as ``[n, Hkv, D]``."""
+        """K or V of logical tokens [token_begin, token_end) as ``[n, Hkv, D]``
+        (in the pool's storage type: FP8 codes for an 8-bit cache)."""
         stream = STREAM_K if which == "k" else STREAM_V
         w = self.num_kv_heads * self.head_dim
-        vals = normal_as(stream_key(self.seed, stream), token_begin * w,
-                         (token_end - token_begin) * w, self.dtype, device)
+        n = (token_end - token_begin) * w
+        if self.kv_dtype:
+            scale = self.k_scale if which == "k" else self.v_scale
+            x = normal(stream_key(self.seed, stream), token_begin * w, n, device).to(torch.float32)
+            vals = (x / scale).to(KV8_DTYPES[self.kv_dtype])
+        else:
+            vals = normal_as(stream_key(self.seed, stream), token_begin * w, n, self.dtype, device)
         return vals.view(token_end - token_begin, self.num_kv_heads, self.head_dim)
 
     def materialize(self, device="cpu") -> dict:
@@ -313,7 +333,8 @@ def tables_from_lengths(lens, page_size: int, page_order: Optional[np.ndarray] =
 
 def make_workload(name, lens, *, num_qo_heads, num_kv_heads, head_dim=128, page_size=16,
                   dtype="f16", seed=0, shuffle=True, extra_pages=0, prefix_len=0,
-                  sm_scale=0.0, qo_lens=None) -> PagedWorkload:
+                  sm_scale=0.0, qo_lens=None, kv_dtype=None, k_scale=1.0,
+                  v_scale=1.0) -> PagedWorkload:
     """A paged problem whose pool holds exactly the pages used (+ ``extra_pages``).
 
     ``shuffle`` places every page at a random pool position (one permutation
@@ -334,7 +355,8 @@ def make_workload(name, lens, *, num_qo_heads, num_kv_heads, head_dim=128, page_
                          num_kv_heads=num_kv_heads, head_dim=head_dim, page_size=page_size,
                          dtype=dtype, seed=seed, num_pages=num_pages, kv_indptr=indptr,
                          kv_indices=indices, last_page_len=last, prefix_len=prefix_len,
-                         prefix_indices=prefix_indices, sm_scale=sm_scale, qo_lens=qo_lens)
+                         prefix_indices=prefix_indices, sm_scale=sm_scale, qo_lens=qo_lens,
+                         kv_dtype=kv_dtype, k_scale=k_scale, v_scale=v_scale)
 
 
 # ---------------------------------------------------------------------------
