@@ -11,7 +11,8 @@ single-request decode usage example) and the flashinfer-cubin registry page
 
 * ``paged_decode`` — the attention definition in fp64 (``paged_attention.c``),
   over 16-bit pools or 8-bit (FP8 E4M3 / E5M2) pools with a K and a V scale
-  (README core feature 3: low-precision attention for a compressed KV-Cache).
+  (README core feature 3: low-precision attention for a compressed KV-Cache),
+  optionally with LLaMA-style rotary positions applied on the fly.
 * ``merge_state`` / ``merge_states`` — combining attention states by their
   log-sum-exp (what split-KV and cascade attention rely on).
 * ``cascade_decode`` — shared prefix merged with per-request suffix.
@@ -60,7 +61,8 @@ def _load():
         lib.oracle_widen.argtypes = [ctypes.c_uint16, i32]
         lib.oracle_widen.restype = dbl
         lib.oracle_paged_decode_kv.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
-                                               i32, i32, dbl, dbl, dbl, vp, i64, vp, vp, i32]
+                                               i32, i32, dbl, dbl, dbl, dbl, vp, i64, vp, vp,
+                                               i32]
         lib.oracle_paged_decode_kv.restype = ctypes.c_int
         lib.oracle_widen8.argtypes = [ctypes.c_uint8, i32]
         lib.oracle_widen8.restype = dbl
@@ -112,13 +114,17 @@ def widen8(code: int, kv_dtype: str) -> float:
 
 def paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, *, num_qo_heads,
                  num_kv_heads, head_dim, page_size, dtype, sm_scale, rows=None, threads=1,
-                 kv_dtype=None, k_scale=1.0, v_scale=1.0):
+                 kv_dtype=None, k_scale=1.0, v_scale=1.0, rope_theta=None):
     """fp64 attention of every (b, hq) row (or the listed ``rows`` = b*Hq+hq).
 
     ``dtype`` is q's (fp16 / bf16).  With ``kv_dtype=None`` the pools hold the
     same 16-bit type; with ``kv_dtype`` ``"e4m3"`` or ``"e5m2"`` they hold
     8-bit codes and each cached key is ``k_scale * code`` (values:
     ``v_scale * code``).
+
+    ``rope_theta`` (README usage example: decode with LLaMA-style RoPE on the
+    fly) rotates q to position L_b - 1 and key t to position t before the dot
+    product: element pairs (d, d + D/2) turn by pos * rope_theta^(-2d/D).
 
     Returns ``(o, lse)``: o ``[n_rows, D]`` fp64 and lse ``[n_rows]`` fp64
     (natural log; -inf for an empty request).  With ``rows=None`` the result
@@ -146,7 +152,7 @@ def paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, *, num
         qa.ctypes.data, ka.ctypes.data, va.ctypes.data, indptr.ctypes.data, indices.ctypes.data,
         last.ctypes.data if last.size else None, batch, num_qo_heads, num_kv_heads, head_dim,
         page_size, DTYPE_CODE[dtype], fmt, float(sm_scale), float(k_scale), float(v_scale),
-        rows_arr.ctypes.data if rows_arr is not None else None, n_rows, o.ctypes.data,
+        float(rope_theta) if rope_theta else 0.0, rows_arr.ctypes.data if rows_arr is not None else None, n_rows, o.ctypes.data,
         lse.ctypes.data, int(threads))
     if rc != 0:
         raise ValueError("oracle_paged_decode rejected its arguments")
@@ -157,7 +163,7 @@ def paged_decode(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, *, num
 
 def paged_decode_requests(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, requests, *,
                           num_qo_heads, num_kv_heads, head_dim, page_size, dtype, sm_scale,
-                          threads=1, kv_dtype=None, k_scale=1.0, v_scale=1.0):
+                          threads=1, kv_dtype=None, k_scale=1.0, v_scale=1.0, rope_theta=None):
     """``paged_decode`` for every q head of the listed requests only.
 
     q and the pools may be large torch tensors on any device: only the pages
@@ -185,7 +191,7 @@ def paged_decode_requests(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_le
                         num_qo_heads=num_qo_heads, num_kv_heads=num_kv_heads,
                         head_dim=head_dim, page_size=page_size, dtype=dtype,
                         sm_scale=sm_scale, threads=threads, kv_dtype=kv_dtype,
-                        k_scale=k_scale, v_scale=v_scale)
+                        k_scale=k_scale, v_scale=v_scale, rope_theta=rope_theta)
 
 
 def merge_state(o_a, lse_a, o_b, lse_b):

@@ -28,6 +28,12 @@
  * 8-bit floats (OCP FP8 E4M3 without infinities, or E5M2) with one scale
  * for K and one for V; the cached value is scale * code, and q stays fp16 /
  * bf16.
+ *
+ * Rotary positions on the fly (README usage example: decode with LLaMA-style
+ * RoPE, pos_encoding_mode="ROPE_LLAMA"), when rope_theta > 0: before the dot
+ * product q is rotated to its position L_b - 1 (the new token is the last in
+ * the cache) and key t to position t; element pairs (d, d + D/2) turn by
+ * pos * rope_theta^(-2d/D).  Values are not rotated.
  */
 #include <math.h>
 #include <pthread.h>
@@ -107,7 +113,7 @@ typedef struct {
   const void *k_pool, *v_pool;
   const int32_t *kv_indptr, *kv_indices, *last_page_len;
   int32_t batch, num_qo_heads, num_kv_heads, head_dim, page_size, dtype, kv_fmt;
-  double sm_scale, k_scale, v_scale;
+  double sm_scale, k_scale, v_scale, rope_theta;
   const int64_t *rows;
   int64_t n_rows;
   double *out_o, *out_lse;
@@ -120,6 +126,18 @@ typedef struct {
 static double kv_elem(const job_t *J, const void *pool, int64_t i, double scale) {
   if (J->kv_fmt < 0) return widen(((const uint16_t *)pool)[i], J->dtype);
   return scale * widen8(((const uint8_t *)pool)[i], J->kv_fmt);
+}
+
+/* Rotate x (D elements) to position pos: pairs (d, d + D/2) by pos * theta^(-2d/D). */
+static void rope(double *x, int D, double pos, double theta) {
+  const int half = D / 2;
+  for (int d = 0; d < half; ++d) {
+    const double a = pos * pow(theta, -2.0 * d / D);
+    const double c = cos(a), sn = sin(a);
+    const double x0 = x[d], x1 = x[d + half];
+    x[d] = x0 * c - x1 * sn;
+    x[d + half] = x1 * c + x0 * sn;
+  }
 }
 
 static void one_row(job_t *J, int64_t r, int64_t out_index, double *s, double *q) {
@@ -135,6 +153,9 @@ static void one_row(job_t *J, int64_t r, int64_t out_index, double *s, double *q
     return;
   }
   for (int d = 0; d < D; ++d) q[d] = widen(J->q[(b * Hq + hq) * D + d], J->dtype);
+  const int rotary = J->rope_theta > 0.0;
+  if (rotary) rope(q, D, (double)(L - 1), J->rope_theta);
+  double *kr = q + D; /* room for one rotated key */
 
   /* scores */
   double M = -INFINITY;
@@ -142,7 +163,13 @@ static void one_row(job_t *J, int64_t r, int64_t out_index, double *s, double *q
     int64_t row = (int64_t)J->kv_indices[J->kv_indptr[b] + t / P] * P + t % P;
     const int64_t k0 = (row * Hkv + h) * D;
     double acc = 0.0;
-    for (int d = 0; d < D; ++d) acc += q[d] * kv_elem(J, J->k_pool, k0 + d, J->k_scale);
+    if (rotary) {
+      for (int d = 0; d < D; ++d) kr[d] = kv_elem(J, J->k_pool, k0 + d, J->k_scale);
+      rope(kr, D, (double)t, J->rope_theta);
+      for (int d = 0; d < D; ++d) acc += q[d] * kr[d];
+    } else {
+      for (int d = 0; d < D; ++d) acc += q[d] * kv_elem(J, J->k_pool, k0 + d, J->k_scale);
+    }
     s[t] = J->sm_scale * acc;
     if (s[t] > M) M = s[t];
   }
@@ -174,7 +201,7 @@ static void *worker(void *arg) {
   job_t *J = (job_t *)arg;
   int64_t Lmax = max_len(J);
   double *s = (double *)malloc(sizeof(double) * (size_t)(Lmax > 0 ? Lmax : 1));
-  double *q = (double *)malloc(sizeof(double) * (size_t)J->head_dim);
+  double *q = (double *)malloc(sizeof(double) * 2 * (size_t)J->head_dim);
   if (!s || !q) {
     pthread_mutex_lock(&J->lock);
     J->error = 1;
@@ -201,17 +228,19 @@ static void *worker(void *arg) {
  * all B * Hq rows in order).  out_o is [n_rows, D] fp64, out_lse [n_rows].
  * dtype (of q, and of the pools when kv_fmt < 0): 0 = fp16, 1 = bf16.
  * kv_fmt: -1 = 16-bit pools; 0 = E4M3 or 1 = E5M2 pools, each value times
- * k_scale (K) or v_scale (V).  Returns 0, or 1 on bad arguments / no memory.
+ * k_scale (K) or v_scale (V).  rope_theta > 0 turns on rotary positions (an
+ * even head_dim is then required).  Returns 0, or 1 on bad arguments / no
+ * memory.
  */
 int oracle_paged_decode_kv(const uint16_t *q, const void *k_pool, const void *v_pool,
                            const int32_t *kv_indptr, const int32_t *kv_indices,
                            const int32_t *last_page_len, int32_t batch, int32_t num_qo_heads,
                            int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
                            int32_t dtype, int32_t kv_fmt, double sm_scale, double k_scale,
-                           double v_scale, const int64_t *rows, int64_t n_rows, double *out_o,
-                           double *out_lse, int32_t n_threads) {
+                           double v_scale, double rope_theta, const int64_t *rows,
+                           int64_t n_rows, double *out_o, double *out_lse, int32_t n_threads) {
   if (batch < 0 || num_kv_heads <= 0 || num_qo_heads % num_kv_heads || head_dim <= 0 ||
-      page_size <= 0 || kv_fmt < -1 || kv_fmt > 1)
+      page_size <= 0 || kv_fmt < -1 || kv_fmt > 1 || (rope_theta > 0.0 && head_dim % 2))
     return 1;
   job_t J;
   memset(&J, 0, sizeof J);
@@ -231,6 +260,7 @@ int oracle_paged_decode_kv(const uint16_t *q, const void *k_pool, const void *v_
   J.sm_scale = sm_scale;
   J.k_scale = k_scale;
   J.v_scale = v_scale;
+  J.rope_theta = rope_theta;
   J.rows = rows;
   J.n_rows = rows ? n_rows : (int64_t)batch * num_qo_heads;
   J.out_o = out_o;
@@ -257,5 +287,6 @@ int oracle_paged_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_
                         double *out_o, double *out_lse, int32_t n_threads) {
   return oracle_paged_decode_kv(q, k_pool, v_pool, kv_indptr, kv_indices, last_page_len, batch,
                                 num_qo_heads, num_kv_heads, head_dim, page_size, dtype, -1,
-                                sm_scale, 1.0, 1.0, rows, n_rows, out_o, out_lse, n_threads);
+                                sm_scale, 1.0, 1.0, 0.0, rows, n_rows, out_o, out_lse,
+                                n_threads);
 }
