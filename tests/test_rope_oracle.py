@@ -50,8 +50,8 @@ def test_position_zero_is_the_identity():
 def test_only_relative_positions_matter(dtype):
     """RoPE(q, m) . RoPE(k, n) = q . RoPE(k, n - m): dense attention with q as
     it is and key t turned by t - (L_b - 1) must give the same result."""
-    w = W.make_workload("rope_rel", [37, 5, 0, 64], num_qo_heads=8, num_kv_heads=2, head_dim=32,
-                        page_size=8, dtype=dtype, seed=52)
+    w = W.make_workload("rope_rel", [37, 5, 0, 64], num_qo_heads=8, num_kv_heads=2,
+                        head_dim=32, page_size=8, dtype=dtype, seed=52)
     t = w.materialize()
     o, lse = _decode(w, t, rope_theta=THETA)
     q = t["q"].to(torch.float64).numpy()
