@@ -64,3 +64,27 @@ def test_benchmark_workload_shapes():
     assert 64 <= w5.kv_lens().min() and w5.kv_lens().max() <= 1024
     assert w2.kv_bytes() == 2 * 16 * 4096 * 8 * 128 * 2
     assert abs(w1.sm_scale - 1 / math.sqrt(128)) < 1e-15
+
+
+def test_prefill_flop_accounting():
+    """The bench's per-token flops (4 per visible key and element, all q heads)
+    summed over every new token equal the workload's total, and a causal token
+    sees L_b - Q_b + i + 1 keys: brute force on a small ragged batch."""
+    import numpy as np
+
+    import bench
+    w = W.make_workload("pf_flops", [10, 7, 0, 33], num_qo_heads=4, num_kv_heads=2,
+                        head_dim=16, page_size=4, dtype="f16", seed=9, qo_lens=[10, 3, 0, 5])
+    allq = np.arange(w.query_rows())
+    assert bench.prefill_query_flops(w, allq) == w.prefill_flops()
+    lens, qo = w.kv_lens(), w.qo_indptr
+    brute = 0
+    for b in range(w.batch):
+        Q = qo[b + 1] - qo[b]
+        for i in range(Q):
+            brute += 4 * (int(lens[b]) - Q + i + 1) * w.num_qo_heads * w.head_dim
+    assert brute == w.prefill_flops()
+    # one token alone: the last of request 3 sees all 33 keys
+    assert bench.prefill_query_flops(w, np.array([w.query_rows() - 1])) == 4 * 33 * 4 * 16
+    # workload 6: 8 * 32 * (1024 * 1024 + 1024 * 1025 / 2) pairs * 512
+    assert W.WORKLOADS[6]().prefill_flops() == 8 * 32 * (1024 * 1024 + 1024 * 1025 // 2) * 512
