@@ -127,3 +127,18 @@ def test_plans_run_only_through_their_own_entry_point(C):
     with pytest.raises(C.PagedAttnError) as e:
         C.pa_prefill_run(pf, big, big, big, big, big, None, big, ws_pf - 1, 0)
     assert e.value.status == C.PA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_empty_prefill_plans_run_without_a_launch(C):
+    """No requests, or requests without new tokens: no tiles, and the run
+    returns at once (no CUDA call is made, so this runs on the host)."""
+    empty = C.pa_prefill_plan_create(_problem(C, 0), True, np.zeros(1, np.int32),
+                                     np.zeros(1, np.int32), np.zeros(0, np.int32))
+    assert len(C.pa_plan_prefill_tiles(empty)) == 0
+    nb = C.pa_plan_workspace_bytes(empty)
+    C.pa_prefill_run(empty, None, None, None, None, None, None, 1 << 40, nb, 0)
+    indptr, last = _tables([40, 10], 16)
+    idle = C.pa_prefill_plan_create(_problem(C, 2), True, np.zeros(3, np.int32), indptr, last)
+    assert len(C.pa_plan_prefill_tiles(idle)) == 0
+    big = 1 << 40  # never dereferenced
+    C.pa_prefill_run(idle, big, big, big, big, big, None, big, C.pa_plan_workspace_bytes(idle), 0)
