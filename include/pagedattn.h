@@ -23,8 +23,8 @@
  *   - flashinfer-cubin registry page, quickstart: the paged-table names
  *     kv_indptr, kv_indices, last_page_len and kv_layout (NHD here).
  *   - hysenlabs project review, "Installing FlashInfer and running a first
- *     decode": q is [num_qo_heads, head_dim]; k and v are
- *     [kv_len, num_kv_heads, head_dim] (NHD).
+ *     decode": the decode example's query has shape [num_qo_heads, head_dim],
+ *     its keys and values [kv_len, num_kv_heads, head_dim] (NHD).
  * The merge of partial states by log-sum-exp (pa_merge_state) is not named
  * on the pages; split-KV and cascade both need it.
  *

@@ -225,7 +225,7 @@ def cascade_decode(q, k_pool, v_pool, prefix_indices, prefix_len, kv_indptr, kv_
                    sm_scale, threads=1):
     """Two-level cascade: attention over the shared prefix, attention over each
     request's own pages, merged by log-sum-exp (FlashInfer README, core
-    feature 3 "Cascade Attention for hierarchical KV-Cache")."""
+    feature 3: cascade attention over a hierarchical KV cache)."""
     batch = len(_as_i32(last_page_len))
     npre = prefix_len // page_size
     pre_indptr = np.arange(batch + 1, dtype=np.int32) * npre

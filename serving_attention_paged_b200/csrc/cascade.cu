@@ -1,8 +1,8 @@
 // Cascade level 1: every request's queries against the shared prefix, on the
 // sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// FlashInfer README, core feature 3 ("Cascade Attention for hierarchical
-// KV-Cache") and the news item on cascade inference for shared-prefix batch
+// FlashInfer README, core feature 3 (cascade attention over a hierarchical
+// KV cache) and the news item on cascade inference for shared-prefix batch
 // decoding: when all B requests share a prefix, attention over the prefix is
 // one dense problem per kv head — the B*G query rows of that head (G q heads
 // per kv head, head-query fusion) against the prefix's K and V — so it is

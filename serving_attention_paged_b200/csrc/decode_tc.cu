@@ -1,7 +1,7 @@
 // Batched paged decode with head-query fusion on the sm_100a tensor cores.
 //
-// FlashInfer README, core feature 3 ("Head-Query fusion for accelerating
-// Grouped-Query Attention") and core feature 1 (tensor-core templates for
+// FlashInfer README, core feature 3 (head-query fusion, to speed up grouped-
+// query attention) and core feature 1 (tensor-core templates for
 // paged KV).  For G = Hq / Hkv >= 4 the G query heads of one kv head turn each
 // 128-token tile into a small dense contraction: S^T = K Q^T (M = 128 tokens,
 // N = 16 with the G heads padded, K = 128) and O^T += V^T P^T (M = 128 head
