@@ -291,7 +291,8 @@ pa_status pa_default_schedule(int32_t device, int32_t num_qo_heads, int32_t num_
                               int32_t* ctas_per_sm);
 
 /* 1 if the plan's decode level runs on the tensor-core kernel, 0 if on the
- * CUDA-core kernel, -1 for a null plan. */
+ * CUDA-core kernel, -1 for a null plan.  Prefill plans always run on the
+ * tensor cores (1). */
 int32_t pa_plan_uses_tensor_cores(pa_plan_t plan);
 
 void pa_plan_destroy(pa_plan_t plan);

@@ -403,7 +403,8 @@ const char* pa_status_string(pa_status s) {
 }
 
 int32_t pa_plan_uses_tensor_cores(pa_plan_t plan) {
-  return plan ? int32_t(pa::decode_uses_tensor_cores(plan->prob)) : -1;
+  if (!plan) return -1;
+  return plan->prefill ? 1 : int32_t(pa::decode_uses_tensor_cores(plan->prob));
 }
 
 int32_t pa_abi_version(void) { return PA_ABI_VERSION; }

@@ -142,3 +142,11 @@ def test_empty_prefill_plans_run_without_a_launch(C):
     assert len(C.pa_plan_prefill_tiles(idle)) == 0
     big = 1 << 40  # never dereferenced
     C.pa_prefill_run(idle, big, big, big, big, big, None, big, C.pa_plan_workspace_bytes(idle), 0)
+
+
+def test_prefill_plans_report_tensor_cores(C):
+    indptr, last = _tables([40, 10], 16)
+    for flags in (0, C.PA_FLAG_CUDA_CORES):
+        plan = C.pa_prefill_plan_create(_problem(C, 2, flags=flags), True,
+                                        np.array([0, 4, 6], np.int32), indptr, last)
+        assert C.pa_plan_uses_tensor_cores(plan) is True
