@@ -150,3 +150,17 @@ def test_prefill_plans_report_tensor_cores(C):
         plan = C.pa_prefill_plan_create(_problem(C, 2, flags=flags), True,
                                         np.array([0, 4, 6], np.int32), indptr, last)
         assert C.pa_plan_uses_tensor_cores(plan) is True
+
+
+def test_prefill_refuses_pools_beyond_signed_32bit_rows(C):
+    """Page rows are TMA coordinates (signed 32-bit): a pool of 2^31 - 1 rows or
+    more is refused before anything runs."""
+    indptr, last = _tables([40, 10], 16)
+    big = C.make_problem(batch=2, num_qo_heads=32, num_kv_heads=8, page_size=16, dtype="f16",
+                         sm_scale=0.088, num_sms=1, ctas_per_sm=1, num_pages=(1 << 31) // 16)
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_prefill_plan_create(big, True, np.array([0, 4, 6], np.int32), indptr, last)
+    assert e.value.status == C.PA_ERR_UNSUPPORTED
+    ok = C.make_problem(batch=2, num_qo_heads=32, num_kv_heads=8, page_size=16, dtype="f16",
+                        sm_scale=0.088, num_sms=1, ctas_per_sm=1, num_pages=(1 << 27))
+    C.pa_prefill_plan_create(ok, True, np.array([0, 4, 6], np.int32), indptr, last)
