@@ -162,5 +162,5 @@ def test_prefill_refuses_pools_beyond_signed_32bit_rows(C):
         C.pa_prefill_plan_create(big, True, np.array([0, 4, 6], np.int32), indptr, last)
     assert e.value.status == C.PA_ERR_UNSUPPORTED
     ok = C.make_problem(batch=2, num_qo_heads=32, num_kv_heads=8, page_size=16, dtype="f16",
-                        sm_scale=0.088, num_sms=1, ctas_per_sm=1, num_pages=(1 << 27))
+                        sm_scale=0.088, num_sms=1, ctas_per_sm=1, num_pages=(1 << 26))
     C.pa_prefill_plan_create(ok, True, np.array([0, 4, 6], np.int32), indptr, last)
