@@ -30,7 +30,6 @@ worked numeric example, so nothing is pinned to a published output value.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 import subprocess
 

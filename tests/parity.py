@@ -8,10 +8,7 @@ bf16 that exceeds 2e-3 once |o| >= 1 (fp16: |o| >= 8).  Where the dtype's
 half-ulp at the reference value is itself >= 2e-3, the allowance is
 2e-3 + that half-ulp.  An empty request must give exactly o = 0, lse = -inf.
 """
-import math
-
 import numpy as np
-import torch
 
 import oracle
 

@@ -11,7 +11,6 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
 from parity import assert_close, oracle_full, oracle_sampled, to_np
 from serving_attention_paged_b200 import workloads as W
 

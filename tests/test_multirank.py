@@ -7,8 +7,6 @@ value takes the slowest rank's time and all ranks' bytes (weak scaling).
 import os
 import socket
 
-import numpy as np
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp

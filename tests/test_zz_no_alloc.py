@@ -9,7 +9,6 @@ row, within the parity tolerance, and checks that a plan too large for the
 fixed array is refused before anything runs.  It lives in its own file,
 collected last, and passes alone in a fresh process as well.
 """
-import numpy as np
 import pytest
 import torch
 
