@@ -1,21 +1,28 @@
 #!/usr/bin/env python3
 """Paged decode attention benchmark: effective KV HBM GB/s, % of peak, µs/step.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 4] [--impl ours|reference]
 
 One step = one decode step of the workload through the run stage (plan made
 beforehand, as a serving engine does once per step and reuses across
 layers): for the plain workloads one ``pa_run`` launch, for the cascade
 ``pa_cascade_run``.  Inputs are resident in HBM; L2 is flushed (a 256 MB
-write) before every timed step, outside the CUDA events.  ``value`` is the
-algorithmic K/V bytes of all ranks' steps divided by the max-over-ranks
-device time.  ``e2e`` repeats the step through the public API from host
-buffers: plan on the host, upload of the work list, copies of q and
-kv_indices from pinned memory, the run, and the copy of o and lse back.
+write, then a 256 MB read) before every timed step, outside the CUDA events.
+``value`` is the algorithmic K/V bytes of all ranks' steps divided by the
+max-over-ranks device time.  ``e2e`` repeats the step through the public API
+from host buffers: plan on the host, upload of the work list, copies of q
+and kv_indices from pinned memory, the run, and the copy of o and lse back.
+
+The default workload is 4 (vector-sparse decode: B 256, GQA 64/8, page size
+1, bf16, 4.59 GB of K/V per step), the largest configuration on one GPU.  On
+one GPU its run also times, each with the same flush-and-events protocol:
+its contiguous page-size-16 twin (``vector_sparse_vs_contiguous``: the
+bandwidth ratio), and workloads 1, 2, 3, 5 (decode; for the cascade also its
+prefix level alone) and 6 (prefill / append) under ``per_config``.
 
 With N > 1 (torchrun) every rank runs its own replica of the workload on
 its own GPU (no collective on the data path; the requests of a batch are
-independent), so scaling is weak.
+independent), so scaling is weak; the extra workloads are skipped.
 
 ``--impl reference``: the fp64 CPU oracle timed on the host cores on a
 bounded sample of the same workload (rank 0 only).
@@ -42,6 +49,8 @@ METRIC = "paged decode: effective KV HBM GB/s and % of B200 peak; µs per decode
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
+EXTRA_SOAK_S = 0.3          # run-in before each extra workload's timed steps
+CPU_BASELINE_SECONDS = 10.0  # target CPU time of the oracle's bounded sample
 
 
 def parse_args():
@@ -49,8 +58,10 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="2",
-                    help="1 2 3 4 4c 4s 5 (decode), 6 (prefill / append); default: 2")
+    ap.add_argument("--workload", default="4",
+                    help="1 2 3 4 4c 4s 5 (decode), 6 (prefill / append); default: 4, the "
+                         "largest single-GPU configuration, whose run also times 4c and "
+                         "workloads 1, 2, 3, 5 and 6 as extra keys")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="untimed run-in after warm-up so clocks settle and get sampled")
@@ -66,6 +77,8 @@ def parse_args():
                          "< 0 = none")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the chosen workload (no contiguous twin, no per_config)")
     return ap.parse_args()
 
 
@@ -187,26 +200,36 @@ def aggregate_gbs(world: int, bytes_per_rank: int, max_seconds: float) -> float:
     return world * bytes_per_rank / max_seconds / 1e9
 
 
-def cpu_baseline(w, dev, max_requests):
-    """The oracle as it stands, on the host cores, over a bounded sample of
-    the same workload (whole requests, every q head)."""
+def cpu_baseline(w, dev, seconds):
+    """The oracle as it stands, on the host cores, over a bounded sample of the
+    same workload: whole requests (every q head), in request order, as many as
+    fit about ``seconds`` of CPU time (estimated from the first request)."""
     import oracle
     lens = w.kv_lens()
-    reqs = list(range(min(max_requests, w.batch)))
     threads = os.cpu_count() or 1
     indptr, indices, last = w.flat_tables()
-    t0 = time.perf_counter()
-    oracle.paged_decode_requests(dev["q"], dev["k_pool"], dev["v_pool"], indptr, indices, last,
-                                 reqs, num_qo_heads=w.num_qo_heads,
-                                 num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
-                                 page_size=w.page_size, dtype=w.dtype, sm_scale=w.sm_scale,
-                                 threads=threads)
-    dt = time.perf_counter() - t0
+    kw = dict(num_qo_heads=w.num_qo_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+              page_size=w.page_size, dtype=w.dtype, sm_scale=w.sm_scale, threads=threads)
+
+    def run(reqs):
+        t0 = time.perf_counter()
+        oracle.paged_decode_requests(dev["q"], dev["k_pool"], dev["v_pool"], indptr, indices,
+                                     last, reqs, **kw)
+        return time.perf_counter() - t0
+
+    t1 = run([0])
+    per_token = t1 / max(1, int(lens[0]) + w.prefix_len)
+    n, toks = 0, 0
+    while n < w.batch and (toks + int(lens[n]) + w.prefix_len) * per_token <= seconds:
+        toks += int(lens[n]) + w.prefix_len
+        n += 1
+    reqs = list(range(max(1, n)))
+    dt = run(reqs)
     toks = sum(int(lens[b]) + w.prefix_len for b in reqs)
     nbytes = 2 * toks * w.num_kv_heads * w.head_dim * 2
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"{len(reqs)} of {w.batch} requests (all {w.num_qo_heads} q heads each), "
-                      f"{toks} tokens, {nbytes} KV bytes, {dt:.2f} s, fp64"}
+            "sample": f"the first {len(reqs)} of {w.batch} requests (all {w.num_qo_heads} q "
+                      f"heads each), {toks} tokens, {nbytes} KV bytes, {dt:.2f} s, fp64"}
 
 
 def run_reference(args):
@@ -321,7 +344,7 @@ def make_l2_flush(dev_t):
     return flush_l2
 
 
-def timed_steps(step, flush_l2, args, stream, dev_t, world):
+def timed_steps(step, flush_l2, args, stream, dev_t, world, soak_seconds):
     """W warm-up steps, an untimed soak while the clocks are sampled, then K
     steps each bracketed by CUDA events on the launching stream (L2 flushed
     before each, outside the events).  Returns the max-over-ranks mean step
@@ -336,7 +359,7 @@ def timed_steps(step, flush_l2, args, stream, dev_t, world):
     uuid = str(torch.cuda.get_device_properties(dev_t).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     sampler.start()
-    t_end = time.perf_counter() + args.soak_seconds
+    t_end = time.perf_counter() + soak_seconds
     while time.perf_counter() < t_end:
         for _ in range(20):
             flush_l2()
@@ -404,6 +427,29 @@ def prefill_query_flops(w, queries):
     return int(4 * visible.sum() * w.num_qo_heads * w.head_dim)
 
 
+def prefill_timing(args, w, dev, stream, dev_t, world, flush_l2):
+    """The prefill / append workload as a per-config entry: µs per step and
+    causal attention TFLOP/s against the measured dense tensor peak."""
+    from serving_attention_paged_b200.wrapper import PagedPrefill
+    pf = PagedPrefill(w.qo_indptr, w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
+                      num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
+                      sm_scale=w.sm_scale, num_pages=w.num_pages, causal=True, device=dev_t)
+    o, lse = pf.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"])
+
+    def step():
+        pf.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"], o, lse, stream=stream)
+
+    ms, step_ms, clocks = timed_steps(step, flush_l2, args, stream, dev_t, world,
+                                      soak_seconds=EXTRA_SOAK_S)
+    flops = w.prefill_flops()
+    tf = flops / (ms * 1e-3) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+    return {"workload": w.name, **step_stats(step_ms), "flops_per_step": flops,
+            "tflop_s": round(tf, 1), "pct_of_tensor_peak": round(100.0 * tf / peak, 2),
+            "tensor_peak_kind": peak_kind, "kernel": "paged_prefill_kernel",
+            "sm_mhz": clocks["sm_mhz"], "clock_reasons": clocks["reasons"]}, ms
+
+
 def run_prefill(args, w, dev, stream, dev_t, world, rank):
     """Prefill / append step: one pa_prefill_run launch over all new tokens."""
     import torch
@@ -425,7 +471,8 @@ def run_prefill(args, w, dev, stream, dev_t, world, rank):
         pf.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"], o, lse, stream=stream)
 
     flush_l2 = make_l2_flush(dev_t)
-    ms, step_ms, clocks = timed_steps(step, flush_l2, args, stream, dev_t, world)
+    ms, step_ms, clocks = timed_steps(step, flush_l2, args, stream, dev_t, world,
+                                      soak_seconds=args.soak_seconds)
     flops = w.prefill_flops()
     value = world * flops / (ms * 1e-3) / 1e12
     achieved = flops / (ms * 1e-3) / 1e12
@@ -500,6 +547,98 @@ def run_prefill(args, w, dev, stream, dev_t, world, rank):
         }))
 
 
+def make_decode(w, args, dev_t, C):
+    """Plan (and workspace) for a decode workload, in the bench's launch configuration."""
+    from serving_attention_paged_b200.wrapper import PagedDecode
+    return PagedDecode(w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
+                       num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
+                       sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
+                       device=dev_t, min_chunk_tokens=args.min_chunk_tokens,
+                       ctas_per_sm=args.ctas_per_sm or None,
+                       flags={"auto": 0, "cuda_cores": C.PA_FLAG_CUDA_CORES,
+                              "tensor_cores": C.PA_FLAG_TENSOR_CORES}[args.kernel],
+                       piece_cost_tokens=args.piece_cost_tokens)
+
+
+def step_stats(step_ms):
+    return {"us_p10_p50_p90": [round(float(np.percentile(step_ms, p)) * 1e3, 2)
+                               for p in (10, 50, 90)],
+            "us_mean": round(sum(step_ms) / len(step_ms) * 1e3, 2)}
+
+
+def decode_kernel_name(C, pd):
+    return "paged_decode_tc_kernel" if C.pa_plan_uses_tensor_cores(pd.plan) else \
+        "paged_decode_kernel"
+
+
+def extra_decode(key, args, dev_t, stream, flush_l2, peak, C):
+    """One more decode workload, timed like the headline (1 GPU, own clocks):
+    µs per step, effective GB/s and % of the HBM peak."""
+    import torch
+    w = workload(key)
+    dev = w.materialize(dev_t)
+    pd = make_decode(w, args, dev_t, C)
+    o, lse = pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"],
+                    prefix_indices=dev.get("prefix_indices"))
+
+    def step():
+        pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"], o, lse,
+               prefix_indices=dev.get("prefix_indices"), stream=stream)
+
+    ms, step_ms, clocks = timed_steps(step, flush_l2, args, stream, dev_t, 1,
+                                      soak_seconds=EXTRA_SOAK_S)
+    nbytes = w.kv_bytes()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    entry = {"workload": w.name, **step_stats(step_ms), "gb_s": round(gbs, 1),
+             "pct_of_peak": round(100.0 * gbs / peak, 2), "kv_bytes_per_step": nbytes,
+             "kernel": decode_kernel_name(C, pd), "sm_mhz": clocks["sm_mhz"],
+             "clock_reasons": clocks["reasons"]}
+    if w.prefix_len:
+        # the prefix level with a near-empty second level: the same cascade with
+        # every suffix cut to its first token (the decode level then reads one
+        # token per request and merges the prefix chunks of each row)
+        one_indptr = np.arange(w.batch + 1, dtype=np.int32)
+        one_last = np.ones(w.batch, dtype=np.int32)
+        first_pages = dev["kv_indices"][torch.from_numpy(w.kv_indptr[:-1].astype(np.int64))
+                                        .to(dev_t)].contiguous()
+        from serving_attention_paged_b200.wrapper import PagedDecode
+        pp = PagedDecode(one_indptr, one_last, num_qo_heads=w.num_qo_heads,
+                         num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
+                         sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
+                         device=dev_t)
+
+        def prefix_step():
+            pp.run(dev["q"], dev["k_pool"], dev["v_pool"], first_pages, o, lse,
+                   prefix_indices=dev["prefix_indices"], stream=stream)
+
+        pms, pstep_ms, _ = timed_steps(prefix_step, flush_l2, args, stream, dev_t, 1,
+                                       soak_seconds=0.0)
+        flops = 4 * w.batch * w.num_qo_heads * w.prefix_len * w.head_dim
+        tpeak, tkind = measured_tensor_peak()
+        tf = flops / (pms * 1e-3) / 1e12
+        entry["prefix_level"] = {
+            **step_stats(pstep_ms), "flops_per_step": flops, "tflop_s": round(tf, 1),
+            "pct_of_tensor_peak": round(100.0 * tf / tpeak, 2), "tensor_peak_kind": tkind,
+            "includes": "cascade_prefix_kernel + a decode launch over one suffix token per "
+                        "request that merges the prefix chunks of every row"}
+    del dev, o, lse
+    torch.cuda.empty_cache()
+    return w, entry, ms
+
+
+def launch_floor(args, dev_t, stream, flush_l2):
+    """Event-timed cost of one near-empty kernel in the bench's timing pattern
+    (L2 flush, start event, one kernel, end event): the fixed per-step floor."""
+    import torch
+    x = torch.zeros(1, device=dev_t)
+
+    def step():
+        x.add_(1.0)
+
+    ms, step_ms, _ = timed_steps(step, flush_l2, args, stream, dev_t, 1, soak_seconds=0.0)
+    return step_stats(step_ms)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -522,7 +661,6 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     from serving_attention_paged_b200 import pagedattn as C
-    from serving_attention_paged_b200.wrapper import PagedDecode
 
     w = workload(args.workload)
     dev = w.materialize(dev_t)
@@ -534,14 +672,7 @@ def run_ours(args):
             dist.destroy_process_group()
         return
     t0 = time.perf_counter()
-    pd = PagedDecode(w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
-                     num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
-                     sm_scale=w.sm_scale, num_pages=w.num_pages, prefix_len=w.prefix_len,
-                     device=dev_t, min_chunk_tokens=args.min_chunk_tokens,
-                     ctas_per_sm=args.ctas_per_sm or None,
-                     flags={"auto": 0, "cuda_cores": C.PA_FLAG_CUDA_CORES,
-                            "tensor_cores": C.PA_FLAG_TENSOR_CORES}[args.kernel],
-                     piece_cost_tokens=args.piece_cost_tokens)
+    pd = make_decode(w, args, dev_t, C)
     tensor_cores = C.pa_plan_uses_tensor_cores(pd.plan)
     setup_us = (time.perf_counter() - t0) * 1e6
     reps = 20
@@ -559,7 +690,8 @@ def run_ours(args):
                prefix_indices=dev.get("prefix_indices"), stream=stream)
 
     flush_l2 = make_l2_flush(dev_t)
-    ms, step_ms, clocks = timed_steps(step, flush_l2, args, stream, dev_t, world)
+    ms, step_ms, clocks = timed_steps(step, flush_l2, args, stream, dev_t, world,
+                                      soak_seconds=args.soak_seconds)
 
     nbytes = w.kv_bytes()
     value = aggregate_gbs(world, nbytes, ms * 1e-3)
@@ -605,9 +737,8 @@ def run_ours(args):
             if i >= max(args.warmup, 3):
                 e2e_s.append(time.perf_counter() - t0)
         e2e_max = max_over_ranks(sum(e2e_s) / len(e2e_s), dev_t)
-        from serving_attention_paged_b200 import pagedattn as Cb
         items = len(pd.work_items())
-        n_cta = len(Cb.pa_plan_cta_indptr(pd.plan)) - 1
+        n_cta = len(C.pa_plan_cta_indptr(pd.plan)) - 1
         h2d = (q_h.numel() * q_h.element_size() + idx_h.numel() * 4 + items * 24 +
                (n_cta + 1) * 4 + (w.batch * w.num_kv_heads + 1) * 4)
         e2e = {"value": aggregate_gbs(world, nbytes, e2e_max), "unit": "GB/s",
@@ -615,11 +746,36 @@ def run_ours(args):
                "d2h_bytes_per_step": int(o_h.numel() * o_h.element_size() + lse_h.numel() * 4),
                "us_per_step": e2e_max * 1e6,
                "includes": "host plan + work-list upload + q/kv_indices H2D + run + o/lse D2H"}
+        del q_h, idx_h, o_h, lse_h, q_d, idx_d
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        max_req = {"batch_decode_uniform": 16, "single_request_decode": 1}.get(w.name, 4)
-        cpu = cpu_baseline(w, dev, max_req)
+        cpu = cpu_baseline(w, dev, CPU_BASELINE_SECONDS)
+
+    # Every other configuration, timed the same way on this GPU (1 GPU only:
+    # they characterise the kernels; the headline above is the job's number).
+    extras = {}
+    if world == 1 and not args.headline_only and w.name == "vector_sparse_decode":
+        del dev, o, lse
+        torch.cuda.empty_cache()
+        tw, twin, _ = extra_decode("4c", args, dev_t, stream, flush_l2, peak, C)
+        extras["vector_sparse_vs_contiguous"] = {
+            "ratio": round(value / twin["gb_s"], 4), "target": 0.85,
+            "page_size_1_gb_s": round(value, 1), "contiguous": twin}
+        per = {}
+        for key in (1, 2, 3, 5):
+            kw, entry, _ = extra_decode(str(key), args, dev_t, stream, flush_l2, peak, C)
+            per[str(key)] = entry
+        per["1"]["launch_floor"] = launch_floor(args, dev_t, stream, flush_l2)
+        per["1"]["launch_floor"]["what"] = (
+            "the same timing pattern (flush, start event, one 1-element torch kernel, end "
+            "event): the fixed cost every event-timed step carries")
+        pw = workload("6")
+        pdev = pw.materialize(dev_t)
+        per["6"] = prefill_timing(args, pw, pdev, stream, dev_t, 1, flush_l2)[0]
+        del pdev
+        torch.cuda.empty_cache()
+        extras["per_config"] = per
 
     if rank == 0:
         line = {
@@ -638,6 +794,7 @@ def run_ours(args):
             "gpu_launches": args.steps * launches_per_step,
             "plan_us": plan_us, "setup_us": setup_us,
             "step_ms_p10_p50_p90": [float(np.percentile(step_ms, p)) for p in (10, 50, 90)],
+            **extras,
         }
         print(json.dumps(line))
     if world > 1:
