@@ -214,6 +214,13 @@ pa_status pa_plan_prefill_tiles(pa_plan_t plan, const pa_prefill_tile** tiles, i
  * aligned. */
 pa_status pa_plan_workspace_bytes(pa_plan_t plan, size_t* bytes);
 
+/* Byte offset, within the workspace, of the two 64-bit status words that
+ * pa_plan_check reads: word 0 holds the first out-of-range kv_indices
+ * position a PA_FLAG_CHECK_INDICES run met (all ones: none), word 1 is
+ * nonzero once a kernel abandoned a bounded wait.  pa_plan_upload writes
+ * both as "nothing seen"; 8-byte aligned. */
+pa_status pa_plan_status_offset(pa_plan_t plan, size_t* offset);
+
 /* Copy the work list into the workspace and zero its counters (enqueued on
  * `stream`, a cudaStream_t or NULL for the legacy default stream).  Once per
  * plan and workspace; any number of runs may follow.  The counters return to
@@ -269,11 +276,22 @@ pa_status pa_merge_state(const void* o_a, const float* lse_a, const void* o_b,
  * prefill plans with PA_ERR_INVALID_ARG.  Nothing is allocated: each call uploads the plan
  * into the array (as pa_plan_upload) and runs it (as pa_run).  The first call
  * on a device looks the array up (cudaGetSymbolAddress), so make it before any
- * stream capture.  All calls share the array: calls that overlap on the GPU
+ * stream capture.  The looked-up address is kept for the life of the
+ * process: after a cudaDeviceReset on that device this entry point must not
+ * be used again.  All calls share the array: calls that overlap on the GPU
  * (different streams or threads) race. */
 pa_status pa_run_static_workspace(pa_plan_t plan, const void* q, const void* k_pool,
                                   const void* v_pool, const int32_t* d_kv_indices, void* o,
                                   float* lse, void* stream);
+
+/* pa_plan_check for the library's fixed workspace: synchronously reads and
+ * clears the status words that the last pa_run_static_workspace call on this
+ * device left in it, with the same results as pa_plan_check (PA_ERR_DEVICE_TIMEOUT,
+ * PA_ERR_DEVICE_CHECK with *bad_position, or PA_OK).  Call it after that run
+ * and before the next one, which clears the words again.  `plan` must be the
+ * plan of that run (its layout locates the words); plans that
+ * pa_run_static_workspace refuses are refused here with the same status. */
+pa_status pa_static_workspace_check(pa_plan_t plan, int64_t* bad_position, void* stream);
 
 /* Synchronously read and clear the device status words of a workspace.
  * Returns PA_ERR_DEVICE_TIMEOUT if a kernel abandoned one of its bounded

@@ -380,6 +380,12 @@ pa_status pa_plan_prefix_chunks(pa_plan_t plan, int32_t* n_chunks, int32_t* chun
   return PA_OK;
 }
 
+pa_status pa_plan_status_offset(pa_plan_t plan, size_t* offset) {
+  if (!plan || !offset) return PA_ERR_INVALID_ARG;
+  *offset = plan->ws.error;
+  return PA_OK;
+}
+
 pa_status pa_plan_workspace_bytes(pa_plan_t plan, size_t* bytes) {
   if (!plan || !bytes) return PA_ERR_INVALID_ARG;
   *bytes = plan->ws.total;

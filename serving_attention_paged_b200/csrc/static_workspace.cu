@@ -12,10 +12,16 @@
 // stays allocated until the process exits.  Its device address is looked up
 // with cudaGetSymbolAddress on the first call made on each device (with that
 // device current); that first call should therefore come before any stream
-// capture.  Every call shares the one array and leaves its contents behind;
-// each call re-uploads the work list and re-zeroes the arrival counters and
-// status words, so calls that run one after another are independent, but two
-// calls whose work overlaps on the GPU (other streams, other threads) race.
+// capture.  The address is cached per device for the life of the process: a
+// cudaDeviceReset (or anything else that destroys the device's primary
+// context) invalidates it, and the entry point must not be used on that
+// device afterwards.  Every call shares the one array and leaves its contents
+// behind; each call re-uploads the work list and re-zeroes the arrival
+// counters and status words, so calls that run one after another are
+// independent, but two calls whose work overlaps on the GPU (other streams,
+// other threads) race.  pa_static_workspace_check reads the status words a
+// call left there (a bad page index under PA_FLAG_CHECK_INDICES, an abandoned
+// bounded wait) before the next call clears them.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -60,4 +66,14 @@ extern "C" pa_status pa_run_static_workspace(pa_plan_t plan, const void* q, cons
   st = pa_plan_upload(plan, ws, kStaticWorkspaceBytes, stream);
   if (st != PA_OK) return st;
   return pa_run(plan, q, k_pool, v_pool, d_kv_indices, o, lse, ws, kStaticWorkspaceBytes, stream);
+}
+
+extern "C" pa_status pa_static_workspace_check(pa_plan_t plan, int64_t* bad_position,
+                                               void* stream) {
+  if (!plan || plan->cascade || plan->prefill) return PA_ERR_INVALID_ARG;
+  if (plan->ws.total > kStaticWorkspaceBytes) return PA_ERR_WORKSPACE_TOO_SMALL;
+  void* ws = nullptr;
+  const pa_status st = static_workspace_address(&ws);
+  if (st != PA_OK) return st;
+  return pa_plan_check(plan, ws, bad_position, stream);
 }

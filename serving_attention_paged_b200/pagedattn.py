@@ -65,12 +65,14 @@ _SIGS = {
     "pa_plan_num_partials": [_vp, _P(_i64)],
     "pa_plan_prefix_chunks": [_vp, _P(_i32), _P(_i32)],
     "pa_plan_workspace_bytes": [_vp, _P(_sz)],
+    "pa_plan_status_offset": [_vp, _P(_sz)],
     "pa_plan_upload": [_vp, _vp, _sz, _vp],
     "pa_run": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "pa_cascade_run": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "pa_merge_state": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp],
     "pa_run_static_workspace": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "pa_plan_check": [_vp, _vp, _P(_i64), _vp],
+    "pa_static_workspace_check": [_vp, _P(_i64), _vp],
     "pa_default_schedule": [_i32, _i32, _i32, _i32, ctypes.c_uint32, _P(_i32), _P(_i32)],
 }
 for _name, _args in _SIGS.items():
@@ -238,6 +240,12 @@ def pa_plan_workspace_bytes(plan: Plan) -> int:
     return n.value
 
 
+def pa_plan_status_offset(plan: Plan) -> int:
+    n = _sz()
+    _check(lib.pa_plan_status_offset(plan.handle, ctypes.byref(n)), "pa_plan_status_offset")
+    return n.value
+
+
 def pa_plan_upload(plan: Plan, workspace, workspace_bytes: int, stream=None):
     _check(lib.pa_plan_upload(plan.handle, _ptr(workspace), workspace_bytes, _stream(stream)),
            "pa_plan_upload")
@@ -292,6 +300,19 @@ def pa_plan_check(plan: Plan, workspace, stream=None) -> int:
         err.position = pos.value
         raise err
     _check(st, "pa_plan_check")
+    return pos.value
+
+
+def pa_static_workspace_check(plan: Plan, stream=None) -> int:
+    """pa_plan_check for the status words of the library's fixed workspace,
+    as the last ``pa_run_static_workspace`` call left them."""
+    pos = _i64()
+    st = lib.pa_static_workspace_check(plan.handle, ctypes.byref(pos), _stream(stream))
+    if st == PA_ERR_DEVICE_CHECK:
+        err = PagedAttnError(st, "pa_static_workspace_check")
+        err.position = pos.value
+        raise err
+    _check(st, "pa_static_workspace_check")
     return pos.value
 
 

@@ -201,3 +201,34 @@ def test_default_piece_cost_follows_the_kernel(C):
                                     w.last_page_len)
         assert np.array_equal(C.pa_plan_work_items(default), C.pa_plan_work_items(explicit))
         assert C.pa_plan_quota_tokens(default) == C.pa_plan_quota_tokens(explicit)
+
+
+def test_plan_hand_worked_examples_library(C):
+    """The library's work list against the hand-worked fixtures directly (not
+    only through the oracle's restatement)."""
+    import json
+    path = os.path.join(ROOT, "tests", "golden", "plan_small.json")
+    for g in json.load(open(path))["cases"]:
+        hkv = g["num_kv_heads"]
+        B = len(g["last_page_len"])
+        prob = C.make_problem(batch=B, num_qo_heads=hkv, num_kv_heads=hkv,
+                              page_size=g["page_size"], dtype="f16", sm_scale=0.1,
+                              num_sms=g["num_sms"], ctas_per_sm=g["ctas_per_sm"],
+                              min_chunk_tokens=g["min_chunk_tokens"], num_pages=1 << 20,
+                              piece_cost_tokens=g.get("piece_cost_tokens", 0) or -1)
+        plan = C.pa_plan_create(prob, np.array(g["kv_indptr"]), np.array(g["last_page_len"]))
+        assert C.pa_plan_quota_tokens(plan) == g["quota"]
+        assert C.pa_plan_work_items(plan).tolist() == g["items"]
+        assert C.pa_plan_cta_indptr(plan).tolist() == g["cta_indptr"]
+        assert C.pa_plan_merge_indptr(plan, B * hkv).tolist() == g["merge_indptr"]
+
+
+def test_status_offset_lies_inside_the_workspace(C):
+    for lens in ([], [5, 0, 3000], [100] * 40):
+        indptr, _, last = W.tables_from_lengths(lens, 16)
+        prob = C.make_problem(batch=len(lens), num_qo_heads=32, num_kv_heads=8, page_size=16,
+                              dtype="bf16", sm_scale=0.1, num_sms=148, ctas_per_sm=1,
+                              num_pages=1 << 16)
+        plan = C.pa_plan_create(prob, indptr, last)
+        off = C.pa_plan_status_offset(plan)
+        assert off % 8 == 0 and off + 16 <= C.pa_plan_workspace_bytes(plan)

@@ -135,3 +135,45 @@ def test_piece_cost_shifts_tokens_to_single_piece_groups():
             by_k.setdefault(k, []).append(tok)
         assert set(by_k) == {1, 2}
         assert np.mean(by_k[1]) - np.mean(by_k[2]) > c / 2
+
+
+def sliced_work_list(lens, indptr, hkv, q):
+    """The c = 0 rule stated a second way, without the walk: lay the requests'
+    tokens end to end (request b at positions [s_b, s_b + L_b)); group g is
+    the positions [g q, (g + 1) q) and holds, in request order, every request
+    that overlaps it, cut to the overlap.  An empty request sits at s_b and
+    belongs to the group of that position (the last group if s_b = T)."""
+    lens = [int(x) for x in lens]
+    T = sum(lens)
+    n_groups = max(1, -(-T // q)) if lens else 0
+    groups = [[] for _ in range(n_groups)]
+    s = 0
+    for b, L in enumerate(lens):
+        if L == 0:
+            groups[min(s // q, n_groups - 1)].append((b, 0, 0))
+        for g in range(s // q, min(n_groups, -(-(s + L) // q))):
+            lo, hi = max(s, g * q), min(s + L, (g + 1) * q)
+            if hi > lo:
+                groups[g].append((b, lo - s, hi - s))
+        s += L
+    return [[b, h, int(indptr[b]), t0, t1] for g in groups for h in range(hkv)
+            for (b, t0, t1) in g]
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_plan_without_piece_cost_is_a_slicing_of_the_tokens(seed):
+    """Pins the walk against its own definition written as arithmetic on
+    token positions: an off-by-one in when a group closes, or in where an
+    empty request lands, changes the sliced list."""
+    rng = np.random.default_rng(500 + seed)
+    B = int(rng.integers(1, 30))
+    P = int(rng.choice([1, 4, 16]))
+    lens = rng.integers(0, 700, size=B) * (rng.random(B) > 0.25)
+    if seed % 4 == 0:  # requests ending exactly on group boundaries
+        lens = np.where(lens > 0, 64 * (1 + lens // 200), 0)
+    indptr, _, last = W.tables_from_lengths(lens, P)
+    hkv = int(rng.choice([1, 2, 4]))
+    sms = int(rng.integers(1, 40))
+    q, items, ci, _ = oracle.plan(indptr, last, page_size=P, num_kv_heads=hkv, num_sms=sms,
+                                  ctas_per_sm=1, min_chunk_tokens=32, piece_cost=0)
+    assert items[:, :5].tolist() == sliced_work_list(lens, indptr, hkv, q)

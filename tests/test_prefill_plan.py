@@ -164,3 +164,26 @@ def test_prefill_refuses_pools_beyond_signed_32bit_rows(C):
     ok = C.make_problem(batch=2, num_qo_heads=32, num_kv_heads=8, page_size=16, dtype="f16",
                         sm_scale=0.088, num_sms=1, ctas_per_sm=1, num_pages=(1 << 26))
     C.pa_prefill_plan_create(ok, True, np.array([0, 4, 6], np.int32), indptr, last)
+
+
+def test_prefill_pool_row_limit_at_its_edge(C):
+    """The edge of the limit: with page size 8 (the smallest the prefill
+    kernel moves), 2^28 - 1 pages (2^31 - 8 rows, the largest pool whose rows
+    and the one-past-the-end fill row fit a signed 32-bit coordinate) are
+    accepted and 2^28 pages (2^31 rows) refused; the same holds for cascade
+    plans with a prefix."""
+    indptr, last = _tables([40, 10], 8)
+
+    def prob(num_pages):
+        return C.make_problem(batch=2, num_qo_heads=32, num_kv_heads=8, page_size=8,
+                              dtype="f16", sm_scale=0.088, num_sms=1, ctas_per_sm=1,
+                              num_pages=num_pages)
+
+    qo = np.array([0, 4, 6], np.int32)
+    C.pa_prefill_plan_create(prob((1 << 28) - 1), True, qo, indptr, last)
+    C.pa_cascade_plan_create(prob((1 << 28) - 1), 64, indptr, last)
+    for make in (lambda p: C.pa_prefill_plan_create(p, True, qo, indptr, last),
+                 lambda p: C.pa_cascade_plan_create(p, 64, indptr, last)):
+        with pytest.raises(C.PagedAttnError) as e:
+            make(prob(1 << 28))
+        assert e.value.status == C.PA_ERR_UNSUPPORTED

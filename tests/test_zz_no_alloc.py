@@ -66,3 +66,30 @@ def test_static_workspace_refuses_oversized_plans():
     with pytest.raises(C.PagedAttnError) as e:
         C.pa_run_static_workspace(plan, 1 << 40, 1 << 40, 1 << 40, 1 << 40, 1 << 40, None)
     assert e.value.status == C.PA_ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+def test_static_workspace_reports_bad_index(kernel):
+    """With PA_FLAG_CHECK_INDICES a run on the fixed workspace records an
+    out-of-range page index there; pa_static_workspace_check reports its
+    position and clears it, as pa_plan_check does for a caller workspace."""
+    from serving_attention_paged_b200 import pagedattn as C
+    w = W.make_workload("static_chk", [40, 40], num_qo_heads=8, num_kv_heads=2, page_size=16,
+                        dtype="f16", seed=93)
+    dev = {k: v.cuda() for k, v in w.materialize().items()}
+    flags = C.PA_FLAG_CHECK_INDICES | (C.PA_FLAG_TENSOR_CORES if kernel == "tensor_cores"
+                                       else C.PA_FLAG_CUDA_CORES)
+    plan = C.pa_plan_create(_problem(C, w, ctas_per_sm=1, flags=flags), w.kv_indptr,
+                            w.last_page_len)
+    o = torch.empty_like(dev["q"])
+    lse = torch.empty(w.batch, w.num_qo_heads, device="cuda")
+    C.pa_run_static_workspace(plan, dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"],
+                              o, lse)
+    assert C.pa_static_workspace_check(plan) == -1
+    bad = dev["kv_indices"].clone()
+    bad[4] = w.num_pages + 7  # skipped by the checked kernel and recorded
+    C.pa_run_static_workspace(plan, dev["q"], dev["k_pool"], dev["v_pool"], bad, o, lse)
+    with pytest.raises(C.PagedAttnError) as e:
+        C.pa_static_workspace_check(plan)
+    assert e.value.status == C.PA_ERR_DEVICE_CHECK and e.value.position == 4
+    assert C.pa_static_workspace_check(plan) == -1  # the word was cleared
