@@ -18,7 +18,9 @@ The default workload is 4 (vector-sparse decode: B 256, GQA 64/8, page size
 one GPU its run also times, each with the same flush-and-events protocol:
 its contiguous page-size-16 twin (``vector_sparse_vs_contiguous``: the
 bandwidth ratio), and workloads 1, 2, 3, 5 (decode; for the cascade also its
-prefix level alone) and 6 (prefill / append) under ``per_config``.
+prefix level), 2f8 and 3f8 (workloads 2 and 3 with 8-bit E4M3 caches), 2rope
+(workload 2 with rotary positions applied on the fly) and 6 (prefill /
+append) under ``per_config``.
 
 With N > 1 (torchrun) every rank runs its own replica of the workload on
 its own GPU (no collective on the data path; the requests of a batch are
@@ -547,7 +549,7 @@ def run_prefill(args, w, dev, stream, dev_t, world, rank):
         }))
 
 
-def make_decode(w, args, dev_t, C):
+def make_decode(w, args, dev_t, C, rope_theta=0.0):
     """Plan (and workspace) for a decode workload, in the bench's launch configuration."""
     from serving_attention_paged_b200.wrapper import PagedDecode
     return PagedDecode(w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
@@ -557,7 +559,8 @@ def make_decode(w, args, dev_t, C):
                        ctas_per_sm=args.ctas_per_sm or None,
                        flags={"auto": 0, "cuda_cores": C.PA_FLAG_CUDA_CORES,
                               "tensor_cores": C.PA_FLAG_TENSOR_CORES}[args.kernel],
-                       piece_cost_tokens=args.piece_cost_tokens)
+                       piece_cost_tokens=args.piece_cost_tokens, kv_dtype=w.kv_dtype,
+                       k_scale=w.k_scale, v_scale=w.v_scale, rope_theta=rope_theta)
 
 
 def step_stats(step_ms):
@@ -571,13 +574,13 @@ def decode_kernel_name(C, pd):
         "paged_decode_kernel"
 
 
-def extra_decode(key, args, dev_t, stream, flush_l2, peak, C):
+def extra_decode(key, args, dev_t, stream, flush_l2, peak, C, rope_theta=0.0):
     """One more decode workload, timed like the headline (1 GPU, own clocks):
     µs per step, effective GB/s and % of the HBM peak."""
     import torch
     w = workload(key)
     dev = w.materialize(dev_t)
-    pd = make_decode(w, args, dev_t, C)
+    pd = make_decode(w, args, dev_t, C, rope_theta)
     o, lse = pd.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"],
                     prefix_indices=dev.get("prefix_indices"))
 
@@ -593,6 +596,11 @@ def extra_decode(key, args, dev_t, stream, flush_l2, peak, C):
              "pct_of_peak": round(100.0 * gbs / peak, 2), "kv_bytes_per_step": nbytes,
              "kernel": decode_kernel_name(C, pd), "sm_mhz": clocks["sm_mhz"],
              "clock_reasons": clocks["reasons"]}
+    if w.kv_dtype:
+        entry["kv_cache"] = {"format": w.kv_dtype, "k_scale": w.k_scale, "v_scale": w.v_scale,
+                             "bytes_per_element": 1}
+    if rope_theta:
+        entry["rope_theta"] = rope_theta
     if w.prefix_len:
         # the prefix level with a near-empty second level: the same cascade with
         # every suffix cut to its first token (the decode level then reads one
@@ -766,6 +774,14 @@ def run_ours(args):
         for key in (1, 2, 3, 5):
             kw, entry, _ = extra_decode(str(key), args, dev_t, stream, flush_l2, peak, C)
             per[str(key)] = entry
+        # 8-bit (E4M3) caches of workloads 2 and 3: GB/s on the halved bytes
+        for key in ("2f8", "3f8"):
+            _, entry, _ = extra_decode(key, args, dev_t, stream, flush_l2, peak, C)
+            per[key] = entry
+        # rotary positions on the fly, workload 2: the cost against plain decode
+        _, rope, _ = extra_decode("2", args, dev_t, stream, flush_l2, peak, C, rope_theta=1e4)
+        rope["time_vs_plain"] = round(rope["us_mean"] / per["2"]["us_mean"], 3)
+        per["2rope"] = rope
         per["1"]["launch_floor"] = launch_floor(args, dev_t, stream, flush_l2)
         per["1"]["launch_floor"]["what"] = (
             "the same timing pattern (flush, start event, one 1-element torch kernel, end "

@@ -48,8 +48,10 @@
  * until pa_plan_destroy.  Functions return a pa_status; nothing throws
  * across the ABI.  Launch failures return PA_ERR_CUDA.
  *
- * Supported: head_dim 128; num_qo_heads / num_kv_heads in {1, 2, 4, 8, 16};
- * page_size a power of two in [1, 1024]; fp16 and bf16.
+ * Supported: head_dim 128; num_qo_heads / num_kv_heads in {1, 2, 4, 8};
+ * page_size a power of two in [1, 1024]; fp16 and bf16 q (and pools), and for
+ * decode also 8-bit FP8 pools (E4M3 / E5M2 with a K and a V scale) and rotary
+ * positions applied on the fly (pa_problem.kv_dtype, rope_theta).
  */
 #ifndef PAGEDATTN_H_
 #define PAGEDATTN_H_
@@ -61,7 +63,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 4
+#define PA_ABI_VERSION 5
 
 typedef enum {
   PA_OK = 0,
@@ -74,7 +76,13 @@ typedef enum {
   PA_ERR_DEVICE_TIMEOUT = 7        /* a kernel gave up on a bounded wait (see pa_plan_check) */
 } pa_status;
 
-typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 /* pa_merge_state only */ } pa_dtype;
+typedef enum {
+  PA_F16 = 0,
+  PA_BF16 = 1,
+  PA_F32 = 2,   /* pa_merge_state only */
+  PA_E4M3 = 3,  /* 8-bit KV cache (pa_problem.kv_dtype): OCP FP8 E4M3, no infinities, max 448 */
+  PA_E5M2 = 4   /* 8-bit KV cache (pa_problem.kv_dtype): OCP FP8 E5M2 */
+} pa_dtype;
 
 /* Flags for pa_problem.flags. */
 #define PA_FLAG_CHECK_INDICES 1u /* kernels bounds-check every page index against
@@ -106,6 +114,25 @@ typedef struct {
                                 (see pa_plan_create): 0 = the default of the decode
                                 kernel the problem runs (400 CUDA cores, 128 tensor
                                 cores), > 0 that many tokens, < 0 none */
+  /* Compressed KV cache (README core feature 3: low-precision attention for a
+   * compressed KV-Cache).  kv_dtype PA_E4M3 or PA_E5M2: the pools hold 8-bit
+   * codes, [num_pages, page_size, num_kv_heads, head_dim] bytes, and the cached
+   * key is k_scale * code, the value v_scale * code (one scale per tensor;
+   * both finite and > 0).  q and o stay in `dtype`.  Any other kv_dtype
+   * (PA_F16 / PA_BF16) means the pools hold `dtype` and the scales are unused.
+   * 8-bit caches run on the CUDA-core decode kernel (pa_run,
+   * pa_run_static_workspace); cascade plans with a prefix, prefill plans and
+   * PA_FLAG_TENSOR_CORES refuse them with PA_ERR_UNSUPPORTED. */
+  pa_dtype kv_dtype;
+  float k_scale, v_scale;
+  /* Rotary positions on the fly (README usage example: decode with
+   * pos_encoding_mode="ROPE_LLAMA"), when rope_theta > 0: before the dot
+   * product, q is rotated to position L_b - 1 (the new token is the last one
+   * in the cache) and the key of token t to position t; element pairs
+   * (d, d + 64) turn by the angle pos * rope_theta^(-2d/128) (rotate-half
+   * pairing; values are not rotated).  0 = no rotation.  Decode only, on the
+   * CUDA-core kernel, as for 8-bit caches. */
+  float rope_theta;
 } pa_problem;
 
 /* One piece of run-stage work: tokens [token_begin, token_end) of kv head
@@ -306,6 +333,13 @@ pa_status pa_plan_check(pa_plan_t plan, void* d_workspace, int64_t* bad_position
  * runs fit on one SM.  The tensor-core kernel holds one CTA per SM. */
 pa_status pa_default_schedule(int32_t device, int32_t num_qo_heads, int32_t num_kv_heads,
                               pa_dtype dtype, uint32_t flags, int32_t* num_sms,
+                              int32_t* ctas_per_sm);
+
+/* pa_default_schedule for a whole problem: the SM count of `device` and how
+ * many CTAs of the decode kernel that `problem` runs fit on one SM, its
+ * 8-bit cache and rotary positions included (only the shape, dtype, flags,
+ * kv_dtype and rope_theta fields are read). */
+pa_status pa_problem_schedule(const pa_problem* problem, int32_t device, int32_t* num_sms,
                               int32_t* ctas_per_sm);
 
 /* 1 if the plan's decode level runs on the tensor-core kernel, 0 if on the

@@ -21,8 +21,8 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpagedattn.so")
 
-SOURCES = ["plan.cpp", "api.cu", "decode.cu", "decode_tc.cu", "merge_state.cu", "cascade.cu",
-           "prefill.cu", "static_workspace.cu"]
+SOURCES = ["plan.cpp", "api.cu", "decode.cu", "decode_f32.cu", "decode_tc.cu", "merge_state.cu",
+           "cascade.cu", "prefill.cu", "static_workspace.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

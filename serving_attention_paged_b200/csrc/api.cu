@@ -158,4 +158,28 @@ pa_status pa_default_schedule(int32_t device, int32_t num_qo_heads, int32_t num_
   return PA_OK;
 }
 
+pa_status pa_problem_schedule(const pa_problem* problem, int32_t device, int32_t* num_sms,
+                              int32_t* ctas_per_sm) {
+  if (!problem || !num_sms || !ctas_per_sm || problem->num_kv_heads <= 0 ||
+      problem->num_qo_heads % problem->num_kv_heads)
+    return PA_ERR_INVALID_ARG;
+  const int32_t group = problem->num_qo_heads / problem->num_kv_heads;
+  if (!pa::decode_group_supported(group)) return PA_ERR_UNSUPPORTED;
+  if (!pa::decode_needs_cuda_cores(*problem))
+    return pa_default_schedule(device, problem->num_qo_heads, problem->num_kv_heads,
+                               problem->dtype, problem->flags, num_sms, ctas_per_sm);
+  int prev = 0;
+  cudaError_t e = cudaGetDevice(&prev);
+  if (e == cudaSuccess) e = cudaSetDevice(device);
+  int sms = 0;
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  int32_t k = 0;
+  if (e == cudaSuccess) e = cudaError_t(pa::decode_f32_ctas_per_sm(*problem, &k));
+  cudaSetDevice(prev);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  *num_sms = sms;
+  *ctas_per_sm = k;
+  return PA_OK;
+}
+
 }  // extern "C"

@@ -7,35 +7,51 @@
 // one dense problem per kv head — the B*G query rows of that head (G q heads
 // per kv head, head-query fusion) against the prefix's K and V — so it is
 // computed once as a tensor-core contraction instead of B times from HBM.
-// Its (o, lse) per prefix chunk are merged with the per-request suffix by
-// log-sum-exp in the level-2 decode kernel.
+// The prefix is cut into chunks across CTAs; a small merge kernel combines
+// each row's chunk states by log-sum-exp into one (o, lse), which the
+// level-2 decode kernel merges with the per-request suffix.
 //
-// CTA = (kv head h, 128-row query tile, prefix chunk); one CTA per SM.
-//   warp 4  (TMA):     Q tile once; K and V of each 64-key tile as page-row
-//                      boxes (the prefix is paged), 128-byte swizzle, into a
-//                      4-stage ring so three tiles are always in flight; rows
-//                      past the chunk are fetched out of range, which TMA fills
-//                      with zeros.
-//   warp 5  (MMA):     S = Q K^T into one of two TMEM buffers (M = 128, N = 64,
-//                      K = 128), then O += P V (V read as an MN-major operand)
-//                      into a third; completion is committed to mbarriers.
-//   warps 0-3 (rows):  thread i owns query row i = TMEM lane i: reads S with
-//                      tcgen05.ld, keeps a lazy running max (O is rescaled in
-//                      TMEM only when the max grows by more than 2^8), computes
-//                      P rounded to the input type while the tensor core runs
-//                      the previous P V, and writes it into one of two shared
-//                      buffers in the swizzled K-major layout; at the end it
-//                      normalises O.
+// CTA = (kv head h, 256 query rows as two halves of 128, prefix chunk); one
+// CTA per SM, 12 warps:
+//   warp 8  (TMA):     both halves of Q once; K and V of each 128-key tile as
+//                      page-row boxes (the prefix is paged), 128-byte swizzle,
+//                      K into a 3-stage ring and V into a 2-stage ring; boxes
+//                      past the chunk read out of range (zero fill).
+//   warp 9  (MMA):     one thread issues, in a fixed order, P V(half 0, t - 1)
+//                      then S(half 0, t) = Q K^T (M = 128, N = 128, K = 128),
+//                      then the same for half 1: the tensor core works on one
+//                      half while the other half's softmax runs.  P is read
+//                      from TMEM (A operand) and V is an MN-major operand in
+//                      shared memory.  S(half, t) overwrites the TMEM that
+//                      P V(half, t - 1) reads; it is issued right behind it on
+//                      the same thread, and one thread's tcgen05.mma execute in
+//                      issue order, so nothing waits for that P V to finish.
+//   warps 10-11:       idle (they complete the producer warpgroup, whose
+//                      registers go to the softmax warpgroups).
+//   warps 0-3, 4-7:    one warpgroup per half; thread i owns row i of its
+//                      half = TMEM lane i: reads S(t) with tcgen05.ld, masks
+//                      keys past the chunk, keeps a lazy running max (O is
+//                      rescaled in TMEM only when the max grows by more than
+//                      2^8; S(t) having completed means P V(t - 1) has too),
+//                      writes P in the input type over S with tcgen05.st, and
+//                      at the end normalises O into the chunk's fp32 state.
+//                      bf16 P is written as hi = bf16(p) and lo = bf16(p - hi)
+//                      in the two 64-column halves of the S columns, with one
+//                      P V for each, so the weights carry ~16 bits.
+// TMEM: half h owns columns [256 h, 256 h + 128) for S / P and the next 128
+// for O: all 512 columns.  The S barrier of a half completes once per tile
+// and once more after its last P V (the epilogue's signal).
 // Every mbarrier wait is bounded; on a timeout the kernel records it in the
-// workspace status word and unwinds instead of hanging.  Waits are by phase
-// parity, so every wait targets a barrier whose previous phase the waiting
-// thread has itself observed (a parity wait two phases behind would pass).
+// workspace status word and unwinds instead of hanging.  Every parity wait
+// targets a barrier whose previous phase the waiting thread has itself
+// observed.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "pa_internal.h"
@@ -45,29 +61,35 @@ namespace pa {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int kRows = 128;                  // query rows per tile (M)
-constexpr int kKeys = 64;                   // keys per tile
-constexpr int kThreads = 32 * 6;            // 4 row warps, 1 TMA warp, 1 MMA warp
+constexpr int kRows = 128;                  // rows of one MMA tile (M)
+constexpr int kHalves = 2;                  // MMA tiles per CTA, one softmax warpgroup each
+constexpr int kKeys = 128;                  // keys per K/V tile (N of S)
+constexpr int kThreads = 32 * 12;           // 8 softmax warps, TMA, MMA, 2 idle warps
+constexpr int kWarpTma = 8, kWarpMma = 9;
+// Register split per warpgroup (setmaxnreg): the block is launched with 168
+// registers a thread (384 x 168 = 64512); the producer warpgroup (TMA, MMA
+// and two idle warps) gives up to 56 so that each softmax thread can hold a
+// whole 128-key score row: 128 x 56 + 256 x 224 = 64512.
+constexpr int kRegsProducer = 56, kRegsSoftmax = 224;
+static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * 168, "register split");
 constexpr int kQHalf = kRows * 128;         // 128 rows x 64 16-bit columns (16 KB)
-constexpr int kKVHalf = kKeys * 128;        // 64 keys x 64 16-bit columns (8 KB)
-constexpr int kQBytes = 2 * kQHalf;         // Q tile: 128 rows x 128 head elements
-constexpr int kKVBytes = 2 * kKVHalf;       // K or V tile: 64 keys x 128 head elements
-constexpr int kPBytes = kRows * kKeys * 2;  // P tile: 128 rows x 64 keys (one 128-byte row each)
-constexpr int kStages = 4;                  // K/V ring depth: three tiles in flight
+constexpr int kKVHalf = kKeys * 128;        // 128 keys x 64 16-bit columns (16 KB)
+constexpr int kQBytes = 2 * kQHalf;         // one half of Q: 128 rows x 128 elements
+constexpr int kKVBytes = 2 * kKVHalf;       // one K or V tile
+constexpr int kKStages = 3, kVStages = 2;
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kStages * kKVBytes;
-constexpr int kOffP = kOffV + kStages * kKVBytes;  // two P buffers
-constexpr int kOffBar = kOffP + 2 * kPBytes;
-constexpr int kNumBars = 21;
+constexpr int kOffK = kOffQ + kHalves * kQBytes;
+constexpr int kOffV = kOffK + kKStages * kKVBytes;
+constexpr int kOffBar = kOffV + kVStages * kKVBytes;
+// mbarriers: Q; K full / empty; V full / empty; per half S done, P written
+constexpr int kBarQ = 0, kBarKFull = 1, kBarKEmpty = kBarKFull + kKStages,
+              kBarVFull = kBarKEmpty + kKStages, kBarVEmpty = kBarVFull + kVStages,
+              kBarS = kBarVEmpty + kVStages, kBarP = kBarS + kHalves,
+              kNumBars = kBarP + kHalves;
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 8 + 1024;  // + slack to align to 1 KB
-constexpr uint32_t kTmemCols = 256;         // S0 [0,64) S1 [64,128) O [128,256)
-constexpr uint32_t kColO = 128;
+constexpr uint32_t kTmemCols = 512;
 constexpr float kSlack = 8.f;
-
-// mbarrier slots
-constexpr int kBarQ = 0, kBarFullK = 1, kBarFullV = 5, kBarEmpty = 9, kBarS = 13, kBarSFree = 15,
-              kBarPReady = 17, kBarPFree = 19;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 struct CascadeArgs {
   const int32_t* prefix_indices;
@@ -75,7 +97,7 @@ struct CascadeArgs {
   float* prefix_lse;               // [chunks][B][Hq], base 2
   unsigned long long* status;      // timeout flag
   int32_t batch, num_qo_heads, group, page_size, log2_page, box_rows;
-  int32_t prefix_len, chunk_tokens, chunks, q_tiles;
+  int32_t prefix_len, chunks, row_pairs;
   int32_t oob_row;                 // a pool row past the end (TMA zero fill)
   float score_scale;               // sm_scale * log2(e)
 };
@@ -84,14 +106,7 @@ template <typename Tag> struct Fmt;
 template <> struct Fmt<F16> { static constexpr int v = 0; };
 template <> struct Fmt<BF16> { static constexpr int v = 1; };
 
-// Round two fp32 to the 16-bit input type, packed; returns them widened again.
-__device__ __forceinline__ uint32_t pack2(F16, float a, float b, float& ra, float& rb) {
-  const __half2 h = __floats2half2_rn(a, b);
-  const float2 f = __half22float2(h);
-  ra = f.x;
-  rb = f.y;
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
+// Round two fp32 to bf16, packed; returns them widened again (the hi / lo split).
 __device__ __forceinline__ uint32_t pack2(BF16, float a, float b, float& ra, float& rb) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
@@ -102,11 +117,46 @@ __device__ __forceinline__ uint32_t pack2(BF16, float a, float b, float& ra, flo
 
 __device__ __forceinline__ void flag_timeout(const CascadeArgs& a) { atomicOr(a.status, 1ull); }
 
+// 2^x on the FMA pipe, for part of the exponentials so that the MUFU unit
+// (16 per clock per SM) is not the softmax's only bound.  x is split as
+// n + f with n = round(x) (the 1.5 * 2^23 shifter leaves n in the low bits of
+// t) and f in [-0.5, 0.5]; 2^f is a polynomial whose coefficients are a Remez
+// fit of relative error on that interval, computed for this kernel: degree 3
+// (error 7.5e-5, below an fp16 P's rounding) or degree 4 (2.7e-6, for the
+// two-term bf16 P); 2^n is added to the exponent field.  x is clamped to
+// -125 so the exponent stays normal: such p are < 2^-124 and round to 0 in
+// fp16 (they are 1e-38 in a bf16 P: nothing next to the other weights).
+template <int kDeg>
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float p;
+  if constexpr (kDeg == 3) {
+    p = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111251115799f), f, 0.6932609677314758f), f,
+             0.9999280571937561f);
+  } else {
+    p = fmaf(fmaf(fmaf(fmaf(0.009570102207362652f, f, 0.05591785907745361f), f,
+                       0.240247443318367f),
+                  f, 0.6931217908859253f),
+             f, 0.9999992847442627f);
+  }
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Key tiles [t0, t1) of chunk c: the prefix's 128-key tiles split as evenly
+// as possible over the chunks.
+__device__ __forceinline__ void chunk_tiles(int c, int chunks, int ktiles, int& t0, int& t1) {
+  t0 = int((int64_t(c) * ktiles) / chunks);
+  t1 = int((int64_t(c + 1) * ktiles) / chunks);
+}
+
 template <typename Tag>
 __global__ void __launch_bounds__(kThreads, 1)
     cascade_prefix_kernel(const __grid_constant__ CUtensorMap tmap_q,
                           const __grid_constant__ CUtensorMap tmap_k,
                           const __grid_constant__ CUtensorMap tmap_v, const CascadeArgs a) {
+  constexpr bool kSplit = std::is_same<Tag, BF16>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -116,29 +166,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.group;
-  const int mt = blockIdx.x % a.q_tiles;
-  const int rest = blockIdx.x / a.q_tiles;
+  const int rp = blockIdx.x % a.row_pairs;
+  const int rest = blockIdx.x / a.row_pairs;
   const int chunk = rest % a.chunks;
   const int h = rest / a.chunks;
-  const int k0 = chunk * a.chunk_tokens;
-  const int k1 = min(k0 + a.chunk_tokens, a.prefix_len);
-  const int ntiles = (k1 - k0 + kKeys - 1) / kKeys;
+  const int ktiles = (a.prefix_len + kKeys - 1) / kKeys;
+  int t0, t1;
+  chunk_tiles(chunk, a.chunks, ktiles, t0, t1);
+  const int k0 = t0 * kKeys;
+  const int k1 = min(t1 * kKeys, a.prefix_len);
+  const int nt = t1 - t0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kBarFullK + s), 1);
-      mbar_init(bar(kBarFullV + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kBarS + s), 1);
-      mbar_init(bar(kBarSFree + s), 4);
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
     }
-    mbar_init(bar(kBarPReady), 4);
-    mbar_init(bar(kBarPReady + 1), 4);
-    mbar_init(bar(kBarPFree), 1);
-    mbar_init(bar(kBarPFree + 1), 1);
+    for (int hf = 0; hf < kHalves; ++hf) {
+      mbar_init(bar(kBarS + hf), 1);
+      mbar_init(bar(kBarP + hf), 4);
+    }
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -150,212 +202,274 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp >= 8) {
+   // ------------------------- producer warpgroup -------------------------
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsProducer) : "memory");
+   if (warp == kWarpTma) {
     // ------------------------------ TMA producer ------------------------------
-    // Lane j owns box j of every tile (a page, or a 64-row part of one): it
+    // Lane j owns box j of every tile (a page, or a 128-row part of one): it
     // reads that page's index one tile ahead and issues the box's copies.
     const int box = a.box_rows, pmask = a.page_size - 1;
     const int nbox = kKeys / box;
     auto row_of = [&](int kt) -> int {
       const int key = k0 + kt * kKeys + lane * box;
-      if (lane >= nbox || kt >= ntiles) return 0;
+      if (lane >= nbox || kt >= nt) return 0;
       return key < k1 ? __ldg(a.prefix_indices + (key >> a.log2_page)) * a.page_size +
                             (key & pmask)
                       : a.oob_row;
     };
     if (lane == 0) {
       const int rows_per_b = kRows / G;
-      mbar_arrive_expect_tx(bar(kBarQ), kQBytes);
-      tc::tma_load_3d(sb + kOffQ, &tmap_q, 0, h * G, mt * rows_per_b, bar(kBarQ));
-      tc::tma_load_3d(sb + kOffQ + kQHalf, &tmap_q, 64, h * G, mt * rows_per_b, bar(kBarQ));
-    }
-    int rowA = row_of(0), rowB = row_of(1);  // unrolled by two: no copy of a pending load
-    auto produce = [&](int kt, int row) -> bool {
-      const int s = kt % kStages;
-      if (kt >= kStages && !mbar_wait(bar(kBarEmpty + s), ((kt / kStages) - 1) & 1)) return false;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(kBarFullK + s), kKVBytes);
-        mbar_arrive_expect_tx(bar(kBarFullV + s), kKVBytes);
+      mbar_arrive_expect_tx(bar(kBarQ), kHalves * kQBytes);
+      for (int hf = 0; hf < kHalves; ++hf) {
+        const uint32_t dq = sb + kOffQ + hf * kQBytes;
+        const int z = (rp * kHalves + hf) * rows_per_b;
+        tc::tma_load_3d(dq, &tmap_q, 0, h * G, z, bar(kBarQ));
+        tc::tma_load_3d(dq + kQHalf, &tmap_q, 64, h * G, z, bar(kBarQ));
       }
+    }
+    auto load_tile = [&](const CUtensorMap* map, uint32_t dst, int row, uint32_t full) {
+      if (lane == 0) mbar_arrive_expect_tx(full, kKVBytes);
       __syncwarp();
       if (lane < nbox) {
-        const uint32_t dk = sb + kOffK + s * kKVBytes + lane * box * 128;
-        const uint32_t dv = sb + kOffV + s * kKVBytes + lane * box * 128;
-        tc::tma_load_3d(dk, &tmap_k, 0, h, row, bar(kBarFullK + s));
-        tc::tma_load_3d(dk + kKVHalf, &tmap_k, 64, h, row, bar(kBarFullK + s));
-        tc::tma_load_3d(dv, &tmap_v, 0, h, row, bar(kBarFullV + s));
-        tc::tma_load_3d(dv + kKVHalf, &tmap_v, 64, h, row, bar(kBarFullV + s));
+        tc::tma_load_3d(dst + lane * box * 128, map, 0, h, row, full);
+        tc::tma_load_3d(dst + kKVHalf + lane * box * 128, map, 64, h, row, full);
       }
-      return true;
     };
+    // Order: K(0), then K(t + 1) ahead of V(t), so the keys the next S needs
+    // are never held up behind a V stage still in use.  V(t) reads the rows
+    // K(t) read (kept in rv0 / rv1 by tile parity).
+    int rnext = row_of(0);
+    int rv0 = 0, rv1 = 0;
     bool ok = true;
-    for (int kt = 0; ok && kt < ntiles; kt += 2) {
-      ok = produce(kt, rowA);
-      rowA = row_of(kt + 2);
-      if (ok && kt + 1 < ntiles) {
-        ok = produce(kt + 1, rowB);
-        rowB = row_of(kt + 3);
+    for (int kt = -1; kt < nt; ++kt) {
+      const int kn = kt + 1;  // the K tile issued this step
+      if (kn < nt) {
+        const int s = kn % kKStages;
+        if (kn >= kKStages) ok = mbar_wait(bar(kBarKEmpty + s), ((kn / kKStages) - 1) & 1);
+        if (!ok) break;
+        load_tile(&tmap_k, sb + kOffK + s * kKVBytes, rnext, bar(kBarKFull + s));
+        if (kn & 1) rv1 = rnext;
+        else rv0 = rnext;
+        rnext = row_of(kn + 1);
+      }
+      if (kt >= 0) {
+        const int s = kt % kVStages;
+        if (kt >= kVStages) ok = mbar_wait(bar(kBarVEmpty + s), ((kt / kVStages) - 1) & 1);
+        if (!ok) break;
+        load_tile(&tmap_v, sb + kOffV + s * kKVBytes, (kt & 1) ? rv1 : rv0, bar(kBarVFull + s));
       }
     }
     if (!ok && lane == 0) flag_timeout(a);
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ------------------------------ MMA issuer ------------------------------
-    // S of the next tile and P V of the current one are issued as soon as
-    // their inputs are ready, whichever comes first.
     if (lane == 0) {
       constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
       constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
       // descriptors are built once; a k-step adds its byte offset / 16
-      const uint64_t dq = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
+      const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
       const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffK, 16, 1024);
       const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffV, kKVHalf, 1024);
-      const uint64_t dp0 = tc::smem_desc_sw128(sb + kOffP, 16, 1024);
-      bool ok = mbar_wait(bar(kBarQ), 0);
-      int ns = 0, npv = 0;
-      uint32_t idle = 0;
-      while (ok && npv < ntiles) {
-        bool progress = false;
-        // S(ns) into buffer ns & 1, free once softmax has read S(ns - 2)
-        if (ns < ntiles && ns <= npv + 2 &&
-            (ns < 2 || mbar_try_wait(bar(kBarSFree + (ns & 1)), ((ns - 2) >> 1) & 1)) &&
-            mbar_try_wait(bar(kBarFullK + ns % kStages), (ns / kStages) & 1)) {
-          tc::fence_after_sync();
-          const uint64_t kd = dk0 + ((ns % kStages) * kKVBytes >> 4);
+      auto issue_s = [&](int hf, int kt) {
+        const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
+        const uint64_t kd = dk0 + (((kt % kKStages) * kKVBytes) >> 4);
+        const uint32_t dst = tmem + hf * 256;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-            const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
-            tc::mma_f16_ss(tmem + (ns & 1) * kKeys, dq + off, kd + koff, kIdescQK, kk > 0);
-          }
-          tc::commit(bar(kBarS + (ns & 1)));
-          ++ns;
-          progress = true;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+          const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+          tc::mma_f16_ss(dst, qd + off, kd + koff, kIdescQK, kk > 0);
         }
-        // O += P(npv) V(npv)
-        if (npv < ns && mbar_try_wait(bar(kBarPReady + (npv & 1)), (npv >> 1) & 1) &&
-            mbar_try_wait(bar(kBarFullV + npv % kStages), (npv / kStages) & 1)) {
-          tc::fence_after_sync();
-          const int s = npv % kStages;
-          const uint64_t pd = dp0 + (((npv & 1) * kPBytes) >> 4);
-          const uint64_t vd = dv0 + ((s * kKVBytes) >> 4);
+        tc::commit(bar(kBarS + hf));
+      };
+      auto issue_pv = [&](int hf, int v) {
+        const uint32_t pt = tmem + hf * 256;            // P over S(v)
+        const uint32_t dst = tmem + hf * 256 + 128;     // O of the half
+        const uint64_t vd = dv0 + (((v % kVStages) * kKVBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          tc::mma_f16_ts(dst, pt + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                         (v > 0 || kk > 0) ? 1u : 0u);
+        if (kSplit) {  // the lo term in the other 64 columns
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk)
-            tc::mma_f16_ss(tmem + kColO, pd + ((kk * 32) >> 4), vd + ((kk * 16 * 128) >> 4),
-                           kIdescPV, (npv > 0 || kk > 0) ? 1u : 0u);
-          tc::commit(bar(kBarPFree + (npv & 1)));
-          tc::commit(bar(kBarEmpty + s));
-          ++npv;
-          progress = true;
+            tc::mma_f16_ts(dst, pt + 64 + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
         }
-        idle = progress ? 0u : idle + 1u;
-        if (idle > kSpinLimit) ok = false;
+      };
+      bool ok = mbar_wait(bar(kBarQ), 0);
+      // Fixed order per tile t: for each half, P V(t - 1) then S(t).  The
+      // softmax of a half always finds its next S queued behind the other
+      // half's work.
+      for (int kt = 0; ok && kt <= nt; ++kt) {
+        for (int hf = 0; ok && hf < kHalves; ++hf) {
+          if (kt > 0) {
+            const int v = kt - 1;
+            if (hf == 0) ok = mbar_wait(bar(kBarVFull + v % kVStages), (v / kVStages) & 1);
+            if (ok) ok = mbar_wait(bar(kBarP + hf), v & 1);
+            if (!ok) break;
+            tc::fence_after_sync();
+            issue_pv(hf, v);
+            if (hf == kHalves - 1) tc::commit(bar(kBarVEmpty + v % kVStages));
+          }
+          if (kt < nt) {
+            if (hf == 0) ok = mbar_wait(bar(kBarKFull + kt % kKStages), (kt / kKStages) & 1);
+            if (!ok) break;
+            tc::fence_after_sync();
+            issue_s(hf, kt);  // its commit also signals that P V(kt - 1) is done
+            if (hf == kHalves - 1) tc::commit(bar(kBarKEmpty + kt % kKStages));
+          } else {
+            tc::commit(bar(kBarS + hf));  // the last P V of the half is done
+          }
+        }
       }
       if (!ok) flag_timeout(a);
     }
+   }
   } else {
     // ------------------------- softmax / epilogue rows -------------------------
-    const int i = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t lane_addr = tmem + (uint32_t(warp * 32) << 16);
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax) : "memory");
+    const int hf = warp >> 2;              // which half (warpgroup)
+    const int i = threadIdx.x & 127;       // row within the half == TMEM lane
+    const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16);
+    const uint32_t col_s = hf * 256, col_o = hf * 256 + 128;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int kt = 0; kt < ntiles; ++kt) {
-      const int s = kt & 1;  // S buffer
-      ok = mbar_wait(bar(kBarS + s), (kt >> 1) & 1);
+    for (int kt = 0; kt < nt; ++kt) {
+      ok = mbar_wait(bar(kBarS + hf), kt & 1);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::fence_after_sync();
       float x[kKeys];
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
         float t32[32];
-        tc::tmem_ld32(lane_addr + s * kKeys + 32 * c, t32);
+        tc::tmem_ld32(lane_addr + col_s + 32 * c, t32);
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[32 * c + e] = t32[e];
       }
       tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarSFree + s));
-
       // Raw scores; the scale is folded into the exponent argument below.
       const int valid = min(kKeys, k1 - (k0 + kt * kKeys));
-      if (valid < kKeys) {  // ragged last tile of the chunk (uniform branch)
+      const bool ragged = valid < kKeys;  // last tile of the chunk (uniform branch)
+      if (ragged) {
 #pragma unroll
         for (int c = 0; c < kKeys; ++c)
           if (c >= valid) x[c] = -INFINITY;
       }
-      float tm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // P = 2^(s * scale - m) in the input type, written over S in TMEM 32
+      // keys at a time; l sums p in fp32 (for fp16 P the weights the tensor
+      // core applies are within 2^-11 of these, so o moves by at most that
+      // fraction of its size).  Past the first tile the exponents are taken
+      // against the current reference while the tile maximum is found (no
+      // wait for the maximum); in the rare tile whose maximum beats the
+      // reference by more than 2^8 they are taken again with the new one.
+      auto write_p = [&](float mref, bool poly) -> float {
+        const float nm = -mref;
+        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) tm4[c & 3] = fmaxf(tm4[c & 3], x[c]);
-      const float tmax = fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3])) * a.score_scale;
-      const bool moved = tmax > m + kSlack;
-      const float mnew = moved ? tmax : m;
-      const float alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
-      // P = 2^(s * scale - m), rounded to the input type (l sums exactly what
-      // the MMA sees), computed before waiting on the tensor core.
-      const float nm = -mnew;
-      uint32_t w[kKeys / 2];
-      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c16 = 0; c16 < kKeys / 32; ++c16) {
+          uint32_t w[16], wl[16];
 #pragma unroll
-      for (int e = 0; e < kKeys / 2; ++e) {
-        const float p0 = fast_exp2(fmaf(x[2 * e], a.score_scale, nm));
-        const float p1 = fast_exp2(fmaf(x[2 * e + 1], a.score_scale, nm));
-        float r0, r1;
-        w[e] = pack2(Tag{}, p0, p1, r0, r1);
-        ps4[e & 3] += r0 + r1;
-      }
-      const float psum = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
-      l = l * alpha + psum;
-      m = mnew;
-      // O is rescaled in TMEM once the previous tile's PV is complete.  That is
-      // waited for on the P buffer it read: this thread already saw that
-      // barrier's previous phase (PV of tile kt - 3), so its parity is exact.
-      if (kt > 0 && __any_sync(0xffffffffu, moved)) {
-        ok = mbar_wait(bar(kBarPFree + ((kt - 1) & 1)), ((kt - 1) >> 1) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc::fence_after_sync();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float ov[32];
-          tc::tmem_ld32(lane_addr + kColO + 32 * c, ov);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-          tc::tmem_st32(lane_addr + kColO + 32 * c, ov);
+          for (int e = 0; e < 16; ++e) {
+            const int c = 32 * c16 + 2 * e;
+            const float a0 = fmaf(x[c], a.score_scale, nm), a1 = fmaf(x[c + 1], a.score_scale, nm);
+            float p0, p1;
+            if (poly && (e & 3) < 2) {  // half of the pairs on the FMA pipe
+              p0 = exp2_poly<kSplit ? 4 : 3>(a0);
+              p1 = exp2_poly<kSplit ? 4 : 3>(a1);
+            } else {
+              p0 = fast_exp2(a0);
+              p1 = fast_exp2(a1);
+            }
+            float r0, r1;
+            if constexpr (kSplit) {  // hi + lo carries p to ~2^-16
+              w[e] = pack2(Tag{}, p0, p1, r0, r1);
+              float q0, q1;
+              wl[e] = pack2(Tag{}, p0 - r0, p1 - r1, q0, q1);
+            } else {
+              const __half2 hp = __floats2half2_rn(p0, p1);
+              w[e] = *reinterpret_cast<const uint32_t*>(&hp);
+            }
+            ps4[e & 3] += p0 + p1;
+          }
+          tc::tmem_st16(lane_addr + col_s + 16 * c16, w);
+          if constexpr (kSplit) tc::tmem_st16(lane_addr + col_s + 64 + 16 * c16, wl);
         }
-        tc::tmem_wait_st();
-      }
-      // This tile's P buffer was last read by the PV of tile kt - 2.
-      if (kt >= 2) {
-        ok = mbar_wait(bar(kBarPFree + (kt & 1)), ((kt - 2) >> 1) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      uint8_t* prow = smem + kOffP + (kt & 1) * kPBytes + i * 128;
+        return (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+      };
+      auto tile_max = [&]() {
+        float tm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c8 = 0; c8 < kKeys / 8; ++c8)  // 16-byte chunk c8 of the 128-byte row
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (i & 7)) << 4)) =
-            make_uint4(w[4 * c8], w[4 * c8 + 1], w[4 * c8 + 2], w[4 * c8 + 3]);
-      fence_proxy_async_smem();
+        for (int c = 0; c < kKeys; ++c) tm4[c & 3] = fmaxf(tm4[c & 3], x[c]);
+        return fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3])) * a.score_scale;
+      };
+      float psum, alpha = 1.f;
+      if (kt == 0 || ragged) {
+        const float tmax = tile_max();
+        const bool moved = tmax > m + kSlack;
+        const float mnew = moved ? tmax : m;
+        alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
+        if (kt > 0 && __any_sync(0xffffffffu, moved)) {
+          // O holds every earlier tile: S(kt) completing means P V(kt - 1) has
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
+          }
+        }
+        psum = write_p(mnew, false);
+        m = mnew;
+      } else {
+        psum = write_p(m, true);
+        const float tmax = tile_max();
+        const bool moved = tmax > m + kSlack;
+        if (__any_sync(0xffffffffu, moved)) {
+          const float mnew = moved ? tmax : m;
+          alpha = moved ? fast_exp2(m - mnew) : 1.f;
+          tc::tmem_wait_st();  // the first P writes are done before they are replaced
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
+          }
+          psum = write_p(mnew, true);
+          m = mnew;
+        }
+      }
+      l = l * alpha + psum;
+      tc::tmem_wait_st();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarPReady + (kt & 1)));
+      if (lane == 0) mbar_arrive(bar(kBarP + hf));
     }
-    // epilogue: O / l of this row, and the row's lse (base 2)
-    if (ok && ntiles > 0) ok = mbar_wait(bar(kBarPFree + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1);
+    // epilogue: the half's last P V has completed (its extra S commit)
+    if (ok && nt > 0) ok = mbar_wait(bar(kBarS + hf), nt & 1);
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (!all_ok && lane == 0) flag_timeout(a);
     if (all_ok) {
       tc::fence_after_sync();
-      const int r = mt * kRows + i;
+      const int r = (rp * kHalves + hf) * kRows + i;
       const int rows = a.batch * G;
       const int b = r / G, j = r - (r / G) * G;
-      float* dst = a.prefix_o +
-                   ((int64_t(chunk) * a.batch + b) * a.num_qo_heads + h * G + j) * D;
+      float* dst = a.prefix_o + ((int64_t(chunk) * a.batch + b) * a.num_qo_heads + h * G + j) * D;
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float ov[32];
-        tc::tmem_ld32(lane_addr + kColO + 32 * c, ov);
-        tc::tmem_wait_ld();
+        if (nt > 0) {
+          tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
+          tc::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = 0.f;
+        }
         if (r < rows) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
@@ -375,6 +489,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+// Merge the prefix chunks of every (request, q head) row by log-sum-exp into
+// chunk slot 0 (base-2 lse), one warp per row, 4 head elements per lane.
+// Each warp reads all chunks of its row before writing slot 0.
+__global__ void __launch_bounds__(256) cascade_merge_kernel(float* prefix_o, float* prefix_lse,
+                                                            int64_t rows, int chunks) {
+  const int64_t row = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float M = -INFINITY, L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = 0; c < chunks; ++c) {
+    const float lse = prefix_lse[int64_t(c) * rows + row];
+    const float4 o = *reinterpret_cast<const float4*>(prefix_o + (int64_t(c) * rows + row) * D +
+                                                      4 * lane);
+    if (lse == -INFINITY) continue;
+    if (lse > M) {
+      const float s = fast_exp2(M - lse);  // M = -inf -> 0
+      L = L * s + 1.f;
+      acc = make_float4(acc.x * s + o.x, acc.y * s + o.y, acc.z * s + o.z, acc.w * s + o.w);
+      M = lse;
+    } else {
+      const float w = fast_exp2(lse - M);
+      L += w;
+      acc = make_float4(acc.x + w * o.x, acc.y + w * o.y, acc.z + w * o.z, acc.w + w * o.w);
+    }
+  }
+  const float inv = M == -INFINITY ? 0.f : 1.f / L;
+  __syncwarp();  // every lane has read slot 0 of this row
+  *reinterpret_cast<float4*>(prefix_o + row * D + 4 * lane) =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (lane == 0) prefix_lse[row] = M == -INFINITY ? -INFINITY : M + fast_log2(L);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -389,7 +536,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D map over (dim0 = 128 head elements, dim1, dim2) with 128-byte swizzle.
+// 3-D map over (dim0 = 128 head elements, dim1, dim2) with 128-byte swizzle;
+// boxes of 64 x box1 x box2 elements.
 bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t d1,
               uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box1, uint32_t box2) {
   auto fn = encode_fn();
@@ -454,15 +602,19 @@ int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* str
   a.log2_page = plan.log2_page;
   a.box_rows = box_rows;
   a.prefix_len = plan.prefix_len;
-  a.chunk_tokens = plan.prefix_chunk_tokens;
   a.chunks = plan.prefix_chunks;
-  a.q_tiles = plan.q_tiles;
+  a.row_pairs = plan.q_tiles;
   a.oob_row = int32_t(pool_rows);  // one past the last row: TMA fills the box with zeros
   a.score_scale = pr.sm_scale * kLog2e;
   const int grid = pr.num_kv_heads * plan.q_tiles * plan.prefix_chunks;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return int(pr.dtype == PA_BF16 ? launch_t<BF16>(a, tq, tk, tv, grid, s)
-                                 : launch_t<F16>(a, tq, tk, tv, grid, s));
+  cudaError_t e = pr.dtype == PA_BF16 ? launch_t<BF16>(a, tq, tk, tv, grid, s)
+                                      : launch_t<F16>(a, tq, tk, tv, grid, s);
+  if (e != cudaSuccess || plan.prefix_chunks == 1) return int(e);
+  const int64_t rows = int64_t(pr.batch) * pr.num_qo_heads;
+  cascade_merge_kernel<<<unsigned((rows + 7) / 8), 256, 0, s>>>(a.prefix_o, a.prefix_lse, rows,
+                                                                 plan.prefix_chunks);
+  return int(cudaGetLastError());
 }
 
 }  // namespace pa

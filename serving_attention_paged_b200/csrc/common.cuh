@@ -73,6 +73,13 @@ __device__ __forceinline__ void cp_async16_imm(uint32_t smem_addr, uint64_t gadd
                "l"(gaddr), "r"(src_bytes), "n"(kDst), "n"(kSrc)
                : "memory");
 }
+// 8-byte form (cp.async.cg takes only 16 bytes; .ca also allocates in L1).
+template <int kDst, int kSrc = kDst>
+__device__ __forceinline__ void cp_async8_imm(uint32_t smem_addr, uint64_t gaddr, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0+%3], [%1+%4], 8, %2;\n" ::"r"(smem_addr),
+               "l"(gaddr), "r"(src_bytes), "n"(kDst), "n"(kSrc)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }

@@ -780,7 +780,8 @@ int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream) 
   a.num_qo_heads = pr.num_qo_heads;
   a.num_kv_heads = pr.num_kv_heads;
   a.log2_page = plan.log2_page;
-  a.prefix_chunks = plan.cascade ? plan.prefix_chunks : 0;
+  // the prefix level leaves each row's merged prefix state in chunk slot 0
+  a.prefix_chunks = plan.cascade && plan.prefix_chunks > 0 ? 1 : 0;
   a.score_scale = pr.sm_scale * kLog2e;
   const bool check = (pr.flags & PA_FLAG_CHECK_INDICES) != 0;
   const int64_t n = int64_t(plan.cta_indptr.size()) - 1;

@@ -24,17 +24,20 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 //   prefill_tiles [n_tiles]            pa_prefill_tile (prefill plans only)
 //   cta_indptr   [n_cta + 1]           int32, pieces of CTA i
 //   merge_indptr [B * Hkv + 1]         int32, partial slots of segment (b, h)
+//   kv_len       [B]                   int32, tokens per request (rotary plans only:
+//                                      the query's position is kv_len - 1)
 //   counters     [B * Hkv * kCounterSlots]  int32, zero between runs (decode levels only)
 //   error        [2]                   uint64: first bad kv_indices position (~0 = none),
 //                                      then a timeout flag (0 = none)
 //   partial_o    [n_partials, G, D]    fp32, outputs of pieces of split segments
 //                                      (normalised; G = q heads of the kv head)
 //   partial_lse  [n_partials, G]       fp32, their log-sum-exp in base 2
-//   prefix_o     [prefix_chunks, B, Hq, D]  fp32 (cascade only)
+//   prefix_o     [prefix_chunks, B, Hq, D]  fp32 (cascade only); after the
+//                                      prefix level, chunk 0 holds the merged state
 //   prefix_lse   [prefix_chunks, B, Hq]     fp32, base 2 (cascade only)
 struct WorkspaceLayout {
-  size_t items = 0, prefill_tiles = 0, cta_indptr = 0, merge_indptr = 0, counters = 0, error = 0,
-         partial_o = 0, partial_lse = 0, prefix_o = 0, prefix_lse = 0, total = 0;
+  size_t items = 0, prefill_tiles = 0, cta_indptr = 0, merge_indptr = 0, kv_len = 0, counters = 0,
+         error = 0, partial_o = 0, partial_lse = 0, prefix_o = 0, prefix_lse = 0, total = 0;
 };
 
 }  // namespace pa
@@ -53,8 +56,8 @@ struct pa_plan_s {
   bool cascade = false;
   int32_t prefix_len = 0;
   int32_t prefix_chunks = 0;        // split of the prefix across CTAs
-  int32_t prefix_chunk_tokens = 0;  // tokens per chunk (multiple of the 128-key tile)
-  int32_t q_tiles = 0;              // 128-row tiles over the B * G query rows of one kv head
+  int32_t prefix_chunk_tokens = 0;  // tokens of the largest chunk (whole 128-key tiles)
+  int32_t q_tiles = 0;              // 256-row CTA tiles over the B * G query rows of one kv head
   // prefill / append (pa_prefill_plan_create): query tiles, longest first
   bool prefill = false;
   int64_t total_q = 0;
@@ -82,7 +85,18 @@ struct RunPointers {
   uint8_t* ws;
 };
 
+// 8-bit (FP8) KV cache; rotary positions on the fly.  Both run on the
+// CUDA-core decode kernel only.
+inline bool kv_is_8bit(const pa_problem& p) {
+  return p.kv_dtype == PA_E4M3 || p.kv_dtype == PA_E5M2;
+}
+inline bool decode_needs_cuda_cores(const pa_problem& p) {
+  return kv_is_8bit(p) || p.rope_theta > 0.f;
+}
+
 int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream);
+// Resident CTAs per SM of the fp32-path kernel (8-bit pools, rotary) a problem runs.
+int decode_f32_ctas_per_sm(const pa_problem& p, int32_t* out);
 int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream);
 bool decode_tc_supported(int32_t group, pa_dtype dtype);
 int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out);
@@ -92,7 +106,9 @@ int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out);
 // faster, the padded MMA buying nothing once HBM is the bound.
 inline bool decode_uses_tensor_cores(const pa_problem& p) {
   const int32_t group = p.num_qo_heads / p.num_kv_heads;
-  if (!decode_tc_supported(group, p.dtype) || (p.flags & PA_FLAG_CUDA_CORES)) return false;
+  if (!decode_tc_supported(group, p.dtype) || (p.flags & PA_FLAG_CUDA_CORES) ||
+      decode_needs_cuda_cores(p))
+    return false;
   return (p.flags & PA_FLAG_TENSOR_CORES) || group >= 8;
 }
 // Plan cost of a piece boundary, in tokens of the kernel's steady-state rate.

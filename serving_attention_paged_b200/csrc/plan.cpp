@@ -10,6 +10,7 @@
 // tokens, one CTA per kv head.  Host code only: no CUDA call.
 #include <algorithm>
 #include <array>
+#include <cmath>
 #include <cstring>
 #include <new>
 
@@ -36,6 +37,16 @@ pa_status validate_problem(const pa_problem* p) {
   if (p->num_qo_heads % p->num_kv_heads) return PA_ERR_INVALID_ARG;
   if (!(p->sm_scale == p->sm_scale)) return PA_ERR_INVALID_ARG;  // NaN
   if (p->dtype != PA_F16 && p->dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (p->kv_dtype != PA_F16 && p->kv_dtype != PA_BF16 && !pa::kv_is_8bit(*p))
+    return PA_ERR_INVALID_ARG;
+  if (pa::kv_is_8bit(*p) && !(std::isfinite(p->k_scale) && p->k_scale > 0.f &&
+                              std::isfinite(p->v_scale) && p->v_scale > 0.f))
+    return PA_ERR_INVALID_ARG;
+  if (!(std::isfinite(p->rope_theta) && p->rope_theta >= 0.f)) return PA_ERR_INVALID_ARG;
+  // 8-bit caches and rotary positions are built for the CUDA-core decode kernel
+  if (pa::decode_needs_cuda_cores(*p) && (p->flags & PA_FLAG_TENSOR_CORES) &&
+      !(p->flags & PA_FLAG_CUDA_CORES))
+    return PA_ERR_UNSUPPORTED;
   if (p->head_dim != pa::kHeadDim) return PA_ERR_UNSUPPORTED;
   if (!is_pow2(p->page_size) || p->page_size > 1024) return PA_ERR_UNSUPPORTED;
   if (!pa::decode_group_supported(p->num_qo_heads / p->num_kv_heads)) return PA_ERR_UNSUPPORTED;
@@ -57,6 +68,8 @@ pa_status build(pa_plan_s* plan, const int32_t* indptr, const int32_t* last) {
     if (n > 0 && (last[b] < 1 || last[b] > P)) return PA_ERR_INVALID_ARG;
     L[b] = n > 0 ? (n - 1) * P + last[b] : 0;
     if (L[b] > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    // rotary positions are formed as exact fp32 integers in the kernel
+    if (p.rope_theta > 0.f && L[b] > (int64_t(1) << 24)) return PA_ERR_UNSUPPORTED;
     total += L[b];
   }
   if (indptr) plan->kv_indptr.assign(indptr, indptr + B + 1);
@@ -175,6 +188,7 @@ void layout_workspace(pa_plan_s* plan) {
   w.prefill_tiles = take(plan->prefill_tiles.size() * sizeof(pa_prefill_tile));
   w.cta_indptr = take(plan->cta_indptr.size() * sizeof(int32_t));
   w.merge_indptr = take(plan->merge_indptr.size() * sizeof(int32_t));
+  w.kv_len = take(p.rope_theta > 0.f && !plan->prefill ? B * sizeof(int32_t) : 0);
   w.counters = take(plan->prefill ? 0 : B * p.num_kv_heads * pa::kCounterSlots * sizeof(int32_t));
   w.error = take(2 * sizeof(uint64_t));  // first bad index, timeout flag
   const size_t G = plan->group;
@@ -198,16 +212,26 @@ void build_upload_image(pa_plan_s* plan) {
               plan->cta_indptr.size() * sizeof(int32_t));
   std::memcpy(img.data() + w.merge_indptr, plan->merge_indptr.data(),
               plan->merge_indptr.size() * sizeof(int32_t));
+  if (plan->prob.rope_theta > 0.f && !plan->prefill) {
+    const pa_problem& p = plan->prob;
+    for (int32_t b = 0; b < p.batch; ++b) {
+      const int64_t n = int64_t(plan->kv_indptr[b + 1]) - plan->kv_indptr[b];
+      const int32_t L = n > 0 ? int32_t((n - 1) * p.page_size + plan->last_page_len[b]) : 0;
+      std::memcpy(img.data() + w.kv_len + b * sizeof(int32_t), &L, sizeof L);
+    }
+  }
   std::memset(img.data() + w.error, 0xff, sizeof(uint64_t));  // first bad index: none
 }
 
-// Level-1 cascade schedule: (kv head, 128-row query tile, prefix chunk) tiles,
-// about one per SM; each chunk a whole number of 128-key tiles.
+// Level-1 cascade schedule: (kv head, pair of 128-row query tiles, prefix
+// chunk) CTAs, about one per SM; the prefix's 128-key tiles are split as
+// evenly as possible over the chunks (the largest chunk has ceil(tiles /
+// chunks) of them).
 void schedule_prefix(pa_plan_s* plan) {
   const pa_problem& p = plan->prob;
-  constexpr int64_t kTileKeys = 128, kTileRows = 128;
+  constexpr int64_t kTileKeys = 128, kRowsPerCta = 256;
   const int64_t rows = int64_t(p.batch) * plan->group;
-  plan->q_tiles = int32_t(std::max<int64_t>(1, ceil_div(rows, kTileRows)));
+  plan->q_tiles = int32_t(std::max<int64_t>(1, ceil_div(rows, kRowsPerCta)));
   const int64_t key_tiles = ceil_div(plan->prefix_len, kTileKeys);
   if (plan->prefix_len == 0 || p.batch == 0) {
     plan->prefix_chunks = 0;
@@ -215,11 +239,9 @@ void schedule_prefix(pa_plan_s* plan) {
     return;
   }
   const int64_t base = int64_t(p.num_kv_heads) * plan->q_tiles;
-  int64_t chunks = std::max<int64_t>(1, std::min<int64_t>(int64_t(p.num_sms) / base, key_tiles));
-  const int64_t tiles_per_chunk = ceil_div(key_tiles, chunks);
-  chunks = ceil_div(key_tiles, tiles_per_chunk);
+  const int64_t chunks = std::max<int64_t>(1, std::min<int64_t>(int64_t(p.num_sms) / base, key_tiles));
   plan->prefix_chunks = int32_t(chunks);
-  plan->prefix_chunk_tokens = int32_t(tiles_per_chunk * kTileKeys);
+  plan->prefix_chunk_tokens = int32_t(ceil_div(key_tiles, chunks) * kTileKeys);
 }
 
 // Prefill / append tiles: each request's new tokens cut into runs of 256 / G
@@ -277,6 +299,10 @@ pa_status create(const pa_problem* problem, int32_t prefix_len, Mode mode, bool 
   pa_status st = validate_problem(problem);
   if (st != PA_OK) return st;
   if (cascade && (prefix_len < 0 || prefix_len % problem->page_size)) return PA_ERR_INVALID_ARG;
+  // the prefix level and prefill read 16-bit pools with TMA, without rotation
+  if (((cascade && prefix_len > 0) || mode == Mode::kPrefill) &&
+      pa::decode_needs_cuda_cores(*problem))
+    return PA_ERR_UNSUPPORTED;
   // the prefix level moves whole pages (>= 8 rows) with TMA, whose row
   // coordinates are signed 32-bit
   if (((cascade && prefix_len > 0) || mode == Mode::kPrefill) &&

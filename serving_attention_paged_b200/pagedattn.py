@@ -23,11 +23,12 @@ lib = ctypes.CDLL(_LIB_PATH)
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL = 0, 1, 2, 3
 PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_NO_MEMORY, PA_ERR_DEVICE_TIMEOUT = 4, 5, 6, 7
-PA_F16, PA_BF16, PA_F32 = 0, 1, 2
+PA_F16, PA_BF16, PA_F32, PA_E4M3, PA_E5M2 = 0, 1, 2, 3, 4
 PA_FLAG_CHECK_INDICES = 1
 PA_FLAG_CUDA_CORES = 2
 PA_FLAG_TENSOR_CORES = 4
-DTYPE_CODES = {"f16": PA_F16, "bf16": PA_BF16, "f32": PA_F32}
+DTYPE_CODES = {"f16": PA_F16, "bf16": PA_BF16, "f32": PA_F32, "e4m3": PA_E4M3,
+               "e5m2": PA_E5M2}
 
 
 class pa_problem(ctypes.Structure):
@@ -37,7 +38,9 @@ class pa_problem(ctypes.Structure):
                 ("sm_scale", ctypes.c_float), ("num_sms", ctypes.c_int32),
                 ("ctas_per_sm", ctypes.c_int32), ("min_chunk_tokens", ctypes.c_int32),
                 ("num_pages", ctypes.c_int64), ("flags", ctypes.c_uint32),
-                ("piece_cost_tokens", ctypes.c_int32)]
+                ("piece_cost_tokens", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
+                ("rope_theta", ctypes.c_float)]
 
 
 class pa_work_item(ctypes.Structure):
@@ -74,6 +77,7 @@ _SIGS = {
     "pa_plan_check": [_vp, _vp, _P(_i64), _vp],
     "pa_static_workspace_check": [_vp, _P(_i64), _vp],
     "pa_default_schedule": [_i32, _i32, _i32, _i32, ctypes.c_uint32, _P(_i32), _P(_i32)],
+    "pa_problem_schedule": [_P(pa_problem), _i32, _P(_i32), _P(_i32)],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name)
@@ -139,12 +143,20 @@ class Plan:
 
 def make_problem(*, batch, num_qo_heads, num_kv_heads, head_dim=128, page_size, dtype,
                  sm_scale, num_sms, ctas_per_sm, min_chunk_tokens=0, num_pages=0,
-                 flags=0, piece_cost_tokens=0) -> pa_problem:
+                 flags=0, piece_cost_tokens=0, kv_dtype=None, k_scale=1.0, v_scale=1.0,
+                 rope_theta=0.0) -> pa_problem:
+    """``kv_dtype`` None: the pools hold ``dtype``; "e4m3" / "e5m2": 8-bit
+    pools with ``k_scale`` / ``v_scale``.  ``rope_theta`` > 0: rotary
+    positions applied on the fly."""
     if isinstance(dtype, str):
         dtype = DTYPE_CODES[dtype]
+    if kv_dtype is None:
+        kv_dtype = dtype
+    elif isinstance(kv_dtype, str):
+        kv_dtype = DTYPE_CODES[kv_dtype]
     return pa_problem(batch, num_qo_heads, num_kv_heads, head_dim, page_size, dtype, sm_scale,
                       num_sms, ctas_per_sm, min_chunk_tokens, num_pages, flags,
-                      piece_cost_tokens)
+                      piece_cost_tokens, kv_dtype, k_scale, v_scale, rope_theta or 0.0)
 
 
 def pa_plan_create(problem: pa_problem, kv_indptr_host, last_page_len_host) -> Plan:
@@ -322,6 +334,14 @@ def pa_default_schedule(device: int, num_qo_heads: int, num_kv_heads: int, dtype
     sms, k = _i32(), _i32()
     _check(lib.pa_default_schedule(device, num_qo_heads, num_kv_heads, dtype, flags,
                                    ctypes.byref(sms), ctypes.byref(k)), "pa_default_schedule")
+    return sms.value, k.value
+
+
+def pa_problem_schedule(problem: pa_problem, device: int):
+    """(SM count, resident CTAs per SM) of the decode kernel ``problem`` runs."""
+    sms, k = _i32(), _i32()
+    _check(lib.pa_problem_schedule(ctypes.byref(problem), device, ctypes.byref(sms),
+                                   ctypes.byref(k)), "pa_problem_schedule")
     return sms.value, k.value
 
 

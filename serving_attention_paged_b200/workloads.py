@@ -261,7 +261,9 @@ class PagedWorkload:
         key = stream_key(self.seed, stream)
         w = self.num_kv_heads * self.head_dim
         pool_dtype = KV8_DTYPES[self.kv_dtype] if self.kv_dtype else DTYPES[self.dtype]
-        pool = torch.zeros(self.num_pages * self.page_size, w, dtype=pool_dtype, device=device)
+        pool = torch.zeros(self.num_pages * self.page_size, w,
+                           dtype=torch.uint8 if self.kv_dtype else pool_dtype,
+                           device=device).view(pool_dtype)  # 8-bit: byte 0 is +0.0
         if rows is None:
             rows = self.token_rows()
         rows_t = torch.from_numpy(rows).to(device)
@@ -271,9 +273,12 @@ class PagedWorkload:
                 scale = self.k_scale if which == "k" else self.v_scale
                 x = normal(key, j0 * w, (j1 - j0) * w, device).to(torch.float32) / scale
                 vals = x.to(pool_dtype).view(j1 - j0, w)
+                # scatter the codes as bytes (indexing of 8-bit float tensors is not
+                # available everywhere)
+                pool.view(torch.uint8)[rows_t[j0:j1]] = vals.view(torch.uint8)
             else:
                 vals = normal_as(key, j0 * w, (j1 - j0) * w, self.dtype, device).view(j1 - j0, w)
-            pool[rows_t[j0:j1]] = vals
+                pool[rows_t[j0:j1]] = vals
         return pool.view(self.num_pages, self.page_size, self.num_kv_heads, self.head_dim)
 
     def logical_kv(self, which: str, token_begin: int, token_end: int, device="cpu") -> torch.Tensor:
@@ -447,6 +452,22 @@ def prefill_append(seed=1006) -> PagedWorkload:
                          page_size=16, dtype="f16", seed=seed, qo_lens=[1024] * 8)
 
 
+def batch_decode_uniform_fp8(seed=1002) -> PagedWorkload:
+    """Workload 2 with an 8-bit E4M3 cache: the same draws stored as codes with
+    per-tensor scales (K 0.02, V 0.02: the largest draw, ~6.5, maps below the
+    format's 448)."""
+    return make_workload("batch_decode_uniform_fp8", [4096] * 16, num_qo_heads=32,
+                         num_kv_heads=8, page_size=16, dtype="f16", seed=seed, kv_dtype="e4m3",
+                         k_scale=0.02, v_scale=0.02)
+
+
+def batch_decode_ragged_fp8(seed=1003) -> PagedWorkload:
+    """Workload 3 (bf16 q) with an 8-bit E4M3 cache, scales as for 2f8."""
+    return make_workload("batch_decode_ragged_fp8", ragged_lengths(seed), num_qo_heads=32,
+                         num_kv_heads=8, page_size=16, dtype="bf16", seed=seed, kv_dtype="e4m3",
+                         k_scale=0.02, v_scale=0.02)
+
+
 WORKLOADS = {
     1: single_request_decode,
     2: batch_decode_uniform,
@@ -456,4 +477,6 @@ WORKLOADS = {
     "4c": vector_sparse_contiguous_twin,
     "4s": vector_sparse_small,
     6: prefill_append,
+    "2f8": batch_decode_uniform_fp8,
+    "3f8": batch_decode_ragged_fp8,
 }

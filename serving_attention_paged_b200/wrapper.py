@@ -26,23 +26,30 @@ class PagedDecode:
     def __init__(self, kv_indptr, last_page_len, *, num_qo_heads, num_kv_heads, page_size,
                  dtype, sm_scale, num_pages, head_dim=128, device=None, num_sms=None,
                  ctas_per_sm=None, min_chunk_tokens=0, prefix_len=0, flags=0,
-                 piece_cost_tokens=0, stream=None):
+                 piece_cost_tokens=0, kv_dtype=None, k_scale=1.0, v_scale=1.0,
+                 rope_theta=0.0, stream=None):
         self.device = torch.device(device if device is not None else "cuda")
         dev_index = self.device.index if self.device.index is not None else torch.cuda.current_device()
-        if num_sms is None or ctas_per_sm is None:
-            sms, k = C.pa_default_schedule(dev_index, num_qo_heads, num_kv_heads, dtype, flags)
-            num_sms = sms if num_sms is None else num_sms
-            ctas_per_sm = k if ctas_per_sm is None else ctas_per_sm
         self.dtype = dtype
         self.batch = len(last_page_len)
         self.num_qo_heads, self.head_dim = num_qo_heads, head_dim
         self.prefix_len = prefix_len
+        extra = dict(kv_dtype=kv_dtype, k_scale=k_scale, v_scale=v_scale, rope_theta=rope_theta)
+        if num_sms is None or ctas_per_sm is None:
+            shape = C.make_problem(batch=self.batch, num_qo_heads=num_qo_heads,
+                                   num_kv_heads=num_kv_heads, head_dim=head_dim,
+                                   page_size=page_size, dtype=dtype, sm_scale=sm_scale,
+                                   num_sms=1, ctas_per_sm=1, flags=flags, **extra)
+            sms, k = C.pa_problem_schedule(shape, dev_index)
+            num_sms = sms if num_sms is None else num_sms
+            ctas_per_sm = k if ctas_per_sm is None else ctas_per_sm
         self.problem = C.make_problem(batch=self.batch, num_qo_heads=num_qo_heads,
                                       num_kv_heads=num_kv_heads, head_dim=head_dim,
                                       page_size=page_size, dtype=dtype, sm_scale=sm_scale,
                                       num_sms=num_sms, ctas_per_sm=ctas_per_sm,
                                       min_chunk_tokens=min_chunk_tokens, num_pages=num_pages,
-                                      flags=flags, piece_cost_tokens=piece_cost_tokens)
+                                      flags=flags, piece_cost_tokens=piece_cost_tokens,
+                                      **extra)
         if prefix_len:
             self.plan = C.pa_cascade_plan_create(self.problem, prefix_len, kv_indptr, last_page_len)
         else:

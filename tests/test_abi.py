@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(C):
     assert len(names) >= 15
     for n in names:
         assert hasattr(C.lib, n), n
-    assert C.pa_abi_version() == 4
+    assert C.pa_abi_version() == 5
 
 
 def _problem(C, w, num_sms=148, k=2, mct=0, flags=0):
@@ -232,3 +232,76 @@ def test_status_offset_lies_inside_the_workspace(C):
         plan = C.pa_plan_create(prob, indptr, last)
         off = C.pa_plan_status_offset(plan)
         assert off % 8 == 0 and off + 16 <= C.pa_plan_workspace_bytes(plan)
+
+
+def test_kv8_and_rope_validation(C):
+    """8-bit caches and rotary positions: bad scales, bad types and unbuilt
+    combinations are refused before anything runs."""
+    w = W.make_workload("v8", [20, 40], num_qo_heads=16, num_kv_heads=2, page_size=16,
+                        dtype="f16", seed=1)
+    qo = np.array([0, 4, 6], np.int32)
+
+    def prob(**kw):
+        base = dict(batch=w.batch, num_qo_heads=16, num_kv_heads=2, page_size=16, dtype="f16",
+                    sm_scale=0.1, num_sms=148, ctas_per_sm=2, num_pages=w.num_pages)
+        base.update(kw)
+        return C.make_problem(**base)
+
+    def status(make):
+        with pytest.raises(C.PagedAttnError) as e:
+            make()
+        return e.value.status
+
+    def plan(p):
+        return lambda: C.pa_plan_create(p, w.kv_indptr, w.last_page_len)
+
+    ok8 = prob(kv_dtype="e4m3", k_scale=0.5, v_scale=2.0)
+    p8 = C.pa_plan_create(ok8, w.kv_indptr, w.last_page_len)
+    assert C.pa_plan_uses_tensor_cores(p8) is False  # group 8 defaults to tensor cores otherwise
+    C.pa_plan_create(prob(kv_dtype="e5m2", k_scale=1.0, v_scale=1.0), w.kv_indptr,
+                     w.last_page_len)
+    okr = prob(rope_theta=1e4)
+    assert C.pa_plan_uses_tensor_cores(C.pa_plan_create(okr, w.kv_indptr, w.last_page_len)) is False
+    C.pa_plan_create(prob(kv_dtype="e4m3", rope_theta=5e5), w.kv_indptr, w.last_page_len)
+    for bad in (dict(kv_dtype="e4m3", k_scale=0.0), dict(kv_dtype="e4m3", v_scale=-1.0),
+                dict(kv_dtype="e5m2", k_scale=float("nan")), dict(kv_dtype="e4m3",
+                                                                  v_scale=float("inf")),
+                dict(kv_dtype="f32"), dict(rope_theta=-1.0), dict(rope_theta=float("nan"))):
+        assert status(plan(prob(**bad))) == C.PA_ERR_INVALID_ARG, bad
+    # not built: tensor cores, the cascade prefix level and prefill with either
+    assert status(plan(prob(kv_dtype="e4m3", flags=C.PA_FLAG_TENSOR_CORES))) == \
+        C.PA_ERR_UNSUPPORTED
+    assert status(plan(prob(rope_theta=1e4, flags=C.PA_FLAG_TENSOR_CORES))) == \
+        C.PA_ERR_UNSUPPORTED
+    C.pa_plan_create(prob(kv_dtype="e4m3", flags=C.PA_FLAG_TENSOR_CORES | C.PA_FLAG_CUDA_CORES),
+                     w.kv_indptr, w.last_page_len)
+    for kw in (dict(kv_dtype="e4m3"), dict(rope_theta=1e4)):
+        assert status(lambda: C.pa_cascade_plan_create(prob(**kw), 32, w.kv_indptr,
+                                                       w.last_page_len)) == C.PA_ERR_UNSUPPORTED
+        assert status(lambda: C.pa_prefill_plan_create(prob(**kw), True, qo, w.kv_indptr,
+                                                       w.last_page_len)) == C.PA_ERR_UNSUPPORTED
+    # a cascade without a prefix is a plain decode: allowed
+    C.pa_cascade_plan_create(prob(kv_dtype="e4m3"), 0, w.kv_indptr, w.last_page_len)
+    # rotary positions are exact fp32 integers: requests beyond 2^24 tokens are refused
+    indptr = np.array([0, (1 << 24) // 16 + 1], np.int32)
+    big = C.make_problem(batch=1, num_qo_heads=16, num_kv_heads=2, page_size=16, dtype="f16",
+                         sm_scale=0.1, num_sms=148, ctas_per_sm=2, num_pages=1 << 21,
+                         rope_theta=1e4)
+    assert status(lambda: C.pa_plan_create(big, indptr, np.array([1], np.int32))) == \
+        C.PA_ERR_UNSUPPORTED
+    big.rope_theta = 0.0
+    C.pa_plan_create(big, indptr, np.array([1], np.int32))
+
+
+def test_rope_plans_upload_each_request_length(C):
+    """Rotary plans carry each request's length in the workspace (the query's
+    position); others do not grow."""
+    w = W.make_workload("rl", [20, 0, 40, 1000], num_qo_heads=8, num_kv_heads=2, page_size=16,
+                        dtype="f16", seed=1)
+    args = dict(batch=w.batch, num_qo_heads=8, num_kv_heads=2, page_size=16, dtype="f16",
+                sm_scale=0.1, num_sms=4, ctas_per_sm=1, num_pages=w.num_pages)
+    plain = C.pa_plan_create(C.make_problem(**args), w.kv_indptr, w.last_page_len)
+    rope = C.pa_plan_create(C.make_problem(rope_theta=1e4, **args), w.kv_indptr,
+                            w.last_page_len)
+    assert C.pa_plan_workspace_bytes(rope) >= C.pa_plan_workspace_bytes(plain)
+    assert np.array_equal(C.pa_plan_work_items(rope), C.pa_plan_work_items(plain))
