@@ -213,9 +213,10 @@ typedef struct {
  * qo_indptr[batch]; lse is [total_q, num_qo_heads]; the pools as above.
  * Work: the query tokens of each request are cut into tiles of 256 / G
  * consecutive tokens (G = Hq / Hkv; the last tile of a request may be
- * shorter); the run launches one CTA per (tile, kv head), tiles in
- * decreasing order of 64-key tiles ceil(kv_end / 64), ties in request then
- * token order.  num_sms, ctas_per_sm, min_chunk_tokens and
+ * shorter); the run launches one CTA per (tile, kv head).  Tile order: the
+ * tiles of one request together, requests in decreasing order of their
+ * longest tile's ceil(kv_end / 128) (ties by request index), and within a
+ * request decreasing ceil(kv_end / 128), ties in token order.  num_sms, ctas_per_sm, min_chunk_tokens and
  * piece_cost_tokens are not used.
  * Validates as pa_plan_create, plus: qo_indptr[0] == 0 and non-decreasing,
  * total_q < 2^31, and Q_b <= L_b when causal.  page_size must be >= 8

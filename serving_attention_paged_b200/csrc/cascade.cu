@@ -55,6 +55,7 @@
 
 #include "common.cuh"
 #include "pa_internal.h"
+#include "attn_tile.cuh"
 #include "tcgen05.cuh"
 
 namespace pa {
@@ -89,6 +90,9 @@ constexpr int kBarQ = 0, kBarKFull = 1, kBarKEmpty = kBarKFull + kKStages,
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 8 + 1024;  // + slack to align to 1 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr float kSlack = 8.f;
+// Pairs of exponentials (out of every 8) taken on the FMA pipe by a
+// polynomial instead of the MUFU unit: balances the two with issue slots.
+constexpr int kPolyPairsPer8 = 2;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 struct CascadeArgs {
@@ -102,47 +106,13 @@ struct CascadeArgs {
   float score_scale;               // sm_scale * log2(e)
 };
 
-template <typename Tag> struct Fmt;
-template <> struct Fmt<F16> { static constexpr int v = 0; };
-template <> struct Fmt<BF16> { static constexpr int v = 1; };
-
-// Round two fp32 to bf16, packed; returns them widened again (the hi / lo split).
-__device__ __forceinline__ uint32_t pack2(BF16, float a, float b, float& ra, float& rb) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
-  ra = __uint_as_float(u << 16);
-  rb = __uint_as_float(u & 0xffff0000u);
-  return u;
-}
+using at::Fmt;
+using at::exp2_poly2;
+using at::make_map;
+using at::max3;
+using at::pack2;
 
 __device__ __forceinline__ void flag_timeout(const CascadeArgs& a) { atomicOr(a.status, 1ull); }
-
-// 2^x on the FMA pipe, for part of the exponentials so that the MUFU unit
-// (16 per clock per SM) is not the softmax's only bound.  x is split as
-// n + f with n = round(x) (the 1.5 * 2^23 shifter leaves n in the low bits of
-// t) and f in [-0.5, 0.5]; 2^f is a polynomial whose coefficients are a Remez
-// fit of relative error on that interval, computed for this kernel: degree 3
-// (error 7.5e-5, below an fp16 P's rounding) or degree 4 (2.7e-6, for the
-// two-term bf16 P); 2^n is added to the exponent field.  x is clamped to
-// -125 so the exponent stays normal: such p are < 2^-124 and round to 0 in
-// fp16 (they are 1e-38 in a bf16 P: nothing next to the other weights).
-template <int kDeg>
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float p;
-  if constexpr (kDeg == 3) {
-    p = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111251115799f), f, 0.6932609677314758f), f,
-             0.9999280571937561f);
-  } else {
-    p = fmaf(fmaf(fmaf(fmaf(0.009570102207362652f, f, 0.05591785907745361f), f,
-                       0.240247443318367f),
-                  f, 0.6931217908859253f),
-             f, 0.9999992847442627f);
-  }
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
 
 // Key tiles [t0, t1) of chunk c: the prefix's 128-key tiles split as evenly
 // as possible over the chunks.
@@ -363,44 +333,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       // wait for the maximum); in the rare tile whose maximum beats the
       // reference by more than 2^8 they are taken again with the new one.
       auto write_p = [&](float mref, bool poly) -> float {
-        const float nm = -mref;
-        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 sc2 = make_float2(a.score_scale, a.score_scale);
+        const float2 nm2 = make_float2(-mref, -mref);
+        float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c16 = 0; c16 < kKeys / 32; ++c16) {
           uint32_t w[16], wl[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c = 32 * c16 + 2 * e;
-            const float a0 = fmaf(x[c], a.score_scale, nm), a1 = fmaf(x[c + 1], a.score_scale, nm);
-            float p0, p1;
-            if (poly && (e & 3) < 2) {  // half of the pairs on the FMA pipe
-              p0 = exp2_poly<kSplit ? 4 : 3>(a0);
-              p1 = exp2_poly<kSplit ? 4 : 3>(a1);
+            const float2 a2 = __ffma2_rn(make_float2(x[c], x[c + 1]), sc2, nm2);
+            float2 p2;
+            if (poly && (e & 7) < kPolyPairsPer8) {  // on the FMA pipe
+              p2 = exp2_poly2<kSplit ? 4 : 3>(a2);
             } else {
-              p0 = fast_exp2(a0);
-              p1 = fast_exp2(a1);
+              p2 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
             }
-            float r0, r1;
             if constexpr (kSplit) {  // hi + lo carries p to ~2^-16
-              w[e] = pack2(Tag{}, p0, p1, r0, r1);
+              float r0, r1;
+              w[e] = pack2(Tag{}, p2.x, p2.y, r0, r1);
               float q0, q1;
-              wl[e] = pack2(Tag{}, p0 - r0, p1 - r1, q0, q1);
+              wl[e] = pack2(Tag{}, p2.x - r0, p2.y - r1, q0, q1);
             } else {
-              const __half2 hp = __floats2half2_rn(p0, p1);
+              const __half2 hp = __floats2half2_rn(p2.x, p2.y);
               w[e] = *reinterpret_cast<const uint32_t*>(&hp);
             }
-            ps4[e & 3] += p0 + p1;
+            ps2[e & 1] = __fadd2_rn(ps2[e & 1], p2);
           }
           tc::tmem_st16(lane_addr + col_s + 16 * c16, w);
           if constexpr (kSplit) tc::tmem_st16(lane_addr + col_s + 64 + 16 * c16, wl);
         }
-        return (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+        const float2 t = __fadd2_rn(ps2[0], ps2[1]);
+        return t.x + t.y;
       };
       auto tile_max = [&]() {
-        float tm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float t0 = fmaxf(x[0], x[4]), t1 = fmaxf(x[1], x[5]), t2 = fmaxf(x[2], x[6]),
+              t3 = fmaxf(x[3], x[7]);
 #pragma unroll
-        for (int c = 0; c < kKeys; ++c) tm4[c & 3] = fmaxf(tm4[c & 3], x[c]);
-        return fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3])) * a.score_scale;
+        for (int c = 8; c < kKeys; c += 8) {
+          t0 = max3(t0, x[c], x[c + 4]);
+          t1 = max3(t1, x[c + 1], x[c + 5]);
+          t2 = max3(t2, x[c + 2], x[c + 6]);
+          t3 = max3(t3, x[c + 3], x[c + 7]);
+        }
+        return max3(t0, t1, fmaxf(t2, t3)) * a.score_scale;
       };
       float psum, alpha = 1.f;
       if (kt == 0 || ragged) {
@@ -491,28 +467,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merge the prefix chunks of every (request, q head) row by log-sum-exp into
 // chunk slot 0 (base-2 lse), one warp per row, 4 head elements per lane.
-// Each warp reads all chunks of its row before writing slot 0.
+// The loads of a batch of chunks are all issued before any is used (the
+// merge is a chain of dependent L2 round trips otherwise), and each warp
+// reads all chunks of its row before writing slot 0.
 __global__ void __launch_bounds__(256) cascade_merge_kernel(float* prefix_o, float* prefix_lse,
                                                             int64_t rows, int chunks) {
+  constexpr int kBatch = 16;  // the chunks of a row in one round of loads, up to 16
   const int64_t row = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   float M = -INFINITY, L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c = 0; c < chunks; ++c) {
-    const float lse = prefix_lse[int64_t(c) * rows + row];
-    const float4 o = *reinterpret_cast<const float4*>(prefix_o + (int64_t(c) * rows + row) * D +
-                                                      4 * lane);
-    if (lse == -INFINITY) continue;
-    if (lse > M) {
-      const float s = fast_exp2(M - lse);  // M = -inf -> 0
-      L = L * s + 1.f;
-      acc = make_float4(acc.x * s + o.x, acc.y * s + o.y, acc.z * s + o.z, acc.w * s + o.w);
-      M = lse;
-    } else {
-      const float w = fast_exp2(lse - M);
-      L += w;
-      acc = make_float4(acc.x + w * o.x, acc.y + w * o.y, acc.z + w * o.z, acc.w + w * o.w);
+  for (int c0 = 0; c0 < chunks; c0 += kBatch) {
+    float lse[kBatch];
+    float4 o[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const bool in = c0 + j < chunks;
+      const int64_t c = in ? c0 + j : 0;
+      lse[j] = in ? prefix_lse[c * rows + row] : -INFINITY;
+      o[j] = *reinterpret_cast<const float4*>(prefix_o + (c * rows + row) * D + 4 * lane);
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      if (lse[j] == -INFINITY) continue;
+      if (lse[j] > M) {
+        const float s = fast_exp2(M - lse[j]);  // M = -inf -> 0
+        L = L * s + 1.f;
+        acc = make_float4(acc.x * s + o[j].x, acc.y * s + o[j].y, acc.z * s + o[j].z,
+                          acc.w * s + o[j].w);
+        M = lse[j];
+      } else {
+        const float w = fast_exp2(lse[j] - M);
+        L += w;
+        acc = make_float4(acc.x + w * o[j].x, acc.y + w * o[j].y, acc.z + w * o[j].z,
+                          acc.w + w * o[j].w);
+      }
     }
   }
   const float inv = M == -INFINITY ? 0.f : 1.f / L;
@@ -520,35 +510,6 @@ __global__ void __launch_bounds__(256) cascade_merge_kernel(float* prefix_o, flo
   *reinterpret_cast<float4*>(prefix_o + row * D + 4 * lane) =
       make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   if (lane == 0) prefix_lse[row] = M == -INFINITY ? -INFINITY : M + fast_log2(L);
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 3-D map over (dim0 = 128 head elements, dim1, dim2) with 128-byte swizzle;
-// boxes of 64 x box1 x box2 elements.
-bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t d1,
-              uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box1, uint32_t box2) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(d1), cuuint64_t(d2)};
-  const cuuint64_t strides[2] = {cuuint64_t(stride1), cuuint64_t(stride2)};
-  const cuuint32_t box[3] = {64, box1, box2};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename Tag>

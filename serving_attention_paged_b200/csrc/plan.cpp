@@ -245,8 +245,10 @@ void schedule_prefix(pa_plan_s* plan) {
 }
 
 // Prefill / append tiles: each request's new tokens cut into runs of 256 / G
-// (two 128-row tensor-core tiles of (token, q head) rows per kv head, one CTA),
-// listed in decreasing order of 64-key tiles so that the long ones start first.
+// (two 128-row tensor-core tiles of (token, q head) rows per kv head, one CTA).
+// A request's tiles are listed together (the CTAs running at a time then share
+// its K/V in L2), requests in decreasing order of their longest tile, and the
+// tiles of a request longest first; lengths count 128-key tiles.
 pa_status build_prefill(pa_plan_s* plan, bool causal, const int32_t* qo, const int32_t* indptr,
                         const int32_t* last) {
   const pa_problem& p = plan->prob;
@@ -254,7 +256,7 @@ pa_status build_prefill(pa_plan_s* plan, bool causal, const int32_t* qo, const i
   if (B > 0 && (!qo || !indptr || !last)) return PA_ERR_INVALID_ARG;
   if ((qo && qo[0] != 0) || (indptr && indptr[0] != 0)) return PA_ERR_INVALID_ARG;
   const int64_t per_tile = 256 / plan->group;
-  constexpr int64_t kTileKeys = 64;
+  constexpr int64_t kTileKeys = 128;
   std::vector<pa_prefill_tile> tiles;
   for (int64_t b = 0; b < B; ++b) {
     if (indptr[b + 1] < indptr[b] || qo[b + 1] < qo[b]) return PA_ERR_INVALID_ARG;
@@ -272,9 +274,16 @@ pa_status build_prefill(pa_plan_s* plan, bool causal, const int32_t* qo, const i
                                       int32_t(base), int32_t(end)});
     }
   }
-  std::stable_sort(tiles.begin(), tiles.end(), [](const pa_prefill_tile& x, const pa_prefill_tile& y) {
-    return ceil_div(x.kv_end, kTileKeys) > ceil_div(y.kv_end, kTileKeys);
-  });
+  std::vector<int64_t> longest(size_t(B), 0);
+  for (const pa_prefill_tile& t : tiles)
+    longest[size_t(t.request)] = std::max(longest[size_t(t.request)], ceil_div(t.kv_end, kTileKeys));
+  std::stable_sort(tiles.begin(), tiles.end(),
+                   [&](const pa_prefill_tile& x, const pa_prefill_tile& y) {
+                     const int64_t lx = longest[size_t(x.request)], ly = longest[size_t(y.request)];
+                     if (lx != ly) return lx > ly;
+                     if (x.request != y.request) return x.request < y.request;
+                     return ceil_div(x.kv_end, kTileKeys) > ceil_div(y.kv_end, kTileKeys);
+                   });
   plan->prefill_tiles = std::move(tiles);
   plan->total_q = B > 0 ? qo[B] : 0;
   if (B > 0) plan->kv_indptr.assign(indptr, indptr + B + 1);

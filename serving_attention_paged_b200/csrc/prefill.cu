@@ -10,56 +10,56 @@
 // attends to all L_b.  The plan's tiles carry both as one rule: token j of a
 // tile sees keys [0, min(kv_base + j + 1, kv_end)).
 //
-// CTA = (query tile, kv head h); one CTA per SM.  A query tile is up to
-// 256 / G consecutive new tokens of one request, as two halves of 128 rows
-// (M of one MMA); a half's rows are its (token, q head of h) pairs,
+// CTA = (query tile, kv head h); one CTA per SM, 12 warps.  A query tile is
+// up to 256 / G consecutive new tokens of one request, as two halves of 128
+// rows (M of one MMA); a half's rows are its (token, q head of h) pairs,
 // token-major, so one K/V load serves all G heads of the kv head
-// (head-query fusion) and both halves.  The host plan lists the tiles
-// longest first, so the block scheduler starts the long ones first.
-//   warp 8  (TMA):     both halves of Q once; K and V of each 64-key tile as
-//                      page-row boxes, 128-byte swizzle, into a 5-stage ring;
-//                      boxes wholly past the tile's last key read out of
-//                      range (zero fill).
-//   warp 9  (MMA):     per half, S = Q K^T into one of two TMEM buffers
-//                      (M = 128, N = 64, K = 128) and O += P V with P read
-//                      from TMEM (V an MN-major operand in shared memory)
-//                      into the half's O; completion goes to mbarriers, and
-//                      a K/V stage is released when both halves are done
-//                      with it.  Before the first P V of the last tile it
-//                      zeroes the V rows that were copied from a page but
-//                      lie past the tile's keys (a partly used last page may
-//                      hold anything, NaN included, and 0 * NaN would reach
-//                      O).
+// (head-query fusion) and both halves.  The plan groups each request's tiles
+// (so the CTAs in flight share its K/V in L2) and lists long tiles first.
+//   warp 8  (TMA):     both halves of Q once; K and V of each 128-key tile as
+//                      page-row boxes, 128-byte swizzle, K into a 3-stage and
+//                      V into a 2-stage ring; boxes wholly past the tile's
+//                      last key read out of range (zero fill).
+//   warp 9  (MMA):     one thread issues, in a fixed order, P V(half 0, t - 1)
+//                      then S(half 0, t) = Q K^T (M = 128, N = 128, K = 128),
+//                      then the same for half 1 (a half whose rows see fewer
+//                      keys stops early): the tensor core works on one half
+//                      while the other half's softmax runs.  P is read from
+//                      TMEM (A operand), V is an MN-major operand in shared
+//                      memory; S(half, t) is issued right behind the P V that
+//                      reads its columns (one thread's tcgen05.mma execute in
+//                      issue order).  Before the last tile's P V the warp
+//                      zeroes the V rows copied from a partly used last page
+//                      past the tile's keys (they may hold anything, NaN
+//                      included, and 0 * NaN would reach O).
+//   warps 10-11:       idle (they complete the producer warpgroup, whose
+//                      registers go to the softmax warpgroups).
 //   warps 0-3, 4-7:    one warpgroup per half; thread i owns row i of its
-//                      half = TMEM lane i: reads S with tcgen05.ld, masks
-//                      the keys its token may not see, keeps a lazy running
-//                      max (O is rescaled in TMEM only when the max grows by
-//                      more than 2^8), writes P in the input type over S in
-//                      TMEM with tcgen05.st, and at the end writes o = O / l
-//                      in the input type and lse = ln l + max straight to
-//                      the outputs.  Two independent softmax chains per SM
-//                      keep the tensor core fed while each waits on its own
-//                      latencies.  For bf16, P is written as two bf16 terms
-//                      (hi and the rounding remainder lo, in the buffer's
-//                      two 32-column halves) and P V is issued for both, so
-//                      the weights carry ~16 bits like the fp16 path
-//                      instead of 8.
-// TMEM: S / P (half, buffer) at columns 64 (2 half + buffer), O of a half at
-// 256 + 128 half: all 512 columns, one CTA per SM.  Keeping P out of shared
-// memory leaves room for five K/V stages: the K/V tiles come through L2 with
-// microseconds of latency, and the ring depth sets how many are in flight.
+//                      half = TMEM lane i: reads S(t), masks the keys its
+//                      token may not see (a select: the score of a stale row
+//                      may be anything), keeps a lazy running max (O is
+//                      rescaled in TMEM only when the max grows by more than
+//                      2^8), writes P in the input type over S with
+//                      tcgen05.st, and at the end writes o = O / l in the
+//                      input type and lse = (m + log2 l) ln 2.  bf16 P is
+//                      written as hi = bf16(p) and lo = bf16(p - hi) with one
+//                      P V for each (~16 bits).  Part of the exponentials run
+//                      as a polynomial on the FMA pipe.
+// TMEM: half h owns columns [256 h, 256 h + 128) for S / P and the next 128
+// for O.  A half's S barrier completes once per tile it computes and once
+// more after its last P V.
 // Every mbarrier wait is bounded; on a timeout the kernel records it in the
-// workspace status word and unwinds instead of hanging.  Waits are by phase
-// parity, and every wait targets a barrier whose previous phase the waiting
-// thread has itself observed, so no wait can match a phase two ahead.
+// workspace status word and unwinds instead of hanging.  Every parity wait
+// targets a barrier whose previous phase the waiting thread has itself
+// observed.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
 #include <atomic>
-#include <mutex>
 #include <type_traits>
 
+#include "attn_tile.cuh"
 #include "common.cuh"
 #include "pa_internal.h"
 #include "tcgen05.cuh"
@@ -67,39 +67,41 @@
 namespace pa {
 namespace {
 
+using at::exp2_poly2;
+using at::Fmt;
+using at::make_map;
+using at::max3;
+using at::pack2;
+
 constexpr int D = kHeadDim;
 constexpr int kRows = 128;                  // rows of one MMA tile (M): query tokens x G heads
 constexpr int kHalves = 2;                  // MMA tiles per CTA, one softmax warpgroup each
-constexpr int kKeys = 64;                   // keys per K/V tile
-constexpr int kThreads = 32 * 10;           // 8 softmax warps, 1 TMA warp, 1 MMA warp
+constexpr int kKeys = 128;                  // keys per K/V tile (N of S)
+constexpr int kThreads = 32 * 12;           // 8 softmax warps, TMA, MMA, 2 idle warps
 constexpr int kWarpTma = 8, kWarpMma = 9;
+// Register split per warpgroup (setmaxnreg), as in the cascade kernel:
+// 128 x 56 + 256 x 224 = 384 x 168.
+constexpr int kRegsProducer = 56, kRegsSoftmax = 224;
+static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * 168, "register split");
 constexpr int kQHalf = kRows * 128;         // 128 rows x 64 16-bit columns (16 KB)
-constexpr int kKVHalf = kKeys * 128;        // 64 keys x 64 16-bit columns (8 KB)
-constexpr int kQBytes = 2 * kQHalf;         // one MMA tile of Q: 128 rows x 128 elements
+constexpr int kKVHalf = kKeys * 128;        // 128 keys x 64 16-bit columns (16 KB)
+constexpr int kQBytes = 2 * kQHalf;
 constexpr int kKVBytes = 2 * kKVHalf;
-constexpr int kStages = 5;
-constexpr int kOffQ = 0;                                  // Q of half 0, then half 1
+constexpr int kKStages = 3, kVStages = 2;
+constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kHalves * kQBytes;
-constexpr int kOffV = kOffK + kStages * kKVBytes;
-constexpr int kOffBar = kOffV + kStages * kKVBytes;
-constexpr uint32_t kTmemCols = 512;  // S: 4 x 64 columns, O: 2 x 128 columns
-constexpr uint32_t kColO = 256;
+constexpr int kOffV = kOffK + kKStages * kKVBytes;
+constexpr int kOffBar = kOffV + kVStages * kKVBytes;
+constexpr int kBarQ = 0, kBarKFull = 1, kBarKEmpty = kBarKFull + kKStages,
+              kBarVFull = kBarKEmpty + kKStages, kBarVEmpty = kBarVFull + kVStages,
+              kBarS = kBarVEmpty + kVStages, kBarP = kBarS + kHalves,
+              kNumBars = kBarP + kHalves;
+constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 8 + 1024;  // + slack to align to 1 KB
+constexpr uint32_t kTmemCols = 512;
 constexpr float kSlack = 8.f;
+constexpr int kPolyPairsPer8 = 2;  // pairs of exponentials (of 8) on the FMA pipe
 constexpr float kLn2 = 0.6931471805599453f;
-
-// mbarriers: Q, then per K/V stage full K, full V, empty; then per (half,
-// buffer) S ready, P ready (in TMEM, over S), P V done.
-constexpr int kBarQ = 0, kBarFullK = 1, kBarFullV = kBarFullK + kStages,
-              kBarEmpty = kBarFullV + kStages, kBarS = kBarEmpty + kStages,
-              kBarPReady = kBarS + 4, kBarPFree = kBarPReady + 4, kNumBars = kBarPFree + 4;
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 8 + 1024;  // + 1 KB alignment slack
-static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
-
-// P is written over its own S in TMEM: 64 keys of 16 bits fill 32 of the
-// buffer's 64 columns; bf16 puts its lo term in the other 32.
-template <typename Tag> struct PTraits {
-  static constexpr bool kSplit = std::is_same<Tag, BF16>::value;
-};
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 struct PrefillArgs {
   const int32_t* kv_indices;
@@ -113,26 +115,6 @@ struct PrefillArgs {
   float score_scale;                // sm_scale * log2(e)
 };
 
-template <typename Tag> struct Fmt;
-template <> struct Fmt<F16> { static constexpr int v = 0; };
-template <> struct Fmt<BF16> { static constexpr int v = 1; };
-
-// Round two fp32 to the 16-bit type, packed; returns them widened again.
-__device__ __forceinline__ uint32_t pack2(F16, float a, float b, float& ra, float& rb) {
-  const __half2 h = __floats2half2_rn(a, b);
-  const float2 f = __half22float2(h);
-  ra = f.x;
-  rb = f.y;
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-__device__ __forceinline__ uint32_t pack2(BF16, float a, float b, float& ra, float& rb) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
-  ra = __uint_as_float(u << 16);
-  rb = __uint_as_float(u & 0xffff0000u);
-  return u;
-}
-
 __device__ __forceinline__ void flag_timeout(const PrefillArgs& a) {
   atomicOr(a.error_pos + 1, 1ull);
 }
@@ -142,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v, const PrefillArgs a) {
-  using PT = PTraits<Tag>;
+  constexpr bool kSplit = std::is_same<Tag, BF16>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -169,15 +151,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kBarFullK + s), 1);
-      mbar_init(bar(kBarFullV + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
     }
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(bar(kBarS + s), 1);
-      mbar_init(bar(kBarPReady + s), 4);
-      mbar_init(bar(kBarPFree + s), 1);
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+    }
+    for (int hf = 0; hf < kHalves; ++hf) {
+      mbar_init(bar(kBarS + hf), 1);
+      mbar_init(bar(kBarP + hf), 4);
     }
     fence_mbar_init();
   }
@@ -190,9 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == kWarpTma) {
+  if (warp >= 8) {
+   // ------------------------- producer warpgroup -------------------------
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsProducer) : "memory");
+   if (warp == kWarpTma) {
     // ------------------------------ TMA producer ------------------------------
-    // Lane j owns box j of every tile (a page, or a 64-row part of one): it
+    // Lane j owns box j of every tile (a page, or a 128-row part of one): it
     // reads that page's index one tile ahead and issues the box's copies.
     const int box = a.box_rows, pmask = a.page_size - 1;
     const int nbox = kKeys / box;
@@ -216,133 +203,135 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_3d(dq + kQHalf, &tmap_q, 64, h * G, q_begin + hf * per_half, bar(kBarQ));
       }
     }
-    int rowA = row_of(0), rowB = row_of(1);  // unrolled by two: no copy of a pending load
-    auto produce = [&](int kt, int row) -> bool {
-      const int s = kt % kStages;
-      if (kt >= kStages && !mbar_wait(bar(kBarEmpty + s), ((kt / kStages) - 1) & 1)) return false;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(kBarFullK + s), kKVBytes);
-        mbar_arrive_expect_tx(bar(kBarFullV + s), kKVBytes);
-      }
+    auto load_tile = [&](const CUtensorMap* map, uint32_t dst, int row, uint32_t full) {
+      if (lane == 0) mbar_arrive_expect_tx(full, kKVBytes);
       __syncwarp();
       if (lane < nbox) {
-        const uint32_t dk = sb + kOffK + s * kKVBytes + lane * box * 128;
-        const uint32_t dv = sb + kOffV + s * kKVBytes + lane * box * 128;
-        tc::tma_load_3d(dk, &tmap_k, 0, h, row, bar(kBarFullK + s));
-        tc::tma_load_3d(dk + kKVHalf, &tmap_k, 64, h, row, bar(kBarFullK + s));
-        tc::tma_load_3d(dv, &tmap_v, 0, h, row, bar(kBarFullV + s));
-        tc::tma_load_3d(dv + kKVHalf, &tmap_v, 64, h, row, bar(kBarFullV + s));
+        tc::tma_load_3d(dst + lane * box * 128, map, 0, h, row, full);
+        tc::tma_load_3d(dst + kKVHalf + lane * box * 128, map, 64, h, row, full);
       }
-      return true;
     };
+    // K(t + 1) ahead of V(t); V(t) reads the rows K(t) read.
+    int rnext = row_of(0);
+    int rv0 = 0, rv1 = 0;
     bool ok = true;
-    for (int kt = 0; ok && kt < ntiles; kt += 2) {
-      ok = produce(kt, rowA);
-      rowA = row_of(kt + 2);
-      if (ok && kt + 1 < ntiles) {
-        ok = produce(kt + 1, rowB);
-        rowB = row_of(kt + 3);
+    for (int kt = -1; kt < ntiles; ++kt) {
+      const int kn = kt + 1;
+      if (kn < ntiles) {
+        const int s = kn % kKStages;
+        if (kn >= kKStages) ok = mbar_wait(bar(kBarKEmpty + s), ((kn / kKStages) - 1) & 1);
+        if (!ok) break;
+        load_tile(&tmap_k, sb + kOffK + s * kKVBytes, rnext, bar(kBarKFull + s));
+        if (kn & 1) rv1 = rnext;
+        else rv0 = rnext;
+        rnext = row_of(kn + 1);
+      }
+      if (kt >= 0) {
+        const int s = kt % kVStages;
+        if (kt >= kVStages) ok = mbar_wait(bar(kBarVEmpty + s), ((kt / kVStages) - 1) & 1);
+        if (!ok) break;
+        load_tile(&tmap_v, sb + kOffV + s * kKVBytes, (kt & 1) ? rv1 : rv0, bar(kBarVFull + s));
       }
     }
     if (!ok && lane == 0) flag_timeout(a);
-  } else if (warp == kWarpMma) {
+   } else if (warp == kWarpMma) {
     // ------------------------------ MMA issuer ------------------------------
-    // The whole warp runs the schedule (it zeroes stale V rows before the
-    // P V of the last tile); every lane waits, lane 0 issues.  Each half runs
-    // its own S and P V sequence over the shared K/V ring; a stage is
-    // released once every half that uses the tile has issued its P V.
-    // Rows [zero_from, zero_to) of the last tile were copied from the page
-    // that holds the tile's last key but lie past it.
-    const int zero_from = kv_end - (ntiles - 1) * kKeys;
-    const int zero_to = min(kKeys, (zero_from + a.box_rows - 1) / a.box_rows * a.box_rows);
+    // Every lane waits (ok stays warp-uniform, and the lanes zero stale V rows
+    // together); lane 0 issues.
     constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
     constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
-    // descriptors are built once; a k-step adds its byte offset / 16
     const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
     const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffK, 16, 1024);
     const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffV, kKVHalf, 1024);
     const int nt[2] = {nt0, nt1};
-    // Fixed order, one blocking wait per input: S of tile kt for both halves,
-    // then P V of tile kt - 1 for both.  The softmax of a half always finds
-    // the next S issued while it works on the current tile.  S(kt) overwrites
-    // the TMEM buffer P V(kt - 2) reads P from; it is issued after that P V by
-    // this same thread, and the tensor pipe runs one thread's tcgen05.mma in
-    // issue order, so it is queued without waiting for the P V to finish and
-    // the pipe never drains between tiles.
-    // Every lane waits and ok stays warp-uniform, so the lanes take the same
-    // branches to the __syncwarp calls.
+    // Rows [zero_from, zero_to) of the last tile were copied from the page
+    // that holds the tile's last key but lie past it.
+    const int zero_from = kv_end - (ntiles - 1) * kKeys;
+    const int zero_to = min(kKeys, (zero_from + a.box_rows - 1) / a.box_rows * a.box_rows);
     auto wait_all = [&](int b, int parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar(b), parity));
     };
+    auto issue_s = [&](int hf, int kt) {
+      const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
+      const uint64_t kd = dk0 + (((kt % kKStages) * kKVBytes) >> 4);
+      const uint32_t dst = tmem + hf * 256;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+        const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+        tc::mma_f16_ss(dst, qd + off, kd + koff, kIdescQK, kk > 0);
+      }
+      tc::commit(bar(kBarS + hf));
+    };
+    auto issue_pv = [&](int hf, int v) {
+      const uint32_t pt = tmem + hf * 256;
+      const uint32_t dst = tmem + hf * 256 + 128;
+      const uint64_t vd = dv0 + (((v % kVStages) * kKVBytes) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < kKeys / 16; ++kk)
+        tc::mma_f16_ts(dst, pt + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                       (v > 0 || kk > 0) ? 1u : 0u);
+      if (kSplit) {
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          tc::mma_f16_ts(dst, pt + 64 + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
+      }
+    };
     bool ok = wait_all(kBarQ, 0);
+    // Fixed order per tile t: for each half, P V(t - 1) then S(t); a half
+    // past its own tile count only finishes (its last P V, then the extra
+    // S-barrier commit).
     for (int kt = 0; ok && kt <= ntiles; ++kt) {
-      if (kt < ntiles) {
-        const int s = kt % kStages;
-        ok = wait_all(kBarFullK + s, (kt / kStages) & 1);
-#pragma unroll
-        for (int hf = 0; hf < kHalves; ++hf) {
-          if (!ok || kt >= nt[hf]) continue;
-          if (ok && lane == 0) {
-            tc::fence_after_sync();
-            const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
-            const uint64_t kd = dk0 + ((s * kKVBytes) >> 4);
-            const uint32_t dst = tmem + (2 * hf + (kt & 1)) * kKeys;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-              const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
-              tc::mma_f16_ss(dst, qd + off, kd + koff, kIdescQK, kk > 0);
+      for (int hf = 0; ok && hf < kHalves; ++hf) {
+        const int v = kt - 1;
+        if (v >= 0 && v < nt[hf]) {
+          if (hf == 0 || v >= nt[0]) {  // the first half to use V(v) waits for it
+            ok = wait_all(kBarVFull + v % kVStages, (v / kVStages) & 1);
+            if (ok && v == ntiles - 1 && zero_from < zero_to) {
+              uint8_t* vt = smem + kOffV + (v % kVStages) * kKVBytes;
+              const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
+              for (int c = lane; c < n16; c += 32) {
+                const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
+                *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
             }
-            tc::commit(bar(kBarS + 2 * hf + (kt & 1)));
+          }
+          if (ok) ok = wait_all(kBarP + hf, v & 1);
+          if (!ok) break;
+          if (lane == 0) {
+            tc::fence_after_sync();
+            issue_pv(hf, v);
           }
           __syncwarp();
         }
-      }
-      if (ok && kt >= 1) {
-        // O(half) += P(v) V(v), P read from TMEM
-        const int v = kt - 1, s = v % kStages;
-        ok = wait_all(kBarFullV + s, (v / kStages) & 1);
-        if (ok && v == ntiles - 1 && zero_from < zero_to) {
-          // every lane has observed the landed copy itself before overwriting it
-          uint8_t* vt = smem + kOffV + s * kKVBytes;
-          const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
-          for (int c = lane; c < n16; c += 32) {
-            const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
-            *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();  // the zeros are written (and fenced) before lane 0 issues
-        }
-#pragma unroll
-        for (int hf = 0; hf < kHalves; ++hf) {
-          if (!ok || v >= nt[hf]) continue;
-          ok = wait_all(kBarPReady + 2 * hf + (v & 1), (v >> 1) & 1);
-          if (ok && lane == 0) {
+        if (kt < nt[hf]) {
+          if (hf == 0 || kt >= nt[0]) ok = wait_all(kBarKFull + kt % kKStages, (kt / kKStages) & 1);
+          if (!ok) break;
+          if (lane == 0) {
             tc::fence_after_sync();
-            const uint32_t pt = tmem + (2 * hf + (v & 1)) * kKeys;  // P over S(v)
-            const uint64_t vd = dv0 + ((s * kKVBytes) >> 4);
-            const uint32_t dst = tmem + kColO + hf * D;
-#pragma unroll
-            for (int kk = 0; kk < kKeys / 16; ++kk)
-              tc::mma_f16_ts(dst, pt + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
-                             (v > 0 || kk > 0) ? 1u : 0u);
-            if (PT::kSplit) {  // the lo term in the buffer's other 32 columns
-#pragma unroll
-              for (int kk = 0; kk < kKeys / 16; ++kk)
-                tc::mma_f16_ts(dst, pt + kKeys / 2 + kk * 8, vd + ((kk * 16 * 128) >> 4),
-                               kIdescPV, 1u);
-            }
-            tc::commit(bar(kBarPFree + 2 * hf + (v & 1)));
+            issue_s(hf, kt);
           }
           __syncwarp();
+        } else if (kt == nt[hf] && nt[hf] > 0) {
+          if (lane == 0) tc::commit(bar(kBarS + hf));  // the half's last P V is done
+          __syncwarp();
         }
-        if (ok && lane == 0) tc::commit(bar(kBarEmpty + s));  // both halves are done with v
       }
+      // release the stages the tile's last user has finished with
+      if (ok && lane == 0) {
+        if (kt < ntiles) tc::commit(bar(kBarKEmpty + kt % kKStages));
+        if (kt >= 1) tc::commit(bar(kBarVEmpty + (kt - 1) % kVStages));
+      }
+      __syncwarp();
     }
     if (!ok && lane == 0) flag_timeout(a);
+   }
   } else {
     // ------------------------- softmax / epilogue rows -------------------------
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax) : "memory");
     const int hf = warp >> 2;              // which half (warpgroup)
     const int i = threadIdx.x & 127;       // row within the half == TMEM lane
     const int jq = hf * per_half + i / G;  // token within the tile
@@ -354,106 +343,128 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lim = min(kv_base + jq + 1, kv_end);
     const int lim_min = min(kv_base + hf * per_half + 1, kv_end);
     const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16);
-    const uint32_t col_s = 2 * hf * kKeys, col_o = kColO + hf * D;
+    const uint32_t col_s = hf * 256, col_o = hf * 256 + 128;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int kt = 0; kt < nt; ++kt) {
-      const int s = kt & 1;  // S buffer
-      ok = mbar_wait(bar(kBarS + 2 * hf + s), (kt >> 1) & 1);
+      ok = mbar_wait(bar(kBarS + hf), kt & 1);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::fence_after_sync();
       float x[kKeys];
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
         float t32[32];
-        tc::tmem_ld32(lane_addr + col_s + s * kKeys + 32 * c, t32);
+        tc::tmem_ld32(lane_addr + col_s + 32 * c, t32);
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[32 * c + e] = t32[e];
       }
       tc::tmem_wait_ld();
-
-      // Raw scores; the scale is folded into the exponent argument below.
       // Keys at or past a row's limit are masked (a select: the score of a
-      // stale row may be anything).  Tiles wholly below every row's limit
-      // need no mask (uniform branch).
+      // stale row may be anything); tiles wholly below every row's limit need
+      // no mask (uniform branch).
       const int key0 = kt * kKeys;
-      if (key0 + kKeys > lim_min) {
+      const bool masked = key0 + kKeys > lim_min;
+      if (masked) {
 #pragma unroll
         for (int c = 0; c < kKeys; ++c) x[c] = key0 + c < lim ? x[c] : -INFINITY;
       }
-      float tm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      auto write_p = [&](float mref, bool poly) -> float {
+        const float2 sc2 = make_float2(a.score_scale, a.score_scale);
+        const float2 nm2 = make_float2(-mref, -mref);
+        float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) tm4[c & 3] = fmaxf(tm4[c & 3], x[c]);
-      const float tmax = fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3])) * a.score_scale;
-      const bool moved = tmax > m + kSlack;
-      const float mnew = moved ? tmax : m;
-      const float alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
-      // P V(kt - 2) has finished: S(kt) was issued after it and its commit
-      // counts every earlier MMA.  Waiting for it anyway (it returns at once)
-      // lets this thread see every phase of each P V barrier in order, which
-      // keeps the rescale wait below exact.
-      if (kt >= 2) {
-        const int pv = kt - 2;
-        ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      // O is rescaled in TMEM once the previous tile's P V is complete.
-      if (kt > 0 && __any_sync(0xffffffffu, moved)) {
-        const int pv = kt - 1;
-        ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc::fence_after_sync();
+        for (int c16 = 0; c16 < kKeys / 32; ++c16) {
+          uint32_t w[16], wl[16];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float ov[32];
-          tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-          tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
+          for (int e = 0; e < 16; ++e) {
+            const int c = 32 * c16 + 2 * e;
+            const float2 a2 = __ffma2_rn(make_float2(x[c], x[c + 1]), sc2, nm2);
+            float2 p2;
+            if (poly && (e & 7) < kPolyPairsPer8) {  // on the FMA pipe
+              p2 = exp2_poly2<kSplit ? 4 : 3>(a2);
+            } else {
+              p2 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
+            }
+            if constexpr (kSplit) {  // hi + lo carries p to ~2^-16
+              float r0, r1;
+              w[e] = pack2(Tag{}, p2.x, p2.y, r0, r1);
+              float q0, q1;
+              wl[e] = pack2(Tag{}, p2.x - r0, p2.y - r1, q0, q1);
+            } else {
+              const __half2 hp = __floats2half2_rn(p2.x, p2.y);
+              w[e] = *reinterpret_cast<const uint32_t*>(&hp);
+            }
+            ps2[e & 1] = __fadd2_rn(ps2[e & 1], p2);
+          }
+          tc::tmem_st16(lane_addr + col_s + 16 * c16, w);
+          if constexpr (kSplit) tc::tmem_st16(lane_addr + col_s + 64 + 16 * c16, wl);
         }
-      }
-      // P = 2^(s * scale - m) in the input type, written over S in TMEM (the
-      // P V that last read this buffer has finished, see above), 32 keys at a
-      // time; l sums what the tensor core multiplies.
-      const float nm = -mnew;
-      const uint32_t p_addr = lane_addr + col_s + s * kKeys;
-      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 t = __fadd2_rn(ps2[0], ps2[1]);
+        return t.x + t.y;
+      };
+      auto tile_max = [&]() {
+        float t0 = fmaxf(x[0], x[4]), t1 = fmaxf(x[1], x[5]), t2 = fmaxf(x[2], x[6]),
+              t3 = fmaxf(x[3], x[7]);
 #pragma unroll
-      for (int c16 = 0; c16 < kKeys / 32; ++c16) {
-        uint32_t w[16], wl[16];
+        for (int c = 8; c < kKeys; c += 8) {
+          t0 = max3(t0, x[c], x[c + 4]);
+          t1 = max3(t1, x[c + 1], x[c + 5]);
+          t2 = max3(t2, x[c + 2], x[c + 6]);
+          t3 = max3(t3, x[c + 3], x[c + 7]);
+        }
+        return max3(t0, t1, fmaxf(t2, t3)) * a.score_scale;
+      };
+      float psum, alpha = 1.f;
+      if (kt == 0 || masked) {
+        const float tmax = tile_max();
+        const bool moved = tmax > m + kSlack;
+        const float mnew = moved ? tmax : m;
+        alpha = moved ? fast_exp2(m - mnew) : 1.f;  // m = -inf -> 0
+        if (kt > 0 && __any_sync(0xffffffffu, moved)) {
+          // O holds every earlier tile: S(kt) completing means P V(kt - 1) has
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = 32 * c16 + 2 * e;
-          const float p0 = fast_exp2(fmaf(x[c], a.score_scale, nm));
-          const float p1 = fast_exp2(fmaf(x[c + 1], a.score_scale, nm));
-          float r0, r1;
-          w[e] = pack2(Tag{}, p0, p1, r0, r1);
-          if constexpr (PT::kSplit) {  // hi + lo carries p to ~2^-16: sum p itself
-            float q0, q1;
-            wl[e] = pack2(Tag{}, p0 - r0, p1 - r1, q0, q1);
-            ps4[e & 3] += p0 + p1;
-          } else {
-            ps4[e & 3] += r0 + r1;
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
           }
         }
-        tc::tmem_st16(p_addr + 16 * c16, w);
-        if constexpr (PT::kSplit) tc::tmem_st16(p_addr + kKeys / 2 + 16 * c16, wl);
+        psum = write_p(mnew, false);
+        m = mnew;
+      } else {
+        psum = write_p(m, true);
+        const float tmax = tile_max();
+        const bool moved = tmax > m + kSlack;
+        if (__any_sync(0xffffffffu, moved)) {
+          const float mnew = moved ? tmax : m;
+          alpha = moved ? fast_exp2(m - mnew) : 1.f;
+          tc::tmem_wait_st();  // the first P writes are done before they are replaced
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tc::tmem_ld32(lane_addr + col_o + 32 * c, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tc::tmem_st32(lane_addr + col_o + 32 * c, ov);
+          }
+          psum = write_p(mnew, true);
+          m = mnew;
+        }
       }
-      l = l * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
-      m = mnew;
+      l = l * alpha + psum;
       tc::tmem_wait_st();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarPReady + 2 * hf + s));
+      if (lane == 0) mbar_arrive(bar(kBarP + hf));
     }
-    // epilogue: o = O / l in the input type and lse = (m + log2 l) ln 2; a
-    // half without keys (no mask, empty request) writes o = 0, lse = -inf.
-    // The wait for the last P V is exact: this thread saw P V(nt - 3) finish.
-    if (ok && nt > 0) {
-      const int pv = nt - 1;
-      ok = mbar_wait(bar(kBarPFree + 2 * hf + (pv & 1)), (pv >> 1) & 1);
-    }
+    // epilogue: the half's last P V has completed (its extra S commit);
+    // o = O / l in the input type and lse = (m + log2 l) ln 2; a half without
+    // keys (no mask, empty request) writes o = 0, lse = -inf.
+    if (ok && nt > 0) ok = mbar_wait(bar(kBarS + hf), nt & 1);
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (!all_ok && lane == 0) flag_timeout(a);
     if (all_ok && nqh > 0) {
@@ -475,12 +486,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (valid) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
-            float t0, t1;
-            const uint4 u = make_uint4(pack2(Tag{}, ov[e] * inv, ov[e + 1] * inv, t0, t1),
-                                       pack2(Tag{}, ov[e + 2] * inv, ov[e + 3] * inv, t0, t1),
-                                       pack2(Tag{}, ov[e + 4] * inv, ov[e + 5] * inv, t0, t1),
-                                       pack2(Tag{}, ov[e + 6] * inv, ov[e + 7] * inv, t0, t1));
-            *reinterpret_cast<uint4*>(dst + (32 * c + e) * 2) = u;
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if constexpr (kSplit) {
+                float t0, t1;
+                w[k] = pack2(Tag{}, ov[e + 2 * k] * inv, ov[e + 2 * k + 1] * inv, t0, t1);
+              } else {
+                const __half2 hp = __floats2half2_rn(ov[e + 2 * k] * inv, ov[e + 2 * k + 1] * inv);
+                w[k] = *reinterpret_cast<const uint32_t*>(&hp);
+              }
+            }
+            *reinterpret_cast<uint4*>(dst + (32 * c + e) * 2) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
@@ -494,51 +511,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 3-D map over (dim0 = 128 head elements, dim1, dim2) with 128-byte swizzle;
-// boxes of 64 x box1 x box2 elements.
-bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t d1,
-              uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box1, uint32_t box2) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(d1), cuuint64_t(d2)};
-  const cuuint64_t strides[2] = {cuuint64_t(stride1), cuuint64_t(stride2)};
-  const cuuint32_t box[3] = {64, box1, box2};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename Tag, bool kCheck>
 cudaError_t launch_t(const PrefillArgs& args, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t stream) {
   auto kern = paged_prefill_kernel<Tag, kCheck>;
-  constexpr int smem = kSmemBytes;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = uint64_t(1) << (dev & 63);
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, args);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, args);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,8 @@
 """The prefill / append plan on the host (no GPU): its tiles cover every new
 query token of every request exactly once, in runs of at most 256 / G
 tokens of one request, with the key range of the causal rule (or all keys
-without the mask), longest first; malformed tables are rejected before
-anything runs."""
+without the mask), grouped by request with long tiles first; malformed
+tables are rejected before anything runs."""
 import numpy as np
 import pytest
 
@@ -60,12 +60,22 @@ def test_tiles_cover_every_query_once_longest_first(C, causal, hq, hkv):
     expected = _expected_tiles(kv_lens, qo_lens, G, causal)
     # the same set of tiles ...
     assert sorted(map(tuple, tiles.tolist())) == sorted(expected)
-    # ... in decreasing order of 64-key tiles, ties in (request, token) order
-    keys = -(-tiles[:, 5] // 64)
-    assert np.all(np.diff(keys) <= 0)
-    for k in np.unique(keys):
-        grp = tiles[keys == k]
-        assert np.all(np.diff(grp[:, 1]) > 0)
+    # ... each request's tiles together, requests by decreasing longest tile
+    # (ties by request), a request's tiles by decreasing ceil(kv_end / 128)
+    # (ties in token order)
+    keys = -(-tiles[:, 5] // 128)
+    reqs = tiles[:, 0]
+    starts = np.flatnonzero(np.r_[True, np.diff(reqs) != 0])
+    assert len(starts) == len(np.unique(reqs))  # contiguous per request
+    longest = [keys[reqs == r].max() for r in reqs[starts]]
+    order = list(zip([-x for x in longest], reqs[starts].tolist()))
+    assert order == sorted(order)
+    for r in np.unique(reqs):
+        mine = tiles[reqs == r]
+        k = -(-mine[:, 5] // 128)
+        assert np.all(np.diff(k) <= 0)
+        for kk in np.unique(k):
+            assert np.all(np.diff(mine[k == kk][:, 1]) > 0)
     # every new token of every request exactly once
     seen = np.zeros(qo_indptr[-1], np.int32)
     for r, q0, n, pb, base, end in tiles:
