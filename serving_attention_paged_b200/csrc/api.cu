@@ -165,9 +165,12 @@ pa_status pa_problem_schedule(const pa_problem* problem, int32_t device, int32_t
     return PA_ERR_INVALID_ARG;
   const int32_t group = problem->num_qo_heads / problem->num_kv_heads;
   if (!pa::decode_group_supported(group)) return PA_ERR_UNSUPPORTED;
-  if (!pa::decode_needs_cuda_cores(*problem))
+  if (pa::decode_uses_tensor_cores(*problem) || !pa::decode_f32_path(*problem))
     return pa_default_schedule(device, problem->num_qo_heads, problem->num_kv_heads,
-                               problem->dtype, problem->flags, num_sms, ctas_per_sm);
+                               problem->dtype, problem->flags | (pa::decode_uses_tensor_cores(*problem)
+                                                                     ? PA_FLAG_TENSOR_CORES
+                                                                     : 0u),
+                               num_sms, ctas_per_sm);
   int prev = 0;
   cudaError_t e = cudaGetDevice(&prev);
   if (e == cudaSuccess) e = cudaSetDevice(device);

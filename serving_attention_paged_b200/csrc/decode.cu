@@ -124,7 +124,7 @@ int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream) {
   const pa_problem& pr = plan.prob;
   DecodeArgs a;
   fill_decode_args(plan, p, &a);
-  if (decode_needs_cuda_cores(pr)) return launch_decode_f32(plan, a, stream);
+  if (decode_f32_path(pr)) return launch_decode_f32(plan, a, stream);
   using dec::KV16;
   const bool check = (pr.flags & PA_FLAG_CHECK_INDICES) != 0;
   const int64_t n = int64_t(plan.cta_indptr.size()) - 1;  // CTAs

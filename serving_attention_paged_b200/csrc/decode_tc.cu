@@ -44,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 #include "pa_internal.h"
@@ -55,25 +56,15 @@ namespace {
 constexpr int D = kHeadDim;
 constexpr int kTok = 128;                    // tokens per tile (MMA M of S^T)
 constexpr int kN = 16;                       // padded heads (MMA N)
-constexpr int kStages = 3;
 constexpr int kHalfKV = kTok * 128;          // 128 token rows x 64 elements: 16 KB
 constexpr int kTileKV = 2 * kHalfKV;         // K or V of a tile: 32 KB
-constexpr int kStageBytes = 2 * kTileKV;     // K then V
 constexpr int kHalfQ = kN * 128;             // 16 head rows x 64 elements: 2 KB
 constexpr int kQBytes = 2 * kHalfQ;          // Q^T: 16 rows x 128 elements
 constexpr int kPHalf = kN * 128;             // 16 head rows x 64 tokens: 2 KB
 constexpr int kPBytes = 2 * kPHalf;          // P^T: 16 rows x 128 tokens
-constexpr int kOffRing = 0;
-constexpr int kOffQ = kOffRing + kStages * kStageBytes;
-constexpr int kOffP = kOffQ + 2 * kQBytes;
-constexpr int kOffX = kOffP + 2 * kPBytes;     // tile maxima [2][4 warps][16]
-constexpr int kOffL = kOffX + 2 * 4 * kN * 4;  // row sums    [2][4 warps][16]
-constexpr int kOffM = kOffL + 2 * 4 * kN * 4;  // a piece's final maxima [2][16]
-constexpr int kOffBar = kOffM + 2 * kN * 4;
 
-// mbarriers: a K/V ring of full / empty pairs, then double-buffered pairs.
-constexpr int kBarFull = 0, kBarEmpty = kStages;
-constexpr int kBarS = 2 * kStages;      // S^T(t) written              (MMA commit)
+// mbarriers shared by both pool types, then those of each path.
+constexpr int kBarS = 0;                // S^T(t) written              (MMA commit)
 constexpr int kBarSFree = kBarS + 2;    // S^T(t) read                 (4 softmax warps)
 constexpr int kBarPReady = kBarS + 4;   // P^T(t) written, O^T rescaled (4 softmax warps)
 constexpr int kBarPFree = kBarS + 6;    // PV(t) done                  (MMA commit)
@@ -83,20 +74,62 @@ constexpr int kBarOFree = kBarS + 12;   // O^T of a piece read         (4 epilog
 constexpr int kBarXReady = kBarS + 14;  // tile maxima written         (4 softmax warps)
 constexpr int kBarLReady = kBarS + 16;  // piece maxima, row sums written (4 softmax warps)
 constexpr int kBarLFree = kBarS + 18;   // ... and read                (4 epilogue warps)
-constexpr int kNumBars = kBarS + 20;
+constexpr int kBarPath = kBarS + 20;
 
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;  // + alignment slack
+// 16-bit pools: a ring of kStages K/V tiles, copied straight into the layout
+// the MMA reads; full (the loaders' copies landed) / empty (PV done) pairs.
+// 8-bit pools: a ring of kRawStages raw tiles (8-bit rows, 16-byte chunks
+// swizzled by row), widened by the loader threads: K into one of two TMEM
+// buffers (the A operand of S^T), V into one of two shared-memory tiles.
+template <bool k8> struct Lay;
+template <> struct Lay<false> {
+  static constexpr int kStages = 3;
+  static constexpr int kStageBytes = 2 * kTileKV;   // K then V
+  static constexpr int kOffRing = 0;
+  static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+  static constexpr int kBarFull = kBarPath, kBarEmpty = kBarFull + kStages;
+  static constexpr int kNumBars = kBarEmpty + kStages;
+  static constexpr uint32_t kTmemCols = 64;         // S0, S1, O0, O1: 16 columns each
+};
+template <> struct Lay<true> {
+  static constexpr int kRawStages = 3;
+  static constexpr int kVStages = 3;                // widened V tiles
+  static constexpr int kRawHalf = kTok * 128;       // 128 raw rows of 128 bytes: 16 KB
+  static constexpr int kRawStage = 2 * kRawHalf;    // K then V
+  static constexpr int kOffRaw = 0;
+  static constexpr int kOffV = kOffRaw + kRawStages * kRawStage;  // widened V tiles
+  static constexpr int kOffQ = kOffV + kVStages * kTileKV;
+  static constexpr int kBarRawFull = kBarPath;                    // copies landed (128)
+  static constexpr int kBarRawFree = kBarRawFull + kRawStages;    // stage read (128)
+  static constexpr int kBarKReady = kBarRawFree + kRawStages;     // K(t) in TMEM (4 warps)
+  static constexpr int kBarKFree = kBarKReady + 2;                // S^T(t) done (MMA commit)
+  static constexpr int kBarVReady = kBarKFree + 2;                // V(t) widened (4 warps)
+  static constexpr int kBarVFree = kBarVReady + kVStages;         // PV(t) done (MMA commit)
+  static constexpr int kNumBars = kBarVFree + kVStages;
+  static constexpr uint32_t kTmemCols = 256;  // S0, S1, O0, O1 (16 each), K0, K1 (64 each)
+  static constexpr uint32_t kColK = 64;
+};
+template <bool k8> struct Off {
+  static constexpr int kOffQ = Lay<k8>::kOffQ;
+  static constexpr int kOffP = kOffQ + 2 * kQBytes;
+  static constexpr int kOffX = kOffP + 2 * kPBytes;     // tile maxima [2][4 warps][16]
+  static constexpr int kOffL = kOffX + 2 * 4 * kN * 4;  // row sums    [2][4 warps][16]
+  static constexpr int kOffM = kOffL + 2 * 4 * kN * 4;  // a piece's final maxima [2][16]
+  static constexpr int kOffBar = kOffM + 2 * kN * 4;
+  static constexpr int kSmemBytes = kOffBar + Lay<k8>::kNumBars * 8 + 16 + 1024;  // + alignment
+  static_assert(kSmemBytes <= 232448, "shared memory");
+  static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0,
+                "128-byte swizzle atoms need 1 KB alignment");
+};
+
 constexpr int kThreads = 13 * 32;
-constexpr uint32_t kTmemCols = 64;  // S0, S1, O0, O1: 16 columns each
 constexpr float kSlack = 8.f;       // lazy max: rescale only past 2^8
 
-static_assert(kSmemBytes <= 232448, "shared memory");
-static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "128-byte swizzle atoms need 1 KB alignment");
 
 struct TcArgs {
   const uint16_t* q;
-  const uint16_t* k_pool;
-  const uint16_t* v_pool;
+  const uint8_t* k_pool;  // 16-bit values or 8-bit codes
+  const uint8_t* v_pool;
   const int32_t* kv_indices;
   const pa_work_item* items;
   const int32_t* cta_indptr;
@@ -111,7 +144,8 @@ struct TcArgs {
   float* lse;
   int64_t num_pages;
   int32_t batch, num_qo_heads, num_kv_heads, log2_page, prefix_chunks;
-  float score_scale;
+  float score_scale;  // sm_scale * log2(e) (* k_scale for 8-bit pools)
+  float v_scale;      // 8-bit pools: value = v_scale * code
 };
 
 template <typename Tag> struct Fmt;
@@ -191,6 +225,43 @@ template <> __device__ __forceinline__ void tmem_st<16>(uint32_t taddr, const ui
       : "memory");
 }
 
+template <> __device__ __forceinline__ void tmem_st<32>(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Four 8-bit codes (little-endian in w) widened exactly to two pairs of q's
+// 16-bit type: cvt to fp16 pairs (every E4M3 / E5M2 value is an fp16 value),
+// and for bf16 through fp32 (every such value is a bf16 value too).
+template <typename Tag, int KV8>
+__device__ __forceinline__ void widen4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  if constexpr (KV8 == 1)
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n"
+        " cvt.rn.f16x2.e4m3x2 %1, h;\n}\n"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+  else
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e5m2x2 %0, l;\n"
+        " cvt.rn.f16x2.e5m2x2 %1, h;\n}\n"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+  if constexpr (Fmt<Tag>::v == 1) {
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+    const __nv_bfloat162 x = __floats2bfloat162_rn(a.x, a.y), y = __floats2bfloat162_rn(b.x, b.y);
+    lo = *reinterpret_cast<const uint32_t*>(&x);
+    hi = *reinterpret_cast<const uint32_t*>(&y);
+  }
+}
+
 // Byte offset of 16-byte chunk c (0..15) of row r in a 128-byte-swizzled
 // tile stored as two 64-element halves of `half_bytes` each.
 __device__ __forceinline__ uint32_t sw_chunk(int r, int c, int half_bytes) {
@@ -210,10 +281,24 @@ __device__ __forceinline__ int next_nonempty(const pa_work_item* items, int pc, 
   return pc;
 }
 
-template <typename Tag, int G, bool kCheck>
+// 8-bit pools: the code type (1 = E4M3, 2 = E5M2), 0 for 16-bit pools.
+template <typename Tag, int KV8, int G, bool kCheck>
 __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcArgs a) {
-  // bf16: P^T rows [0, G) hold hi, rows [G, 2G) lo; O^T columns likewise
-  constexpr bool kSplit = Fmt<Tag>::v == 1;
+  constexpr bool k8 = KV8 != 0;
+  // P^T and V in the type of the PV MMA: q's type for 16-bit pools; fp16 for
+  // 8-bit pools (every code widens exactly to fp16, so V costs one conversion
+  // per pair whatever q's type).
+  using PTag = std::conditional_t<k8, F16, Tag>;
+  // Two-term P: P^T rows [0, G) hold hi = round(p), rows [G, 2G) lo =
+  // round(p - hi); O^T columns likewise, added in the epilogue.  Needed for
+  // bf16 P (8 bits), and for the fp16 P of 8-bit pools, whose scaled values
+  // can be large: 11 bits of weight would move o by up to 2^-11 |v - o|.
+  constexpr bool kSplit = k8 || Fmt<PTag>::v == 1;
+  using L = Lay<k8>;
+  constexpr int kOffQ = Off<k8>::kOffQ, kOffP = Off<k8>::kOffP, kOffX = Off<k8>::kOffX,
+                kOffL = Off<k8>::kOffL, kOffM = Off<k8>::kOffM, kOffBar = Off<k8>::kOffBar;
+  constexpr int kNumBars = L::kNumBars;
+  constexpr uint32_t kTmemCols = L::kTmemCols;
   constexpr int kCols = kSplit ? 2 * G : G;
   static_assert(kCols <= kN, "hi and lo rows must fit the padded MMA N");
   extern __shared__ uint8_t smem_raw[];
@@ -227,9 +312,24 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
   const int p0 = a.cta_indptr[blockIdx.x], p1 = a.cta_indptr[blockIdx.x + 1];
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kBarFull + s), 128);
-      mbar_init(bar(kBarEmpty + s), 1);
+    if constexpr (k8) {
+      for (int s = 0; s < Lay<true>::kRawStages; ++s) {
+        mbar_init(bar(Lay<true>::kBarRawFull + s), 128);
+        mbar_init(bar(Lay<true>::kBarRawFree + s), 128);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(bar(Lay<true>::kBarKReady + b), 4);
+        mbar_init(bar(Lay<true>::kBarKFree + b), 1);
+      }
+      for (int b = 0; b < Lay<true>::kVStages; ++b) {
+        mbar_init(bar(Lay<true>::kBarVReady + b), 4);
+        mbar_init(bar(Lay<true>::kBarVFree + b), 1);
+      }
+    } else {
+      for (int s = 0; s < Lay<false>::kStages; ++s) {
+        mbar_init(bar(Lay<false>::kBarFull + s), 128);
+        mbar_init(bar(Lay<false>::kBarEmpty + s), 1);
+      }
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(kBarS + b), 1);
@@ -255,10 +355,156 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
   const uint32_t tmem = *tmem_holder;
 
   if (warp >= 4 && warp < 8) {
+   if constexpr (k8) {
+    // ------------------------- loaders (8-bit pools) -------------------------
+    // Thread j copies, for every tile, the 16-byte chunk j % 8 of raw rows
+    // j / 8 + 16 k (k = 0..7) of K and V (8 lanes per 128-byte row: coalesced)
+    // into a raw stage, chunk c of row r at byte r * 128 + ((c ^ (r % 8)) * 16)
+    // so that the row-per-thread reads below are conflict-free; the stage's
+    // mbarrier counts the copies.  Then thread j widens token row j of tile t:
+    // K into TMEM lane j (64 columns, two 16-bit elements each, the A operand
+    // of S^T = K Q^T), V into the 128-byte-swizzled 16-bit tile the PV MMA
+    // reads.  Rows past a piece are zero-filled and widen to zeros.
+    using LL = Lay<true>;
+    const int j = threadIdx.x - 128;  // token row of the tile this thread widens
+    const int lw = warp - 4;
+    const int lp = a.log2_page;
+    const uint32_t pmask = (1u << lp) - 1u;
+    const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * D;
+    const int cc = j & 7, cr = j >> 3;  // copied chunk, first copied row
+    // copy walker over the tiles of the CTA's non-empty pieces
+    int pi = next_nonempty(a.items, p0, p1), tt = 0, len = 0;
+    pa_work_item it{};
+    int total = 0;
+    for (int pc = pi; pc < p1; ++pc)
+      total += (a.items[pc].token_end - a.items[pc].token_begin + kTok - 1) / kTok;
+    if (pi < p1) {
+      it = a.items[pi];
+      len = it.token_end - it.token_begin;
+    }
+    // Page of each row this thread copies, for the tile copied next: looked up
+    // a tile ahead so the copies never wait on an index load.
+    int pgn[8];
+    auto lookup = [&]() {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int pos = tt * kTok + cr + 16 * k;
+        int pg = -1;
+        if (pi < p1 && pos < len) {
+          const int idx = (it.token_begin + pos) >> lp;
+          pg = __ldg(a.kv_indices + it.page_begin + idx);
+          if (kCheck && (pg < 0 || int64_t(pg) >= a.num_pages)) {
+            atomicMin(a.error_pos, (unsigned long long)(it.page_begin + idx));
+            pg = -1;
+          }
+        }
+        pgn[k] = pg;
+      }
+    };
+    lookup();
+    auto copy_tile = [&](int c) {
+      const int s = c % LL::kRawStages;
+      const uint32_t base = sb + LL::kOffRaw + s * LL::kRawStage;
+      const uint8_t* kb = a.k_pool + int64_t(it.kv_head) * D + cc * 16;
+      const uint8_t* vb = a.v_pool + int64_t(it.kv_head) * D + cc * 16;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int r = cr + 16 * k;
+        const int pos = tt * kTok + r;
+        const int pg = pgn[k];
+        const uint32_t row = pg >= 0 ? ((uint32_t(pg) << lp) | (uint32_t(it.token_begin + pos) & pmask)) : 0u;
+        const uint32_t nbytes = pg >= 0 ? 16u : 0u;  // 0: zero-fill, nothing read
+        const uint64_t off = uint64_t(row) * pool_row_bytes;
+        const uint32_t dst = base + r * 128 + ((cc ^ (r & 7)) << 4);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst),
+                     "l"(kb + off), "r"(nbytes) : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst + LL::kRawHalf),
+                     "l"(vb + off), "r"(nbytes) : "memory");
+      }
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(
+                       bar(LL::kBarRawFull + s)) : "memory");
+      if (++tt * kTok >= len) {  // advance the walker
+        tt = 0;
+        pi = next_nonempty(a.items, pi + 1, p1);
+        if (pi < p1) {
+          it = a.items[pi];
+          len = it.token_end - it.token_begin;
+        }
+      }
+      lookup();
+    };
+    const uint32_t lane_k = tmem + LL::kColK + (uint32_t(lw * 32) << 16);
+    bool ok = true;
+    for (int c = 0; c < LL::kRawStages - 1 && c < total; ++c) copy_tile(c);
+    for (int t = 0; ok && t < total; ++t) {
+      const int c = t + LL::kRawStages - 1;
+      if (c < total) {
+        if (c >= LL::kRawStages)  // the stage's previous tile has been read by every thread
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(LL::kBarRawFree + c % LL::kRawStages),
+                                                 ((c / LL::kRawStages) - 1) & 1));
+        if (!ok) break;
+        copy_tile(c);
+      }
+      const int s = t % LL::kRawStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(LL::kBarRawFull + s), (t / LL::kRawStages) & 1));
+      if (!ok) break;
+      const uint8_t* raw = smem + LL::kOffRaw + s * LL::kRawStage + j * 128;
+      // K row j -> TMEM lane j of buffer t & 1, once S^T(t - 2) has read it
+      {
+        uint32_t w[64];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 u = *reinterpret_cast<const uint4*>(raw + ((ch ^ (j & 7)) << 4));
+          widen4<Tag, KV8>(u.x, w[8 * ch + 0], w[8 * ch + 1]);
+          widen4<Tag, KV8>(u.y, w[8 * ch + 2], w[8 * ch + 3]);
+          widen4<Tag, KV8>(u.z, w[8 * ch + 4], w[8 * ch + 5]);
+          widen4<Tag, KV8>(u.w, w[8 * ch + 6], w[8 * ch + 7]);
+        }
+        if (t >= 2) ok = mbar_wait(bar(LL::kBarKFree + (t & 1)), ((t >> 1) - 1) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc::fence_after_sync();
+        tmem_st<32>(lane_k + (t & 1) * 64, *reinterpret_cast<const uint32_t(*)[32]>(w));
+        tmem_st<32>(lane_k + (t & 1) * 64 + 32, *reinterpret_cast<const uint32_t(*)[32]>(w + 32));
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(LL::kBarKReady + (t & 1)));
+      }
+      // V row j -> the widened tile t & 1, once PV(t - 2) has read it
+      {
+        uint4 v[16];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 u = *reinterpret_cast<const uint4*>(raw + LL::kRawHalf + ((ch ^ (j & 7)) << 4));
+          widen4<PTag, KV8>(u.x, v[2 * ch].x, v[2 * ch].y);
+          widen4<PTag, KV8>(u.y, v[2 * ch].z, v[2 * ch].w);
+          widen4<PTag, KV8>(u.z, v[2 * ch + 1].x, v[2 * ch + 1].y);
+          widen4<PTag, KV8>(u.w, v[2 * ch + 1].z, v[2 * ch + 1].w);
+        }
+        mbar_arrive(bar(LL::kBarRawFree + s));  // this thread is done with the raw stage
+        const int vs = t % LL::kVStages;
+        if (t >= LL::kVStages)
+          ok = mbar_wait(bar(LL::kBarVFree + vs), ((t / LL::kVStages) - 1) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        uint8_t* vt = smem + LL::kOffV + vs * kTileKV;
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch)
+          *reinterpret_cast<uint4*>(vt + sw_chunk(j, ch, kHalfKV)) = v[ch];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(LL::kBarVReady + vs));
+      }
+    }
+    if (!ok) {
+      asm volatile("cp.async.wait_all;\n" ::: "memory");
+      if (lane == 0) flag_timeout(a);
+    }
+   } else {
     // ------------------------------ loaders ------------------------------
     const int lw = warp - 4;
     const int lp = a.log2_page;
     const uint32_t pmask = (1u << lp) - 1u;
+    constexpr int kStages = Lay<false>::kStages, kStageBytes = Lay<false>::kStageBytes;
     const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * D * 2;
     const int c = lane & 15;  // 16-byte chunk of a 256-byte row
     // Page of this lane's row (32 * lw + lane) of tile tt of a piece; -1 past
@@ -289,13 +535,13 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
     bool ok = true;
     while (pi < p1) {
       const int s = t % kStages;
-      if (t >= kStages && !mbar_wait(bar(kBarEmpty + s), ((t / kStages) - 1) & 1)) {
+      if (t >= kStages && !mbar_wait(bar(Lay<false>::kBarEmpty + s), ((t / kStages) - 1) & 1)) {
         ok = false;
         break;
       }
-      const uint64_t kb = reinterpret_cast<uint64_t>(a.k_pool + int64_t(it.kv_head) * D) + c * 16;
-      const uint64_t vb = reinterpret_cast<uint64_t>(a.v_pool + int64_t(it.kv_head) * D) + c * 16;
-      const uint32_t kdst = sb + kOffRing + s * kStageBytes;
+      const uint64_t kb = reinterpret_cast<uint64_t>(a.k_pool + int64_t(it.kv_head) * D * 2) + c * 16;
+      const uint64_t vb = reinterpret_cast<uint64_t>(a.v_pool + int64_t(it.kv_head) * D * 2) + c * 16;
+      const uint32_t kdst = sb + Lay<false>::kOffRing + s * kStageBytes;
       const uint32_t vdst = kdst + kTileKV;
 #pragma unroll 4
       for (int k = 0; k < 16; ++k) {
@@ -318,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       }
       // the stage's barrier counts this thread once all its copies above land
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(
-                       bar(kBarFull + s))
+                       bar(Lay<false>::kBarFull + s))
                    : "memory");
       ++t;
       if (++tt * kTok >= len) {
@@ -335,14 +581,20 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       asm volatile("cp.async.wait_all;\n" ::: "memory");
       if (lane == 0) flag_timeout(a);
     }
+   }
   } else if (warp == 8) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
       constexpr uint32_t kIdescS = tc::idesc_f16(Fmt<Tag>::v, 0, kTok, kN);
       // O^T = V^T P^T: A = V^T (M = head elements, MN-major), B = P^T (K-major)
-      constexpr uint32_t kIdescO = tc::idesc_f16(Fmt<Tag>::v, 0, D, kN) | (1u << 15);
-      const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffRing, 16, 1024);
-      const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffRing + kTileKV, kHalfKV, 1024);
+      constexpr uint32_t kIdescO = tc::idesc_f16(Fmt<PTag>::v, 0, D, kN) | (1u << 15);
+      // 16-bit pools: K and V of a tile in one ring stage; 8-bit pools: K in a
+      // TMEM buffer, widened V in one of two shared-memory tiles
+      constexpr int kStages = Lay<false>::kStages, kStageBytes = Lay<false>::kStageBytes;
+      const uint64_t dk0 = tc::smem_desc_sw128(sb + Lay<false>::kOffRing, 16, 1024);
+      const uint64_t dv0 =
+          k8 ? tc::smem_desc_sw128(sb + Lay<true>::kOffV, kHalfKV, 1024)
+             : tc::smem_desc_sw128(sb + Lay<false>::kOffRing + kTileKV, kHalfKV, 1024);
       const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
       const uint64_t dp0 = tc::smem_desc_sw128(sb + kOffP, 16, 1024);
       // S^T(ts) and PV(tv) walk the pieces in step with their counters
@@ -358,19 +610,33 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       bool ok = true;
       while (v_piece < p1) {
         bool progress = false;
+        auto k_ready = [&]() {
+          return k8 ? mbar_test_wait(bar(Lay<true>::kBarKReady + (ts & 1)), (ts >> 1) & 1)
+                    : mbar_test_wait(bar(Lay<false>::kBarFull + ts % kStages), (ts / kStages) & 1);
+        };
         if (s_piece < p1 &&
             (ts < 2 || mbar_test_wait(bar(kBarSFree + (ts & 1)), ((ts - 2) >> 1) & 1)) &&
-            mbar_test_wait(bar(kBarFull + ts % kStages), (ts / kStages) & 1) &&
-            mbar_test_wait(bar(kBarQReady + (s_np & 1)), (s_np >> 1) & 1)) {
+            k_ready() && mbar_test_wait(bar(kBarQReady + (s_np & 1)), (s_np >> 1) & 1)) {
           fence_proxy_async_smem();  // the loaders' cp.async writes, seen by the tensor core
           tc::fence_after_sync();
-          const uint64_t kd = dk0 + uint64_t(((ts % kStages) * kStageBytes) >> 4);
           const uint64_t qd = dq0 + uint64_t(((s_np & 1) * kQBytes) >> 4);
+          if constexpr (k8) {
+            // A = K from TMEM (lane = token, 8 columns per 16 head elements)
+            const uint32_t ka = tmem + Lay<true>::kColK + (ts & 1) * 64;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = ((kk >> 2) * kHalfKV + (kk & 3) * 32) >> 4;
-            const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
-            tc::mma_f16_ss(tmem + (ts & 1) * kN, kd + koff, qd + qoff, kIdescS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
+              tc::mma_f16_ts(tmem + (ts & 1) * kN, ka + kk * 8, qd + qoff, kIdescS, kk > 0);
+            }
+            tc::commit(bar(Lay<true>::kBarKFree + (ts & 1)));
+          } else {
+            const uint64_t kd = dk0 + uint64_t(((ts % kStages) * kStageBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t koff = ((kk >> 2) * kHalfKV + (kk & 3) * 32) >> 4;
+              const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
+              tc::mma_f16_ss(tmem + (ts & 1) * kN, kd + koff, qd + qoff, kIdescS, kk > 0);
+            }
           }
           tc::commit(bar(kBarS + (ts & 1)));
           ++ts;
@@ -383,10 +649,13 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           progress = true;
         }
         if (tv < ts && mbar_test_wait(bar(kBarPReady + (tv & 1)), (tv >> 1) & 1) &&
+            (!k8 || mbar_test_wait(bar(Lay<true>::kBarVReady + tv % Lay<true>::kVStages),
+                                   (tv / Lay<true>::kVStages) & 1)) &&
             (v_tile > 0 || v_np < 2 ||
              mbar_test_wait(bar(kBarOFree + (v_np & 1)), ((v_np - 2) >> 1) & 1))) {
           tc::fence_after_sync();
-          const uint64_t vd = dv0 + uint64_t(((tv % kStages) * kStageBytes) >> 4);
+          const uint64_t vd = k8 ? dv0 + uint64_t(((tv % Lay<true>::kVStages) * kTileKV) >> 4)
+                                 : dv0 + uint64_t(((tv % kStages) * kStageBytes) >> 4);
           const uint64_t pd = dp0 + uint64_t(((tv & 1) * kPBytes) >> 4);
           const uint32_t od = tmem + 2 * kN + (v_np & 1) * kN;
 #pragma unroll
@@ -396,7 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
             tc::mma_f16_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
           }
           tc::commit(bar(kBarPFree + (tv & 1)));
-          tc::commit(bar(kBarEmpty + tv % kStages));
+          if constexpr (k8) tc::commit(bar(Lay<true>::kBarVFree + tv % Lay<true>::kVStages));
+          else tc::commit(bar(Lay<false>::kBarEmpty + tv % kStages));
           ++tv;
           if (++v_tile == v_ntiles) {
             tc::commit(bar(kBarODone + (v_np & 1)));
@@ -510,11 +780,11 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
         for (int hh = 0; hh < G; ++hh) {
           const float p = valid ? fast_exp2(fmaf(sv[hh], a.score_scale, -mn[hh])) : 0.f;
           float pr;
-          const uint16_t bits = round16(Tag{}, p, pr);
+          const uint16_t bits = round16(PTag{}, p, pr);
           *reinterpret_cast<uint16_t*>(pt + hh * 128 + ((pc ^ (hh & 7)) << 4)) = bits;
           if constexpr (kSplit) {  // p - hi is exact in fp32
             float lo;
-            const uint16_t lbits = round16(Tag{}, p - pr, lo);
+            const uint16_t lbits = round16(PTag{}, p - pr, lo);
             *reinterpret_cast<uint16_t*>(pt + (G + hh) * 128 + ((pc ^ ((G + hh) & 7)) << 4)) = lbits;
             pr += lo;
           }
@@ -635,6 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           const float acc = kSplit ? __uint_as_float(r[hh]) + __uint_as_float(r[(G + hh) % kCols])
                                    : __uint_as_float(r[hh]);
           res[hh] = acc / l[hh];
+          if constexpr (k8) res[hh] *= a.v_scale;  // cached value = v_scale * code
           lse2[hh] = m[hh] + fast_log2(l[hh]);
         }
         ++np;
@@ -702,33 +973,48 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
   if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-template <typename Tag, int G, bool kCheck>
+template <typename Tag, int KV8, int G, bool kCheck>
 cudaError_t launch_tc_t(const TcArgs& a, int64_t n_cta, cudaStream_t stream) {
-  auto kern = paged_decode_tc_kernel<Tag, G, kCheck>;
+  auto kern = paged_decode_tc_kernel<Tag, KV8, G, kCheck>;
+  constexpr int kSmem = Off<KV8 != 0>::kSmemBytes;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = uint64_t(1) << (dev & 63);
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   if (n_cta <= 0) return cudaSuccess;
-  kern<<<dim3(unsigned(n_cta)), kThreads, kSmemBytes, stream>>>(a);
+  kern<<<dim3(unsigned(n_cta)), kThreads, kSmem, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <typename Tag, bool kCheck>
+template <typename Tag, int KV8, bool kCheck>
 cudaError_t dispatch_tc(int group, const TcArgs& a, int64_t n, cudaStream_t s) {
   switch (group) {
-    case 1: return launch_tc_t<Tag, 1, kCheck>(a, n, s);
-    case 2: return launch_tc_t<Tag, 2, kCheck>(a, n, s);
-    case 4: return launch_tc_t<Tag, 4, kCheck>(a, n, s);
-    case 8: return launch_tc_t<Tag, 8, kCheck>(a, n, s);
+    case 1: return launch_tc_t<Tag, KV8, 1, kCheck>(a, n, s);
+    case 2: return launch_tc_t<Tag, KV8, 2, kCheck>(a, n, s);
+    case 4: return launch_tc_t<Tag, KV8, 4, kCheck>(a, n, s);
+    case 8: return launch_tc_t<Tag, KV8, 8, kCheck>(a, n, s);
   }
   return cudaErrorInvalidValue;
+}
+
+template <typename Tag, int KV8>
+cudaError_t dispatch_tc_check(bool check, int group, const TcArgs& a, int64_t n, cudaStream_t s) {
+  return check ? dispatch_tc<Tag, KV8, true>(group, a, n, s)
+               : dispatch_tc<Tag, KV8, false>(group, a, n, s);
+}
+
+template <typename Tag>
+cudaError_t dispatch_tc_kv(pa_dtype kv, bool check, int group, const TcArgs& a, int64_t n,
+                           cudaStream_t s) {
+  if (kv == PA_E4M3) return dispatch_tc_check<Tag, 1>(check, group, a, n, s);
+  if (kv == PA_E5M2) return dispatch_tc_check<Tag, 2>(check, group, a, n, s);
+  return dispatch_tc_check<Tag, 0>(check, group, a, n, s);
 }
 
 }  // namespace
@@ -739,30 +1025,25 @@ bool decode_tc_supported(int32_t group, pa_dtype dtype) {
 }
 
 int decode_tc_ctas_per_sm(int32_t group, pa_dtype dtype, int32_t* out) {
-  auto get = [&](auto kern) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, kSmemBytes);
-  };
-  const bool bf = dtype == PA_BF16;
-  if (group == 1)
-    return int(bf ? get(paged_decode_tc_kernel<BF16, 1, false>) : get(paged_decode_tc_kernel<F16, 1, false>));
-  if (group == 2)
-    return int(bf ? get(paged_decode_tc_kernel<BF16, 2, false>) : get(paged_decode_tc_kernel<F16, 2, false>));
-  if (group == 4)
-    return int(bf ? get(paged_decode_tc_kernel<BF16, 4, false>) : get(paged_decode_tc_kernel<F16, 4, false>));
-  if (group == 8)
-    return int(bf ? get(paged_decode_tc_kernel<BF16, 8, false>) : get(paged_decode_tc_kernel<F16, 8, false>));
-  return int(cudaErrorInvalidValue);
+  // one CTA per SM whatever the shape: the kernels hold ~200 KB of shared memory
+  (void)group;
+  (void)dtype;
+  auto kern = paged_decode_tc_kernel<F16, 0, 8, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Off<false>::kSmemBytes);
+  int n = 0;
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, Off<false>::kSmemBytes);
+  *out = n;
+  return int(e);
 }
 
 int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream) {
   const pa_problem& pr = plan.prob;
   TcArgs a{};
   a.q = static_cast<const uint16_t*>(p.q);
-  a.k_pool = static_cast<const uint16_t*>(p.k_pool);
-  a.v_pool = static_cast<const uint16_t*>(p.v_pool);
+  a.k_pool = static_cast<const uint8_t*>(p.k_pool);
+  a.v_pool = static_cast<const uint8_t*>(p.v_pool);
   a.kv_indices = p.kv_indices;
   a.items = reinterpret_cast<const pa_work_item*>(p.ws + plan.ws.items);
   a.cta_indptr = reinterpret_cast<const int32_t*>(p.ws + plan.ws.cta_indptr);
@@ -782,17 +1063,15 @@ int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream) 
   a.log2_page = plan.log2_page;
   // the prefix level leaves each row's merged prefix state in chunk slot 0
   a.prefix_chunks = plan.cascade && plan.prefix_chunks > 0 ? 1 : 0;
-  a.score_scale = pr.sm_scale * kLog2e;
+  const bool kv8 = kv_is_8bit(pr);
+  a.score_scale = pr.sm_scale * kLog2e * (kv8 ? pr.k_scale : 1.f);
+  a.v_scale = kv8 ? pr.v_scale : 1.f;
   const bool check = (pr.flags & PA_FLAG_CHECK_INDICES) != 0;
   const int64_t n = int64_t(plan.cta_indptr.size()) - 1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  if (pr.dtype == PA_BF16)
-    e = check ? dispatch_tc<BF16, true>(plan.group, a, n, s)
-              : dispatch_tc<BF16, false>(plan.group, a, n, s);
-  else
-    e = check ? dispatch_tc<F16, true>(plan.group, a, n, s)
-              : dispatch_tc<F16, false>(plan.group, a, n, s);
+  const pa_dtype kv = kv8 ? pr.kv_dtype : pr.dtype;
+  const cudaError_t e = pr.dtype == PA_BF16 ? dispatch_tc_kv<BF16>(kv, check, plan.group, a, n, s)
+                                            : dispatch_tc_kv<F16>(kv, check, plan.group, a, n, s);
   return int(e);
 }
 

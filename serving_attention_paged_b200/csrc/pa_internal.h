@@ -85,14 +85,14 @@ struct RunPointers {
   uint8_t* ws;
 };
 
-// 8-bit (FP8) KV cache; rotary positions on the fly.  Both run on the
-// CUDA-core decode kernel only.
+// 8-bit (FP8) KV cache (both decode kernels); rotary positions on the fly
+// (the CUDA-core decode kernel only).
 inline bool kv_is_8bit(const pa_problem& p) {
   return p.kv_dtype == PA_E4M3 || p.kv_dtype == PA_E5M2;
 }
-inline bool decode_needs_cuda_cores(const pa_problem& p) {
-  return kv_is_8bit(p) || p.rope_theta > 0.f;
-}
+inline bool decode_needs_cuda_cores(const pa_problem& p) { return p.rope_theta > 0.f; }
+// Problems the CUDA-core kernel runs on its fp32 path (decode_f32.cu).
+inline bool decode_f32_path(const pa_problem& p) { return kv_is_8bit(p) || p.rope_theta > 0.f; }
 
 int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream);
 // Resident CTAs per SM of the fp32-path kernel (8-bit pools, rotary) a problem runs.
@@ -109,7 +109,11 @@ inline bool decode_uses_tensor_cores(const pa_problem& p) {
   if (!decode_tc_supported(group, p.dtype) || (p.flags & PA_FLAG_CUDA_CORES) ||
       decode_needs_cuda_cores(p))
     return false;
-  return (p.flags & PA_FLAG_TENSOR_CORES) || group >= 8;
+  // 8-bit caches: the CUDA-core kernel spends as many instructions per
+  // (token, kv head) widening and multiplying as on 16-bit rows, so only the
+  // tensor-core kernel (which widens once into its MMA operands) gains from
+  // the halved bytes
+  return (p.flags & PA_FLAG_TENSOR_CORES) || group >= 8 || kv_is_8bit(p);
 }
 // Plan cost of a piece boundary, in tokens of the kernel's steady-state rate.
 // Per-CTA clock traces on B200 put the extra time of a further piece of a CTA

@@ -43,7 +43,7 @@ pa_status validate_problem(const pa_problem* p) {
                               std::isfinite(p->v_scale) && p->v_scale > 0.f))
     return PA_ERR_INVALID_ARG;
   if (!(std::isfinite(p->rope_theta) && p->rope_theta >= 0.f)) return PA_ERR_INVALID_ARG;
-  // 8-bit caches and rotary positions are built for the CUDA-core decode kernel
+  // rotary positions are built for the CUDA-core decode kernel only
   if (pa::decode_needs_cuda_cores(*p) && (p->flags & PA_FLAG_TENSOR_CORES) &&
       !(p->flags & PA_FLAG_CUDA_CORES))
     return PA_ERR_UNSUPPORTED;
@@ -309,8 +309,7 @@ pa_status create(const pa_problem* problem, int32_t prefix_len, Mode mode, bool 
   if (st != PA_OK) return st;
   if (cascade && (prefix_len < 0 || prefix_len % problem->page_size)) return PA_ERR_INVALID_ARG;
   // the prefix level and prefill read 16-bit pools with TMA, without rotation
-  if (((cascade && prefix_len > 0) || mode == Mode::kPrefill) &&
-      pa::decode_needs_cuda_cores(*problem))
+  if (((cascade && prefix_len > 0) || mode == Mode::kPrefill) && pa::decode_f32_path(*problem))
     return PA_ERR_UNSUPPORTED;
   // the prefix level moves whole pages (>= 8 rows) with TMA, whose row
   // coordinates are signed 32-bit

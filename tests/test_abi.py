@@ -257,7 +257,10 @@ def test_kv8_and_rope_validation(C):
 
     ok8 = prob(kv_dtype="e4m3", k_scale=0.5, v_scale=2.0)
     p8 = C.pa_plan_create(ok8, w.kv_indptr, w.last_page_len)
-    assert C.pa_plan_uses_tensor_cores(p8) is False  # group 8 defaults to tensor cores otherwise
+    assert C.pa_plan_uses_tensor_cores(p8) is True  # 8-bit caches default to tensor cores
+    p8c = C.pa_plan_create(prob(kv_dtype="e4m3", flags=C.PA_FLAG_CUDA_CORES), w.kv_indptr,
+                           w.last_page_len)
+    assert C.pa_plan_uses_tensor_cores(p8c) is False
     C.pa_plan_create(prob(kv_dtype="e5m2", k_scale=1.0, v_scale=1.0), w.kv_indptr,
                      w.last_page_len)
     okr = prob(rope_theta=1e4)
@@ -268,9 +271,10 @@ def test_kv8_and_rope_validation(C):
                                                                   v_scale=float("inf")),
                 dict(kv_dtype="f32"), dict(rope_theta=-1.0), dict(rope_theta=float("nan"))):
         assert status(plan(prob(**bad))) == C.PA_ERR_INVALID_ARG, bad
-    # not built: tensor cores, the cascade prefix level and prefill with either
-    assert status(plan(prob(kv_dtype="e4m3", flags=C.PA_FLAG_TENSOR_CORES))) == \
-        C.PA_ERR_UNSUPPORTED
+    # not built: rotary positions on tensor cores, the cascade prefix level and
+    # prefill with either
+    C.pa_plan_create(prob(kv_dtype="e4m3", flags=C.PA_FLAG_TENSOR_CORES), w.kv_indptr,
+                     w.last_page_len)
     assert status(plan(prob(rope_theta=1e4, flags=C.PA_FLAG_TENSOR_CORES))) == \
         C.PA_ERR_UNSUPPORTED
     C.pa_plan_create(prob(kv_dtype="e4m3", flags=C.PA_FLAG_TENSOR_CORES | C.PA_FLAG_CUDA_CORES),

@@ -4,8 +4,10 @@ README core feature 3: attention over a compressed KV-Cache.  The pools hold
 8-bit codes with one scale for K and one for V; q and o stay fp16 / bf16.
 Small cases span several tiles, ragged tails, empty requests, every GQA
 group, page sizes 1 / 16 / 64, both q types and both formats, with
-non-power-of-two scales, split and unsplit plans.  The full-size uniform and
-ragged batches with E4M3 caches are checked on every row.
+non-power-of-two scales, split and unsplit plans, on both decode kernels
+(the tensor-core one widens K into TMEM and V into shared memory).  The
+full-size uniform and ragged batches with E4M3 caches are checked on every
+row.
 """
 import os
 
@@ -43,11 +45,15 @@ def _decode(w, dev, **kw):
     return pd, o, lse
 
 
+KERNELS = {"cuda_cores": 2, "tensor_cores": 4}  # PA_FLAG_CUDA_CORES / PA_FLAG_TENSOR_CORES
+
+
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
 @pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("P", [1, 16, 64])
-def test_fp8_small_parity(fmt, dtype, group, P):
+def test_fp8_small_parity(fmt, dtype, group, P, kernel):
     hkv = 2
     w = W.make_workload("fp8_small", EDGE_LENS, num_qo_heads=hkv * group, num_kv_heads=hkv,
                         page_size=P, dtype=dtype, seed=300 + group + P, extra_pages=3,
@@ -58,13 +64,15 @@ def test_fp8_small_parity(fmt, dtype, group, P):
     from serving_attention_paged_b200 import pagedattn as C
     for kw in (dict(num_sms=10000, ctas_per_sm=1),
                dict(num_sms=3, ctas_per_sm=1, min_chunk_tokens=16)):
-        pd, o, lse = _decode(w, dev, **kw)
-        assert not C.pa_plan_uses_tensor_cores(pd.plan)
-        assert_close(to_np(o), to_np(lse), o_ref, l_ref, dtype, f"{fmt} G={group} P={P} {kw}")
+        pd, o, lse = _decode(w, dev, flags=KERNELS[kernel], **kw)
+        assert C.pa_plan_uses_tensor_cores(pd.plan) == (kernel == "tensor_cores")
+        assert_close(to_np(o), to_np(lse), o_ref, l_ref, dtype,
+                     f"{kernel} {fmt} G={group} P={P} {kw}")
 
 
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
 @pytest.mark.parametrize("group", [4, 8])
-def test_fp8_sharp_softmax(group):
+def test_fp8_sharp_softmax(group, kernel):
     """Large score spread: the running maximum moves past the lazy slack."""
     w = W.make_workload("fp8_sharp", [2000, 700, 129, 5000, 1], num_qo_heads=2 * group,
                         num_kv_heads=2, page_size=16, dtype="bf16", seed=310 + group,
@@ -72,8 +80,9 @@ def test_fp8_sharp_softmax(group):
     t = w.materialize()
     o_ref, l_ref = _oracle(w, t)
     dev = {k: v.cuda() for k, v in t.items()}
-    pd, o, lse = _decode(w, dev, num_sms=5, ctas_per_sm=1, min_chunk_tokens=300)
-    assert_close(to_np(o), to_np(lse), o_ref, l_ref, "bf16", f"fp8 sharp G={group}")
+    pd, o, lse = _decode(w, dev, num_sms=5, ctas_per_sm=1, min_chunk_tokens=300,
+                         flags=KERNELS[kernel])
+    assert_close(to_np(o), to_np(lse), o_ref, l_ref, "bf16", f"fp8 sharp G={group} {kernel}")
 
 
 def test_fp8_equals_16bit_cache_holding_the_same_values():
@@ -97,7 +106,8 @@ def test_fp8_equals_16bit_cache_holding_the_same_values():
     assert (l8 - l16).abs().max().item() <= 1e-3
 
 
-def test_fp8_checked_indices_and_graph_replay():
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+def test_fp8_checked_indices_and_graph_replay(kernel):
     from serving_attention_paged_b200 import pagedattn as C
     w = W.make_workload("fp8_chk", [4000, 50, 9], num_qo_heads=32, num_kv_heads=8,
                         page_size=16, dtype="bf16", seed=330, kv_dtype="e5m2", k_scale=0.8,
@@ -105,7 +115,7 @@ def test_fp8_checked_indices_and_graph_replay():
     t = w.materialize()
     dev = {k: v.cuda() for k, v in t.items()}
     pd, o_eager, l_eager = _decode(w, dev, num_sms=148, ctas_per_sm=2,
-                                   flags=C.PA_FLAG_CHECK_INDICES)
+                                   flags=C.PA_FLAG_CHECK_INDICES | KERNELS[kernel])
     o_ref, l_ref = _oracle(w, t)
     assert_close(to_np(o_eager), to_np(l_eager), o_ref, l_ref, "bf16", "fp8 checked")
     bad = dev["kv_indices"].clone()
@@ -128,11 +138,12 @@ def test_fp8_checked_indices_and_graph_replay():
         assert torch.equal(o, o_eager) and torch.equal(lse, l_eager)
 
 
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
 @pytest.mark.parametrize("n", ["2f8", "3f8"])
-def test_fp8_full_size_every_row(n):
+def test_fp8_full_size_every_row(n, kernel):
     w = W.WORKLOADS[n]()
     dev = w.materialize("cuda")
-    pd, o, lse = _decode(w, dev)
+    pd, o, lse = _decode(w, dev, flags=KERNELS[kernel])
     indptr, indices, last = w.flat_tables()
     # 8-bit pools cross to the host as raw bytes
     o_ref, l_ref = oracle.paged_decode_requests(
