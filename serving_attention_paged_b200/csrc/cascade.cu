@@ -56,6 +56,7 @@
 #include "common.cuh"
 #include "pa_internal.h"
 #include "attn_tile.cuh"
+#include "launch.cuh"
 #include "tcgen05.cuh"
 
 namespace pa {
@@ -171,6 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
+  // the merge kernel and the decode level may be scheduled from now on: they
+  // wait for this grid before reading its results
+  grid_dependents_launch();
 
   if (warp >= 8) {
    // ------------------------- producer warpgroup -------------------------
@@ -473,6 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(256) cascade_merge_kernel(float* prefix_o, float* prefix_lse,
                                                             int64_t rows, int chunks) {
   constexpr int kBatch = 16;  // the chunks of a row in one round of loads, up to 16
+  grid_dependents_launch();  // the decode level may be scheduled
+  grid_dependency_wait();    // the prefix level has completed
   const int64_t row = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -573,9 +579,9 @@ int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* str
                                       : launch_t<F16>(a, tq, tk, tv, grid, s);
   if (e != cudaSuccess || plan.prefix_chunks == 1) return int(e);
   const int64_t rows = int64_t(pr.batch) * pr.num_qo_heads;
-  cascade_merge_kernel<<<unsigned((rows + 7) / 8), 256, 0, s>>>(a.prefix_o, a.prefix_lse, rows,
-                                                                 plan.prefix_chunks);
-  return int(cudaGetLastError());
+  return int(launch_maybe_dependent(cascade_merge_kernel, dim3(unsigned((rows + 7) / 8)), dim3(256),
+                                    0, s, true, a.prefix_o, a.prefix_lse, rows,
+                                    int(plan.prefix_chunks)));
 }
 
 }  // namespace pa

@@ -174,6 +174,19 @@ __device__ __forceinline__ void axpy2_f16(uint16_t p, uint32_t v, float& o0, flo
       : "r"(v), "h"(p));
 }
 
+// Programmatic dependent launch (grid dependency control).  A kernel calls
+// grid_dependents_launch() once its dependent grid may be scheduled (every
+// CTA of this grid has then started, so the dependent's CTAs never wait for
+// resources this grid still needs); the dependent calls grid_dependency_wait()
+// before it reads anything the previous grid writes: it returns once that grid
+// has completed and its memory is visible (at once for a normal launch).
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -130,12 +130,14 @@ int launch_decode(const pa_plan_s& plan, const RunPointers& p, void* stream) {
   const int64_t n = int64_t(plan.cta_indptr.size()) - 1;  // CTAs
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
+  // a cascade's decode level starts while the prefix level finishes
+  const bool pdl = a.prefix_chunks > 0;
   if (pr.dtype == PA_BF16)
-    e = check ? dec::dispatch_group<BF16, KV16, dec::kChecked, false>(plan.group, a, n, s)
-              : dec::dispatch_group<BF16, KV16, dec::kNoCheck, false>(plan.group, a, n, s);
+    e = check ? dec::dispatch_group<BF16, KV16, dec::kChecked, false>(plan.group, a, n, s, pdl)
+              : dec::dispatch_group<BF16, KV16, dec::kNoCheck, false>(plan.group, a, n, s, pdl);
   else
-    e = check ? dec::dispatch_group<F16, KV16, dec::kChecked, false>(plan.group, a, n, s)
-              : dec::dispatch_group<F16, KV16, dec::kNoCheck, false>(plan.group, a, n, s);
+    e = check ? dec::dispatch_group<F16, KV16, dec::kChecked, false>(plan.group, a, n, s, pdl)
+              : dec::dispatch_group<F16, KV16, dec::kNoCheck, false>(plan.group, a, n, s, pdl);
   return int(e);
 }
 

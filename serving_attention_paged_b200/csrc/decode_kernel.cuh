@@ -10,6 +10,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "launch.cuh"
 #include "pa_internal.h"
 
 namespace pa {
@@ -614,6 +615,7 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
       MergeAcc acc[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) acc[hh].add(res[hh], lse2[hh]);
+      grid_dependency_wait();  // the prefix level has completed
       merge_prefix<G, D>(acc, a.prefix_o, a.prefix_lse, a.prefix_chunks, Bstride, row0, d);
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) write_final<Tag>(a, row0 + hh, d, acc[hh].out(), acc[hh].lse2());
@@ -644,6 +646,7 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
   const int s0 = a.merge_indptr[seg], s1 = a.merge_indptr[seg + 1];
   MergeAcc acc[G];
   merge_partials<G, D>(acc, a.partial_o, a.partial_lse, s0, s1, d);
+  if (a.prefix_chunks > 0) grid_dependency_wait();  // the prefix level has completed
   merge_prefix<G, D>(acc, a.prefix_o, a.prefix_lse, a.prefix_chunks, Bstride, row0, d);
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) write_final<Tag>(a, row0 + hh, d, acc[hh].out(), acc[hh].lse2());
@@ -700,7 +703,7 @@ cudaError_t occupancy_group(int group, int* out) {
 }
 
 template <typename Tag, typename KV, int G, int kCheckMode, bool kRope>
-cudaError_t launch_t(const DecodeArgs& a, int64_t n_cta, cudaStream_t stream) {
+cudaError_t launch_t(const DecodeArgs& a, int64_t n_cta, cudaStream_t stream, bool pdl) {
   auto kern = paged_decode_kernel<Tag, KV, G, kCheckMode, kRope>;
   static std::atomic<uint64_t> configured{0};  // bit per device
   int dev = 0;
@@ -714,17 +717,17 @@ cudaError_t launch_t(const DecodeArgs& a, int64_t n_cta, cudaStream_t stream) {
     configured.fetch_or(bit);
   }
   if (n_cta <= 0) return cudaSuccess;
-  kern<<<dim3(unsigned(n_cta)), kThreads, kSmem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_maybe_dependent(kern, dim3(unsigned(n_cta)), dim3(kThreads), kSmem, stream, pdl, a);
 }
 
 template <typename Tag, typename KV, int kCheckMode, bool kRope>
-cudaError_t dispatch_group(int group, const DecodeArgs& a, int64_t n, cudaStream_t s) {
+cudaError_t dispatch_group(int group, const DecodeArgs& a, int64_t n, cudaStream_t s,
+                           bool pdl = false) {
   switch (group) {
-    case 1: return launch_t<Tag, KV, 1, kCheckMode, kRope>(a, n, s);
-    case 2: return launch_t<Tag, KV, 2, kCheckMode, kRope>(a, n, s);
-    case 4: return launch_t<Tag, KV, 4, kCheckMode, kRope>(a, n, s);
-    case 8: return launch_t<Tag, KV, 8, kCheckMode, kRope>(a, n, s);
+    case 1: return launch_t<Tag, KV, 1, kCheckMode, kRope>(a, n, s, pdl);
+    case 2: return launch_t<Tag, KV, 2, kCheckMode, kRope>(a, n, s, pdl);
+    case 4: return launch_t<Tag, KV, 4, kCheckMode, kRope>(a, n, s, pdl);
+    case 8: return launch_t<Tag, KV, 8, kCheckMode, kRope>(a, n, s, pdl);
   }
   return cudaErrorInvalidValue;
 }

@@ -47,6 +47,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "launch.cuh"
 #include "pa_internal.h"
 #include "tcgen05.cuh"
 
@@ -926,6 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           MergeAcc acc[G];
 #pragma unroll
           for (int hh = 0; hh < G; ++hh) acc[hh].add(res[hh], lse2[hh]);
+          grid_dependency_wait();  // the prefix level has completed
           merge_prefix<G, D>(acc, a.prefix_o, a.prefix_lse, a.prefix_chunks, Bstride, row0, d);
 #pragma unroll
           for (int hh = 0; hh < G; ++hh)
@@ -959,6 +961,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       const int s0 = a.merge_indptr[seg], s1 = a.merge_indptr[seg + 1];
       MergeAcc acc[G];
       merge_partials<G, D>(acc, a.partial_o, a.partial_lse, s0, s1, d);
+      if (a.prefix_chunks > 0) grid_dependency_wait();  // the prefix level has completed
       merge_prefix<G, D>(acc, a.prefix_o, a.prefix_lse, a.prefix_chunks, Bstride, row0, d);
 #pragma unroll
       for (int hh = 0; hh < G; ++hh)
@@ -975,6 +978,8 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
 
 template <typename Tag, int KV8, int G, bool kCheck>
 cudaError_t launch_tc_t(const TcArgs& a, int64_t n_cta, cudaStream_t stream) {
+  // a cascade's decode level starts while the prefix level finishes
+  const bool pdl = a.prefix_chunks > 0;
   auto kern = paged_decode_tc_kernel<Tag, KV8, G, kCheck>;
   constexpr int kSmem = Off<KV8 != 0>::kSmemBytes;
   static std::atomic<uint64_t> configured{0};
@@ -988,8 +993,7 @@ cudaError_t launch_tc_t(const TcArgs& a, int64_t n_cta, cudaStream_t stream) {
     configured.fetch_or(bit);
   }
   if (n_cta <= 0) return cudaSuccess;
-  kern<<<dim3(unsigned(n_cta)), kThreads, kSmem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_maybe_dependent(kern, dim3(unsigned(n_cta)), dim3(kThreads), kSmem, stream, pdl, a);
 }
 
 template <typename Tag, int KV8, bool kCheck>
