@@ -37,6 +37,16 @@
 //     split into hi = bf16(p) and lo = bf16(p - hi), stored in the padding
 //     rows G..2G-1 of the N = 16 operand: the same single MMA then yields
 //     V^T hi and V^T lo in separate columns, which the epilogue adds.
+// 8-bit pools (E4M3 / E5M2 codes with a K and a V scale; README core feature
+// 3, low-precision attention for a compressed KV-cache): the MMAs are
+// kind::f8f6f4 straight on the cached codes, so a tile is 16 KB of K and 16 KB
+// of V copied as they are (a 6-stage ring, the same bytes in flight as the
+// 16-bit ring) with no conversion pass.  The 16-bit operands are split into
+// E4M3 terms, each the rounded residual of the previous ones scaled by 16:
+// q, after a per-head power-of-two scale, into 2 terms for bf16 and 3 for
+// fp16 (exact: 4 significant bits each), P into 4 terms (16 significant
+// bits).  Term k of head h is column k * G + h of S^T (resp. O^T); the
+// softmax (resp. epilogue) adds the columns back with weights 16^-k.
 // Q^T, S^T, P^T and O^T are double buffered so a CTA's next piece starts while
 // the previous one finishes.  The warps meet only on mbarriers; every wait is
 // bounded, and every parity wait targets a barrier whose previous phase the
@@ -77,11 +87,9 @@ constexpr int kBarLReady = kBarS + 16;  // piece maxima, row sums written (4 sof
 constexpr int kBarLFree = kBarS + 18;   // ... and read                (4 epilogue warps)
 constexpr int kBarPath = kBarS + 20;
 
-// 16-bit pools: a ring of kStages K/V tiles, copied straight into the layout
-// the MMA reads; full (the loaders' copies landed) / empty (PV done) pairs.
-// 8-bit pools: a ring of kRawStages raw tiles (8-bit rows, 16-byte chunks
-// swizzled by row), widened by the loader threads: K into one of two TMEM
-// buffers (the A operand of S^T), V into one of two shared-memory tiles.
+// A ring of kStages K/V tiles, copied straight into the layout the MMA reads;
+// full (the loaders' copies landed) / empty (PV done) barrier pairs.  16-bit
+// pools: 3 stages of 64 KB; 8-bit pools: 6 stages of 32 KB.
 template <bool k8> struct Lay;
 template <> struct Lay<false> {
   static constexpr int kStages = 3;
@@ -93,22 +101,14 @@ template <> struct Lay<false> {
   static constexpr uint32_t kTmemCols = 64;         // S0, S1, O0, O1: 16 columns each
 };
 template <> struct Lay<true> {
-  static constexpr int kRawStages = 3;
-  static constexpr int kVStages = 3;                // widened V tiles
-  static constexpr int kRawHalf = kTok * 128;       // 128 raw rows of 128 bytes: 16 KB
-  static constexpr int kRawStage = 2 * kRawHalf;    // K then V
-  static constexpr int kOffRaw = 0;
-  static constexpr int kOffV = kOffRaw + kRawStages * kRawStage;  // widened V tiles
-  static constexpr int kOffQ = kOffV + kVStages * kTileKV;
-  static constexpr int kBarRawFull = kBarPath;                    // copies landed (128)
-  static constexpr int kBarRawFree = kBarRawFull + kRawStages;    // stage read (128)
-  static constexpr int kBarKReady = kBarRawFree + kRawStages;     // K(t) in TMEM (4 warps)
-  static constexpr int kBarKFree = kBarKReady + 2;                // S^T(t) done (MMA commit)
-  static constexpr int kBarVReady = kBarKFree + 2;                // V(t) widened (4 warps)
-  static constexpr int kBarVFree = kBarVReady + kVStages;         // PV(t) done (MMA commit)
-  static constexpr int kNumBars = kBarVFree + kVStages;
-  static constexpr uint32_t kTmemCols = 256;  // S0, S1, O0, O1 (16 each), K0, K1 (64 each)
-  static constexpr uint32_t kColK = 64;
+  static constexpr int kStages = 6;
+  static constexpr int kTile8 = kTok * 128;        // 128 rows of 128 one-byte codes: 16 KB
+  static constexpr int kStageBytes = 2 * kTile8;   // K then V
+  static constexpr int kOffRing = 0;
+  static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+  static constexpr int kBarFull = kBarPath, kBarEmpty = kBarFull + kStages;
+  static constexpr int kNumBars = kBarEmpty + kStages;
+  static constexpr uint32_t kTmemCols = 128;       // S0, S1, O0, O1: up to 32 columns each
 };
 template <bool k8> struct Off {
   static constexpr int kOffQ = Lay<k8>::kOffQ;
@@ -116,7 +116,8 @@ template <bool k8> struct Off {
   static constexpr int kOffX = kOffP + 2 * kPBytes;     // tile maxima [2][4 warps][16]
   static constexpr int kOffL = kOffX + 2 * 4 * kN * 4;  // row sums    [2][4 warps][16]
   static constexpr int kOffM = kOffL + 2 * 4 * kN * 4;  // a piece's final maxima [2][16]
-  static constexpr int kOffBar = kOffM + 2 * kN * 4;
+  static constexpr int kOffQS = kOffM + 2 * kN * 4;     // 8-bit pools: score scale per head [2][16]
+  static constexpr int kOffBar = kOffQS + 2 * kN * 4;
   static constexpr int kSmemBytes = kOffBar + Lay<k8>::kNumBars * 8 + 16 + 1024;  // + alignment
   static_assert(kSmemBytes <= 232448, "shared memory");
   static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0,
@@ -194,6 +195,18 @@ template <> __device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+template <> __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
 template <int N> __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]);
 template <> __device__ __forceinline__ void tmem_st<1>(uint32_t taddr, const uint32_t (&r)[1]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n" ::"r"(taddr), "r"(r[0])
@@ -239,29 +252,62 @@ template <> __device__ __forceinline__ void tmem_st<32>(uint32_t taddr, const ui
       : "memory");
 }
 
-// Four 8-bit codes (little-endian in w) widened exactly to two pairs of q's
-// 16-bit type: cvt to fp16 pairs (every E4M3 / E5M2 value is an fp16 value),
-// and for bf16 through fp32 (every such value is a bf16 value too).
-template <typename Tag, int KV8>
-__device__ __forceinline__ void widen4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  if constexpr (KV8 == 1)
-    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n"
-        " cvt.rn.f16x2.e4m3x2 %1, h;\n}\n"
-        : "=r"(lo), "=r"(hi)
-        : "r"(w));
-  else
-    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e5m2x2 %0, l;\n"
-        " cvt.rn.f16x2.e5m2x2 %1, h;\n}\n"
-        : "=r"(lo), "=r"(hi)
-        : "r"(w));
-  if constexpr (Fmt<Tag>::v == 1) {
-    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-    const __nv_bfloat162 x = __floats2bfloat162_rn(a.x, a.y), y = __floats2bfloat162_rn(b.x, b.y);
-    lo = *reinterpret_cast<const uint32_t*>(&x);
-    hi = *reinterpret_cast<const uint32_t*>(&y);
+// E4M3 codes of two fp32 values (lo in the low byte); rn, saturating.
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+  uint16_t c;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(c) : "f"(hi), "f"(lo));
+  return c;
+}
+// ... of an fp16 pair.
+__device__ __forceinline__ uint16_t e4m3x2(__half2 h) {
+  uint16_t c;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;\n" : "=h"(c) : "r"(*reinterpret_cast<uint32_t*>(&h)));
+  return c;
+}
+// The values of two E4M3 codes (exact in fp16).
+__device__ __forceinline__ __half2 e4m3x2_value(uint16_t c) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(d) : "h"(c));
+  return *reinterpret_cast<__half2*>(&d);
+}
+
+// Two P values (in [0, 2^8]) as four E4M3 terms p ~ t0 + t1/16 + t2/256 +
+// t3/4096: t0 = e4m3(p); the residual (p - t0) * 16 is exact in fp32 and
+// rounded to fp16 (11 more bits, ~15 in all); t1..t3 take it apart exactly.
+__device__ __forceinline__ void split_p4(float lo, float hi, uint16_t (&t)[4]) {
+  t[0] = e4m3x2(lo, hi);
+  const float2 v = __half22float2(e4m3x2_value(t[0]));
+  __half2 r = __floats2half2_rn((lo - v.x) * 16.f, (hi - v.y) * 16.f);
+  const __half2 k16 = __float2half2_rn(16.f);
+#pragma unroll
+  for (int k = 1; k < 4; ++k) {
+    t[k] = e4m3x2(r);
+    if (k < 3) r = __hmul2(__hsub2(r, e4m3x2_value(t[k])), k16);
   }
 }
+
+// Two scaled q values as `n` E4M3 terms, each the residual of the previous
+// ones times 16, in fp32 (exact for n = 2 on bf16 and n = 3 on fp16 values
+// whose terms stay in E4M3's normal range).
+template <int n>
+__device__ __forceinline__ void split_q(float lo, float hi, uint16_t (&t)[n]) {
+#pragma unroll
+  for (int k = 0; k < n; ++k) {
+    t[k] = e4m3x2(lo, hi);
+    if (k + 1 < n) {
+      const float2 v = __half22float2(e4m3x2_value(t[k]));
+      lo = (lo - v.x) * 16.f;
+      hi = (hi - v.y) * 16.f;
+    }
+  }
+}
+
+__device__ __forceinline__ float to_f32(F16, uint16_t u) {
+  return __half2float(__ushort_as_half(u));
+}
+__device__ __forceinline__ float to_f32(BF16, uint16_t u) { return __uint_as_float(uint32_t(u) << 16); }
+
+__host__ __device__ constexpr int pow2_at_least(int x) { return x <= 1 ? 1 : 2 * pow2_at_least((x + 1) / 2); }
 
 // Byte offset of 16-byte chunk c (0..15) of row r in a 128-byte-swizzled
 // tile stored as two 64-element halves of `half_bytes` each.
@@ -286,22 +332,24 @@ __device__ __forceinline__ int next_nonempty(const pa_work_item* items, int pc, 
 template <typename Tag, int KV8, int G, bool kCheck>
 __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcArgs a) {
   constexpr bool k8 = KV8 != 0;
-  // P^T and V in the type of the PV MMA: q's type for 16-bit pools; fp16 for
-  // 8-bit pools (every code widens exactly to fp16, so V costs one conversion
-  // per pair whatever q's type).
-  using PTag = std::conditional_t<k8, F16, Tag>;
-  // Two-term P: P^T rows [0, G) hold hi = round(p), rows [G, 2G) lo =
-  // round(p - hi); O^T columns likewise, added in the epilogue.  Needed for
-  // bf16 P (8 bits), and for the fp16 P of 8-bit pools, whose scaled values
-  // can be large: 11 bits of weight would move o by up to 2^-11 |v - o|.
-  constexpr bool kSplit = k8 || Fmt<PTag>::v == 1;
+  // 16-bit pools, two-term P: P^T rows [0, G) hold hi = round(p), rows
+  // [G, 2G) lo = round(p - hi); O^T columns likewise, added in the epilogue.
+  // Needed for bf16 P (8 bits).
+  constexpr bool kSplit = !k8 && Fmt<Tag>::v == 1;
+  // 8-bit pools: E4M3 terms of q (kQT) and of P (kPT) per head.
+  constexpr int kQT = Fmt<Tag>::v == 1 ? 2 : 3, kPT = 4;
+  // columns of one S^T / O^T buffer (the MMA N)
+  constexpr int kNC = k8 ? (kPT * G <= 16 ? 16 : 32) : kN;
+  // S^T columns a softmax thread reads, O^T columns the epilogue reads
+  constexpr int kSC = k8 ? pow2_at_least(kQT * G) : G;
+  constexpr int kCols = k8 ? kPT * G : (kSplit ? 2 * G : G);
+  static_assert(kCols <= kNC && kSC <= kNC, "terms must fit the MMA N");
   using L = Lay<k8>;
   constexpr int kOffQ = Off<k8>::kOffQ, kOffP = Off<k8>::kOffP, kOffX = Off<k8>::kOffX,
-                kOffL = Off<k8>::kOffL, kOffM = Off<k8>::kOffM, kOffBar = Off<k8>::kOffBar;
+                kOffL = Off<k8>::kOffL, kOffM = Off<k8>::kOffM, kOffQS = Off<k8>::kOffQS,
+                kOffBar = Off<k8>::kOffBar;
   constexpr int kNumBars = L::kNumBars;
   constexpr uint32_t kTmemCols = L::kTmemCols;
-  constexpr int kCols = kSplit ? 2 * G : G;
-  static_assert(kCols <= kN, "hi and lo rows must fit the padded MMA N");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -313,24 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
   const int p0 = a.cta_indptr[blockIdx.x], p1 = a.cta_indptr[blockIdx.x + 1];
 
   if (threadIdx.x == 0) {
-    if constexpr (k8) {
-      for (int s = 0; s < Lay<true>::kRawStages; ++s) {
-        mbar_init(bar(Lay<true>::kBarRawFull + s), 128);
-        mbar_init(bar(Lay<true>::kBarRawFree + s), 128);
-      }
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(bar(Lay<true>::kBarKReady + b), 4);
-        mbar_init(bar(Lay<true>::kBarKFree + b), 1);
-      }
-      for (int b = 0; b < Lay<true>::kVStages; ++b) {
-        mbar_init(bar(Lay<true>::kBarVReady + b), 4);
-        mbar_init(bar(Lay<true>::kBarVFree + b), 1);
-      }
-    } else {
-      for (int s = 0; s < Lay<false>::kStages; ++s) {
-        mbar_init(bar(Lay<false>::kBarFull + s), 128);
-        mbar_init(bar(Lay<false>::kBarEmpty + s), 1);
-      }
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::kBarFull + s), 128);
+      mbar_init(bar(L::kBarEmpty + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(kBarS + b), 1);
@@ -356,158 +389,19 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
   const uint32_t tmem = *tmem_holder;
 
   if (warp >= 4 && warp < 8) {
-   if constexpr (k8) {
-    // ------------------------- loaders (8-bit pools) -------------------------
-    // Thread j copies, for every tile, the 16-byte chunk j % 8 of raw rows
-    // j / 8 + 16 k (k = 0..7) of K and V (8 lanes per 128-byte row: coalesced)
-    // into a raw stage, chunk c of row r at byte r * 128 + ((c ^ (r % 8)) * 16)
-    // so that the row-per-thread reads below are conflict-free; the stage's
-    // mbarrier counts the copies.  Then thread j widens token row j of tile t:
-    // K into TMEM lane j (64 columns, two 16-bit elements each, the A operand
-    // of S^T = K Q^T), V into the 128-byte-swizzled 16-bit tile the PV MMA
-    // reads.  Rows past a piece are zero-filled and widen to zeros.
-    using LL = Lay<true>;
-    const int j = threadIdx.x - 128;  // token row of the tile this thread widens
-    const int lw = warp - 4;
-    const int lp = a.log2_page;
-    const uint32_t pmask = (1u << lp) - 1u;
-    const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * D;
-    const int cc = j & 7, cr = j >> 3;  // copied chunk, first copied row
-    // copy walker over the tiles of the CTA's non-empty pieces
-    int pi = next_nonempty(a.items, p0, p1), tt = 0, len = 0;
-    pa_work_item it{};
-    int total = 0;
-    for (int pc = pi; pc < p1; ++pc)
-      total += (a.items[pc].token_end - a.items[pc].token_begin + kTok - 1) / kTok;
-    if (pi < p1) {
-      it = a.items[pi];
-      len = it.token_end - it.token_begin;
-    }
-    // Page of each row this thread copies, for the tile copied next: looked up
-    // a tile ahead so the copies never wait on an index load.
-    int pgn[8];
-    auto lookup = [&]() {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int pos = tt * kTok + cr + 16 * k;
-        int pg = -1;
-        if (pi < p1 && pos < len) {
-          const int idx = (it.token_begin + pos) >> lp;
-          pg = __ldg(a.kv_indices + it.page_begin + idx);
-          if (kCheck && (pg < 0 || int64_t(pg) >= a.num_pages)) {
-            atomicMin(a.error_pos, (unsigned long long)(it.page_begin + idx));
-            pg = -1;
-          }
-        }
-        pgn[k] = pg;
-      }
-    };
-    lookup();
-    auto copy_tile = [&](int c) {
-      const int s = c % LL::kRawStages;
-      const uint32_t base = sb + LL::kOffRaw + s * LL::kRawStage;
-      const uint8_t* kb = a.k_pool + int64_t(it.kv_head) * D + cc * 16;
-      const uint8_t* vb = a.v_pool + int64_t(it.kv_head) * D + cc * 16;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int r = cr + 16 * k;
-        const int pos = tt * kTok + r;
-        const int pg = pgn[k];
-        const uint32_t row = pg >= 0 ? ((uint32_t(pg) << lp) | (uint32_t(it.token_begin + pos) & pmask)) : 0u;
-        const uint32_t nbytes = pg >= 0 ? 16u : 0u;  // 0: zero-fill, nothing read
-        const uint64_t off = uint64_t(row) * pool_row_bytes;
-        const uint32_t dst = base + r * 128 + ((cc ^ (r & 7)) << 4);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst),
-                     "l"(kb + off), "r"(nbytes) : "memory");
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst + LL::kRawHalf),
-                     "l"(vb + off), "r"(nbytes) : "memory");
-      }
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(
-                       bar(LL::kBarRawFull + s)) : "memory");
-      if (++tt * kTok >= len) {  // advance the walker
-        tt = 0;
-        pi = next_nonempty(a.items, pi + 1, p1);
-        if (pi < p1) {
-          it = a.items[pi];
-          len = it.token_end - it.token_begin;
-        }
-      }
-      lookup();
-    };
-    const uint32_t lane_k = tmem + LL::kColK + (uint32_t(lw * 32) << 16);
-    bool ok = true;
-    for (int c = 0; c < LL::kRawStages - 1 && c < total; ++c) copy_tile(c);
-    for (int t = 0; ok && t < total; ++t) {
-      const int c = t + LL::kRawStages - 1;
-      if (c < total) {
-        if (c >= LL::kRawStages)  // the stage's previous tile has been read by every thread
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(LL::kBarRawFree + c % LL::kRawStages),
-                                                 ((c / LL::kRawStages) - 1) & 1));
-        if (!ok) break;
-        copy_tile(c);
-      }
-      const int s = t % LL::kRawStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(LL::kBarRawFull + s), (t / LL::kRawStages) & 1));
-      if (!ok) break;
-      const uint8_t* raw = smem + LL::kOffRaw + s * LL::kRawStage + j * 128;
-      // K row j -> TMEM lane j of buffer t & 1, once S^T(t - 2) has read it
-      {
-        uint32_t w[64];
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint4 u = *reinterpret_cast<const uint4*>(raw + ((ch ^ (j & 7)) << 4));
-          widen4<Tag, KV8>(u.x, w[8 * ch + 0], w[8 * ch + 1]);
-          widen4<Tag, KV8>(u.y, w[8 * ch + 2], w[8 * ch + 3]);
-          widen4<Tag, KV8>(u.z, w[8 * ch + 4], w[8 * ch + 5]);
-          widen4<Tag, KV8>(u.w, w[8 * ch + 6], w[8 * ch + 7]);
-        }
-        if (t >= 2) ok = mbar_wait(bar(LL::kBarKFree + (t & 1)), ((t >> 1) - 1) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc::fence_after_sync();
-        tmem_st<32>(lane_k + (t & 1) * 64, *reinterpret_cast<const uint32_t(*)[32]>(w));
-        tmem_st<32>(lane_k + (t & 1) * 64 + 32, *reinterpret_cast<const uint32_t(*)[32]>(w + 32));
-        tc::tmem_wait_st();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(LL::kBarKReady + (t & 1)));
-      }
-      // V row j -> the widened tile t & 1, once PV(t - 2) has read it
-      {
-        uint4 v[16];
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint4 u = *reinterpret_cast<const uint4*>(raw + LL::kRawHalf + ((ch ^ (j & 7)) << 4));
-          widen4<PTag, KV8>(u.x, v[2 * ch].x, v[2 * ch].y);
-          widen4<PTag, KV8>(u.y, v[2 * ch].z, v[2 * ch].w);
-          widen4<PTag, KV8>(u.z, v[2 * ch + 1].x, v[2 * ch + 1].y);
-          widen4<PTag, KV8>(u.w, v[2 * ch + 1].z, v[2 * ch + 1].w);
-        }
-        mbar_arrive(bar(LL::kBarRawFree + s));  // this thread is done with the raw stage
-        const int vs = t % LL::kVStages;
-        if (t >= LL::kVStages)
-          ok = mbar_wait(bar(LL::kBarVFree + vs), ((t / LL::kVStages) - 1) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        uint8_t* vt = smem + LL::kOffV + vs * kTileKV;
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch)
-          *reinterpret_cast<uint4*>(vt + sw_chunk(j, ch, kHalfKV)) = v[ch];
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(LL::kBarVReady + vs));
-      }
-    }
-    if (!ok) {
-      asm volatile("cp.async.wait_all;\n" ::: "memory");
-      if (lane == 0) flag_timeout(a);
-    }
-   } else {
     // ------------------------------ loaders ------------------------------
+    // A (token, kv head) row is 256 bytes (16-bit pools: a half warp per
+    // row) or 128 bytes (8-bit pools: 8 lanes per row); either way 16-byte
+    // chunks, 128-byte swizzled, so the MMA reads the tiles where they land.
     const int lw = warp - 4;
     const int lp = a.log2_page;
     const uint32_t pmask = (1u << lp) - 1u;
-    constexpr int kStages = Lay<false>::kStages, kStageBytes = Lay<false>::kStageBytes;
-    const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * D * 2;
-    const int c = lane & 15;  // 16-byte chunk of a 256-byte row
+    constexpr int kStages = L::kStages, kStageBytes = L::kStageBytes;
+    constexpr int kRowBytes = k8 ? D : 2 * D;
+    constexpr int kLanesRow = kRowBytes / 16, kRowsPer = 32 / kLanesRow;
+    constexpr int kVOff = kStageBytes / 2;  // V after K in a stage
+    const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * kRowBytes;
+    const int c = lane % kLanesRow;  // 16-byte chunk of a row
     // Page of this lane's row (32 * lw + lane) of tile tt of a piece; -1 past
     // the piece or rejected by the bounds check.
     auto page_of = [&](const pa_work_item& w, int wlen, int wtt) -> int {
@@ -536,17 +430,19 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
     bool ok = true;
     while (pi < p1) {
       const int s = t % kStages;
-      if (t >= kStages && !mbar_wait(bar(Lay<false>::kBarEmpty + s), ((t / kStages) - 1) & 1)) {
+      if (t >= kStages && !mbar_wait(bar(L::kBarEmpty + s), ((t / kStages) - 1) & 1)) {
         ok = false;
         break;
       }
-      const uint64_t kb = reinterpret_cast<uint64_t>(a.k_pool + int64_t(it.kv_head) * D * 2) + c * 16;
-      const uint64_t vb = reinterpret_cast<uint64_t>(a.v_pool + int64_t(it.kv_head) * D * 2) + c * 16;
-      const uint32_t kdst = sb + Lay<false>::kOffRing + s * kStageBytes;
-      const uint32_t vdst = kdst + kTileKV;
+      const uint64_t kb =
+          reinterpret_cast<uint64_t>(a.k_pool + int64_t(it.kv_head) * kRowBytes) + c * 16;
+      const uint64_t vb =
+          reinterpret_cast<uint64_t>(a.v_pool + int64_t(it.kv_head) * kRowBytes) + c * 16;
+      const uint32_t kdst = sb + L::kOffRing + s * kStageBytes;
+      const uint32_t vdst = kdst + kVOff;
 #pragma unroll 4
-      for (int k = 0; k < 16; ++k) {
-        const int rr = 2 * k + (lane >> 4);  // row within the warp's 32
+      for (int k = 0; k < 32 / kRowsPer; ++k) {
+        const int rr = kRowsPer * k + lane / kLanesRow;  // row within the warp's 32
         const int r = 32 * lw + rr;           // row within the tile
         const int rpg = __shfl_sync(0xffffffffu, pg, rr);
         const uint32_t pos = uint32_t(it.token_begin + tt * kTok + r);
@@ -565,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       }
       // the stage's barrier counts this thread once all its copies above land
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(
-                       bar(Lay<false>::kBarFull + s))
+                       bar(L::kBarFull + s))
                    : "memory");
       ++t;
       if (++tt * kTok >= len) {
@@ -582,20 +478,20 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       asm volatile("cp.async.wait_all;\n" ::: "memory");
       if (lane == 0) flag_timeout(a);
     }
-   }
   } else if (warp == 8) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
-      constexpr uint32_t kIdescS = tc::idesc_f16(Fmt<Tag>::v, 0, kTok, kN);
-      // O^T = V^T P^T: A = V^T (M = head elements, MN-major), B = P^T (K-major)
-      constexpr uint32_t kIdescO = tc::idesc_f16(Fmt<PTag>::v, 0, D, kN) | (1u << 15);
-      // 16-bit pools: K and V of a tile in one ring stage; 8-bit pools: K in a
-      // TMEM buffer, widened V in one of two shared-memory tiles
-      constexpr int kStages = Lay<false>::kStages, kStageBytes = Lay<false>::kStageBytes;
-      const uint64_t dk0 = tc::smem_desc_sw128(sb + Lay<false>::kOffRing, 16, 1024);
-      const uint64_t dv0 =
-          k8 ? tc::smem_desc_sw128(sb + Lay<true>::kOffV, kHalfKV, 1024)
-             : tc::smem_desc_sw128(sb + Lay<false>::kOffRing + kTileKV, kHalfKV, 1024);
+      // S^T = K Q^T: A = K (M = tokens, K-major), B = Q^T (K-major).
+      // O^T = V^T P^T: A = V^T (M = head elements, MN-major), B = P^T (K-major).
+      // 8-bit pools: A in the cached format, B in E4M3 terms.
+      constexpr uint32_t kIdescS = k8 ? tc::idesc_f8(KV8 - 1, 0, 0, 0, kTok, kNC)
+                                      : tc::idesc_f16(Fmt<Tag>::v, 0, kTok, kN);
+      constexpr uint32_t kIdescO = k8 ? tc::idesc_f8(KV8 - 1, 0, 1, 0, D, kNC)
+                                      : tc::idesc_f16(Fmt<Tag>::v, 0, D, kN) | (1u << 15);
+      constexpr int kStages = L::kStages, kStageBytes = L::kStageBytes;
+      const uint64_t dk0 = tc::smem_desc_sw128(sb + L::kOffRing, 16, 1024);
+      // 16-bit V: two 64-element halves along M (16 KB apart); 8-bit V: one
+      const uint64_t dv0 = tc::smem_desc_sw128(sb + L::kOffRing + kStageBytes / 2, kHalfKV, 1024);
       const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
       const uint64_t dp0 = tc::smem_desc_sw128(sb + kOffP, 16, 1024);
       // S^T(ts) and PV(tv) walk the pieces in step with their counters
@@ -612,8 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       while (v_piece < p1) {
         bool progress = false;
         auto k_ready = [&]() {
-          return k8 ? mbar_test_wait(bar(Lay<true>::kBarKReady + (ts & 1)), (ts >> 1) & 1)
-                    : mbar_test_wait(bar(Lay<false>::kBarFull + ts % kStages), (ts / kStages) & 1);
+          return mbar_test_wait(bar(L::kBarFull + ts % kStages), (ts / kStages) & 1);
         };
         if (s_piece < p1 &&
             (ts < 2 || mbar_test_wait(bar(kBarSFree + (ts & 1)), ((ts - 2) >> 1) & 1)) &&
@@ -621,22 +516,18 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           fence_proxy_async_smem();  // the loaders' cp.async writes, seen by the tensor core
           tc::fence_after_sync();
           const uint64_t qd = dq0 + uint64_t(((s_np & 1) * kQBytes) >> 4);
+          const uint64_t kd = dk0 + uint64_t(((ts % kStages) * kStageBytes) >> 4);
           if constexpr (k8) {
-            // A = K from TMEM (lane = token, 8 columns per 16 head elements)
-            const uint32_t ka = tmem + Lay<true>::kColK + (ts & 1) * 64;
+            // 32 one-byte elements (32 bytes of each 128-byte row) per step
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
-              tc::mma_f16_ts(tmem + (ts & 1) * kN, ka + kk * 8, qd + qoff, kIdescS, kk > 0);
-            }
-            tc::commit(bar(Lay<true>::kBarKFree + (ts & 1)));
+            for (int kk = 0; kk < D / 32; ++kk)
+              tc::mma_f8_ss(tmem + (ts & 1) * kNC, kd + kk * 2, qd + kk * 2, kIdescS, kk > 0);
           } else {
-            const uint64_t kd = dk0 + uint64_t(((ts % kStages) * kStageBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t koff = ((kk >> 2) * kHalfKV + (kk & 3) * 32) >> 4;
               const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
-              tc::mma_f16_ss(tmem + (ts & 1) * kN, kd + koff, qd + qoff, kIdescS, kk > 0);
+              tc::mma_f16_ss(tmem + (ts & 1) * kNC, kd + koff, qd + qoff, kIdescS, kk > 0);
             }
           }
           tc::commit(bar(kBarS + (ts & 1)));
@@ -650,24 +541,28 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           progress = true;
         }
         if (tv < ts && mbar_test_wait(bar(kBarPReady + (tv & 1)), (tv >> 1) & 1) &&
-            (!k8 || mbar_test_wait(bar(Lay<true>::kBarVReady + tv % Lay<true>::kVStages),
-                                   (tv / Lay<true>::kVStages) & 1)) &&
             (v_tile > 0 || v_np < 2 ||
              mbar_test_wait(bar(kBarOFree + (v_np & 1)), ((v_np - 2) >> 1) & 1))) {
           tc::fence_after_sync();
-          const uint64_t vd = k8 ? dv0 + uint64_t(((tv % Lay<true>::kVStages) * kTileKV) >> 4)
-                                 : dv0 + uint64_t(((tv % kStages) * kStageBytes) >> 4);
+          const uint64_t vd = dv0 + uint64_t(((tv % kStages) * kStageBytes) >> 4);
           const uint64_t pd = dp0 + uint64_t(((tv & 1) * kPBytes) >> 4);
-          const uint32_t od = tmem + 2 * kN + (v_np & 1) * kN;
+          const uint32_t od = tmem + 2 * kNC + (v_np & 1) * kNC;
+          if constexpr (k8) {
 #pragma unroll
-          for (int kk = 0; kk < kTok / 16; ++kk) {
-            const uint32_t voff = (kk * 16 * 128) >> 4;  // 16 token rows
-            const uint32_t poff = ((kk >> 2) * kPHalf + (kk & 3) * 32) >> 4;
-            tc::mma_f16_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kTok / 32; ++kk) {
+              const uint32_t voff = (kk * 32 * 128) >> 4;  // 32 token rows
+              tc::mma_f8_ss(od, vd + voff, pd + kk * 2, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kTok / 16; ++kk) {
+              const uint32_t voff = (kk * 16 * 128) >> 4;  // 16 token rows
+              const uint32_t poff = ((kk >> 2) * kPHalf + (kk & 3) * 32) >> 4;
+              tc::mma_f16_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           tc::commit(bar(kBarPFree + (tv & 1)));
-          if constexpr (k8) tc::commit(bar(Lay<true>::kBarVFree + tv % Lay<true>::kVStages));
-          else tc::commit(bar(Lay<false>::kBarEmpty + tv % kStages));
+          tc::commit(bar(L::kBarEmpty + tv % kStages));
           ++tv;
           if (++v_tile == v_ntiles) {
             tc::commit(bar(kBarODone + (v_np & 1)));
@@ -693,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
     float* xmax = reinterpret_cast<float*>(smem + kOffX);  // [2][4][kN]
     float* xsum = reinterpret_cast<float*>(smem + kOffL);  // [2][4][kN]
     float* xm_piece = reinterpret_cast<float*>(smem + kOffM);  // [2][kN]
+    const float* qscale = reinterpret_cast<const float*>(smem + kOffQS);  // [2][kN]
     // P^T rows past the used ones stay zero for the whole kernel
     for (int e = i; e < 2 * kPBytes / 16; e += 128)
       reinterpret_cast<uint4*>(smem + kOffP)[e] = make_uint4(0, 0, 0, 0);
@@ -703,11 +599,19 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       const int len = it.token_end - it.token_begin;
       const int ntiles = (len + kTok - 1) / kTok;
       if (ntiles == 0) continue;  // the epilogue warps write its (0, -inf)
-      float m[G], lsum[G];
+      float m[G], lsum[G], scl[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
         m[hh] = -INFINITY;
         lsum[hh] = 0.f;
+        scl[hh] = a.score_scale;
+      }
+      if constexpr (k8) {
+        // the per-head scale of q's terms comes with the piece's Q^T
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarQReady + (np & 1)), (np >> 1) & 1));
+        if (!ok) break;
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) scl[hh] = qscale[(np & 1) * kN + hh];
       }
       for (int tt = 0; tt < ntiles; ++tt, ++t) {
         const int sbuf = t & 1;
@@ -716,11 +620,20 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
         tc::fence_after_sync();
         float sv[G];
         {
-          uint32_t r[G];
-          tmem_ld<G>(lane_addr + sbuf * kN, r);
+          uint32_t r[kSC];
+          tmem_ld<kSC>(lane_addr + sbuf * kNC, r);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) sv[hh] = __uint_as_float(r[hh]);
+          for (int hh = 0; hh < G; ++hh) {
+            if constexpr (k8) {  // q's terms: sum_k S^T(k G + h) / 16^k
+              float x = __uint_as_float(r[(kQT - 1) * G + hh]);
+#pragma unroll
+              for (int k = kQT - 2; k >= 0; --k) x = fmaf(x, 0.0625f, __uint_as_float(r[k * G + hh]));
+              sv[hh] = x;
+            } else {
+              sv[hh] = __uint_as_float(r[hh]);
+            }
+          }
         }
         tc::fence_before_sync();
         __syncwarp();
@@ -744,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
         for (int hh = 0; hh < G; ++hh) {
           const float tmax =
               fmaxf(fmaxf(xm[hh], xm[kN + hh]), fmaxf(xm[2 * kN + hh], xm[3 * kN + hh])) *
-              a.score_scale;
+              scl[hh];
           alpha[hh] = 1.f;
           mn[hh] = m[hh];
           if (tmax > m[hh] + kSlack) {
@@ -760,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
                           mbar_wait(bar(kBarPFree + ((t - 1) & 1)), ((t - 1) >> 1) & 1));
           if (!ok) break;
           tc::fence_after_sync();
-          const uint32_t oaddr = lane_addr + 2 * kN + (np & 1) * kN;
+          const uint32_t oaddr = lane_addr + 2 * kNC + (np & 1) * kNC;
           uint32_t r[kCols];
           tmem_ld<kCols>(oaddr, r);
           tc::tmem_wait_ld();
@@ -775,22 +688,48 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarPFree + sbuf), ((t - 2) >> 1) & 1));
           if (!ok) break;
         }
-        uint8_t* pt = smem + kOffP + sbuf * kPBytes + (i >> 6) * kPHalf + (i & 7) * 2;
-        const int pc = (i >> 3) & 7;  // 16-byte chunk of the token within its 128-byte row
+        if constexpr (k8) {
+          // P^T row k G + h holds term k of head h, one byte per token
+          uint8_t* pt = smem + kOffP + sbuf * kPBytes + (i & 15);
+          const int pc = i >> 4;  // 16-byte chunk of the token within its 128-byte row
+          float p[G];
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          const float p = valid ? fast_exp2(fmaf(sv[hh], a.score_scale, -mn[hh])) : 0.f;
-          float pr;
-          const uint16_t bits = round16(PTag{}, p, pr);
-          *reinterpret_cast<uint16_t*>(pt + hh * 128 + ((pc ^ (hh & 7)) << 4)) = bits;
-          if constexpr (kSplit) {  // p - hi is exact in fp32
-            float lo;
-            const uint16_t lbits = round16(PTag{}, p - pr, lo);
-            *reinterpret_cast<uint16_t*>(pt + (G + hh) * 128 + ((pc ^ ((G + hh) & 7)) << 4)) = lbits;
-            pr += lo;
+          for (int hh = 0; hh < G; ++hh) {
+            p[hh] = valid ? fast_exp2(fmaf(sv[hh], scl[hh], -mn[hh])) : 0.f;
+            // the MMA's weights agree with p to ~2^-15: the row sums take p
+            lsum[hh] = fmaf(lsum[hh], alpha[hh], p[hh]);
+            m[hh] = mn[hh];
           }
-          lsum[hh] = fmaf(lsum[hh], alpha[hh], pr);
-          m[hh] = mn[hh];
+#pragma unroll
+          for (int hh = 0; hh < G; hh += 2) {
+            uint16_t tm[kPT];
+            split_p4(p[hh], hh + 1 < G ? p[hh + 1] : 0.f, tm);
+#pragma unroll
+            for (int k = 0; k < kPT; ++k) {
+              const int n = k * G + hh;
+              pt[n * 128 + ((pc ^ (n & 7)) << 4)] = uint8_t(tm[k]);
+              if (hh + 1 < G) pt[(n + 1) * 128 + ((pc ^ ((n + 1) & 7)) << 4)] = uint8_t(tm[k] >> 8);
+            }
+          }
+        } else {
+          uint8_t* pt = smem + kOffP + sbuf * kPBytes + (i >> 6) * kPHalf + (i & 7) * 2;
+          const int pc = (i >> 3) & 7;  // 16-byte chunk of the token within its 128-byte row
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            const float p = valid ? fast_exp2(fmaf(sv[hh], scl[hh], -mn[hh])) : 0.f;
+            float pr;
+            const uint16_t bits = round16(Tag{}, p, pr);
+            *reinterpret_cast<uint16_t*>(pt + hh * 128 + ((pc ^ (hh & 7)) << 4)) = bits;
+            if constexpr (kSplit) {  // p - hi is exact in fp32
+              float lo;
+              const uint16_t lbits = round16(Tag{}, p - pr, lo);
+              *reinterpret_cast<uint16_t*>(pt + (G + hh) * 128 + ((pc ^ ((G + hh) & 7)) << 4)) =
+                  lbits;
+              pr += lo;
+            }
+            lsum[hh] = fmaf(lsum[hh], alpha[hh], pr);
+            m[hh] = mn[hh];
+          }
         }
         fence_proxy_async_smem();
         tc::fence_before_sync();
@@ -841,17 +780,68 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
                      : make_uint4(0, 0, 0, 0);
       }
     };
+    float* qscale = reinterpret_cast<float*>(smem + kOffQS);  // [2][kN]
     auto store_q = [&](const uint4 (&v)[2], int np) {
+      if constexpr (k8) {
+        // Row r = j / 16 (a head, r < G), elements 8 (j % 16) .. + 7: scaled by
+        // 2^e so that the row's largest magnitude lies in [128, 256) (E4M3
+        // reaches 448), then split into kQT terms, term k to Q^T row k G + r.
+        const int r = j >> 4, ch = j & 15;
+        const uint16_t* u = reinterpret_cast<const uint16_t*>(&v[0]);
+        float x[8], mx = 0.f;
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int e = j + 128 * k;
-        *reinterpret_cast<uint4*>(smem + kOffQ + (np & 1) * kQBytes +
-                                  sw_chunk(e >> 4, e & 15, kHalfQ)) = v[k];
+        for (int e = 0; e < 8; ++e) {
+          x[e] = to_f32(Tag{}, u[e]);
+          mx = fmaxf(mx, fabsf(x[e]));
+        }
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const int ex = mx > 0.f ? min(134 - int((__float_as_uint(mx) >> 23) & 0xff), 126) : 0;
+        const float up = __int_as_float((127 + ex) << 23), down = __int_as_float((127 - ex) << 23);
+        if (r < G) {
+          uint32_t w[kQT][2];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            uint16_t tq[kQT];
+            split_q<kQT>(x[e] * up, x[e + 1] * up, tq);
+#pragma unroll
+            for (int k = 0; k < kQT; ++k) {
+              const uint32_t sh = 16 * ((e >> 1) & 1);
+              if ((e & 2) == 0) w[k][e >> 2] = uint32_t(tq[k]);
+              else w[k][e >> 2] |= uint32_t(tq[k]) << sh;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kQT; ++k) {
+            const int n = k * G + r;
+            *reinterpret_cast<uint2*>(smem + kOffQ + (np & 1) * kQBytes + n * 128 +
+                                      ((((ch >> 1) ^ (n & 7))) << 4) + (ch & 1) * 8) =
+                make_uint2(w[k][0], w[k][1]);
+          }
+          if (ch == 0) qscale[(np & 1) * kN + r] = down * a.score_scale;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int e = j + 128 * k;
+          *reinterpret_cast<uint4*>(smem + kOffQ + (np & 1) * kQBytes +
+                                    sw_chunk(e >> 4, e & 15, kHalfQ)) = v[k];
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarQReady + (np & 1)));
     };
+    if constexpr (k8) {
+      // Q^T rows past the terms stay zero for the whole kernel (rows below
+      // are rewritten in full for every piece)
+      for (int e = j; e < 2 * kNC * 8; e += 128) {
+        const int n = (e >> 3) % kNC;
+        if (n >= kQT * G)
+          *reinterpret_cast<uint4*>(smem + kOffQ + (e / (kNC * 8)) * kQBytes + n * 128 +
+                                    (e & 7) * 16) = make_uint4(0, 0, 0, 0);
+      }
+    }
     {
       const int pc = next_nonempty(a.items, p0, p1);
       if (pc < p1) {
@@ -894,7 +884,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
         if (!ok) break;
         tc::fence_after_sync();
         uint32_t r[kCols];
-        tmem_ld<kCols>(lane_addr + 2 * kN + (np & 1) * kN, r);
+        tmem_ld<kCols>(lane_addr + 2 * kNC + (np & 1) * kNC, r);
         tc::tmem_wait_ld();
         tc::fence_before_sync();
         __syncwarp();
@@ -903,8 +893,15 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
         if (pnn < p1) store_q(qn, np + 2);
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
-          const float acc = kSplit ? __uint_as_float(r[hh]) + __uint_as_float(r[(G + hh) % kCols])
-                                   : __uint_as_float(r[hh]);
+          float acc;
+          if constexpr (k8) {  // P's terms: sum_k O^T(k G + h) / 16^k
+            acc = __uint_as_float(r[(kPT - 1) * G + hh]);
+#pragma unroll
+            for (int k = kPT - 2; k >= 0; --k) acc = fmaf(acc, 0.0625f, __uint_as_float(r[k * G + hh]));
+          } else {
+            acc = kSplit ? __uint_as_float(r[hh]) + __uint_as_float(r[(G + hh) % kCols])
+                         : __uint_as_float(r[hh]);
+          }
           res[hh] = acc / l[hh];
           if constexpr (k8) res[hh] *= a.v_scale;  // cached value = v_scale * code
           lse2[hh] = m[hh] + fast_log2(l[hh]);

@@ -26,6 +26,26 @@ __host__ __device__ constexpr uint32_t idesc_f16(int ab_format, int b_mn_major, 
          (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
+// ---- instruction descriptor for kind::f8f6f4 with fp32 accumulation -------
+// The same fields; formats 0 = E4M3, 1 = E5M2 (the two 8-bit formats for
+// which an MN-major operand is allowed).  One instruction covers K = 32.
+__host__ __device__ constexpr uint32_t idesc_f8(int a_format, int b_format, int a_mn_major,
+                                                int b_mn_major, int M, int N) {
+  return (1u << 4) | (uint32_t(a_format) << 7) | (uint32_t(b_format) << 10) |
+         (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) |
+         (uint32_t(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem] on 8-bit operands, issued by one thread.
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem], issued by one thread.
 __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {
