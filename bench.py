@@ -94,7 +94,7 @@ def workload_config(w):
     lens = w.kv_lens()
     cfg = {"workload": w.name, "batch": w.batch, "num_qo_heads": w.num_qo_heads,
            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "page_size": w.page_size,
-           "kv_dtype": w.dtype, "accumulate": "f32",
+           "q_dtype": w.dtype, "kv_dtype": w.kv_dtype or w.dtype, "accumulate": "f32",
            "kv_len": (int(lens[0]) if len(set(lens.tolist())) == 1 else
                       {"min": int(lens.min()), "max": int(lens.max()), "sum": int(lens.sum())}),
            "pool_pages": w.num_pages, "kv_bytes_per_step": w.kv_bytes(),
@@ -799,7 +799,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "us_per_step": ms * 1e3, "pct_of_peak": 100.0 * achieved / peak,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.dtype, "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))",
+            "dtype": w.kv_dtype or w.dtype,
+            "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))",
             "config": dict(workload_config(w), parallelism=f"replicas x{world}"),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
