@@ -88,8 +88,9 @@ constexpr int kBarLFree = kBarS + 18;   // ... and read                (4 epilog
 constexpr int kBarPath = kBarS + 20;
 
 // A ring of kStages K/V tiles, copied straight into the layout the MMA reads;
-// full (the loaders' copies landed) / empty (PV done) barrier pairs.  16-bit
-// pools: 3 stages of 64 KB; 8-bit pools: 6 stages of 32 KB.
+// full (the loaders' copies landed) / empty (PV done) barrier pairs: 3 stages
+// of 64 KB, 128-token tiles of 16-bit K/V or 256-token tiles of 8-bit codes
+// (the softmax then pays its per-tile costs once per 64 KB either way).
 template <bool k8> struct Lay;
 template <> struct Lay<false> {
   static constexpr int kStages = 3;
@@ -101,19 +102,22 @@ template <> struct Lay<false> {
   static constexpr uint32_t kTmemCols = 64;         // S0, S1, O0, O1: 16 columns each
 };
 template <> struct Lay<true> {
-  static constexpr int kStages = 6;
-  static constexpr int kTile8 = kTok * 128;        // 128 rows of 128 one-byte codes: 16 KB
+  static constexpr int kStages = 3;
+  static constexpr int kTile8 = 2 * kTok * 128;    // 256 rows of 128 one-byte codes: 32 KB
   static constexpr int kStageBytes = 2 * kTile8;   // K then V
   static constexpr int kOffRing = 0;
   static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
   static constexpr int kBarFull = kBarPath, kBarEmpty = kBarFull + kStages;
   static constexpr int kNumBars = kBarEmpty + kStages;
-  static constexpr uint32_t kTmemCols = 128;       // S0, S1, O0, O1: up to 32 columns each
+  // S0, S1 (two 128-token halves each), O0, O1: up to 32 columns each
+  static constexpr uint32_t kTmemCols = 256;
 };
 template <bool k8> struct Off {
   static constexpr int kOffQ = Lay<k8>::kOffQ;
   static constexpr int kOffP = kOffQ + 2 * kQBytes;
-  static constexpr int kOffX = kOffP + 2 * kPBytes;     // tile maxima [2][4 warps][16]
+  // a P^T buffer: 16 x 128 16-bit, or up to 32 x 256 one-byte terms
+  static constexpr int kPB = k8 ? 2 * 32 * 128 : kPBytes;
+  static constexpr int kOffX = kOffP + 2 * kPB;         // tile maxima [2][4 warps][16]
   static constexpr int kOffL = kOffX + 2 * 4 * kN * 4;  // row sums    [2][4 warps][16]
   static constexpr int kOffM = kOffL + 2 * 4 * kN * 4;  // a piece's final maxima [2][16]
   static constexpr int kOffQS = kOffM + 2 * kN * 4;     // 8-bit pools: score scale per head [2][16]
@@ -344,6 +348,11 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
   constexpr int kSC = k8 ? pow2_at_least(kQT * G) : G;
   constexpr int kCols = k8 ? kPT * G : (kSplit ? 2 * G : G);
   static_assert(kCols <= kNC && kSC <= kNC, "terms must fit the MMA N");
+  // tokens per tile: 128-token halves, each one S^T MMA (M = 128, a TMEM lane
+  // per token) and each handled by the same softmax thread
+  constexpr int kHalves = k8 ? 2 : 1, kTT = kHalves * kTok;
+  constexpr int kColO = 2 * kHalves * kNC;  // O^T buffers after the S^T buffers
+  constexpr int kPB = Off<k8>::kPB;
   using L = Lay<k8>;
   constexpr int kOffQ = Off<k8>::kOffQ, kOffP = Off<k8>::kOffP, kOffX = Off<k8>::kOffX,
                 kOffL = Off<k8>::kOffL, kOffM = Off<k8>::kOffM, kOffQS = Off<k8>::kOffQS,
@@ -402,10 +411,13 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
     constexpr int kVOff = kStageBytes / 2;  // V after K in a stage
     const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * kRowBytes;
     const int c = lane % kLanesRow;  // 16-byte chunk of a row
-    // Page of this lane's row (32 * lw + lane) of tile tt of a piece; -1 past
-    // the piece or rejected by the bounds check.
-    auto page_of = [&](const pa_work_item& w, int wlen, int wtt) -> int {
-      const int mypos = wtt * kTok + 32 * lw + lane;
+    // Page of this lane's row (128 h + 32 lw + lane) of tile tt of a piece;
+    // -1 past the piece or rejected by the bounds check.
+    struct Pg {
+      int v[kHalves];
+    };
+    auto page_of = [&](const pa_work_item& w, int wlen, int wtt, int h) -> int {
+      const int mypos = wtt * kTT + kTok * h + 32 * lw + lane;
       if (mypos >= wlen) return -1;
       const int idx = (w.token_begin + mypos) >> lp;
       int pg = __ldg(a.kv_indices + w.page_begin + idx);
@@ -415,9 +427,12 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       }
       return pg;
     };
-    // One walk over the tiles of the CTA's non-empty pieces.  The next tile's
-    // page indices are fetched before waiting for its stage, so the lookup
-    // overlaps the wait.
+    // One walk over the tiles of the CTA's non-empty pieces.  Page indices
+    // are looked up three tiles ahead by a second walker: at the rate the
+    // ring drains, an index load issued one tile ahead (a dependent load of
+    // ~1 us under full HBM traffic) would set the pace.  The three lookups
+    // in flight live in registers whose roles rotate by name (pg0..pg2), so
+    // no register move waits on a pending load.
     int pi = next_nonempty(a.items, p0, p1);
     pa_work_item it{};
     int len = 0, tt = 0;
@@ -425,14 +440,33 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       it = a.items[pi];
       len = it.token_end - it.token_begin;
     }
-    int pg = pi < p1 ? page_of(it, len, 0) : -1;
+    int lpi = pi, ltt = 0, llen = len;
+    pa_work_item lit = it;
+    auto look = [&]() -> Pg {  // this lane's pages of the lookahead tile, then advance
+      Pg r;
+#pragma unroll
+      for (int h = 0; h < kHalves; ++h) r.v[h] = lpi < p1 ? page_of(lit, llen, ltt, h) : -1;
+      if (lpi >= p1) return r;
+      if (++ltt * kTT >= llen) {
+        ltt = 0;
+        lpi = next_nonempty(a.items, lpi + 1, p1);
+        if (lpi < p1) {
+          lit = a.items[lpi];
+          llen = lit.token_end - lit.token_begin;
+        }
+      }
+      return r;
+    };
+    Pg pg0 = look(), pg1 = look(), pg2 = look();
     int t = 0;
     bool ok = true;
-    while (pi < p1) {
+    // copies tile t with the page indices in pg, then reloads pg three tiles on
+    auto step = [&](Pg& pg) -> bool {
+      if (pi >= p1) return false;
       const int s = t % kStages;
       if (t >= kStages && !mbar_wait(bar(L::kBarEmpty + s), ((t / kStages) - 1) & 1)) {
         ok = false;
-        break;
+        return false;
       }
       const uint64_t kb =
           reinterpret_cast<uint64_t>(a.k_pool + int64_t(it.kv_head) * kRowBytes) + c * 16;
@@ -440,31 +474,36 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           reinterpret_cast<uint64_t>(a.v_pool + int64_t(it.kv_head) * kRowBytes) + c * 16;
       const uint32_t kdst = sb + L::kOffRing + s * kStageBytes;
       const uint32_t vdst = kdst + kVOff;
+#pragma unroll
+      for (int h = 0; h < kHalves; ++h) {
+        const int pgh = pg.v[h];
 #pragma unroll 4
-      for (int k = 0; k < 32 / kRowsPer; ++k) {
-        const int rr = kRowsPer * k + lane / kLanesRow;  // row within the warp's 32
-        const int r = 32 * lw + rr;           // row within the tile
-        const int rpg = __shfl_sync(0xffffffffu, pg, rr);
-        const uint32_t pos = uint32_t(it.token_begin + tt * kTok + r);
-        const uint32_t row = rpg >= 0 ? ((uint32_t(rpg) << lp) | (pos & pmask)) : 0u;
-        const uint32_t nbytes = rpg >= 0 ? 16u : 0u;  // 0: zero-fill, nothing read
-        uint64_t ka, va;
-        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(ka) : "r"(row), "r"(pool_row_bytes), "l"(kb));
-        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(va) : "r"(row), "r"(pool_row_bytes), "l"(vb));
-        const uint32_t off = sw_chunk(r, c, kHalfKV);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(kdst + off),
-                     "l"(ka), "r"(nbytes)
-                     : "memory");
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(vdst + off),
-                     "l"(va), "r"(nbytes)
-                     : "memory");
+        for (int k = 0; k < 32 / kRowsPer; ++k) {
+          const int rr = kRowsPer * k + lane / kLanesRow;  // row within the warp's 32
+          const int r = kTok * h + 32 * lw + rr;            // row within the tile
+          const int rpg = __shfl_sync(0xffffffffu, pgh, rr);
+          const uint32_t pos = uint32_t(it.token_begin + tt * kTT + r);
+          const uint32_t row = rpg >= 0 ? ((uint32_t(rpg) << lp) | (pos & pmask)) : 0u;
+          const uint32_t nbytes = rpg >= 0 ? 16u : 0u;  // 0: zero-fill, nothing read
+          uint64_t ka, va;
+          asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(ka) : "r"(row), "r"(pool_row_bytes), "l"(kb));
+          asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(va) : "r"(row), "r"(pool_row_bytes), "l"(vb));
+          const uint32_t off = sw_chunk(r, c, kHalfKV);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(kdst + off),
+                       "l"(ka), "r"(nbytes)
+                       : "memory");
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(vdst + off),
+                       "l"(va), "r"(nbytes)
+                       : "memory");
+        }
       }
       // the stage's barrier counts this thread once all its copies above land
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(
                        bar(L::kBarFull + s))
                    : "memory");
+      pg = look();
       ++t;
-      if (++tt * kTok >= len) {
+      if (++tt * kTT >= len) {
         tt = 0;
         pi = next_nonempty(a.items, pi + 1, p1);
         if (pi < p1) {
@@ -472,7 +511,9 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           len = it.token_end - it.token_begin;
         }
       }
-      if (pi < p1) pg = page_of(it, len, tt);
+      return true;
+    };
+    while (step(pg0) && step(pg1) && step(pg2)) {
     }
     if (!ok) {
       asm volatile("cp.async.wait_all;\n" ::: "memory");
@@ -498,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       int s_piece = next_nonempty(a.items, p0, p1), s_tile = 0, s_np = 0;
       int v_piece = s_piece, v_tile = 0, v_np = 0;
       auto ntiles_of = [&](int pc) {
-        return (a.items[pc].token_end - a.items[pc].token_begin + kTok - 1) / kTok;
+        return (a.items[pc].token_end - a.items[pc].token_begin + kTT - 1) / kTT;
       };
       int s_ntiles = s_piece < p1 ? ntiles_of(s_piece) : 0;
       int v_ntiles = s_ntiles;
@@ -518,10 +559,16 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           const uint64_t qd = dq0 + uint64_t(((s_np & 1) * kQBytes) >> 4);
           const uint64_t kd = dk0 + uint64_t(((ts % kStages) * kStageBytes) >> 4);
           if constexpr (k8) {
-            // 32 one-byte elements (32 bytes of each 128-byte row) per step
+            // per 128-token half; 32 one-byte elements (32 bytes of each
+            // 128-byte row) per step
 #pragma unroll
-            for (int kk = 0; kk < D / 32; ++kk)
-              tc::mma_f8_ss(tmem + (ts & 1) * kNC, kd + kk * 2, qd + kk * 2, kIdescS, kk > 0);
+            for (int h = 0; h < kHalves; ++h) {
+              const uint32_t sd = tmem + ((ts & 1) * kHalves + h) * kNC;
+              const uint64_t kh = kd + uint64_t((h * kTok * 128) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < D / 32; ++kk)
+                tc::mma_f8_ss(sd, kh + kk * 2, qd + kk * 2, kIdescS, kk > 0);
+            }
           } else {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -545,13 +592,16 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
              mbar_test_wait(bar(kBarOFree + (v_np & 1)), ((v_np - 2) >> 1) & 1))) {
           tc::fence_after_sync();
           const uint64_t vd = dv0 + uint64_t(((tv % kStages) * kStageBytes) >> 4);
-          const uint64_t pd = dp0 + uint64_t(((tv & 1) * kPBytes) >> 4);
-          const uint32_t od = tmem + 2 * kNC + (v_np & 1) * kNC;
+          const uint64_t pd = dp0 + uint64_t(((tv & 1) * kPB) >> 4);
+          const uint32_t od = tmem + kColO + (v_np & 1) * kNC;
           if constexpr (k8) {
+            // 32 tokens per step; P^T holds each 128-token half as kNC rows of
+            // 128 bytes
 #pragma unroll
-            for (int kk = 0; kk < kTok / 32; ++kk) {
+            for (int kk = 0; kk < kTT / 32; ++kk) {
               const uint32_t voff = (kk * 32 * 128) >> 4;  // 32 token rows
-              tc::mma_f8_ss(od, vd + voff, pd + kk * 2, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
+              const uint32_t poff = ((kk >> 2) * kNC * 128 + (kk & 3) * 32) >> 4;
+              tc::mma_f8_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
             }
           } else {
 #pragma unroll
@@ -590,14 +640,14 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
     float* xm_piece = reinterpret_cast<float*>(smem + kOffM);  // [2][kN]
     const float* qscale = reinterpret_cast<const float*>(smem + kOffQS);  // [2][kN]
     // P^T rows past the used ones stay zero for the whole kernel
-    for (int e = i; e < 2 * kPBytes / 16; e += 128)
+    for (int e = i; e < 2 * kPB / 16; e += 128)
       reinterpret_cast<uint4*>(smem + kOffP)[e] = make_uint4(0, 0, 0, 0);
     int t = 0, np = 0;
     bool ok = true;
     for (int pi = p0; ok && pi < p1; ++pi) {
       const pa_work_item it = a.items[pi];
       const int len = it.token_end - it.token_begin;
-      const int ntiles = (len + kTok - 1) / kTok;
+      const int ntiles = (len + kTT - 1) / kTT;
       if (ntiles == 0) continue;  // the epilogue warps write its (0, -inf)
       float m[G], lsum[G], scl[G];
 #pragma unroll
@@ -618,10 +668,12 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
         ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarS + sbuf), (t >> 1) & 1));
         if (!ok) break;
         tc::fence_after_sync();
-        float sv[G];
-        {
+        float sv[kHalves][G];
+        bool valid[kHalves];
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h) {
           uint32_t r[kSC];
-          tmem_ld<kSC>(lane_addr + sbuf * kNC, r);
+          tmem_ld<kSC>(lane_addr + (sbuf * kHalves + h) * kNC, r);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int hh = 0; hh < G; ++hh) {
@@ -629,21 +681,23 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
               float x = __uint_as_float(r[(kQT - 1) * G + hh]);
 #pragma unroll
               for (int k = kQT - 2; k >= 0; --k) x = fmaf(x, 0.0625f, __uint_as_float(r[k * G + hh]));
-              sv[hh] = x;
+              sv[h][hh] = x;
             } else {
-              sv[hh] = __uint_as_float(r[hh]);
+              sv[h][hh] = __uint_as_float(r[hh]);
             }
           }
+          valid[h] = tt * kTT + kTok * h + i < len;
         }
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kBarSFree + sbuf));
-        const bool valid = tt * kTok + i < len;
-        // tile maximum per head over the 128 tokens: shuffles, then the 4 warps
+        // tile maximum per head over the tile's tokens: shuffles, then the 4 warps
         float* xm = xmax + sbuf * 4 * kN;
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
-          float v = valid ? sv[hh] : -INFINITY;
+          float v = valid[0] ? sv[0][hh] : -INFINITY;
+#pragma unroll
+          for (int h = 1; h < kHalves; ++h) v = fmaxf(v, valid[h] ? sv[h][hh] : -INFINITY);
 #pragma unroll
           for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
           if (lane == 0) xm[warp * kN + hh] = v;
@@ -673,7 +727,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
                           mbar_wait(bar(kBarPFree + ((t - 1) & 1)), ((t - 1) >> 1) & 1));
           if (!ok) break;
           tc::fence_after_sync();
-          const uint32_t oaddr = lane_addr + 2 * kNC + (np & 1) * kNC;
+          const uint32_t oaddr = lane_addr + kColO + (np & 1) * kNC;
           uint32_t r[kCols];
           tmem_ld<kCols>(oaddr, r);
           tc::tmem_wait_ld();
@@ -689,34 +743,43 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           if (!ok) break;
         }
         if constexpr (k8) {
-          // P^T row k G + h holds term k of head h, one byte per token
-          uint8_t* pt = smem + kOffP + sbuf * kPBytes + (i & 15);
+          // P^T row k G + h of half j holds term k of head h, one byte per token
           const int pc = i >> 4;  // 16-byte chunk of the token within its 128-byte row
-          float p[G];
+          float p[kHalves][G];
 #pragma unroll
           for (int hh = 0; hh < G; ++hh) {
-            p[hh] = valid ? fast_exp2(fmaf(sv[hh], scl[hh], -mn[hh])) : 0.f;
+            float ps = 0.f;
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h) {
+              p[h][hh] = valid[h] ? fast_exp2(fmaf(sv[h][hh], scl[hh], -mn[hh])) : 0.f;
+              ps += p[h][hh];
+            }
             // the MMA's weights agree with p to ~2^-15: the row sums take p
-            lsum[hh] = fmaf(lsum[hh], alpha[hh], p[hh]);
+            lsum[hh] = fmaf(lsum[hh], alpha[hh], ps);
             m[hh] = mn[hh];
           }
 #pragma unroll
-          for (int hh = 0; hh < G; hh += 2) {
-            uint16_t tm[kPT];
-            split_p4(p[hh], hh + 1 < G ? p[hh + 1] : 0.f, tm);
+          for (int h = 0; h < kHalves; ++h) {
+            uint8_t* pt = smem + kOffP + sbuf * kPB + h * kNC * 128 + (i & 15);
 #pragma unroll
-            for (int k = 0; k < kPT; ++k) {
-              const int n = k * G + hh;
-              pt[n * 128 + ((pc ^ (n & 7)) << 4)] = uint8_t(tm[k]);
-              if (hh + 1 < G) pt[(n + 1) * 128 + ((pc ^ ((n + 1) & 7)) << 4)] = uint8_t(tm[k] >> 8);
+            for (int hh = 0; hh < G; hh += 2) {
+              uint16_t tm[kPT];
+              split_p4(p[h][hh], hh + 1 < G ? p[h][hh + 1] : 0.f, tm);
+#pragma unroll
+              for (int k = 0; k < kPT; ++k) {
+                const int n = k * G + hh;
+                pt[n * 128 + ((pc ^ (n & 7)) << 4)] = uint8_t(tm[k]);
+                if (hh + 1 < G)
+                  pt[(n + 1) * 128 + ((pc ^ ((n + 1) & 7)) << 4)] = uint8_t(tm[k] >> 8);
+              }
             }
           }
         } else {
-          uint8_t* pt = smem + kOffP + sbuf * kPBytes + (i >> 6) * kPHalf + (i & 7) * 2;
+          uint8_t* pt = smem + kOffP + sbuf * kPB + (i >> 6) * kPHalf + (i & 7) * 2;
           const int pc = (i >> 3) & 7;  // 16-byte chunk of the token within its 128-byte row
 #pragma unroll
           for (int hh = 0; hh < G; ++hh) {
-            const float p = valid ? fast_exp2(fmaf(sv[hh], scl[hh], -mn[hh])) : 0.f;
+            const float p = valid[0] ? fast_exp2(fmaf(sv[0][hh], scl[hh], -mn[hh])) : 0.f;
             float pr;
             const uint16_t bits = round16(Tag{}, p, pr);
             *reinterpret_cast<uint16_t*>(pt + hh * 128 + ((pc ^ (hh & 7)) << 4)) = bits;
@@ -860,7 +923,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
     for (int pi = p0; pi < p1; ++pi) {
       const pa_work_item it = a.items[pi];
       const int b = it.request, h = it.kv_head;
-      const int ntiles = (it.token_end - it.token_begin + kTok - 1) / kTok;
+      const int ntiles = (it.token_end - it.token_begin + kTT - 1) / kTT;
       float res[G], lse2[G];
       if (ntiles > 0) {
         // Q^T of the non-empty piece after next goes into this piece's buffer
@@ -884,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
         if (!ok) break;
         tc::fence_after_sync();
         uint32_t r[kCols];
-        tmem_ld<kCols>(lane_addr + 2 * kNC + (np & 1) * kNC, r);
+        tmem_ld<kCols>(lane_addr + kColO + (np & 1) * kNC, r);
         tc::tmem_wait_ld();
         tc::fence_before_sync();
         __syncwarp();
