@@ -114,6 +114,17 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# the sources each kernel is compiled from (a capture in profiles/ holds only
+# while their digest matches)
+_CSRC = "serving_attention_paged_b200/csrc/"
+KERNEL_SOURCES = {
+    "decode_tc": [_CSRC + f for f in ("decode_tc.cu", "common.cuh", "tcgen05.cuh", "launch.cuh")],
+    "decode": [_CSRC + f for f in ("decode.cu", "decode_kernel.cuh", "common.cuh", "launch.cuh")],
+    "cascade": [_CSRC + f for f in ("cascade.cu", "attn_tile.cuh", "tcgen05.cuh")],
+    "prefill": [_CSRC + f for f in ("prefill.cu", "attn_tile.cuh", "tcgen05.cuh", "common.cuh")],
+}
+
+
 def source_digest(files):
     h = hashlib.sha256()
     for f in files:
@@ -479,8 +490,7 @@ def run_prefill(args, w, dev, stream, dev_t, world, rank):
     value = world * flops / (ms * 1e-3) / 1e12
     achieved = flops / (ms * 1e-3) / 1e12
     peak, peak_kind = measured_tensor_peak()
-    traffic = profiled_traffic(["serving_attention_paged_b200/csrc/prefill.cu",
-                                "serving_attention_paged_b200/csrc/common.cuh"], w.name)
+    traffic = profiled_traffic(KERNEL_SOURCES["prefill"], w.name)
 
     e2e = None
     if not args.no_e2e:
@@ -705,12 +715,10 @@ def run_ours(args):
     value = aggregate_gbs(world, nbytes, ms * 1e-3)
     peak, peak_kind = measured_peak()
     achieved = nbytes / (ms * 1e-3) / 1e9  # one GPU's launch: the dominant (only) kernel
-    decode_src = "decode_tc.cu" if tensor_cores else "decode.cu"
     decode_kernel = "paged_decode_tc_kernel" if tensor_cores else "paged_decode_kernel"
-    kernel_sources = ["serving_attention_paged_b200/csrc/" + decode_src,
-                      "serving_attention_paged_b200/csrc/common.cuh"]
+    kernel_sources = list(KERNEL_SOURCES["decode_tc" if tensor_cores else "decode"])
     if w.prefix_len:
-        kernel_sources.append("serving_attention_paged_b200/csrc/cascade.cu")
+        kernel_sources += KERNEL_SOURCES["cascade"]
     traffic = profiled_traffic(kernel_sources, w.name)
 
     # end to end through the public API from host buffers
