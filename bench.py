@@ -222,7 +222,8 @@ def cpu_baseline(w, dev, seconds):
     threads = os.cpu_count() or 1
     indptr, indices, last = w.flat_tables()
     kw = dict(num_qo_heads=w.num_qo_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
-              page_size=w.page_size, dtype=w.dtype, sm_scale=w.sm_scale, threads=threads)
+              page_size=w.page_size, dtype=w.dtype, sm_scale=w.sm_scale, threads=threads,
+              kv_dtype=w.kv_dtype, k_scale=w.k_scale, v_scale=w.v_scale)
 
     def run(reqs):
         t0 = time.perf_counter()
@@ -239,7 +240,7 @@ def cpu_baseline(w, dev, seconds):
     reqs = list(range(max(1, n)))
     dt = run(reqs)
     toks = sum(int(lens[b]) + w.prefix_len for b in reqs)
-    nbytes = 2 * toks * w.num_kv_heads * w.head_dim * 2
+    nbytes = 2 * toks * w.num_kv_heads * w.head_dim * (1 if w.kv_dtype else 2)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"the first {len(reqs)} of {w.batch} requests (all {w.num_qo_heads} q "
                       f"heads each), {toks} tokens, {nbytes} KV bytes, {dt:.2f} s, fp64"}
@@ -262,13 +263,15 @@ def run_reference(args):
     sub = W.make_workload(w.name, lens[:n_req], num_qo_heads=w.num_qo_heads,
                           num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
                           page_size=w.page_size, dtype=w.dtype, seed=w.seed,
-                          prefix_len=w.prefix_len)
+                          prefix_len=w.prefix_len, kv_dtype=w.kv_dtype, k_scale=w.k_scale,
+                          v_scale=w.v_scale)
     t = sub.materialize()
     indptr, indices, last = sub.flat_tables()
     threads = os.cpu_count() or 1
     kw = dict(num_qo_heads=sub.num_qo_heads, num_kv_heads=sub.num_kv_heads,
               head_dim=sub.head_dim, page_size=sub.page_size, dtype=sub.dtype,
-              sm_scale=sub.sm_scale, threads=threads)
+              sm_scale=sub.sm_scale, threads=threads, kv_dtype=sub.kv_dtype,
+              k_scale=sub.k_scale, v_scale=sub.v_scale)
 
     def step():
         oracle.paged_decode(t["q"], t["k_pool"], t["v_pool"], indptr, indices, last, **kw)
@@ -657,6 +660,23 @@ def launch_floor(args, dev_t, stream, flush_l2):
     return step_stats(step_ms)
 
 
+def read_floor(args, dev_t, stream, flush_l2, nbytes):
+    """Event-timed cost of reading `nbytes` from HBM with one library reduction
+    (torch.sum over an fp16 buffer of that size) in the bench's timing pattern:
+    what streaming a single-request step's bytes costs at all, as a reference
+    for that step's time."""
+    import torch
+    buf = torch.ones(nbytes // 2, dtype=torch.float16, device=dev_t)
+    out = torch.empty((), dtype=torch.float32, device=dev_t)
+
+    def step():
+        torch.sum(buf, dim=0, dtype=torch.float32, out=out)
+
+    ms, step_ms, _ = timed_steps(step, flush_l2, args, stream, dev_t, 1, soak_seconds=0.0)
+    del buf
+    return step_stats(step_ms)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -794,6 +814,11 @@ def run_ours(args):
         per["1"]["launch_floor"]["what"] = (
             "the same timing pattern (flush, start event, one 1-element torch kernel, end "
             "event): the fixed cost every event-timed step carries")
+        w1_bytes = workload("1").kv_bytes()
+        per["1"]["read_floor"] = read_floor(args, dev_t, stream, flush_l2, w1_bytes)
+        per["1"]["read_floor"]["what"] = (
+            f"the same timing pattern around torch.sum over {w1_bytes} bytes of fp16 (one "
+            "library reduction reading the step's byte count from HBM)")
         pw = workload("6")
         pdev = pw.materialize(dev_t)
         per["6"] = prefill_timing(args, pw, pdev, stream, dev_t, 1, flush_l2)[0]
