@@ -67,10 +67,15 @@ template <int G, int kKVB, bool kF32 = false, bool kRope = false> struct Cfg {
   static constexpr int kStageBytes = 2 * kHalfStage;
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kPBytesPerGroup = TPG * 8 * 4 + 8 * 4;  // p[TPG][<=8] + alpha[<=8]
-  static constexpr int kSmemBytes = kRingBytes + kGroups * kPBytesPerGroup;
+  // a piece's state per warp ([4][G][D] o, [4][G] m and l): the token groups
+  // of a warp are combined with shuffles, the 4 warps through this region, so
+  // the ring can already hold the next piece's first tiles
+  static constexpr int kCombineOff = kRingBytes + kGroups * kPBytesPerGroup;
+  static constexpr int kCombineBytes = 4 * G * D * 4 + 2 * 4 * G * 4;
+  static constexpr int kSmemBytes = kCombineOff + kCombineBytes;
   static constexpr int kLanesPerHead = LT >> LG;
   static_assert(LG <= LLT, "a head's score must fit in the lanes of a token");
-  static_assert(kGroups * G * D * 4 + 2 * kGroups * G * 4 <= kRingBytes, "merge scratch");
+  static_assert(kCombineOff % 16 == 0, "combine region alignment");
 };
 // Rotary frequency table in shared memory after the kernel's other regions:
 // theta^(-d/64) / (2 pi) as a two-float sum, d = 0..63.
@@ -286,9 +291,95 @@ __device__ __forceinline__ void copy_row(uint32_t dst, uint64_t ka, uint64_t va,
   }
 }
 
-// One piece: tokens [token_begin, token_end) of kv head h of request b.
+// The K/V copies of one piece: every thread copies its own blocks of its TPG
+// rows per tile into ring slots only it reads, so a thread may start a
+// piece's copies as soon as it has consumed its own slots of the previous
+// piece.  Addresses are formed with one 32x32->64-bit multiply-add per row
+// (pool row index x bytes per pool row + this lane's base); the V blocks and
+// the further blocks of a row use immediate offsets.
+template <typename C, int kCheckMode>
+struct PieceCopier {
+  static constexpr int TPG = C::TPG, kTile = C::kTile, kGroups = C::kGroups;
+  static constexpr int kRowBytes = C::kRowBytes, kBlock = C::kBlockBytes;
+  const DecodeArgs& a;
+  const int32_t* page_list;
+  uint64_t kaddr0, vaddr0;
+  uint32_t my_slot, pool_row_bytes, pmask;
+  int tb, len, ntiles, grp, lp, page_begin;
+  bool check;
+  __device__ __forceinline__ PieceCopier(const DecodeArgs& a_, const pa_work_item& it,
+                                         uint8_t* smem)
+      : a(a_) {
+    const int tid = threadIdx.x;
+    const int lt = tid & (C::LT - 1);
+    grp = tid / C::LT;
+    check = kCheckMode == kChecked || (kCheckMode == kRuntimeCheck && a.check);
+    tb = it.token_begin;
+    len = it.token_end - it.token_begin;
+    ntiles = (len + kTile - 1) / kTile;
+    lp = a.log2_page;
+    pmask = (1u << lp) - 1u;
+    pool_row_bytes = uint32_t(a.num_kv_heads) * kRowBytes;
+    kaddr0 = reinterpret_cast<uint64_t>(a.k_pool + int64_t(it.kv_head) * kRowBytes + lt * kBlock);
+    vaddr0 = reinterpret_cast<uint64_t>(a.v_pool + int64_t(it.kv_head) * kRowBytes + lt * kBlock);
+    page_begin = it.page_begin;
+    page_list = a.kv_indices + it.page_begin;
+    my_slot = smem_u32(smem) + grp * kRowBytes + lt * kBlock;
+  }
+  __device__ __forceinline__ void load_pages(int tile, int (&pg)[TPG]) const {
+#pragma unroll
+    for (int j = 0; j < TPG; ++j) {
+      const int pos = tile * kTile + grp + kGroups * j;
+      int p = -1;
+      if (pos < len) {
+        const int idx = (tb + pos) >> lp;
+        p = __ldg(page_list + idx);
+        if (check && (p < 0 || int64_t(p) >= a.num_pages)) {
+          atomicMin(a.error_pos, (unsigned long long)(page_begin + idx));
+          p = -1;  // not copied: the row reads as zeros
+        }
+      }
+      pg[j] = p;
+    }
+  }
+  __device__ __forceinline__ void issue(int tile, uint32_t stage_off, const int (&pg)[TPG]) const {
+    if (tile < ntiles) {
+#pragma unroll
+      for (int j = 0; j < TPG; ++j) {
+        const uint32_t pos = uint32_t(tb + tile * kTile + grp + kGroups * j);
+        const bool ok = pg[j] >= 0;
+        const uint32_t row = ok ? ((uint32_t(pg[j]) << lp) | (pos & pmask)) : 0u;
+        const uint32_t nbytes = ok ? uint32_t(kBlock) : 0u;
+        uint64_t ka, va;
+        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(ka) : "r"(row), "r"(pool_row_bytes), "l"(kaddr0));
+        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(va) : "r"(row), "r"(pool_row_bytes), "l"(vaddr0));
+        const uint32_t dst = my_slot + stage_off + j * kGroups * kRowBytes;
+        copy_row<C::V, C::LT, kBlock, C::kHalfStage>(dst, ka, va, nbytes);
+      }
+    }
+    cp_async_commit();
+  }
+  // the first kStages - 1 tiles into stages 0.., then tile kStages - 1's pages into pg
+  __device__ __forceinline__ void start(int (&pg)[TPG]) const {
+#pragma unroll
+    for (int st = 0; st < C::kStages - 1; ++st) {
+      load_pages(st, pg);
+      issue(st, st * C::kStageBytes, pg);
+    }
+    load_pages(C::kStages - 1, pg);
+  }
+};
+
+// One piece: tokens [token_begin, token_end) of kv head h of request b.  With
+// `started` its first tiles are already being copied (by the previous piece,
+// which left tile kStages - 1's pages in pg); `next` (or null) is the CTA's
+// next piece, whose first copies this piece starts right after its last tile.
 template <typename Tag, typename KV, int G, int kCheckMode, bool kRope>
 __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_item& it,
+                                          const pa_work_item* next, bool started,
+                                          int (&pg)[Cfg<G, KVBytes<KV>::v,
+                                                        !std::is_same<KV, KV16>::value || kRope,
+                                                        kRope>::TPG],
                                           uint8_t* smem, const float* rope_tab,
                                           int& s_is_last) {
   constexpr bool k8 = !std::is_same<KV, KV16>::value;
@@ -386,63 +477,15 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
   const bool writer = (lt & (C::kLanesPerHead - 1)) == 0;
 
   // ---- loads: this thread's blocks of its TPG rows per tile ----
-  // Addresses are formed with one 32x32->64-bit multiply-add per row (pool
-  // row index x bytes per pool row + this lane's base), and the V blocks and
-  // the further blocks of a row use immediate offsets.
-  const int lp = a.log2_page;
-  const uint32_t pmask = (1u << lp) - 1u;
-  const uint32_t pool_row_bytes = uint32_t(a.num_kv_heads) * kRowBytes;
-  const uint64_t kaddr0 = reinterpret_cast<uint64_t>(a.k_pool + int64_t(h) * kRowBytes + lt * kBlock);
-  const uint64_t vaddr0 = reinterpret_cast<uint64_t>(a.v_pool + int64_t(h) * kRowBytes + lt * kBlock);
-  const int32_t* page_list = a.kv_indices + it.page_begin;
-  const uint32_t my_slot = smem_u32(smem) + grp * kRowBytes + lt * kBlock;
-  auto load_pages = [&](int tile, int (&pg)[TPG]) {
-#pragma unroll
-    for (int j = 0; j < TPG; ++j) {
-      const int pos = tile * kTile + grp + kGroups * j;
-      int p = -1;
-      if (pos < len) {
-        const int idx = (tb + pos) >> lp;
-        p = __ldg(page_list + idx);
-        if (check && (p < 0 || int64_t(p) >= a.num_pages)) {
-          atomicMin(a.error_pos, (unsigned long long)(it.page_begin + idx));
-          p = -1;  // not copied: the row reads as zeros
-        }
-      }
-      pg[j] = p;
-    }
-  };
-  auto issue = [&](int tile, uint32_t stage_off, const int (&pg)[TPG]) {
-    if (tile < ntiles) {
-#pragma unroll
-      for (int j = 0; j < TPG; ++j) {
-        const uint32_t pos = uint32_t(tb + tile * kTile + grp + kGroups * j);
-        const bool ok = pg[j] >= 0;
-        const uint32_t row = ok ? ((uint32_t(pg[j]) << lp) | (pos & pmask)) : 0u;
-        const uint32_t nbytes = ok ? uint32_t(kBlock) : 0u;
-        uint64_t ka, va;
-        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(ka) : "r"(row), "r"(pool_row_bytes), "l"(kaddr0));
-        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(va) : "r"(row), "r"(pool_row_bytes), "l"(vaddr0));
-        const uint32_t dst = my_slot + stage_off + j * kGroups * kRowBytes;
-        copy_row<V, LT, kBlock, C::kHalfStage>(dst, ka, va, nbytes);
-      }
-    }
-    cp_async_commit();
-  };
   constexpr int kStages = C::kStages;
-  int pg[TPG];
-#pragma unroll
-  for (int st = 0; st < kStages - 1; ++st) {
-    load_pages(st, pg);
-    issue(st, st * C::kStageBytes, pg);
-  }
-  load_pages(kStages - 1, pg);
+  const PieceCopier<C, kCheckMode> cp(a, it, smem);
+  if (!started) cp.start(pg);
 
   uint32_t issue_off = (kStages - 1) * C::kStageBytes;  // ring slot of tile t + kStages - 1
   uint32_t read_off = 0;                                 // ring slot of tile t
   for (int t = 0; t < ntiles; ++t) {
-    issue(t + kStages - 1, issue_off, pg);
-    load_pages(t + kStages, pg);
+    cp.issue(t + kStages - 1, issue_off, pg);
+    cp.load_pages(t + kStages, pg);
     issue_off = issue_off + C::kStageBytes == C::kRingBytes ? 0u : issue_off + C::kStageBytes;
     cp_async_wait<kStages - 1>();
     const uint8_t* ks = smem + read_off + grp * kRowBytes + lt * kBlock;
@@ -554,30 +597,79 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
     }
     __syncwarp();  // p and alpha of this tile consumed before the next tile writes them
   }
-  cp_async_wait<0>();
-  __syncthreads();
+  // This thread's ring slots are free: start the next piece's copies, so they
+  // land while this piece is combined and written.
+  if (next) {
+    const PieceCopier<C, kCheckMode> np(a, *next, smem);
+    np.start(pg);
+  }
 
-  // Combine the token groups through shared memory (the ring is idle now).
-  float* Os = reinterpret_cast<float*>(smem);  // [kGroups][G][D]
-  float* Ms = Os + kGroups * G * D;            // [kGroups][G]
-  float* Ls = Ms + kGroups * G;
+  // Combine the token groups: within a warp by shuffles (the lanes holding
+  // the same elements of another group are LT, 2 LT, ... lanes away), then
+  // the 4 warps through shared memory.  Each group's (m, l) of head hh sits
+  // in its lanes with my_head == hh.
+  constexpr int kWarps = kThreads / 32;
+  float* Ow = reinterpret_cast<float*>(smem + C::kCombineOff);  // [kWarps][G][D]
+  float* Mw = Ow + kWarps * G * D;                                // [kWarps][G]
+  float* Lw = Mw + kWarps * G;
+  const int lane = tid & 31, wp = tid >> 5;
+  float mh[G], lh[G];
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh)
+  for (int hh = 0; hh < G; ++hh) {
+    const int src = (lane & ~(LT - 1)) + hh * C::kLanesPerHead;
+    mh[hh] = __shfl_sync(0xffffffffu, m, src);
+    lh[hh] = __shfl_sync(0xffffffffu, l, src);
+  }
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-      float4* dst = reinterpret_cast<float4*>(Os + (grp * G + hh) * D + (lt + v * LT) * 8);
+  for (int off = LT; off < 32; off <<= 1) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      const float mo = __shfl_xor_sync(0xffffffffu, mh[hh], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, lh[hh], off);
+      const float M = fmaxf(mh[hh], mo);
+      const float ws = mh[hh] == -INFINITY ? 0.f : fast_exp2(mh[hh] - M);
+      const float wo = mo == -INFINITY ? 0.f : fast_exp2(mo - M);
       if constexpr (kF32) {
-        const float2* x = &o2[hh][4 * v];
-        dst[0] = make_float4(x[0].x, x[0].y, x[1].x, x[1].y);
-        dst[1] = make_float4(x[2].x, x[2].y, x[3].x, x[3].y);
+#pragma unroll
+        for (int e = 0; e < E / 2; ++e) {
+          const float2 x = o2[hh][e];
+          const float2 y = make_float2(__shfl_xor_sync(0xffffffffu, x.x, off),
+                                       __shfl_xor_sync(0xffffffffu, x.y, off));
+          o2[hh][e] = make_float2(fmaf(x.x, ws, y.x * wo), fmaf(x.y, ws, y.y * wo));
+        }
       } else {
-        dst[0] = make_float4(o[hh][8 * v], o[hh][8 * v + 1], o[hh][8 * v + 2], o[hh][8 * v + 3]);
-        dst[1] = make_float4(o[hh][8 * v + 4], o[hh][8 * v + 5], o[hh][8 * v + 6], o[hh][8 * v + 7]);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float y = __shfl_xor_sync(0xffffffffu, o[hh][e], off);
+          o[hh][e] = fmaf(o[hh][e], ws, y * wo);
+        }
+      }
+      lh[hh] = fmaf(lh[hh], ws, lo * wo);
+      mh[hh] = M;
+    }
+  }
+  if (lane < LT) {  // group 0 of the warp now holds the warp's state
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        float4* dst = reinterpret_cast<float4*>(Ow + (wp * G + hh) * D + (lt + v * LT) * 8);
+        if constexpr (kF32) {
+          const float2* x = &o2[hh][4 * v];
+          dst[0] = make_float4(x[0].x, x[0].y, x[1].x, x[1].y);
+          dst[1] = make_float4(x[2].x, x[2].y, x[3].x, x[3].y);
+        } else {
+          dst[0] = make_float4(o[hh][8 * v], o[hh][8 * v + 1], o[hh][8 * v + 2], o[hh][8 * v + 3]);
+          dst[1] = make_float4(o[hh][8 * v + 4], o[hh][8 * v + 5], o[hh][8 * v + 6], o[hh][8 * v + 7]);
+        }
+      }
+    if (lane == 0) {
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        Mw[wp * G + hh] = mh[hh];
+        Lw[wp * G + hh] = lh[hh];
       }
     }
-  if (writer) {
-    Ms[grp * G + my_head] = m;
-    Ls[grp * G + my_head] = l;
   }
   __syncthreads();
 
@@ -586,18 +678,19 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
     float M = -INFINITY;
-#pragma unroll 8
-    for (int g = 0; g < kGroups; ++g) M = fmaxf(M, Ms[g * G + hh]);
+#pragma unroll
+    for (int g = 0; g < kWarps; ++g) M = fmaxf(M, Mw[g * G + hh]);
     if (M == -INFINITY) {
       res[hh] = 0.f;
       lse2[hh] = -INFINITY;
     } else {
       float lsum = 0.f, acc = 0.f;
-#pragma unroll 8
-      for (int g = 0; g < kGroups; ++g) {
-        const float w = fast_exp2(Ms[g * G + hh] - M);
-        lsum = fmaf(w, Ls[g * G + hh], lsum);
-        acc = fmaf(w, Os[(g * G + hh) * D + d], acc);
+#pragma unroll
+      for (int g = 0; g < kWarps; ++g) {
+        const float mg = Mw[g * G + hh];
+        const float w = mg == -INFINITY ? 0.f : fast_exp2(mg - M);
+        lsum = fmaf(w, Lw[g * G + hh], lsum);
+        acc = fmaf(w, Ow[(g * G + hh) * D + d], acc);
       }
       res[hh] = acc / lsum;
       if constexpr (k8) res[hh] *= a.v_scale;  // cached value = v_scale * code
@@ -671,9 +764,11 @@ __global__ void __launch_bounds__(kThreads, (KCfg<Tag, KV, G, kCheckMode, kRope>
     __syncthreads();
   }
   const int p0 = a.cta_indptr[blockIdx.x], p1 = a.cta_indptr[blockIdx.x + 1];
+  int pg[C::TPG];  // tile kStages - 1's pages of a piece whose copies are started
   for (int pi = p0; pi < p1; ++pi) {
-    if (pi > p0) __syncthreads();  // the previous piece is done with shared memory
-    run_piece<Tag, KV, G, kCheckMode, kRope>(a, a.items[pi], smem, rope_tab, s_is_last);
+    if (pi > p0) __syncthreads();  // the previous piece is done with p and the combine region
+    run_piece<Tag, KV, G, kCheckMode, kRope>(a, a.items[pi], pi + 1 < p1 ? a.items + pi + 1 : nullptr,
+                                             pi > p0, pg, smem, rope_tab, s_is_last);
   }
 }
 
