@@ -112,7 +112,7 @@ typedef struct {
   uint32_t flags;           /* PA_FLAG_* */
   int32_t piece_cost_tokens; /* plan budget charged for each further piece of a CTA
                                 (see pa_plan_create): 0 = the default of the decode
-                                kernel the problem runs (400 CUDA cores, 128 tensor
+                                kernel the problem runs (300 CUDA cores, 128 tensor
                                 cores), > 0 that many tokens, < 0 none */
   /* Compressed KV cache (README core feature 3: low-precision attention for a
    * compressed KV-Cache).  kv_dtype PA_E4M3 or PA_E5M2: the pools hold 8-bit

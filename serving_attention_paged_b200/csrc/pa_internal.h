@@ -122,7 +122,7 @@ inline bool decode_uses_tensor_cores(const pa_problem& p) {
 // tensor-core kernel (its loaders run across pieces and epilogue warps work
 // off the critical path); the values are the best of a sweep on the uniform
 // and ragged batches.
-constexpr int32_t kPieceCostCudaCores = 400, kPieceCostTensorCores = 128;
+constexpr int32_t kPieceCostCudaCores = 300, kPieceCostTensorCores = 128;
 inline int32_t default_piece_cost_tokens(const pa_problem& p) {
   return decode_uses_tensor_cores(p) ? kPieceCostTensorCores : kPieceCostCudaCores;
 }

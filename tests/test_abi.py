@@ -165,7 +165,7 @@ def test_cascade_plan_shape(C):
     n, tok = C.pa_plan_prefix_chunks(plan)
     assert n >= 1 and tok % 128 == 0 and n * tok >= w.prefix_len > (n - 1) * tok
     q, items, ci, mi = oracle.plan(w.kv_indptr, w.last_page_len, page_size=16, num_kv_heads=8,
-                                   num_sms=148, ctas_per_sm=2, piece_cost=400)
+                                   num_sms=148, ctas_per_sm=2, piece_cost=300)
     assert np.array_equal(C.pa_plan_work_items(plan), items)
     assert np.array_equal(C.pa_plan_cta_indptr(plan), ci)
 
@@ -190,9 +190,9 @@ def test_decode_kernel_choice(C):
 
 def test_default_piece_cost_follows_the_kernel(C):
     """piece_cost_tokens = 0 takes the default of the decode kernel the plan
-    runs: 400 tokens for the CUDA-core kernel, 128 for the tensor-core one."""
+    runs: 300 tokens for the CUDA-core kernel, 128 for the tensor-core one."""
     w = W.WORKLOADS[3]()
-    for flags, c in ((0, 400), (C.PA_FLAG_TENSOR_CORES, 128)):
+    for flags, c in ((0, 300), (C.PA_FLAG_TENSOR_CORES, 128)):
         base = dict(batch=w.batch, num_qo_heads=w.num_qo_heads, num_kv_heads=w.num_kv_heads,
                     page_size=w.page_size, dtype=w.dtype, sm_scale=w.sm_scale, num_sms=148,
                     ctas_per_sm=2, num_pages=w.num_pages, flags=flags)
