@@ -390,7 +390,6 @@ __device__ __forceinline__ void run_piece(const DecodeArgs& a, const pa_work_ite
   constexpr int kGroups = C::kGroups, kTile = C::kTile;
   constexpr int kRowBytes = C::kRowBytes, kBlock = C::kBlockBytes;
 
-  const bool check = kCheckMode == kChecked || (kCheckMode == kRuntimeCheck && a.check);
   const int tid = threadIdx.x;
   const int lt = tid & (LT - 1);   // lane within the token
   const int grp = tid / LT;        // token group

@@ -236,98 +236,90 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) flag_timeout(a);
    } else if (warp == kWarpMma) {
     // ------------------------------ MMA issuer ------------------------------
-    // Every lane waits (ok stays warp-uniform, and the lanes zero stale V rows
-    // together); lane 0 issues.
-    constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
-    constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
-    const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
-    const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffK, 16, 1024);
-    const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffV, kKVHalf, 1024);
-    const int nt[2] = {nt0, nt1};
-    // Rows [zero_from, zero_to) of the last tile were copied from the page
-    // that holds the tile's last key but lie past it.
-    const int zero_from = kv_end - (ntiles - 1) * kKeys;
-    const int zero_to = min(kKeys, (zero_from + a.box_rows - 1) / a.box_rows * a.box_rows);
-    auto wait_all = [&](int b, int parity) {
-      return __all_sync(0xffffffffu, mbar_wait(bar(b), parity));
-    };
-    auto issue_s = [&](int hf, int kt) {
-      const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
-      const uint64_t kd = dk0 + (((kt % kKStages) * kKVBytes) >> 4);
-      const uint32_t dst = tmem + hf * 256;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-        const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
-        tc::mma_f16_ss(dst, qd + off, kd + koff, kIdescQK, kk > 0);
-      }
-      tc::commit(bar(kBarS + hf));
-    };
-    auto issue_pv = [&](int hf, int v) {
-      const uint32_t pt = tmem + hf * 256;
-      const uint32_t dst = tmem + hf * 256 + 128;
-      const uint64_t vd = dv0 + (((v % kVStages) * kKVBytes) >> 4);
-#pragma unroll
-      for (int kk = 0; kk < kKeys / 16; ++kk)
-        tc::mma_f16_ts(dst, pt + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
-                       (v > 0 || kk > 0) ? 1u : 0u);
-      if (kSplit) {
-#pragma unroll
+    // Lane 0 alone waits, zeroes stale V rows and issues: a whole-warp wait
+    // and vote around every issue measured ~130 cycles per tcgen05.mma
+    // against ~64 (the tensor core's own rate) for a single thread.
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
+      constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
+      const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
+      const uint64_t dk0 = tc::smem_desc_sw128(sb + kOffK, 16, 1024);
+      const uint64_t dv0 = tc::smem_desc_sw128(sb + kOffV, kKVHalf, 1024);
+      const int nt[2] = {nt0, nt1};
+      // Rows [zero_from, zero_to) of the last tile were copied from the page
+      // that holds the tile's last key but lie past it.
+      const int zero_from = kv_end - (ntiles - 1) * kKeys;
+      const int zero_to = min(kKeys, (zero_from + a.box_rows - 1) / a.box_rows * a.box_rows);
+      auto wait_all = [&](int b, int parity) { return mbar_wait(bar(b), parity); };
+      auto issue_s = [&](int hf, int kt) {
+        const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
+        const uint64_t kd = dk0 + (((kt % kKStages) * kKVBytes) >> 4);
+        const uint32_t dst = tmem + hf * 256;
+  #pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+          const uint32_t koff = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+          tc::mma_f16_ss(dst, qd + off, kd + koff, kIdescQK, kk > 0);
+        }
+        tc::commit(bar(kBarS + hf));
+      };
+      auto issue_pv = [&](int hf, int v) {
+        const uint32_t pt = tmem + hf * 256;
+        const uint32_t dst = tmem + hf * 256 + 128;
+        const uint64_t vd = dv0 + (((v % kVStages) * kKVBytes) >> 4);
+  #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          tc::mma_f16_ts(dst, pt + 64 + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
-      }
-    };
-    bool ok = wait_all(kBarQ, 0);
-    // Fixed order per tile t: for each half, P V(t - 1) then S(t); a half
-    // past its own tile count only finishes (its last P V, then the extra
-    // S-barrier commit).
-    for (int kt = 0; ok && kt <= ntiles; ++kt) {
-      for (int hf = 0; ok && hf < kHalves; ++hf) {
-        const int v = kt - 1;
-        if (v >= 0 && v < nt[hf]) {
-          if (hf == 0 || v >= nt[0]) {  // the first half to use V(v) waits for it
-            ok = wait_all(kBarVFull + v % kVStages, (v / kVStages) & 1);
-            if (ok && v == ntiles - 1 && zero_from < zero_to) {
-              uint8_t* vt = smem + kOffV + (v % kVStages) * kKVBytes;
-              const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
-              for (int c = lane; c < n16; c += 32) {
-                const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
-                *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
-                    make_uint4(0u, 0u, 0u, 0u);
+          tc::mma_f16_ts(dst, pt + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                         (v > 0 || kk > 0) ? 1u : 0u);
+        if (kSplit) {
+  #pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk)
+            tc::mma_f16_ts(dst, pt + 64 + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
+        }
+      };
+      bool ok = wait_all(kBarQ, 0);
+      // Fixed order per tile t: for each half, P V(t - 1) then S(t); a half
+      // past its own tile count only finishes (its last P V, then the extra
+      // S-barrier commit).
+      for (int kt = 0; ok && kt <= ntiles; ++kt) {
+        for (int hf = 0; ok && hf < kHalves; ++hf) {
+          const int v = kt - 1;
+          if (v >= 0 && v < nt[hf]) {
+            if (hf == 0 || v >= nt[0]) {  // the first half to use V(v) waits for it
+              ok = wait_all(kBarVFull + v % kVStages, (v / kVStages) & 1);
+              if (ok && v == ntiles - 1 && zero_from < zero_to) {
+                uint8_t* vt = smem + kOffV + (v % kVStages) * kKVBytes;
+                const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
+                for (int c = 0; c < n16; ++c) {
+                  const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
+                  *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
+                      make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
               }
-              fence_proxy_async_smem();
-              __syncwarp();
             }
-          }
-          if (ok) ok = wait_all(kBarP + hf, v & 1);
-          if (!ok) break;
-          if (lane == 0) {
+            if (ok) ok = wait_all(kBarP + hf, v & 1);
+            if (!ok) break;
             tc::fence_after_sync();
             issue_pv(hf, v);
           }
-          __syncwarp();
-        }
-        if (kt < nt[hf]) {
-          if (hf == 0 || kt >= nt[0]) ok = wait_all(kBarKFull + kt % kKStages, (kt / kKStages) & 1);
-          if (!ok) break;
-          if (lane == 0) {
+          if (kt < nt[hf]) {
+            if (hf == 0 || kt >= nt[0]) ok = wait_all(kBarKFull + kt % kKStages, (kt / kKStages) & 1);
+            if (!ok) break;
             tc::fence_after_sync();
             issue_s(hf, kt);
+          } else if (kt == nt[hf] && nt[hf] > 0) {
+            tc::commit(bar(kBarS + hf));  // the half's last P V is done
           }
-          __syncwarp();
-        } else if (kt == nt[hf] && nt[hf] > 0) {
-          if (lane == 0) tc::commit(bar(kBarS + hf));  // the half's last P V is done
-          __syncwarp();
+        }
+        // release the stages the tile's last user has finished with
+        if (ok) {
+          if (kt < ntiles) tc::commit(bar(kBarKEmpty + kt % kKStages));
+          if (kt >= 1) tc::commit(bar(kBarVEmpty + (kt - 1) % kVStages));
         }
       }
-      // release the stages the tile's last user has finished with
-      if (ok && lane == 0) {
-        if (kt < ntiles) tc::commit(bar(kBarKEmpty + kt % kKStages));
-        if (kt >= 1) tc::commit(bar(kBarVEmpty + (kt - 1) % kVStages));
-      }
-      __syncwarp();
+      if (!ok) flag_timeout(a);
     }
-    if (!ok && lane == 0) flag_timeout(a);
    }
   } else {
     // ------------------------- softmax / epilogue rows -------------------------
