@@ -108,6 +108,11 @@ struct CascadeArgs {
 };
 
 using at::Fmt;
+
+// bar.sync on a named barrier among `count` threads (whole warps).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
 using at::exp2_poly2;
 using at::make_map;
 using at::max3;
@@ -429,17 +434,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarP + hf));
     }
-    // epilogue: the half's last P V has completed (its extra S commit)
+    // epilogue: the half's last P V has completed (its extra S commit).  O is
+    // normalised into the idle K/V ring (a 512-byte fp32 row per thread, its
+    // 16-byte chunks swizzled by row so the writes spread over the banks), and
+    // the 8 softmax warps then copy whole rows out, 512 contiguous bytes per
+    // warp instruction: a thread storing its own row straight to global memory
+    // touches 32 half sectors per instruction.
     if (ok && nt > 0) ok = mbar_wait(bar(kBarS + hf), nt & 1);
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (!all_ok && lane == 0) flag_timeout(a);
+    named_barrier_sync(1, 256);  // both halves' MMAs are done: the ring is free
+    float* stage = reinterpret_cast<float*>(smem + kOffK);  // [256 rows][128]
+    const int rowc = hf * kRows + i;                        // row within the CTA
+    auto chunk_pos = [](int c, int row) { return (c & ~7) | ((c & 7) ^ (row & 7)); };
+    const float inv = l > 0.f ? 1.f / l : 0.f;
     if (all_ok) {
       tc::fence_after_sync();
-      const int r = (rp * kHalves + hf) * kRows + i;
-      const int rows = a.batch * G;
-      const int b = r / G, j = r - (r / G) * G;
-      float* dst = a.prefix_o + ((int64_t(chunk) * a.batch + b) * a.num_qo_heads + h * G + j) * D;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float ov[32];
@@ -450,16 +460,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = 0.f;
         }
-        if (r < rows) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + 32 * c + e) =
-                make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv, ov[e + 3] * inv);
-        }
+        for (int k = 0; k < 8; ++k)
+          reinterpret_cast<float4*>(stage + rowc * D)[chunk_pos(8 * c + k, rowc)] =
+              make_float4(ov[4 * k] * inv, ov[4 * k + 1] * inv, ov[4 * k + 2] * inv,
+                          ov[4 * k + 3] * inv);
       }
-      if (r < rows)
+    }
+    const int rows = a.batch * G;
+    {
+      const int r = rp * kHalves * kRows + rowc;
+      if (r < rows) {
+        const int b = r / G, j = r - (r / G) * G;
         a.prefix_lse[(int64_t(chunk) * a.batch + b) * a.num_qo_heads + h * G + j] =
             l > 0.f ? m + fast_log2(l) : -INFINITY;
+      }
+    }
+    named_barrier_sync(1, 256);
+    for (int rr = 0; rr < 32; ++rr) {  // warp w copies rows 32 w .. 32 w + 31
+      const int row = warp * 32 + rr;
+      const int r = rp * kHalves * kRows + row;
+      if (r >= rows) break;
+      const int b = r / G, j = r - (r / G) * G;
+      float* dst = a.prefix_o + ((int64_t(chunk) * a.batch + b) * a.num_qo_heads + h * G + j) * D;
+      reinterpret_cast<float4*>(dst)[lane] =
+          reinterpret_cast<const float4*>(stage + row * D)[chunk_pos(lane, row)];
     }
   }
 

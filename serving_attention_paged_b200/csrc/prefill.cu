@@ -68,6 +68,11 @@ namespace pa {
 namespace {
 
 using at::exp2_poly2;
+
+// bar.sync on a named barrier among `count` threads (whole warps).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
 using at::Fmt;
 using at::make_map;
 using at::max3;
@@ -455,15 +460,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // epilogue: the half's last P V has completed (its extra S commit);
     // o = O / l in the input type and lse = (m + log2 l) ln 2; a half without
-    // keys (no mask, empty request) writes o = 0, lse = -inf.
+    // keys (no mask, empty request) writes o = 0, lse = -inf.  o is staged in
+    // the idle K/V ring (a 256-byte row per thread, 16-byte chunks swizzled by
+    // row) and copied out by whole rows, 512 contiguous bytes per warp
+    // instruction.
     if (ok && nt > 0) ok = mbar_wait(bar(kBarS + hf), nt & 1);
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (!all_ok && lane == 0) flag_timeout(a);
+    named_barrier_sync(1, 256);  // both halves' MMAs are done: the ring is free
+    uint8_t* stage = smem + kOffK;                  // [256 rows][128 x 16 bits]
+    const int rowc = hf * kRows + i;                // row within the CTA
+    auto chunk_pos = [](int c, int row) { return (c & ~7) | ((c & 7) ^ (row & 7)); };
     if (all_ok && nqh > 0) {
       tc::fence_after_sync();
-      const bool valid = jq < n_q;
-      const int64_t orow = int64_t(q_begin + jq) * a.num_qo_heads + h * G + jh;
-      uint8_t* dst = static_cast<uint8_t*>(a.o) + orow * (D * 2);
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -475,25 +484,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = 0.f;
         }
-        if (valid) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint32_t w[4];
+        for (int e = 0; e < 32; e += 8) {
+          uint32_t w[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              if constexpr (kSplit) {
-                float t0, t1;
-                w[k] = pack2(Tag{}, ov[e + 2 * k] * inv, ov[e + 2 * k + 1] * inv, t0, t1);
-              } else {
-                const __half2 hp = __floats2half2_rn(ov[e + 2 * k] * inv, ov[e + 2 * k + 1] * inv);
-                w[k] = *reinterpret_cast<const uint32_t*>(&hp);
-              }
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (kSplit) {
+              float t0, t1;
+              w[k] = pack2(Tag{}, ov[e + 2 * k] * inv, ov[e + 2 * k + 1] * inv, t0, t1);
+            } else {
+              const __half2 hp = __floats2half2_rn(ov[e + 2 * k] * inv, ov[e + 2 * k + 1] * inv);
+              w[k] = *reinterpret_cast<const uint32_t*>(&hp);
             }
-            *reinterpret_cast<uint4*>(dst + (32 * c + e) * 2) = make_uint4(w[0], w[1], w[2], w[3]);
           }
+          reinterpret_cast<uint4*>(stage + rowc * (D * 2))[chunk_pos((32 * c + e) / 8, rowc)] =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      if (valid && a.lse) a.lse[orow] = l > 0.f ? (m + fast_log2(l)) * kLn2 : -INFINITY;
+      if (jq < n_q && a.lse) {
+        const int64_t orow = int64_t(q_begin + jq) * a.num_qo_heads + h * G + jh;
+        a.lse[orow] = l > 0.f ? (m + fast_log2(l)) * kLn2 : -INFINITY;
+      }
+    }
+    named_barrier_sync(1, 256);
+    // warp w copies rows 32 w .. 32 w + 31, two per instruction (16 lanes a row)
+    for (int rr = 0; rr < 32; rr += 2) {
+      const int row = warp * 32 + rr + (lane >> 4);
+      const int rh = row >> 7, ri = row & (kRows - 1);
+      const int rq = rh * per_half + ri / G;  // token of the row within the tile
+      if ((rh ? nq1 : nq0) > 0 && rq < n_q) {
+        const int64_t orow = int64_t(q_begin + rq) * a.num_qo_heads + h * G + ri % G;
+        reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.o) + orow * (D * 2))[lane & 15] =
+            reinterpret_cast<const uint4*>(stage + row * (D * 2))[chunk_pos(lane & 15, row)];
+      }
     }
   }
 
