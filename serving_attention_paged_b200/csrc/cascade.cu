@@ -242,7 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) flag_timeout(a);
   } else if (warp == kWarpMma) {
     // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
+    // The whole warp runs the loop (its values stay warp-uniform); one elected
+    // lane issues the MMAs and their commits.
+    {
       constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
       constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
       // descriptors are built once; a k-step adds its byte offset / 16
@@ -275,7 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mma_f16_ts(dst, pt + 64 + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
         }
       };
-      bool ok = mbar_wait(bar(kBarQ), 0);
+      auto wait = [&](int b, int parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar(b), parity));
+      };
+      bool ok = wait(kBarQ, 0);
       // Fixed order per tile t: for each half, P V(t - 1) then S(t).  The
       // softmax of a half always finds its next S queued behind the other
       // half's work.
@@ -283,25 +288,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hf = 0; ok && hf < kHalves; ++hf) {
           if (kt > 0) {
             const int v = kt - 1;
-            if (hf == 0) ok = mbar_wait(bar(kBarVFull + v % kVStages), (v / kVStages) & 1);
-            if (ok) ok = mbar_wait(bar(kBarP + hf), v & 1);
+            if (hf == 0) ok = wait(kBarVFull + v % kVStages, (v / kVStages) & 1);
+            if (ok) ok = wait(kBarP + hf, v & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            issue_pv(hf, v);
-            if (hf == kHalves - 1) tc::commit(bar(kBarVEmpty + v % kVStages));
+            if (tc::elect_one_sync()) {
+              issue_pv(hf, v);
+              if (hf == kHalves - 1) tc::commit(bar(kBarVEmpty + v % kVStages));
+            }
+            __syncwarp();
           }
           if (kt < nt) {
-            if (hf == 0) ok = mbar_wait(bar(kBarKFull + kt % kKStages), (kt / kKStages) & 1);
+            if (hf == 0) ok = wait(kBarKFull + kt % kKStages, (kt / kKStages) & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            issue_s(hf, kt);  // its commit also signals that P V(kt - 1) is done
-            if (hf == kHalves - 1) tc::commit(bar(kBarKEmpty + kt % kKStages));
+            if (tc::elect_one_sync()) {
+              issue_s(hf, kt);  // its commit also signals that P V(kt - 1) is done
+              if (hf == kHalves - 1) tc::commit(bar(kBarKEmpty + kt % kKStages));
+            }
+            __syncwarp();
           } else {
-            tc::commit(bar(kBarS + hf));  // the last P V of the half is done
+            if (tc::elect_one_sync()) tc::commit(bar(kBarS + hf));  // the half's last P V is done
+            __syncwarp();
           }
         }
       }
-      if (!ok) flag_timeout(a);
+      if (!ok && lane == 0) flag_timeout(a);
     }
    }
   } else {

@@ -521,7 +521,13 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
     }
   } else if (warp == 8) {
     // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
+    // The whole warp runs the polling loop (every barrier test is lane 0's
+    // result, so its values stay warp-uniform); one elected lane issues the
+    // MMAs and their commits.
+    {
+      auto test = [&](int b, uint32_t parity) {
+        return __shfl_sync(0xffffffffu, int(mbar_test_wait(bar(b), parity)), 0) != 0;
+      };
       // S^T = K Q^T: A = K (M = tokens, K-major), B = Q^T (K-major).
       // O^T = V^T P^T: A = V^T (M = head elements, MN-major), B = P^T (K-major).
       // 8-bit pools: A in the cached format, B in E4M3 terms.
@@ -549,35 +555,38 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
       while (v_piece < p1) {
         bool progress = false;
         auto k_ready = [&]() {
-          return mbar_test_wait(bar(L::kBarFull + ts % kStages), (ts / kStages) & 1);
+          return test(L::kBarFull + ts % kStages, (ts / kStages) & 1);
         };
         if (s_piece < p1 &&
-            (ts < 2 || mbar_test_wait(bar(kBarSFree + (ts & 1)), ((ts - 2) >> 1) & 1)) &&
-            k_ready() && mbar_test_wait(bar(kBarQReady + (s_np & 1)), (s_np >> 1) & 1)) {
+            (ts < 2 || test(kBarSFree + (ts & 1), ((ts - 2) >> 1) & 1)) &&
+            k_ready() && test(kBarQReady + (s_np & 1), (s_np >> 1) & 1)) {
           fence_proxy_async_smem();  // the loaders' cp.async writes, seen by the tensor core
           tc::fence_after_sync();
           const uint64_t qd = dq0 + uint64_t(((s_np & 1) * kQBytes) >> 4);
           const uint64_t kd = dk0 + uint64_t(((ts % kStages) * kStageBytes) >> 4);
-          if constexpr (k8) {
-            // per 128-token half; 32 one-byte elements (32 bytes of each
-            // 128-byte row) per step
+          if (tc::elect_one_sync()) {
+            if constexpr (k8) {
+              // per 128-token half; 32 one-byte elements (32 bytes of each
+              // 128-byte row) per step
 #pragma unroll
-            for (int h = 0; h < kHalves; ++h) {
-              const uint32_t sd = tmem + ((ts & 1) * kHalves + h) * kNC;
-              const uint64_t kh = kd + uint64_t((h * kTok * 128) >> 4);
+              for (int h = 0; h < kHalves; ++h) {
+                const uint32_t sd = tmem + ((ts & 1) * kHalves + h) * kNC;
+                const uint64_t kh = kd + uint64_t((h * kTok * 128) >> 4);
 #pragma unroll
-              for (int kk = 0; kk < D / 32; ++kk)
-                tc::mma_f8_ss(sd, kh + kk * 2, qd + kk * 2, kIdescS, kk > 0);
+                for (int kk = 0; kk < D / 32; ++kk)
+                  tc::mma_f8_ss(sd, kh + kk * 2, qd + kk * 2, kIdescS, kk > 0);
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = ((kk >> 2) * kHalfKV + (kk & 3) * 32) >> 4;
+                const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
+                tc::mma_f16_ss(tmem + (ts & 1) * kNC, kd + koff, qd + qoff, kIdescS, kk > 0);
+              }
             }
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t koff = ((kk >> 2) * kHalfKV + (kk & 3) * 32) >> 4;
-              const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
-              tc::mma_f16_ss(tmem + (ts & 1) * kNC, kd + koff, qd + qoff, kIdescS, kk > 0);
-            }
+            tc::commit(bar(kBarS + (ts & 1)));
           }
-          tc::commit(bar(kBarS + (ts & 1)));
+          __syncwarp();
           ++ts;
           if (++s_tile == s_ntiles) {
             s_tile = 0;
@@ -587,35 +596,38 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           }
           progress = true;
         }
-        if (tv < ts && mbar_test_wait(bar(kBarPReady + (tv & 1)), (tv >> 1) & 1) &&
-            (v_tile > 0 || v_np < 2 ||
-             mbar_test_wait(bar(kBarOFree + (v_np & 1)), ((v_np - 2) >> 1) & 1))) {
+        if (tv < ts && test(kBarPReady + (tv & 1), (tv >> 1) & 1) &&
+            (v_tile > 0 || v_np < 2 || test(kBarOFree + (v_np & 1), ((v_np - 2) >> 1) & 1))) {
           tc::fence_after_sync();
           const uint64_t vd = dv0 + uint64_t(((tv % kStages) * kStageBytes) >> 4);
           const uint64_t pd = dp0 + uint64_t(((tv & 1) * kPB) >> 4);
           const uint32_t od = tmem + kColO + (v_np & 1) * kNC;
-          if constexpr (k8) {
-            // 32 tokens per step; P^T holds each 128-token half as kNC rows of
-            // 128 bytes
+          const bool last = v_tile + 1 == v_ntiles;
+          if (tc::elect_one_sync()) {
+            if constexpr (k8) {
+              // 32 tokens per step; P^T holds each 128-token half as kNC rows of
+              // 128 bytes
 #pragma unroll
-            for (int kk = 0; kk < kTT / 32; ++kk) {
-              const uint32_t voff = (kk * 32 * 128) >> 4;  // 32 token rows
-              const uint32_t poff = ((kk >> 2) * kNC * 128 + (kk & 3) * 32) >> 4;
-              tc::mma_f8_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
-            }
-          } else {
+              for (int kk = 0; kk < kTT / 32; ++kk) {
+                const uint32_t voff = (kk * 32 * 128) >> 4;  // 32 token rows
+                const uint32_t poff = ((kk >> 2) * kNC * 128 + (kk & 3) * 32) >> 4;
+                tc::mma_f8_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
+              }
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < kTok / 16; ++kk) {
-              const uint32_t voff = (kk * 16 * 128) >> 4;  // 16 token rows
-              const uint32_t poff = ((kk >> 2) * kPHalf + (kk & 3) * 32) >> 4;
-              tc::mma_f16_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kTok / 16; ++kk) {
+                const uint32_t voff = (kk * 16 * 128) >> 4;  // 16 token rows
+                const uint32_t poff = ((kk >> 2) * kPHalf + (kk & 3) * 32) >> 4;
+                tc::mma_f16_ss(od, vd + voff, pd + poff, kIdescO, (v_tile > 0 || kk > 0) ? 1u : 0u);
+              }
             }
+            tc::commit(bar(kBarPFree + (tv & 1)));
+            tc::commit(bar(L::kBarEmpty + tv % kStages));
+            if (last) tc::commit(bar(kBarODone + (v_np & 1)));
           }
-          tc::commit(bar(kBarPFree + (tv & 1)));
-          tc::commit(bar(L::kBarEmpty + tv % kStages));
+          __syncwarp();
           ++tv;
           if (++v_tile == v_ntiles) {
-            tc::commit(bar(kBarODone + (v_np & 1)));
             v_tile = 0;
             ++v_np;
             v_piece = next_nonempty(a.items, v_piece + 1, p1);
@@ -629,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_decode_tc_kernel(const TcAr
           break;
         }
       }
-      if (!ok) flag_timeout(a);
+      if (!ok && lane == 0) flag_timeout(a);
     }
   } else if (warp < 4) {
     // ------------------------------- softmax -------------------------------

@@ -241,10 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) flag_timeout(a);
    } else if (warp == kWarpMma) {
     // ------------------------------ MMA issuer ------------------------------
-    // Lane 0 alone waits, zeroes stale V rows and issues: a whole-warp wait
-    // and vote around every issue measured ~130 cycles per tcgen05.mma
-    // against ~64 (the tensor core's own rate) for a single thread.
-    if (lane == 0) {
+    // The whole warp runs the loop (its values stay warp-uniform) and zeroes
+    // stale V rows; one elected lane issues the MMAs and their commits.
+    {
       constexpr uint32_t kIdescQK = tc::idesc_f16(Fmt<Tag>::v, 0, kRows, kKeys);
       constexpr uint32_t kIdescPV = tc::idesc_f16(Fmt<Tag>::v, 1, kRows, D);
       const uint64_t dq0 = tc::smem_desc_sw128(sb + kOffQ, 16, 1024);
@@ -255,7 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // that holds the tile's last key but lie past it.
       const int zero_from = kv_end - (ntiles - 1) * kKeys;
       const int zero_to = min(kKeys, (zero_from + a.box_rows - 1) / a.box_rows * a.box_rows);
-      auto wait_all = [&](int b, int parity) { return mbar_wait(bar(b), parity); };
+      auto wait_all = [&](int b, int parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar(b), parity));
+      };
       auto issue_s = [&](int hf, int kt) {
         const uint64_t qd = dq0 + ((hf * kQBytes) >> 4);
         const uint64_t kd = dk0 + (((kt % kKStages) * kKVBytes) >> 4);
@@ -295,35 +296,40 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (ok && v == ntiles - 1 && zero_from < zero_to) {
                 uint8_t* vt = smem + kOffV + (v % kVStages) * kKVBytes;
                 const int n16 = (zero_to - zero_from) * 16;  // 16-byte chunks: 8 per row and half
-                for (int c = 0; c < n16; ++c) {
+                for (int c = lane; c < n16; c += 32) {
                   const int r = zero_from + (c >> 4), half = (c >> 3) & 1, ch = c & 7;
                   *reinterpret_cast<uint4*>(vt + half * kKVHalf + r * 128 + ch * 16) =
                       make_uint4(0u, 0u, 0u, 0u);
                 }
                 fence_proxy_async_smem();
+                __syncwarp();
               }
             }
             if (ok) ok = wait_all(kBarP + hf, v & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            issue_pv(hf, v);
+            if (tc::elect_one_sync()) issue_pv(hf, v);
+            __syncwarp();
           }
           if (kt < nt[hf]) {
             if (hf == 0 || kt >= nt[0]) ok = wait_all(kBarKFull + kt % kKStages, (kt / kKStages) & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            issue_s(hf, kt);
+            if (tc::elect_one_sync()) issue_s(hf, kt);
+            __syncwarp();
           } else if (kt == nt[hf] && nt[hf] > 0) {
-            tc::commit(bar(kBarS + hf));  // the half's last P V is done
+            if (tc::elect_one_sync()) tc::commit(bar(kBarS + hf));  // the half's last P V is done
+            __syncwarp();
           }
         }
         // release the stages the tile's last user has finished with
-        if (ok) {
+        if (ok && tc::elect_one_sync()) {
           if (kt < ntiles) tc::commit(bar(kBarKEmpty + kt % kKStages));
           if (kt >= 1) tc::commit(bar(kBarVEmpty + (kt - 1) % kVStages));
         }
+        __syncwarp();
       }
-      if (!ok) flag_timeout(a);
+      if (!ok && lane == 0) flag_timeout(a);
     }
    }
   } else {

@@ -68,6 +68,19 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
+// One lane of a converged warp (elect.sync over the full mask; the same lane
+// every time the whole warp executes it).  An MMA-issuing loop run by the
+// whole warp, with the issue under this election, keeps its values
+// warp-uniform: measured ~73 cycles per M 128, N 128, K 16 MMA in groups of
+// 8 behind a barrier wait and a fence, against ~93 for the same loop run by
+// lane 0 alone.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred = 0;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(pred));
+  return pred != 0;
+}
+
 // Arrive on an mbarrier once all previously issued tcgen05.mma of this thread
 // have completed.
 __device__ __forceinline__ void commit(uint32_t bar) {
