@@ -70,9 +70,10 @@ constexpr int kThreads = 32 * 12;           // 8 softmax warps, TMA, MMA, 2 idle
 constexpr int kWarpTma = 8, kWarpMma = 9;
 // Register split per warpgroup (setmaxnreg): the block is launched with 168
 // registers a thread (384 x 168 = 64512); the producer warpgroup (TMA, MMA
-// and two idle warps) gives up to 56 so that each softmax thread can hold a
-// whole 128-key score row: 128 x 56 + 256 x 224 = 64512.
-constexpr int kRegsProducer = 56, kRegsSoftmax = 224;
+// and two idle warps) gives up to 72 so that each softmax thread can hold a
+// whole 128-key score row: 128 x 72 + 256 x 216 = 64512 (at 56 / 224 the
+// whole-warp MMA loop spilled).
+constexpr int kRegsProducer = 72, kRegsSoftmax = 216;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * 168, "register split");
 constexpr int kQHalf = kRows * 128;         // 128 rows x 64 16-bit columns (16 KB)
 constexpr int kKVHalf = kKeys * 128;        // 128 keys x 64 16-bit columns (16 KB)

@@ -85,8 +85,8 @@ constexpr int kKeys = 128;                  // keys per K/V tile (N of S)
 constexpr int kThreads = 32 * 12;           // 8 softmax warps, TMA, MMA, 2 idle warps
 constexpr int kWarpTma = 8, kWarpMma = 9;
 // Register split per warpgroup (setmaxnreg), as in the cascade kernel:
-// 128 x 56 + 256 x 224 = 384 x 168.
-constexpr int kRegsProducer = 56, kRegsSoftmax = 224;
+// 128 x 72 + 256 x 216 = 384 x 168.
+constexpr int kRegsProducer = 72, kRegsSoftmax = 216;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * 168, "register split");
 constexpr int kQHalf = kRows * 128;         // 128 rows x 64 16-bit columns (16 KB)
 constexpr int kKVHalf = kKeys * 128;        // 128 keys x 64 16-bit columns (16 KB)
