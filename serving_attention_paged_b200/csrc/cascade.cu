@@ -94,7 +94,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kSlack = 8.f;
 // Pairs of exponentials (out of every 8) taken on the FMA pipe by a
 // polynomial instead of the MUFU unit: balances the two with issue slots.
-constexpr int kPolyPairsPer8 = 2;
+constexpr int kPolyPairsPer8 = 1;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 struct CascadeArgs {

@@ -104,7 +104,7 @@ constexpr int kBarQ = 0, kBarKFull = 1, kBarKEmpty = kBarKFull + kKStages,
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 8 + 1024;  // + slack to align to 1 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr float kSlack = 8.f;
-constexpr int kPolyPairsPer8 = 2;  // pairs of exponentials (of 8) on the FMA pipe
+constexpr int kPolyPairsPer8 = 1;  // pairs of exponentials (of 8) on the FMA pipe
 constexpr float kLn2 = 0.6931471805599453f;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
