@@ -303,9 +303,8 @@ pa_status pa_merge_state(const void* o_a, const float* lse_a, const void* o_b,
  * PA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued, and cascade and
  * prefill plans with PA_ERR_INVALID_ARG.  Nothing is allocated: each call uploads the plan
  * into the array (as pa_plan_upload) and runs it (as pa_run).  The first call
- * on a device looks the array up (cudaGetSymbolAddress), so make it before any
- * stream capture.  The looked-up address is kept for the life of the
- * process: after a cudaDeviceReset on that device this entry point must not
+ * on a device looks the array up (cudaGetSymbolAddress); the looked-up address
+ * is kept for the life of the process: after a cudaDeviceReset on that device this entry point must not
  * be used again.  All calls share the array: calls that overlap on the GPU
  * (different streams or threads) race. */
 pa_status pa_run_static_workspace(pa_plan_t plan, const void* q, const void* k_pool,

@@ -11,8 +11,7 @@
 // The array is kStaticWorkspaceBytes on every GPU that loads the library and
 // stays allocated until the process exits.  Its device address is looked up
 // with cudaGetSymbolAddress on the first call made on each device (with that
-// device current); that first call should therefore come before any stream
-// capture.  The address is cached per device for the life of the process: a
+// device current).  The address is cached per device for the life of the process: a
 // cudaDeviceReset (or anything else that destroys the device's primary
 // context) invalidates it, and the entry point must not be used on that
 // device afterwards.  Every call shares the one array and leaves its contents
