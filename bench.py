@@ -121,7 +121,8 @@ KERNEL_SOURCES = {
     "decode_tc": [_CSRC + f for f in ("decode_tc.cu", "common.cuh", "tcgen05.cuh", "launch.cuh")],
     "decode": [_CSRC + f for f in ("decode.cu", "decode_kernel.cuh", "common.cuh", "launch.cuh")],
     "cascade": [_CSRC + f for f in ("cascade.cu", "attn_tile.cuh", "tcgen05.cuh")],
-    "prefill": [_CSRC + f for f in ("prefill.cu", "attn_tile.cuh", "tcgen05.cuh", "common.cuh")],
+    "prefill": [_CSRC + f for f in ("prefill.cu", "attn_tile.cuh", "tcgen05.cuh", "common.cuh",
+                                    "plan.cpp")],
 }
 
 

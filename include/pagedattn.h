@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 5
+#define PA_ABI_VERSION 6
 
 typedef enum {
   PA_OK = 0,
@@ -213,11 +213,19 @@ typedef struct {
  * qo_indptr[batch]; lse is [total_q, num_qo_heads]; the pools as above.
  * Work: the query tokens of each request are cut into tiles of 256 / G
  * consecutive tokens (G = Hq / Hkv; the last tile of a request may be
- * shorter); the run launches one CTA per (tile, kv head).  Tile order: the
+ * shorter).  Tile order: the
  * tiles of one request together, requests in decreasing order of their
  * longest tile's ceil(kv_end / 128) (ties by request index), and within a
- * request decreasing ceil(kv_end / 128), ties in token order.  num_sms, ctas_per_sm, min_chunk_tokens and
- * piece_cost_tokens are not used.
+ * request decreasing ceil(kv_end / 128), ties in token order.  Item
+ * w = tile * num_kv_heads + kv head is the work of one (tile, kv head).
+ * The run launches min(num_sms, items) persistent CTAs (one per SM; pass the
+ * device's SM count), each running its own list of items in order: the items
+ * are dealt in order w = 0, 1, ... to the CTA with the least estimated load
+ * so far (ties to the lower CTA), an item's load being the 128-key tiles of
+ * its two 128-row halves (ceil(min(kv_base + n0, kv_end) / 128) and, if the
+ * tile has more than n0 = 128 / G tokens, ceil(kv_end / 128)) plus 2.
+ * pa_plan_cta_indptr and pa_plan_prefill_schedule return the lists.
+ * ctas_per_sm, min_chunk_tokens and piece_cost_tokens are not used.
  * Validates as pa_plan_create, plus: qo_indptr[0] == 0 and non-decreasing,
  * total_q < 2^31, and Q_b <= L_b when causal.  page_size must be >= 8
  * (pages move as tensor-memory-access boxes of >= 8 rows) and num_pages *
@@ -230,6 +238,10 @@ pa_status pa_plan_quota_tokens(pa_plan_t plan, int32_t* quota);
 pa_status pa_plan_work_items(pa_plan_t plan, const pa_work_item** items, int64_t* n_items);
 pa_status pa_plan_cta_indptr(pa_plan_t plan, const int32_t** cta_indptr /* [n_cta+1] */,
                              int64_t* n_cta);
+/* Prefill plans: the items of CTA c are items[cta_indptr[c] .. cta_indptr[c + 1]),
+ * each w = tile * num_kv_heads + kv head; n_items = tiles * num_kv_heads
+ * (decode and cascade plans: none). */
+pa_status pa_plan_prefill_schedule(pa_plan_t plan, const int32_t** items, int64_t* n_items);
 pa_status pa_plan_merge_indptr(pa_plan_t plan,
                                const int32_t** merge_indptr /* [B*Hkv+1] */);
 pa_status pa_plan_num_partials(pa_plan_t plan, int64_t* n_partials);

@@ -22,7 +22,9 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 // Device workspace, in this order (each region 256-byte aligned):
 //   items        [n_items]             pa_work_item (pieces, grouped by CTA)
 //   prefill_tiles [n_tiles]            pa_prefill_tile (prefill plans only)
-//   cta_indptr   [n_cta + 1]           int32, pieces of CTA i
+//   prefill_sched [n_tiles * Hkv]      int32 items (tile * Hkv + kv head), grouped by CTA
+//                                      (prefill plans only)
+//   cta_indptr   [n_cta + 1]           int32, pieces (prefill: items) of CTA i
 //   merge_indptr [B * Hkv + 1]         int32, partial slots of segment (b, h)
 //   kv_len       [B]                   int32, tokens per request (rotary plans only:
 //                                      the query's position is kv_len - 1)
@@ -36,7 +38,7 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 //                                      prefix level, chunk 0 holds the merged state
 //   prefix_lse   [prefix_chunks, B, Hq]     fp32, base 2 (cascade only)
 struct WorkspaceLayout {
-  size_t items = 0, prefill_tiles = 0, cta_indptr = 0, merge_indptr = 0, kv_len = 0, counters = 0,
+  size_t items = 0, prefill_tiles = 0, prefill_sched = 0, cta_indptr = 0, merge_indptr = 0, kv_len = 0, counters = 0,
          error = 0, partial_o = 0, partial_lse = 0, prefix_o = 0, prefix_lse = 0, total = 0;
 };
 
@@ -63,6 +65,7 @@ struct pa_plan_s {
   int64_t total_q = 0;
   std::vector<int32_t> qo_indptr;
   std::vector<pa_prefill_tile> prefill_tiles;
+  std::vector<int32_t> prefill_sched;  // items (tile * Hkv + kv head), grouped by CTA
   pa::WorkspaceLayout ws;
   // Bytes [0, ws.partial_o) of the workspace as pa_plan_upload writes them:
   // work list, CTA and merge offsets, zeroed counters and the status words

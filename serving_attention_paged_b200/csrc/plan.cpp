@@ -12,7 +12,10 @@
 #include <array>
 #include <cmath>
 #include <cstring>
+#include <functional>
 #include <new>
+#include <queue>
+#include <utility>
 
 #include "pa_internal.h"
 
@@ -186,6 +189,7 @@ void layout_workspace(pa_plan_s* plan) {
   const size_t Hq = p.num_qo_heads, D = p.head_dim, B = p.batch;
   w.items = take(plan->items.size() * sizeof(pa_work_item));
   w.prefill_tiles = take(plan->prefill_tiles.size() * sizeof(pa_prefill_tile));
+  w.prefill_sched = take(plan->prefill_sched.size() * sizeof(int32_t));
   w.cta_indptr = take(plan->cta_indptr.size() * sizeof(int32_t));
   w.merge_indptr = take(plan->merge_indptr.size() * sizeof(int32_t));
   w.kv_len = take(p.rope_theta > 0.f && !plan->prefill ? B * sizeof(int32_t) : 0);
@@ -208,6 +212,9 @@ void build_upload_image(pa_plan_s* plan) {
   if (!plan->prefill_tiles.empty())
     std::memcpy(img.data() + w.prefill_tiles, plan->prefill_tiles.data(),
                 plan->prefill_tiles.size() * sizeof(pa_prefill_tile));
+  if (!plan->prefill_sched.empty())
+    std::memcpy(img.data() + w.prefill_sched, plan->prefill_sched.data(),
+                plan->prefill_sched.size() * sizeof(int32_t));
   std::memcpy(img.data() + w.cta_indptr, plan->cta_indptr.data(),
               plan->cta_indptr.size() * sizeof(int32_t));
   std::memcpy(img.data() + w.merge_indptr, plan->merge_indptr.data(),
@@ -242,6 +249,51 @@ void schedule_prefix(pa_plan_s* plan) {
   const int64_t chunks = std::max<int64_t>(1, std::min<int64_t>(int64_t(p.num_sms) / base, key_tiles));
   plan->prefix_chunks = int32_t(chunks);
   plan->prefix_chunk_tokens = int32_t(ceil_div(key_tiles, chunks) * kTileKeys);
+}
+
+// Prefill CTAs are persistent: min(num_sms, items) CTAs, each running a list
+// of (tile, kv head) items (item w = tile * Hkv + kv head).  The items are
+// dealt in the plan's tile order by list scheduling: each goes to the CTA
+// whose estimated load is least (ties to the lower CTA), the load of an item
+// being the 128-key tiles its two 128-row halves compute plus a fixed
+// per-item cost.  The CTAs running at a time thus work on neighbouring items
+// of that order (a request's tiles share its K/V in L2), as a launch of one
+// CTA per item would, and the per-CTA lists end within about one item of
+// each other.
+constexpr int64_t kPrefillItemCostTiles = 2;  // fill and drain of one item, in key tiles
+
+int64_t prefill_item_tiles(const pa_prefill_tile& t, int32_t group) {
+  constexpr int64_t kTileKeys = 128;
+  const int64_t per_half = 128 / group;
+  const int64_t nq0 = std::min<int64_t>(t.n_q, per_half), nq1 = t.n_q - nq0;
+  const int64_t nt0 = ceil_div(std::min<int64_t>(int64_t(t.kv_base) + nq0, t.kv_end), kTileKeys);
+  const int64_t nt1 = nq1 > 0 ? ceil_div(t.kv_end, kTileKeys) : 0;
+  return nt0 + nt1;
+}
+
+void schedule_prefill(pa_plan_s* plan) {
+  const int64_t H = plan->prob.num_kv_heads;
+  const int64_t n_items = int64_t(plan->prefill_tiles.size()) * H;
+  const int64_t n_cta = std::min<int64_t>(plan->prob.num_sms, n_items);
+  std::vector<std::vector<int32_t>> lists(size_t(std::max<int64_t>(n_cta, 0)));
+  using Load = std::pair<int64_t, int64_t>;  // (estimated load, CTA)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> least;
+  for (int64_t c = 0; c < n_cta; ++c) least.push({0, c});
+  for (int64_t w = 0; w < n_items; ++w) {
+    const pa_prefill_tile& t = plan->prefill_tiles[size_t(w / H)];
+    const Load top = least.top();
+    least.pop();
+    lists[size_t(top.second)].push_back(int32_t(w));
+    least.push({top.first + prefill_item_tiles(t, plan->group) + kPrefillItemCostTiles,
+                top.second});
+  }
+  plan->prefill_sched.clear();
+  plan->prefill_sched.reserve(size_t(n_items));
+  plan->cta_indptr.assign(1, 0);
+  for (const std::vector<int32_t>& l : lists) {
+    plan->prefill_sched.insert(plan->prefill_sched.end(), l.begin(), l.end());
+    plan->cta_indptr.push_back(int32_t(plan->prefill_sched.size()));
+  }
 }
 
 // Prefill / append tiles: each request's new tokens cut into runs of 256 / G
@@ -291,10 +343,10 @@ pa_status build_prefill(pa_plan_s* plan, bool causal, const int32_t* qo, const i
   plan->last_page_len.assign(last ? last : nullptr, last ? last + B : nullptr);
   if (B > 0) plan->qo_indptr.assign(qo, qo + B + 1);
   else plan->qo_indptr.assign(1, 0);
-  plan->cta_indptr.assign(1, 0);
   plan->merge_indptr.assign(1, 0);
   if (plan->prefill_tiles.size() * size_t(p.num_kv_heads) > size_t(INT32_MAX))
     return PA_ERR_UNSUPPORTED;
+  schedule_prefill(plan);
   return PA_OK;
 }
 
@@ -372,6 +424,13 @@ pa_status pa_plan_prefill_tiles(pa_plan_t plan, const pa_prefill_tile** tiles, i
   if (!plan || !tiles || !n_tiles) return PA_ERR_INVALID_ARG;
   *tiles = plan->prefill_tiles.data();
   *n_tiles = int64_t(plan->prefill_tiles.size());
+  return PA_OK;
+}
+
+pa_status pa_plan_prefill_schedule(pa_plan_t plan, const int32_t** items, int64_t* n_items) {
+  if (!plan || !items || !n_items) return PA_ERR_INVALID_ARG;
+  *items = plan->prefill_sched.data();
+  *n_items = int64_t(plan->prefill_sched.size());
   return PA_OK;
 }
 

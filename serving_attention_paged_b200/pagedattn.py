@@ -63,6 +63,7 @@ _SIGS = {
     "pa_prefill_run": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "pa_plan_quota_tokens": [_vp, _P(_i32)],
     "pa_plan_cta_indptr": [_vp, _P(_P(_i32)), _P(_i64)],
+    "pa_plan_prefill_schedule": [_vp, _P(_P(_i32)), _P(_i64)],
     "pa_plan_work_items": [_vp, _P(_P(pa_work_item)), _P(_i64)],
     "pa_plan_merge_indptr": [_vp, _P(_P(_i32))],
     "pa_plan_num_partials": [_vp, _P(_i64)],
@@ -213,6 +214,17 @@ def pa_plan_cta_indptr(plan: Plan) -> np.ndarray:
     _check(lib.pa_plan_cta_indptr(plan.handle, ctypes.byref(p), ctypes.byref(n)),
            "pa_plan_cta_indptr")
     return np.ctypeslib.as_array(p, shape=(n.value + 1,)).copy()
+
+
+def pa_plan_prefill_schedule(plan: Plan) -> np.ndarray:
+    """A prefill plan's items (tile * num_kv_heads + kv head) grouped by CTA,
+    as an int32 array (a copy); pa_plan_cta_indptr delimits each CTA's list."""
+    p, n = _P(_i32)(), _i64()
+    _check(lib.pa_plan_prefill_schedule(plan.handle, ctypes.byref(p), ctypes.byref(n)),
+           "pa_plan_prefill_schedule")
+    if n.value == 0:
+        return np.zeros(0, dtype=np.int32)
+    return np.ctypeslib.as_array(p, shape=(n.value,)).copy()
 
 
 def pa_plan_work_items(plan: Plan) -> np.ndarray:

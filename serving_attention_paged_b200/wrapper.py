@@ -91,17 +91,20 @@ class PagedPrefill:
 
     def __init__(self, qo_indptr, kv_indptr, last_page_len, *, num_qo_heads, num_kv_heads,
                  page_size, dtype, sm_scale, num_pages, causal=True, head_dim=128, device=None,
-                 flags=0, stream=None):
+                 num_sms=None, flags=0, stream=None):
         self.device = torch.device(device if device is not None else "cuda")
         self.dtype = dtype
         self.batch = len(last_page_len)
         self.total_q = int(qo_indptr[-1]) if self.batch else 0
         self.num_qo_heads, self.head_dim = num_qo_heads, head_dim
-        # the schedule fields do not apply to prefill plans; they only need to be valid
+        # one persistent CTA per SM (ctas_per_sm does not apply to prefill plans)
+        if num_sms is None:
+            num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
         self.problem = C.make_problem(batch=self.batch, num_qo_heads=num_qo_heads,
                                       num_kv_heads=num_kv_heads, head_dim=head_dim,
                                       page_size=page_size, dtype=dtype, sm_scale=sm_scale,
-                                      num_sms=1, ctas_per_sm=1, num_pages=num_pages, flags=flags)
+                                      num_sms=num_sms, ctas_per_sm=1, num_pages=num_pages,
+                                      flags=flags)
         self.plan = C.pa_prefill_plan_create(self.problem, causal, qo_indptr, kv_indptr,
                                              last_page_len)
         self.workspace_bytes = C.pa_plan_workspace_bytes(self.plan)
@@ -111,6 +114,9 @@ class PagedPrefill:
 
     def tiles(self):
         return C.pa_plan_prefill_tiles(self.plan)
+
+    def cta_indptr(self):
+        return C.pa_plan_cta_indptr(self.plan)
 
     def run(self, q, k_pool, v_pool, kv_indices, o=None, lse=None, stream=None):
         if o is None:

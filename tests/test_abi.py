@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(C):
     assert len(names) >= 15
     for n in names:
         assert hasattr(C.lib, n), n
-    assert C.pa_abi_version() == 5
+    assert C.pa_abi_version() == 6
 
 
 def _problem(C, w, num_sms=148, k=2, mct=0, flags=0):

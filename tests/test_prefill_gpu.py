@@ -5,9 +5,9 @@ request's keys up to its limit; the GPU side runs the tensor-core prefill
 kernel through the C ABI.  Cases cover every GQA group, both dtypes, the
 causal rule and attention without the mask, page sizes 8 to 256, requests
 with no new tokens, fresh prefills (Q_b = L_b), single-token appends, ragged
-query tiles and 64-key tiles, stale NaN rows in partly used pages, the
-index bounds check, graph replay, and the full-size prefill workload on
-sampled query tokens.
+query tiles and 64-key tiles, stale NaN rows in partly used pages, few
+persistent CTAs running long item lists, the index bounds check, graph
+replay, and the full-size prefill workload on sampled query tokens.
 """
 import numpy as np
 import pytest
@@ -28,15 +28,16 @@ def _oracle(w, t, causal=True, queries=None):
                                 causal=causal, queries=queries, threads=8)
 
 
-def _prefill(w, causal=True, flags=0):
+def _prefill(w, causal=True, flags=0, num_sms=None):
     from serving_attention_paged_b200.wrapper import PagedPrefill
     return PagedPrefill(w.qo_indptr, w.kv_indptr, w.last_page_len, num_qo_heads=w.num_qo_heads,
                         num_kv_heads=w.num_kv_heads, page_size=w.page_size, dtype=w.dtype,
-                        sm_scale=w.sm_scale, num_pages=w.num_pages, causal=causal, flags=flags)
+                        sm_scale=w.sm_scale, num_pages=w.num_pages, causal=causal, flags=flags,
+                        num_sms=num_sms)
 
 
-def _run(w, dev, causal=True, flags=0):
-    pf = _prefill(w, causal, flags)
+def _run(w, dev, causal=True, flags=0, num_sms=None):
+    pf = _prefill(w, causal, flags, num_sms)
     o, lse = pf.run(dev["q"], dev["k_pool"], dev["v_pool"], dev["kv_indices"])
     torch.cuda.synchronize()
     return pf, o, lse
@@ -75,6 +76,30 @@ def test_prefill_without_mask(dtype):
     o_ref, l_ref = _oracle(w, t, causal=False)
     dev = {k: v.cuda() for k, v in t.items()}
     _check(w, dev, o_ref, l_ref, False, f"no mask {dtype}")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("num_sms", [1, 3, 7])
+def test_prefill_persistent_ctas_run_many_items(dtype, causal, num_sms):
+    """Few persistent CTAs, so each runs a long list of items back to back:
+    items with one or two halves, halves of different tile counts, items
+    without keys and without tokens, across which the CTA carries its
+    barriers, rings and TMEM.  Results equal the oracle's, and bit for bit
+    those of one CTA per SM (every item's arithmetic is the same)."""
+    kv = [200, 0, 77, 1, 150, 64, 300] if not causal else [200, 77, 1, 150, 64, 300]
+    qo = [200, 3, 40, 1, 0, 33, 129] if not causal else [200, 40, 1, 0, 33, 129]
+    w = W.make_workload("pf_persist", kv, num_qo_heads=8, num_kv_heads=2, page_size=16,
+                        dtype=dtype, seed=170 + num_sms, qo_lens=qo)
+    t = w.materialize()
+    o_ref, l_ref = _oracle(w, t, causal=causal)
+    dev = {k: v.cuda() for k, v in t.items()}
+    pf, o, lse = _run(w, dev, causal, num_sms=num_sms)
+    assert pf.check() == -1
+    assert len(pf.cta_indptr()) - 1 == min(num_sms, len(pf.tiles()) * w.num_kv_heads)
+    assert_close(to_np(o), to_np(lse), o_ref, l_ref, dtype, f"{num_sms} CTAs {dtype}")
+    _, o_all, lse_all = _run(w, dev, causal)
+    assert torch.equal(o, o_all) and torch.equal(lse, lse_all)
 
 
 @pytest.mark.parametrize("P", [8, 32, 64, 256])

@@ -17,10 +17,31 @@ def C():
     return pagedattn
 
 
-def _problem(C, batch, hq=32, hkv=8, P=16, flags=0):
+def _problem(C, batch, hq=32, hkv=8, P=16, flags=0, num_sms=1):
     return C.make_problem(batch=batch, num_qo_heads=hq, num_kv_heads=hkv, page_size=P,
-                          dtype="f16", sm_scale=0.088, num_sms=1, ctas_per_sm=1,
+                          dtype="f16", sm_scale=0.088, num_sms=num_sms, ctas_per_sm=1,
                           num_pages=1 << 16, flags=flags)
+
+
+def _item_load(tile, G):
+    """The load the schedule counts for one item, from its tile: the 128-key
+    tiles of its two 128-row halves plus 2."""
+    _, _, n, _, base, end = (int(x) for x in tile)
+    n0 = min(n, 128 // G)
+    nt0 = -(-min(base + n0, end) // 128)
+    nt1 = -(-end // 128) if n > n0 else 0
+    return nt0 + nt1 + 2
+
+
+def _list_schedule(loads, n_cta):
+    """Greedy list scheduling written with an explicit scan (no heap): item w
+    goes to the CTA with the least load so far, the lowest such CTA on ties."""
+    lists, total = [[] for _ in range(n_cta)], [0] * n_cta
+    for w, x in enumerate(loads):
+        c = min(range(n_cta), key=lambda k: (total[k], k))
+        lists[c].append(w)
+        total[c] += x
+    return lists, total
 
 
 def _tables(kv_lens, P):
@@ -197,3 +218,49 @@ def test_prefill_pool_row_limit_at_its_edge(C):
         with pytest.raises(C.PagedAttnError) as e:
             make(prob(1 << 28))
         assert e.value.status == C.PA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("num_sms", [1, 5, 148, 1000])
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (16, 2)])
+def test_persistent_schedule_deals_items_by_least_load(C, num_sms, hq, hkv):
+    """min(num_sms, items) CTAs; every item (tile * Hkv + kv head) exactly once;
+    the lists equal greedy list scheduling in item order by the estimated
+    load; the CTAs' loads end within one item of each other."""
+    rng = np.random.default_rng(num_sms + hq)
+    kv_lens = [int(x) for x in rng.integers(1, 4000, 19)] + [1, 300]
+    qo_lens = [int(rng.integers(0, L + 1)) for L in kv_lens]
+    indptr, last = _tables(kv_lens, 16)
+    qo_indptr = np.concatenate([[0], np.cumsum(qo_lens)]).astype(np.int32)
+    plan = C.pa_prefill_plan_create(_problem(C, len(kv_lens), hq, hkv, num_sms=num_sms), True,
+                                    qo_indptr, indptr, last)
+    tiles = C.pa_plan_prefill_tiles(plan)
+    sched = C.pa_plan_prefill_schedule(plan)
+    ci = C.pa_plan_cta_indptr(plan)
+    n_items = len(tiles) * hkv
+    n_cta = min(num_sms, n_items)
+    assert len(ci) == n_cta + 1 and ci[0] == 0 and ci[-1] == n_items
+    assert np.all(np.diff(ci) >= 0)
+    assert sorted(sched.tolist()) == list(range(n_items))
+    loads = [_item_load(tiles[w // hkv], hq // hkv) for w in range(n_items)]
+    lists, total = _list_schedule(loads, n_cta)
+    assert [sched[ci[c]:ci[c + 1]].tolist() for c in range(n_cta)] == lists
+    assert max(total) - min(total) <= max(loads)
+    assert C.pa_plan_workspace_bytes(plan) >= tiles.nbytes + sched.nbytes
+
+
+def test_item_load_of_a_hand_worked_tile():
+    """G = 4 (32 tokens a half): a causal tile of 64 tokens at keys 1000..1063
+    has half 0 seeing up to key 1032 (9 tiles of 128) and half 1 up to 1064
+    (9 tiles); 20 with the fixed 2.  A 20-token tile has no second half."""
+    assert _item_load((0, 0, 64, 0, 1000, 1064), 4) == 9 + 9 + 2
+    assert _item_load((0, 0, 20, 0, 1000, 1020), 4) == 8 + 0 + 2
+    assert _item_load((0, 0, 64, 0, 1023, 1087), 4) == 9 + 9 + 2
+    assert _item_load((0, 0, 64, 0, 1000, 1024), 8) == 8 + 8 + 2
+
+
+def test_empty_prefill_plan_has_no_ctas(C):
+    indptr, last = _tables([40, 10], 16)
+    plan = C.pa_prefill_plan_create(_problem(C, 2, num_sms=148), True, np.zeros(3, np.int32),
+                                    indptr, last)
+    assert len(C.pa_plan_prefill_schedule(plan)) == 0
+    assert C.pa_plan_cta_indptr(plan).tolist() == [0]
