@@ -7,9 +7,11 @@
 // one dense problem per kv head — the B*G query rows of that head (G q heads
 // per kv head, head-query fusion) against the prefix's K and V — so it is
 // computed once as a tensor-core contraction instead of B times from HBM.
-// The prefix is cut into chunks across CTAs; a small merge kernel combines
-// each row's chunk states by log-sum-exp into one (o, lse), which the
-// level-2 decode kernel merges with the per-request suffix.
+// The prefix is cut into chunks across CTAs, each leaving its rows' states
+// (o, lse) in the workspace; the level-2 decode kernel, launched as a
+// dependent of this one, streams the per-request suffixes while the chunks
+// finish and merges every chunk state of a row with its suffix state by
+// log-sum-exp.
 //
 // CTA = (kv head h, 256 query rows as two halves of 128, prefix chunk); one
 // CTA per SM, 12 warps:
@@ -56,7 +58,6 @@
 #include "common.cuh"
 #include "pa_internal.h"
 #include "attn_tile.cuh"
-#include "launch.cuh"
 #include "tcgen05.cuh"
 
 namespace pa {
@@ -178,8 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
-  // the merge kernel and the decode level may be scheduled from now on: they
-  // wait for this grid before reading its results
+  // the decode level may be scheduled from now on: it waits for this grid
+  // before reading its results
   grid_dependents_launch();
 
   if (warp >= 8) {
@@ -507,55 +508,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Merge the prefix chunks of every (request, q head) row by log-sum-exp into
-// chunk slot 0 (base-2 lse), one warp per row, 4 head elements per lane.
-// The loads of a batch of chunks are all issued before any is used (the
-// merge is a chain of dependent L2 round trips otherwise), and each warp
-// reads all chunks of its row before writing slot 0.
-__global__ void __launch_bounds__(256) cascade_merge_kernel(float* prefix_o, float* prefix_lse,
-                                                            int64_t rows, int chunks) {
-  constexpr int kBatch = 16;  // the chunks of a row in one round of loads, up to 16
-  grid_dependents_launch();  // the decode level may be scheduled
-  grid_dependency_wait();    // the prefix level has completed
-  const int64_t row = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  float M = -INFINITY, L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c0 = 0; c0 < chunks; c0 += kBatch) {
-    float lse[kBatch];
-    float4 o[kBatch];
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      const bool in = c0 + j < chunks;
-      const int64_t c = in ? c0 + j : 0;
-      lse[j] = in ? prefix_lse[c * rows + row] : -INFINITY;
-      o[j] = *reinterpret_cast<const float4*>(prefix_o + (c * rows + row) * D + 4 * lane);
-    }
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      if (lse[j] == -INFINITY) continue;
-      if (lse[j] > M) {
-        const float s = fast_exp2(M - lse[j]);  // M = -inf -> 0
-        L = L * s + 1.f;
-        acc = make_float4(acc.x * s + o[j].x, acc.y * s + o[j].y, acc.z * s + o[j].z,
-                          acc.w * s + o[j].w);
-        M = lse[j];
-      } else {
-        const float w = fast_exp2(lse[j] - M);
-        L += w;
-        acc = make_float4(acc.x + w * o[j].x, acc.y + w * o[j].y, acc.z + w * o[j].z,
-                          acc.w + w * o[j].w);
-      }
-    }
-  }
-  const float inv = M == -INFINITY ? 0.f : 1.f / L;
-  __syncwarp();  // every lane has read slot 0 of this row
-  *reinterpret_cast<float4*>(prefix_o + row * D + 4 * lane) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (lane == 0) prefix_lse[row] = M == -INFINITY ? -INFINITY : M + fast_log2(L);
-}
-
 template <typename Tag>
 cudaError_t launch_t(const CascadeArgs& args, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t stream) {
@@ -615,11 +567,7 @@ int launch_cascade_prefix(const pa_plan_s& plan, const RunPointers& p, void* str
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = pr.dtype == PA_BF16 ? launch_t<BF16>(a, tq, tk, tv, grid, s)
                                       : launch_t<F16>(a, tq, tk, tv, grid, s);
-  if (e != cudaSuccess || plan.prefix_chunks == 1) return int(e);
-  const int64_t rows = int64_t(pr.batch) * pr.num_qo_heads;
-  return int(launch_maybe_dependent(cascade_merge_kernel, dim3(unsigned((rows + 7) / 8)), dim3(256),
-                                    0, s, true, a.prefix_o, a.prefix_lse, rows,
-                                    int(plan.prefix_chunks)));
+  return int(e);
 }
 
 }  // namespace pa

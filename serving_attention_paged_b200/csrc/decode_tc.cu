@@ -1137,8 +1137,8 @@ int launch_decode_tc(const pa_plan_s& plan, const RunPointers& p, void* stream) 
   a.num_qo_heads = pr.num_qo_heads;
   a.num_kv_heads = pr.num_kv_heads;
   a.log2_page = plan.log2_page;
-  // the prefix level leaves each row's merged prefix state in chunk slot 0
-  a.prefix_chunks = plan.cascade && plan.prefix_chunks > 0 ? 1 : 0;
+  // the prefix level leaves prefix_chunks states per row; the epilogue merges them all
+  a.prefix_chunks = plan.cascade ? plan.prefix_chunks : 0;
   const bool kv8 = kv_is_8bit(pr);
   a.score_scale = pr.sm_scale * kLog2e * (kv8 ? pr.k_scale : 1.f);
   a.v_scale = kv8 ? pr.v_scale : 1.f;

@@ -34,8 +34,8 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 //   partial_o    [n_partials, G, D]    fp32, outputs of pieces of split segments
 //                                      (normalised; G = q heads of the kv head)
 //   partial_lse  [n_partials, G]       fp32, their log-sum-exp in base 2
-//   prefix_o     [prefix_chunks, B, Hq, D]  fp32 (cascade only); after the
-//                                      prefix level, chunk 0 holds the merged state
+//   prefix_o     [prefix_chunks, B, Hq, D]  fp32 (cascade only): each prefix
+//                                      chunk's state of every row (normalised)
 //   prefix_lse   [prefix_chunks, B, Hq]     fp32, base 2 (cascade only)
 struct WorkspaceLayout {
   size_t items = 0, prefill_tiles = 0, prefill_sched = 0, cta_indptr = 0, merge_indptr = 0, kv_len = 0, counters = 0,
