@@ -279,7 +279,11 @@ pa_status pa_run(pa_plan_t plan, const void* q, const void* k_pool, const void* 
 /* Cascade run: level 1 attends all B * Hq query rows to the shared prefix
  * (pages d_prefix_indices[0 .. prefix_len / P)) on the tensor cores; level 2
  * is the paged decode over each request's own pages; both are merged by
- * log-sum-exp into o and lse.  The plan must come from pa_cascade_plan_create. */
+ * log-sum-exp into o and lse.  Two launches: level 1 leaves one state per
+ * prefix chunk and row in the workspace, and level 2 (a programmatic
+ * dependent of level 1, which may start while level 1 finishes) merges all
+ * of a row's chunk states with its own in its epilogue.  The plan must come
+ * from pa_cascade_plan_create. */
 pa_status pa_cascade_run(pa_plan_t plan, const void* q, const void* k_pool,
                          const void* v_pool, const int32_t* d_prefix_indices,
                          const int32_t* d_kv_indices, void* o, float* lse, void* d_workspace,
